@@ -1,0 +1,8 @@
+"""Plain CPU oracle of the TTT-Linear scan (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package. It shares no code with the CUDA path.
+"""
+
+from .ttt_oracle import (GRAD_LNJAC, MINIBATCH, NO_LN, build, forward,  # noqa: F401
+                         forward_heads, lngrad, max_threads)

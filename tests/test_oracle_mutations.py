@@ -1,0 +1,82 @@
+"""The oracle's pins must catch plausible slips.
+
+Each case below plants one mistake in a temporary copy of the oracle source
+(on the CPU, never in the CUDA path), builds it, and runs the pin suite
+against that build in a child process. Every mutant must make at least one pin
+fail; the unmodified source must pass.
+"""
+
+import os
+import subprocess
+import sys
+import tempfile
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+SRC = ROOT / "oracle" / "ttt_oracle.cpp"
+
+# (name, text in the oracle source, replacement)
+MUTATIONS = [
+    ("update_sign", "W[r * d + cc] -= eta * G[r] * kt[cc];", "W[r * d + cc] += eta * G[r] * kt[cc];"),
+    ("update_transposed", "W[r * d + cc] -= eta * G[r] * kt[cc];", "W[r * d + cc] -= eta * G[cc] * kt[r];"),
+    ("eta_without_1_over_d", "const S eta = update ? sigmoid(eta_logit[t]) / S(d) : S(0);",
+     "const S eta = update ? sigmoid(eta_logit[t]) : S(0);"),
+    ("output_before_update",
+     "for (int r = 0; r < d; ++r)\n          for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];\n"
+     "        matvec(W.data(), qt, d, Wq.data());",
+     "matvec(W.data(), qt, d, Wq.data());\n        for (int r = 0; r < d; ++r)\n"
+     "          for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];"),
+    ("lnjac_drop_mean_g", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - xhat[f] * mean_gx) / s;"),
+    ("lnjac_drop_xhat_term", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - mean_g) / s;"),
+    ("lnjac_drop_gamma", "g[f] = gamma[f] * (pred[f] - v[f]);", "g[f] = (pred[f] - v[f]);"),
+    ("lnjac_no_1_over_s", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx);"),
+    ("eps_outside_sqrt", "const S s = std::sqrt(var + eps);", "const S s = std::sqrt(var) + eps;"),
+    ("unbiased_variance", "var /= S(d);", "var /= S(d - 1);"),
+    ("drop_beta", "pred[f] = gamma[f] * xhat[f] + beta[f];", "pred[f] = gamma[f] * xhat[f];"),
+    ("no_gate_per_token", "const S gate = gate_logit ? sigmoid(gate_logit[t]) : S(1);\n        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];\n      }\n    } else {",
+     "const S gate = S(1);\n        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];\n      }\n    } else {"),
+    ("minibatch_exclusive_prefix", "for (int j = 0; j <= i; ++j) {", "for (int j = 0; j < i; ++j) {"),
+    ("minibatch_wrong_key_index", "const S a = etas[j] * dot(k + (size_t)(t0 + j) * d, qt, d);",
+     "const S a = etas[j] * dot(k + (size_t)(t0 + i) * d, qt, d);"),
+    ("mask_ignored", "(mask_row == nullptr) || (mask_row[c] != 0)", "true"),
+    ("tail_chunk_dropped", "const int n_chunks = (T + b - 1) / b;\n  std::vector<S> W(",
+     "const int n_chunks = T / b;\n  std::vector<S> W("),
+    ("minibatch_update_uses_q", "const S* kj = k + (size_t)(t0 + j) * d;", "const S* kj = q + (size_t)(t0 + j) * d;"),
+]
+
+
+def _build(src_text, out):
+    with tempfile.NamedTemporaryFile("w", suffix=".cpp", delete=False) as f:
+        f.write(src_text)
+        path = f.name
+    try:
+        subprocess.run(["g++", "-O1", "-std=c++17", "-fopenmp", "-fPIC", "-shared",
+                        "-ffp-contract=off", path, "-o", out], check=True)
+    finally:
+        os.unlink(path)
+
+
+def _run_pins(lib):
+    env = dict(os.environ, TTT_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        str(ROOT / "tests" / "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(name, old, new, tmp_path):
+    text = SRC.read_text()
+    assert text.count(old) >= 1, f"mutation {name}: anchor text not found in the oracle"
+    mutated = text.replace(old, new, 1)
+    lib = str(tmp_path / f"lib_{name}.so")
+    _build(mutated, lib)
+    assert _run_pins(lib) != 0, f"no pin failed for the planted slip '{name}'"
+
+
+def test_unmutated_oracle_passes_pins(tmp_path):
+    lib = str(tmp_path / "lib_clean.so")
+    _build(SRC.read_text(), lib)
+    assert _run_pins(lib) == 0
