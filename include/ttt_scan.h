@@ -1,0 +1,113 @@
+/*
+ * ttt_scan.h -- C ABI of the B200 (sm_100a) TTT-Linear inner-loop scan.
+ *
+ * The scan is the per-(batch row, head) recurrence of "Edifice.Recurrent.TTT",
+ * section "Equations (TTT-Linear)": the hidden state is a d x d fast-weight
+ * matrix W (z = W k, stored row-major as W[out][in]); for every token t
+ *
+ *     eta_t  = sigmoid(eta_logit_t) / d
+ *     pred_t = LayerNorm_{gamma,beta}(W_{t-1} k_t),   err_t = pred_t - v_t
+ *     W_t    = W_{t-1} - eta_t * G_t k_t^T
+ *     o_t    = (W_t q_t) * sigmoid(gate_logit_t)
+ *
+ * where G_t is the simplified gradient err_t (the Equations section) or the full
+ * squared-error gradient through the LayerNorm Jacobian, g = gamma*err,
+ * G = (g - mean(g) - xhat*mean(g*xhat)) / sqrt(var + eps) ("Error Correction in
+ * Trained TTT Layers", Abstract). LayerNorm is over the d features of one head
+ * with biased variance and eps inside the square root.
+ *
+ * Mini-batch mode is the dual form of PonderTTT ("Technical Architecture",
+ * dual-form updates): in each chunk of b tokens every gradient is taken at the
+ * chunk-start state W_s, o_i = sigmoid(gate_i)*(W_s q_i - sum_{j<=i} eta_j
+ * (k_j.q_i) G_j) and W advances once by - sum_j eta_j G_j k_j^T. The last chunk
+ * may be partial (cortex_rust src/layers/ttt.rs, forward_chunkwise).
+ *
+ * The optional mask holds one SKIP/UPDATE byte per chunk of b tokens and per
+ * batch row (PonderTTT, "Core Idea: Binary Gating via Gumbel-Softmax"); a SKIP
+ * chunk has eta = 0 for all its tokens, leaves W bit-for-bit unchanged and still
+ * produces outputs. The granularity is b in both modes.
+ */
+#ifndef TTT_SCAN_H
+#define TTT_SCAN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. Argument errors are reported before anything is launched. */
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = -1,    /* null/misaligned pointer, bad size, aliasing, unknown mode bit */
+  TTT_ERR_UNSUPPORTED = -2,    /* valid arguments this build does not implement (d, b, dtype mix) */
+  TTT_ERR_CUDA = -3,           /* a CUDA runtime call or a launch failed */
+  TTT_ERR_DEVICE_TIMEOUT = -4  /* a bounded in-kernel wait gave up; outputs are not valid */
+} ttt_status;
+
+/* Mode bit flags. */
+enum {
+  TTT_MODE_MINIBATCH = 1u << 0, /* dual-form chunk update; else the exact per-token recurrence */
+  TTT_GRAD_LNJAC = 1u << 1,     /* gradient through the LayerNorm Jacobian; else G = err */
+  TTT_NO_LN = 1u << 2,          /* no LayerNorm: pred = z, G = z - v (delta rule); gamma/beta unused */
+  TTT_IN_BF16 = 1u << 3,        /* q, k, v, eta_logit, gate_logit are bf16; else fp32 */
+  TTT_OUT_BF16 = 1u << 4,       /* o is bf16; else fp32 */
+  TTT_KERNEL_SIMT = 1u << 5     /* run the CUDA-core kernel even where the tensor-core kernel applies */
+};
+
+/*
+ * Run the scan on `cuda_stream` (a cudaStream_t; 0 = legacy default stream).
+ * Enqueue-only: returns once the kernel is launched. Device-side failures are
+ * read with ttt_check_device_status().
+ *
+ * All pointers are DEVICE pointers owned by the caller, 16-byte aligned,
+ * contiguous row-major (a pointer may be NULL when the tensor it names has no
+ * elements, e.g. q..o when T == 0, everything when B*H == 0):
+ *   q, k, v      [B, H, T, d]   fp32, or bf16 with TTT_IN_BF16
+ *   eta_logit    [B, H, T]      same dtype as q
+ *   gate_logit   [B, H, T]      same dtype as q; NULL = no output gate (factor 1)
+ *   W0           [B, H, d, d]   fp32 initial fast weights, z = W k
+ *   gamma, beta  [H, d]         fp32 inner-LayerNorm affine; may be NULL with TTT_NO_LN
+ *   mask         [B, ceil(T/b)] bytes, nonzero = UPDATE, 0 = SKIP; NULL = all UPDATE
+ *   o            [B, H, T, d]   out: fp32, or bf16 with TTT_OUT_BF16; must not overlap any input
+ *   W_T          [B, H, d, d]   out: fp32 final fast weights; may equal W0 (in place), must not
+ *                               otherwise overlap it
+ *   W_chunks     NULL, or out [B, H, ceil(T/b) + 1, d, d] fp32: W before every chunk of b tokens
+ *                and, in the last slot, W after the last token (a debugging aid)
+ * Sizes: B, H, T >= 0 (B*H == 0 launches nothing; T == 0 copies W0 to W_T),
+ *   d in {16, 64}, b >= 1, eps >= 0 (finite).
+ * Kernels: per-token mode runs the CUDA-core kernel for any b. Mini-batch mode
+ *   runs the tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs, and
+ *   otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which takes b <= 16.
+ *   Other combinations return TTT_ERR_UNSUPPORTED.
+ * The library allocates no device memory per call.
+ */
+int ttt_scan_forward(const void* q, const void* k, const void* v,
+                     const void* eta_logit, const void* gate_logit,
+                     const float* W0, const float* gamma, const float* beta,
+                     int B, int H, int T, int d, float eps, unsigned mode, int b,
+                     const unsigned char* mask, void* o, float* W_T,
+                     float* W_chunks, void* cuda_stream);
+
+/*
+ * Synchronise `cuda_stream`, then report and clear the device status word that
+ * the kernels set when a bounded wait gives up. Returns TTT_OK,
+ * TTT_ERR_DEVICE_TIMEOUT, or TTT_ERR_CUDA (a sticky or asynchronous CUDA error).
+ */
+int ttt_check_device_status(void* cuda_stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* ttt_status_string(int status);
+
+/*
+ * Upper bound on the number of polls of each bounded in-kernel wait, for all
+ * later launches of this process (default 2^26). A value of 0 makes every such wait give up at
+ * once, which exercises the timeout path without hanging; waits that only
+ * drain work already in flight keep their own bound. Returns TTT_OK or
+ * TTT_ERR_CUDA.
+ */
+int ttt_set_wait_limit(long long polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_SCAN_H */

@@ -1,0 +1,167 @@
+// C-ABI entry points of the TTT-Linear scan: argument checks, kernel choice,
+// launch, and the device status word. See include/ttt_scan.h for the contract.
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+
+#include "ttt_scan.h"
+#include "common.cuh"
+#include "scan_simt.cuh"
+
+namespace {
+
+// Set to a nonzero code by a kernel whose bounded wait gave up; read and
+// cleared by ttt_check_device_status(). One word per device, no allocation.
+__device__ int g_ttt_status;
+
+long long g_wait_limit = 1LL << 26;
+
+constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
+                                 TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT;
+
+bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Largest divisor of b that is <= cap.
+int largest_divisor_upto(int b, int cap) {
+  for (int c = cap < b ? cap : b; c > 1; --c)
+    if (b % c == 0) return c;
+  return 1;
+}
+
+template <int D, typename InT, typename OutT>
+int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
+  using L = ttt::SimtLayout<D>;
+  auto kernel = ttt::scan_simt_kernel<D, InT, OutT>;
+  if (L::bytes > 48 * 1024) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)L::bytes) != cudaSuccess)
+      return TTT_ERR_CUDA;
+  }
+  kernel<<<(unsigned)(p.B * p.H), L::NT, L::bytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+template <int D>
+int dispatch_simt_dtypes(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
+  const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
+  if (in_bf16 && out_bf16) return launch_simt<D, __nv_bfloat16, __nv_bfloat16>(p, s);
+  if (in_bf16) return launch_simt<D, __nv_bfloat16, float>(p, s);
+  if (out_bf16) return launch_simt<D, float, __nv_bfloat16>(p, s);
+  return launch_simt<D, float, float>(p, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ttt_status_string(int status) {
+  switch (status) {
+    case TTT_OK: return "TTT_OK";
+    case TTT_ERR_INVALID_ARG: return "TTT_ERR_INVALID_ARG";
+    case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED";
+    case TTT_ERR_CUDA: return "TTT_ERR_CUDA";
+    case TTT_ERR_DEVICE_TIMEOUT: return "TTT_ERR_DEVICE_TIMEOUT";
+    default: return "TTT_UNKNOWN_STATUS";
+  }
+}
+
+int ttt_set_wait_limit(long long polls) {
+  if (polls < 0) return TTT_ERR_INVALID_ARG;
+  g_wait_limit = polls;
+  return TTT_OK;
+}
+
+int ttt_check_device_status(void* cuda_stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TTT_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_ttt_status, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_ttt_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+    return TTT_ERR_DEVICE_TIMEOUT;
+  }
+  return TTT_OK;
+}
+
+int ttt_scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
+                     const void* gate_logit, const float* W0, const float* gamma,
+                     const float* beta, int B, int H, int T, int d, float eps, unsigned mode,
+                     int b, const unsigned char* mask, void* o, float* W_T, float* W_chunks,
+                     void* cuda_stream) {
+  // ---- argument checks (nothing is launched on failure) ----
+  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
+  const bool no_ln = mode & TTT_NO_LN;
+  // a pointer may be null only where the tensor it names is empty
+  const bool has_heads = (long long)B * H > 0;
+  if (has_heads && T > 0 && (!q || !k || !v || !eta_logit || !o)) return TTT_ERR_INVALID_ARG;
+  if (has_heads && (!W0 || !W_T)) return TTT_ERR_INVALID_ARG;
+  if (has_heads && !no_ln && (!gamma || !beta)) return TTT_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask, o, W_T, W_chunks};
+  for (const void* p : ptrs)
+    if (misaligned(p)) return TTT_ERR_INVALID_ARG;
+  if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+
+  const size_t heads = (size_t)B * H;
+  const int n_mask_chunks = (T + b - 1) / b;
+  const size_t in_elt = (mode & TTT_IN_BF16) ? 2 : 4;
+  const size_t out_elt = (mode & TTT_OUT_BF16) ? 2 : 4;
+  const size_t tok_bytes = heads * (size_t)T * d * in_elt;
+  const size_t scal_bytes = heads * (size_t)T * in_elt;
+  const size_t o_bytes = heads * (size_t)T * d * out_elt;
+  const size_t w_bytes = heads * (size_t)d * d * sizeof(float);
+  const size_t gb_bytes = (size_t)H * d * sizeof(float);
+  const size_t mask_bytes = (size_t)B * n_mask_chunks;
+  const size_t wc_bytes = heads * (size_t)(n_mask_chunks + 1) * d * d * sizeof(float);
+  struct Span { const void* p; size_t n; };
+  const Span inputs[] = {{q, tok_bytes}, {k, tok_bytes}, {v, tok_bytes},
+                         {eta_logit, scal_bytes}, {gate_logit, scal_bytes},
+                         {W0, w_bytes}, {gamma, no_ln ? 0 : gb_bytes},
+                         {beta, no_ln ? 0 : gb_bytes}, {mask, mask ? mask_bytes : 0}};
+  for (const Span& in : inputs) {
+    if (overlaps(o, o_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+    if (in.p != W0 && overlaps(W_T, w_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+    if (W_chunks && overlaps(W_chunks, wc_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+  }
+  if (W_T != W0 && overlaps(W_T, w_bytes, W0, w_bytes)) return TTT_ERR_INVALID_ARG;
+  if (overlaps(o, o_bytes, W_T, w_bytes)) return TTT_ERR_INVALID_ARG;
+  if (W_chunks && (overlaps(W_chunks, wc_bytes, o, o_bytes) ||
+                   overlaps(W_chunks, wc_bytes, W_T, w_bytes)))
+    return TTT_ERR_INVALID_ARG;
+  if (heads == 0) return TTT_OK;
+
+  ttt::ScanParams p{};
+  p.q = q; p.k = k; p.v = v; p.eta_logit = eta_logit; p.gate_logit = gate_logit;
+  p.W0 = W0; p.gamma = gamma; p.beta = beta; p.mask = mask;
+  p.o = o; p.W_T = W_T; p.W_chunks = W_chunks;
+  p.status = nullptr;
+  p.wait_limit = g_wait_limit;
+  p.B = B; p.H = H; p.T = T; p.b = b; p.n_mask_chunks = n_mask_chunks;
+  p.eps = eps;
+  p.lnjac = (mode & TTT_GRAD_LNJAC) ? 1 : 0;
+  p.no_ln = no_ln ? 1 : 0;
+  p.minibatch = (mode & TTT_MODE_MINIBATCH) ? 1 : 0;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (p.minibatch) {
+    if (b > ttt::kSimtCMax) return TTT_ERR_UNSUPPORTED;
+    p.C = b;
+  } else {
+    // chunks must not straddle a mask / snapshot boundary when either is asked for
+    p.C = (mask || W_chunks) ? largest_divisor_upto(b, ttt::kSimtCMax) : ttt::kSimtCMax;
+  }
+  return d == 64 ? dispatch_simt_dtypes<64>(p, mode, stream)
+                 : dispatch_simt_dtypes<16>(p, mode, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+"""Thin Python binding of ``libttt_scan.so`` (argument marshalling only).
+
+Every step of the scan runs in the library's CUDA kernels; this module checks
+shapes and dtypes, allocates outputs with torch, and passes raw device pointers
+and the current CUDA stream to ``ttt_scan_forward`` (include/ttt_scan.h). There
+is no CPU fallback: if the library cannot be loaded, the first call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+from typing import Optional
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libttt_scan.so"
+
+# Mode bits of include/ttt_scan.h.
+MODE_MINIBATCH = 1 << 0
+GRAD_LNJAC = 1 << 1
+NO_LN = 1 << 2
+IN_BF16 = 1 << 3
+OUT_BF16 = 1 << 4
+KERNEL_SIMT = 1 << 5
+
+TTT_OK = 0
+TTT_ERR_INVALID_ARG = -1
+TTT_ERR_UNSUPPORTED = -2
+TTT_ERR_CUDA = -3
+TTT_ERR_DEVICE_TIMEOUT = -4
+
+
+class TTTScanError(RuntimeError):
+    def __init__(self, status: int, what: str = "ttt_scan_forward"):
+        self.status = status
+        super().__init__(f"{what} failed: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise RuntimeError(
+                f"{_LIB_PATH.name} is missing: build it with "
+                "`python -m test_sequence_layers_02_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(str(_LIB_PATH))
+        vp, i, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        L.ttt_scan_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                       ctypes.c_float, u, i, vp, vp, vp, vp, vp]
+        L.ttt_scan_forward.restype = i
+        L.ttt_check_device_status.argtypes = [vp]
+        L.ttt_check_device_status.restype = i
+        L.ttt_status_string.argtypes = [i]
+        L.ttt_status_string.restype = ctypes.c_char_p
+        L.ttt_set_wait_limit.argtypes = [ctypes.c_longlong]
+        L.ttt_set_wait_limit.restype = i
+        L.ttt_probe_ffma.argtypes = [i, i, i, vp, ctypes.POINTER(ctypes.c_double), vp]
+        L.ttt_probe_ffma.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ttt_status_string(int(status)).decode()
+
+
+def check_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream and return the device status (TTT_OK when clean)."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(lib().ttt_check_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def set_wait_limit(polls: int) -> None:
+    rc = lib().ttt_set_wait_limit(int(polls))
+    if rc != TTT_OK:
+        raise TTTScanError(rc, "ttt_set_wait_limit")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
+         minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
+         b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
+         force_simt: bool = False, want_chunks: bool = False,
+         o: Optional[torch.Tensor] = None, W_T: Optional[torch.Tensor] = None,
+         stream: Optional[torch.cuda.Stream] = None):
+    """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
+
+    q, k, v: [B, H, T, d] fp32 or bf16; eta_logit, gate_logit: [B, H, T] with
+    the same dtype (gate may be None); W0: [B, H, d, d] fp32 (z = W k);
+    gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
+    uint8 or None. ``out_dtype`` defaults to the input dtype.
+
+    CUDA tensors run on ``stream`` (default: the current stream) and return
+    without synchronising. CPU tensors take the end-to-end path: inputs are
+    copied to the current CUDA device, the scan runs there, and o / W_T are
+    copied back to host memory before returning.
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+        q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask = map(
+            mv, (q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask))
+        o_dev, wt_dev = None, None
+    else:
+        o_dev, wt_dev = o, W_T
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, T, d]")
+    B, H, T, d = q.shape
+    in_dtype = q.dtype
+    if in_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("inputs must be float32 or bfloat16")
+    for name, t, shp in (("k", k, (B, H, T, d)), ("v", v, (B, H, T, d)),
+                         ("eta_logit", eta_logit, (B, H, T)), ("gate_logit", gate_logit, (B, H, T))):
+        if t is None and name == "gate_logit":
+            continue
+        if tuple(t.shape) != shp or t.dtype != in_dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous {shp} {in_dtype}")
+    if tuple(W0.shape) != (B, H, d, d) or W0.dtype != torch.float32 or not W0.is_contiguous():
+        raise ValueError("W0: expected contiguous [B, H, d, d] float32")
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if t is None:
+            continue
+        if tuple(t.shape) != (H, d) or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous [H, d] float32")
+    n_chunks = -(-T // b) if b > 0 else 0
+    if mask is not None:
+        if tuple(mask.shape) != (B, n_chunks) or mask.dtype != torch.uint8 or not mask.is_contiguous():
+            raise ValueError(f"mask: expected contiguous [B, {n_chunks}] uint8")
+    out_dtype = out_dtype or in_dtype
+    mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
+            (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
+            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0))
+    if o_dev is None:
+        o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
+    if wt_dev is None:
+        wt_dev = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    wc = (torch.empty((B, H, n_chunks + 1, d, d), dtype=torch.float32, device=q.device)
+          if want_chunks else None)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib().ttt_scan_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W0), _ptr(gamma),
+        _ptr(beta), B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(o_dev), _ptr(wt_dev),
+        _ptr(wc), ctypes.c_void_p(s.cuda_stream))
+    if rc != TTT_OK:
+        raise TTTScanError(rc)
+    if host:
+        o_h = o if o is not None else torch.empty(o_dev.shape, dtype=o_dev.dtype, pin_memory=True)
+        wt_h = W_T if W_T is not None else torch.empty(wt_dev.shape, dtype=torch.float32,
+                                                       pin_memory=True)
+        o_h.copy_(o_dev, non_blocking=True)
+        wt_h.copy_(wt_dev, non_blocking=True)
+        rc = check_device_status(s)
+        if rc != TTT_OK:
+            raise TTTScanError(rc, "device")
+        if want_chunks:
+            return o_h, wt_h, wc.cpu()
+        return o_h, wt_h
+    if want_chunks:
+        return o_dev, wt_dev, wc
+    return o_dev, wt_dev
+
+
+def probe_ffma(blocks: int, threads: int, iters: int, sink: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> float:
+    """Enqueue the FFMA throughput probe; returns the flop count of the launch."""
+    flops = ctypes.c_double(0.0)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    rc = lib().ttt_probe_ffma(blocks, threads, iters, _ptr(sink), ctypes.byref(flops),
+                              ctypes.c_void_p(s.cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"ttt_probe_ffma failed ({rc})")
+    return flops.value

@@ -1,0 +1,126 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments before touching the GPU (these run without a GPU)."""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from test_sequence_layers_02_b200 import build as pkg_build
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkg_build.build()
+    from test_sequence_layers_02_b200 import ttt_scan
+    return ttt_scan.lib()
+
+
+def declared_functions():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(ttt_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_headers_declare_the_boundary():
+    names = declared_functions()
+    for must in ("ttt_scan_forward", "ttt_check_device_status", "ttt_status_string",
+                 "ttt_set_wait_limit", "ttt_probe_ffma"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    from test_sequence_layers_02_b200 import ttt_scan as ts
+    assert ts.status_string(0) == "TTT_OK"
+    assert ts.status_string(-1) == "TTT_ERR_INVALID_ARG"
+    assert ts.status_string(-2) == "TTT_ERR_UNSUPPORTED"
+    assert ts.status_string(-3) == "TTT_ERR_CUDA"
+    assert ts.status_string(-4) == "TTT_ERR_DEVICE_TIMEOUT"
+    assert ts.status_string(12345) == "TTT_UNKNOWN_STATUS"
+
+
+# Fake, 16-byte-aligned, non-overlapping "device" addresses: argument checks
+# reject the calls below before any CUDA call, so nothing is dereferenced.
+BASE = 1 << 40
+STRIDE = 1 << 32
+
+
+def addr(i, off=0):
+    return ctypes.c_void_p(BASE + i * STRIDE + off)
+
+
+def call(lib, **over):
+    a = dict(q=addr(0), k=addr(1), v=addr(2), eta=addr(3), gate=addr(4), W0=addr(5),
+             gamma=addr(6), beta=addr(7), B=2, H=3, T=40, d=64, eps=1e-6, mode=0, b=16,
+             mask=None, o=addr(8), W_T=addr(9), W_chunks=None)
+    a.update(over)
+    return lib.ttt_scan_forward(a["q"], a["k"], a["v"], a["eta"], a["gate"], a["W0"], a["gamma"],
+                                a["beta"], a["B"], a["H"], a["T"], a["d"], a["eps"], a["mode"],
+                                a["b"], a["mask"], a["o"], a["W_T"], a["W_chunks"], None)
+
+
+INVALID, UNSUPPORTED = -1, -2
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(k=None), dict(v=None), dict(eta=None), dict(W0=None), dict(o=None),
+    dict(W_T=None), dict(gamma=None), dict(beta=None),
+    dict(q=addr(0, 4)), dict(o=addr(8, 8)), dict(mask=addr(10, 1)), dict(W_chunks=addr(11, 2)),
+    dict(B=-1), dict(H=-1), dict(T=-1), dict(b=0), dict(b=-3), dict(d=0), dict(d=-64),
+    dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")),
+    dict(mode=1 << 6), dict(mode=1 << 31),
+    dict(o=addr(0)),                      # output over an input
+    dict(o=addr(2, 1 << 12)),             # output inside v
+    dict(W_T=addr(5, 256)),               # W_T partially overlapping W0
+    dict(W_T=addr(8)),                    # W_T over o
+    dict(W_chunks=addr(9)),               # W_chunks over W_T
+], ids=lambda o: ",".join(f"{k}" for k in o))
+def test_invalid_arguments_rejected(lib, over):
+    assert call(lib, **over) == INVALID
+
+
+@pytest.mark.parametrize("over", [dict(d=32), dict(d=128), dict(d=17),
+                                  dict(mode=1, b=17), dict(mode=1 | 32, b=32)])
+def test_unsupported_shapes(lib, over):
+    assert call(lib, **over) == UNSUPPORTED
+
+
+def test_no_ln_needs_no_affine_and_empty_batch_is_noop(lib):
+    # no heads: valid, nothing launched
+    assert call(lib, B=0) == 0
+    assert call(lib, H=0) == 0
+    assert call(lib, B=0, gamma=None, beta=None, mode=4) == 0
+
+
+def test_in_place_W_T_is_accepted_by_the_checks(lib):
+    assert call(lib, B=0, W_T=addr(5)) == 0
+
+
+def test_wait_limit(lib):
+    assert lib.ttt_set_wait_limit(-1) == INVALID
+    assert lib.ttt_set_wait_limit(1 << 26) == 0
+
+
+def test_probe_rejects_bad_arguments(lib):
+    flops = ctypes.c_double()
+    assert lib.ttt_probe_ffma(0, 256, 10, addr(0), ctypes.byref(flops), None) == -1
+    assert lib.ttt_probe_ffma(4, 100, 10, addr(0), ctypes.byref(flops), None) == -1
+    assert lib.ttt_probe_ffma(4, 256, 10, None, ctypes.byref(flops), None) == -1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from test_sequence_layers_02_b200 import ttt_scan as ts
+    monkeypatch.setattr(ts, "_lib", None)
+    monkeypatch.setattr(ts, "_LIB_PATH", tmp_path / "missing.so")
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        ts.lib()

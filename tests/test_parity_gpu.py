@@ -1,0 +1,228 @@
+"""GPU parity: the CUDA path against the CPU oracle on the same seeded inputs.
+
+Tolerances: fp32 per-token / CUDA-core paths |gpu - ref| <= 2e-4 (1 + |ref|)
+elementwise on o and W_T; bf16-output tensor-core paths relative RMS <= 2e-2;
+SKIP chunks bit-exact via the W_chunks snapshots.
+"""
+
+import numpy as np
+import pytest
+
+from test_sequence_layers_02_b200.workloads import WORKLOADS, make_inputs, make_workload
+from tests.helpers import (assert_fp32_close, assert_rrms, gpu_scan, oracle_scan, rel_rms)
+
+pytestmark = pytest.mark.gpu
+
+LNJAC, MINIB, NO_LN = 2, 1, 4
+
+
+def _mode(w):
+    return (MINIB if w.minibatch else 0) | (LNJAC if w.lnjac else 0)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from test_sequence_layers_02_b200 import build, ttt_scan
+    build.build()
+    ttt_scan.lib()
+
+
+# ---------------------------------------------------------------------------
+# The named workloads at their full sizes.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["1", "2s", "2j"])
+def test_workload_fp32_full(name):
+    w = WORKLOADS[name]
+    inp = make_workload(w)
+    o, W_T = gpu_scan(inp, in_bf16=False, eps=w.eps, lnjac=w.lnjac, b=w.b)
+    ro, rW = oracle_scan(inp, eps=w.eps, mode=_mode(w), b=w.b)
+    assert_fp32_close(o, ro, f"{name} o")
+    assert_fp32_close(W_T, rW, f"{name} W_T")
+
+
+def _sample_heads(w, n, seed):
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(w.B * w.H, size=min(n, w.B * w.H), replace=False)
+    return [(int(i) // w.H, int(i) % w.H) for i in sorted(idx)]
+
+
+def _sampled_compare(w, inp, o, W_T, heads, fp32):
+    import oracle
+    res = oracle.forward_heads({k: (np.asarray(v, np.float64) if v is not None and k != "mask" else v)
+                                for k, v in inp.items()}, heads, eps=w.eps, mode=_mode(w), b=w.b)
+    for (bi, h), (ro, rW) in zip(heads, res):
+        if fp32:
+            assert_fp32_close(o[bi, h], ro, f"{w.name} o[{bi},{h}]")
+            assert_fp32_close(W_T[bi, h], rW, f"{w.name} W_T[{bi},{h}]")
+        else:
+            assert_rrms(o[bi, h], ro, f"{w.name} o[{bi},{h}]")
+            assert_rrms(W_T[bi, h], rW, f"{w.name} W_T[{bi},{h}]")
+
+
+def test_workload_4pt_per_token_bf16_in_fp32_out_sampled():
+    w = WORKLOADS["4pt"]
+    inp = make_workload(w)
+    o, W_T = gpu_scan(inp, in_bf16=True, out_bf16=False, eps=w.eps, lnjac=True, b=w.b)
+    _sampled_compare(w, inp, o, W_T, _sample_heads(w, 6, 40), fp32=True)
+
+
+@pytest.mark.parametrize("name", ["3", "4", "5"])
+def test_workload_minibatch_bf16_sampled(name):
+    w = WORKLOADS[name]
+    inp = make_workload(w)
+    o, W_T = gpu_scan(inp, in_bf16=True, out_bf16=True, eps=w.eps, lnjac=True, minibatch=True, b=w.b)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(W_T))
+    _sampled_compare(w, inp, o, W_T, _sample_heads(w, 4, 41), fp32=False)
+
+
+# ---------------------------------------------------------------------------
+# Small cases: several chunks, ragged tails, every mode and dtype mix.
+# ---------------------------------------------------------------------------
+
+CASES = [
+    # (B, H, T, d, mode, b, in_bf16, out_bf16)
+    (2, 3, 53, 16, 0, 16, False, False),
+    (2, 3, 53, 16, LNJAC, 16, False, False),
+    (2, 3, 53, 16, NO_LN, 16, False, False),
+    (2, 3, 77, 64, 0, 16, False, False),
+    (2, 3, 77, 64, LNJAC, 16, False, False),
+    (1, 2, 77, 64, NO_LN, 16, False, False),
+    (2, 2, 70, 64, LNJAC, 24, False, False),     # internal chunk 12 (divides b) with a mask
+    (1, 2, 40, 64, LNJAC, 17, False, False),     # prime b: internal chunk 1
+    (2, 3, 77, 64, LNJAC, 16, True, False),
+    (2, 3, 77, 64, LNJAC, 16, True, True),
+    (2, 3, 77, 64, 0, 16, False, True),
+    (2, 3, 53, 64, MINIB | LNJAC, 16, False, False),
+    (2, 3, 53, 64, MINIB | LNJAC, 7, False, False),
+    (2, 3, 53, 64, MINIB, 16, False, False),
+    (2, 2, 53, 64, MINIB | NO_LN, 5, False, False),
+    (2, 3, 53, 16, MINIB | LNJAC, 16, False, False),
+    (2, 3, 53, 64, MINIB | LNJAC, 16, True, False),
+]
+
+
+@pytest.mark.parametrize("with_mask", [False, True])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}H{c[1]}T{c[2]}d{c[3]}m{c[4]}b{c[5]}"
+                         f"{'i16' if c[6] else ''}{'o16' if c[7] else ''}")
+def test_small_cases(case, with_mask):
+    B, H, T, d, mode, b, in_bf16, out_bf16 = case
+    inp = make_inputs(B, H, T, d, seed=100 + T + d + mode + b, random_affine=True,
+                      in_bf16=in_bf16, mask_p=0.5 if with_mask else None, b=b)
+    eps = 1e-6
+    o, W_T, Wc = gpu_scan(inp, in_bf16=in_bf16, out_bf16=out_bf16, eps=eps, b=b,
+                          lnjac=bool(mode & LNJAC), minibatch=bool(mode & MINIB),
+                          no_ln=bool(mode & NO_LN), force_simt=True, want_chunks=True)
+    ro, rW, rWc = oracle_scan(inp, eps=eps, mode=mode, b=b, want_chunks=True)
+    if out_bf16:
+        assert_rrms(o, ro, "o", tol=1e-2)
+        assert_fp32_close(W_T, rW, "W_T")
+    else:
+        assert_fp32_close(o, ro, "o")
+        assert_fp32_close(W_T, rW, "W_T")
+    assert_fp32_close(Wc, rWc, "W_chunks")
+    if with_mask:
+        m = inp["mask"]
+        for bi in range(B):
+            for c in range(m.shape[1]):
+                same = np.array_equal(Wc[bi, :, c + 1], Wc[bi, :, c])
+                assert same == (m[bi, c] == 0), (bi, c, m[bi, c])
+
+
+def test_minibatch_b1_equals_per_token_on_gpu():
+    inp = make_inputs(2, 2, 45, 64, seed=7, random_affine=True)
+    o1, W1 = gpu_scan(inp, in_bf16=False, eps=1e-6, lnjac=True, b=1)
+    o2, W2 = gpu_scan(inp, in_bf16=False, eps=1e-6, lnjac=True, b=1, minibatch=True)
+    assert_fp32_close(o2, o1, "o")
+    assert_fp32_close(W2, W1, "W_T")
+
+
+def test_eta_zero_and_no_gate():
+    inp = make_inputs(2, 2, 37, 64, seed=8, random_affine=True)
+    inp["eta_logit"] = np.full_like(inp["eta_logit"], -1e4)
+    inp["gate_logit"] = None
+    for mb in (False, True):
+        o, W_T = gpu_scan(inp, in_bf16=False, eps=1e-6, lnjac=True, minibatch=mb, force_simt=True)
+        assert np.array_equal(W_T, inp["W0"].astype(np.float64))
+        ref = np.einsum("bhrc,bhtc->bhtr", inp["W0"].astype(np.float64), inp["q"].astype(np.float64))
+        assert_fp32_close(o, ref, "o")
+
+
+def test_empty_and_single_token():
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    # T = 0: W_T = W0, no outputs
+    inp = make_inputs(2, 2, 0, 64, seed=9)
+    o, W_T = gpu_scan(inp, in_bf16=False, eps=1e-6)
+    assert o.shape == (2, 2, 0, 64)
+    assert np.array_equal(W_T, inp["W0"].astype(np.float64))
+    # T = 1
+    inp = make_inputs(1, 3, 1, 64, seed=10, random_affine=True)
+    for mode in (0, LNJAC, MINIB | LNJAC):
+        o, W_T = gpu_scan(inp, in_bf16=False, eps=1e-6, lnjac=bool(mode & LNJAC),
+                          minibatch=bool(mode & MINIB), force_simt=True)
+        ro, rW = oracle_scan(inp, eps=1e-6, mode=mode, b=16)
+        assert_fp32_close(o, ro, "o")
+        assert_fp32_close(W_T, rW, "W_T")
+    # B*H = 0
+    q = torch.empty((0, 4, 8, 64), device="cuda")
+    z = torch.empty((0, 4, 8), device="cuda")
+    o, W_T = ttt_scan.scan(q, q, q, z, z, torch.empty((0, 4, 64, 64), device="cuda"),
+                           torch.ones((4, 64), device="cuda"), torch.zeros((4, 64), device="cuda"))
+    assert o.shape == (0, 4, 8, 64)
+
+
+def test_in_place_W_T_and_chaining():
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    from tests.helpers import to_torch
+    B, H, T1, T2, d, b = 2, 2, 48, 29, 64, 16
+    inp = make_inputs(B, H, T1 + T2, d, seed=11, random_affine=True, mask_p=0.5, b=b)
+    t = to_torch(inp, "cuda", False)
+    for mb in (False, True):
+        kw = dict(eps=1e-6, lnjac=True, minibatch=mb, b=b, force_simt=True)
+        o, W_T = ttt_scan.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"],
+                               t["gamma"], t["beta"], mask=t["mask"], **kw)
+        n1 = T1 // b
+        W = t["W0"].clone()
+        sl = lambda x, a, z: x[:, :, a:z].contiguous()
+        oa, _ = ttt_scan.scan(sl(t["q"], 0, T1), sl(t["k"], 0, T1), sl(t["v"], 0, T1),
+                              sl(t["eta_logit"], 0, T1), sl(t["gate_logit"], 0, T1), W,
+                              t["gamma"], t["beta"], mask=t["mask"][:, :n1].contiguous(),
+                              W_T=W, **kw)                           # in place
+        ob, Wb = ttt_scan.scan(sl(t["q"], T1, None), sl(t["k"], T1, None), sl(t["v"], T1, None),
+                               sl(t["eta_logit"], T1, None), sl(t["gate_logit"], T1, None), W,
+                               t["gamma"], t["beta"], mask=t["mask"][:, n1:].contiguous(), **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat([oa, ob], dim=2), o)
+        assert torch.equal(Wb, W_T)
+
+
+def test_host_buffers_match_device_path():
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    inp = make_inputs(2, 3, 64, 64, seed=12, random_affine=True)
+    cpu = {k: (None if v is None else torch.from_numpy(np.ascontiguousarray(v)))
+           for k, v in inp.items() if not k.endswith("_bf16")}
+    o_h, W_h = ttt_scan.scan(cpu["q"], cpu["k"], cpu["v"], cpu["eta_logit"], cpu["gate_logit"],
+                             cpu["W0"], cpu["gamma"], cpu["beta"], eps=1e-6, lnjac=True)
+    assert not o_h.is_cuda
+    o_d, W_d = gpu_scan(inp, in_bf16=False, eps=1e-6, lnjac=True)
+    assert np.array_equal(o_h.numpy().astype(np.float64), o_d)
+    assert np.array_equal(W_h.numpy().astype(np.float64), W_d)
+
+
+def test_binding_rejects_bad_shapes():
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    q = torch.zeros((1, 1, 8, 64), device="cuda")
+    with pytest.raises(ValueError):
+        ttt_scan.scan(q, q, q, torch.zeros((1, 1, 7), device="cuda"), None,
+                      torch.zeros((1, 1, 64, 64), device="cuda"), None, None, no_ln=True)
+    with pytest.raises(ttt_scan.TTTScanError) as e:
+        ttt_scan.scan(q, q, q, torch.zeros((1, 1, 8), device="cuda"), None,
+                      torch.zeros((1, 1, 64, 64), device="cuda"), None, None)   # LN needs gamma
+    assert e.value.status == ttt_scan.TTT_ERR_INVALID_ARG
