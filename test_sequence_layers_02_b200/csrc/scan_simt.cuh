@@ -1,276 +1,655 @@
 // CUDA-core (fp32) scan kernel: exact per-token recurrence and mini-batch dual
-// form, any input/output dtype, d in {16, 64}.
+// form, fp32 or bf16 inputs, fp32 or bf16 outputs, d in {16, 64}.
 //
-// One CTA per (batch row, head) keeps W in shared memory in fp32 for the whole
-// sequence. Tokens are processed in chunks of C tokens using the exact
-// chunk identity of the per-token recurrence ("Edifice.Recurrent.TTT",
-// Equations (TTT-Linear)): with W_s the state at the chunk start and
-// a_ij = eta_j (k_j . k_i),
+// One CTA per (batch row, head) keeps W in fp32 for the whole sequence. Tokens
+// run in chunks of C <= 16 through the exact chunk identity of the per-token
+// recurrence ("Edifice.Recurrent.TTT", Equations (TTT-Linear)): with W_s the
+// state at the chunk start and a_mj = eta_j (k_m . k_j),
 //
-//     z_i = W_{i-1} k_i = W_s k_i - sum_{j<i} a_ij G_j
+//     z_m = W_{m-1} k_m = W_s k_m - sum_{j<m} a_mj G_j
 //     o_i = W_i q_i     = W_s q_i - sum_{j<=i} eta_j (k_j . q_i) G_j
-//     W_e = W_s - sum_j eta_j G_j k_j^T
+//     W_e = W_s - sum_j eta_j G_j k_j^T .
 //
-// so the d x d work (W_s K^T, W_s Q^T, the rank-C update) runs on all threads
-// while only the O(C d) gradient chain stays sequential (one warp). Mini-batch
-// mode (PonderTTT, dual-form updates) is the same chunk step without the
-// correction of z_i, with C = b.
+// Mini-batch mode (PonderTTT, dual-form updates) is the same chunk step
+// without the in-chunk correction of z_m (C = b).
+//
+// Warp roles. The last warp is the gradient CHAIN: for chunk c it walks the
+// tokens in order, each needing one LayerNorm reduction (all moments of one
+// token in a single butterfly) and a right-looking update of the pending z's.
+// The other 2d threads are BULK threads that own W in registers (thread t:
+// row r = t % d, columns [d/2 * (t / d), +d/2)) and, while the chain works on
+// chunk c, do everything that does not wait for it:
+//     W_{s,c} = W_{s,c-1} - eta G_{c-1} K_{c-1}      (rank-C update)
+//     Q0_c = Q_c W_{s,c}^T,   P_{c+1} = K_{c+1} W_{s,c}^T
+//     O_{c-1} = gate (Q0_{c-1} - S_{c-1} G_{c-1})      (outputs of chunk c-1)
+//     S_c = tril(Q_c K_c^T) eta, X_{c+1} = K_{c+1} K_c^T eta, A_{c+1} = strict tril(K K^T) eta
+//     cp.async prefetch of the inputs of chunks c+1 / c+2.
+// After both finish, the bulk threads apply the look-ahead correction
+//     z-input of chunk c+1:  Zpre_{c+1} = P_{c+1} - X_{c+1} G_c
+// (because W_{s,c+1} = W_{s,c} - eta G_c K_c), and the next chunk starts.
 #pragma once
 
 #include "common.cuh"
 
 namespace ttt {
 
-constexpr int kSimtCMax = 16;
+constexpr int kC = 16;  // largest chunk of the CUDA-core kernel
 
-template <int D>
-struct SimtLayout {
-  static constexpr int NT = 4 * D;           // threads per CTA
-  static constexpr int NW = NT / 32;         // warps per CTA
-  static constexpr int KP = D + 1;           // padded row stride of the W, K and Q tiles
-  // shared-memory carve-up, in floats
-  static constexpr int oW = 0;                        // W     [D][KP]
-  static constexpr int oK = oW + D * KP;              // K     [CMAX][KP]
-  static constexpr int oQ = oK + kSimtCMax * KP;      // Q     [CMAX][KP]
-  static constexpr int oV = oQ + kSimtCMax * KP;      // V     [CMAX][D]
-  static constexpr int oZ = oV + kSimtCMax * D;       // W_s K^T  [CMAX][D]
-  static constexpr int oQ0 = oZ + kSimtCMax * D;      // W_s Q^T  [CMAX][D]
-  static constexpr int oG = oQ0 + kSimtCMax * D;      // G     [CMAX][D]
-  static constexpr int oAkk = oG + kSimtCMax * D;     // eta_j k_i.k_j, j < i  [CMAX][CMAX]
-  static constexpr int oAqk = oAkk + kSimtCMax * kSimtCMax;  // eta_j q_i.k_j, j <= i
-  static constexpr int oEta = oAqk + kSimtCMax * kSimtCMax;
-  static constexpr int oGate = oEta + kSimtCMax;
-  static constexpr int oGam = oGate + kSimtCMax;
-  static constexpr int oBet = oGam + D;
-  static constexpr int total = oBet + D;
-  static constexpr size_t bytes = sizeof(float) * total;
+template <int D, typename InT>
+struct PipeLayout {
+  static constexpr int NBT = 2 * D;          // bulk threads
+  static constexpr int NT = NBT + 32;        // + the chain warp
+  static constexpr int KH = D / 2;           // columns of W per bulk thread
+  static constexpr int NG = NBT / 32;        // bulk warps
+  static constexpr int ELT = (int)sizeof(InT);
+  static constexpr int ROWB = D * ELT + 16;  // padded row of an input tile (bytes)
+  static constexpr int TILE = kC * ROWB;
+  // byte offsets into dynamic shared memory
+  static constexpr int oK = 0;                         // K tiles, ring of 4
+  static constexpr int oQ = oK + 4 * TILE;             // Q tiles, ring of 2
+  static constexpr int oV = oQ + 2 * TILE;             // V tiles, ring of 2
+  static constexpr int oZ = oV + 2 * TILE;             // P / Zpre   [2][kC][D] f32
+  static constexpr int oG = oZ + 2 * kC * D * 4;       // G          [2][kC][D]
+  static constexpr int oQ0 = oG + 2 * kC * D * 4;      // Q0         [2][kC][D]
+  static constexpr int oPP = oQ0 + 2 * kC * D * 4;     // partial products [2][2kC][D]
+  static constexpr int oA = oPP + 2 * 2 * kC * D * 4;  // in-chunk K Gram [2][kC][kC]
+  static constexpr int oS = oA + 2 * kC * kC * 4;      // Q K Gram   [2][kC][kC]
+  static constexpr int oX = oS + 2 * kC * kC * 4;      // cross Gram [kC][kC]
+  static constexpr int oEta = oX + kC * kC * 4;        // eta        [4][kC]
+  static constexpr int oGate = oEta + 4 * kC * 4;      // gate       [4][kC]
+  static constexpr int oMu = oGate + 4 * kC * 4;       // mean of Zpre rows [2][kC]
+  static constexpr int oMG = oMu + 2 * kC * 4;         // mean of G rows    [2][kC]
+  static constexpr int oFlag = oMG + 2 * kC * 4;       // chunk updates?    [4] int
+  static constexpr int bytes = oFlag + 16;
 };
 
-// Copy n rows of D elements (row stride D in global memory) into shared
-// memory as fp32 rows of stride `stride`, with 16-byte loads.
-template <int D, int NT, typename InT>
-__device__ __forceinline__ void simt_load_rows(const InT* __restrict__ src, int n,
-                                               float* dst, int stride, int tid) {
-  constexpr int VW = Vec16<InT>::N;
-  constexpr int VPR = D / VW;
-  const int nv = n * VPR;
-  for (int idx = tid; idx < nv; idx += NT) {
-    const int row = idx / VPR;
-    const int col = (idx - row * VPR) * VW;
-    float tmp[VW];
-    Vec16<InT>::load(src + (size_t)row * D + col, tmp);
+__device__ __forceinline__ void bulk_barrier(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// 8 consecutive elements of a shared-memory tile row, widened to fp32.
+__device__ __forceinline__ void lds8(const unsigned char* p, float (&x)[8], float) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 16);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void lds8(const unsigned char* p, float (&x)[8], __nv_bfloat16) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int u = 0; u < VW; ++u) dst[row * stride + col + u] = tmp[u];
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ float lds1(const unsigned char* p, float) {
+  return *reinterpret_cast<const float*>(p);
+}
+__device__ __forceinline__ float lds1(const unsigned char* p, __nv_bfloat16) {
+  return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+
+// Asynchronous copy of rows [t0, t0 + n) of a [T][D] head array into a tile
+// (rows >= n are zero-filled).
+template <int D, typename InT>
+__device__ __forceinline__ void tile_load(unsigned char* tile, const InT* src, int t0, int n,
+                                          int tid, int nthreads) {
+  using L = PipeLayout<D, InT>;
+  constexpr int CPR = D * L::ELT / 16;  // 16-byte pieces per row
+  for (int idx = tid; idx < kC * CPR; idx += nthreads) {
+    const int row = idx / CPR;
+    const int piece = idx - row * CPR;
+    const bool ok = row < n;
+    const InT* g = src + (size_t)(t0 + (ok ? row : 0)) * D + piece * (16 / L::ELT);
+    cp_async16(tile + row * L::ROWB + piece * 16, g, ok ? 16 : 0);
   }
 }
 
-// Inner LayerNorm + gradient for token i of the chunk, one warp, lane owns
-// features lane, lane + 32, ... Writes G_i to sG[i]. With `correct`, z_i is
-// W_s k_i minus the contribution of the earlier tokens of the chunk.
-template <int D>
-__device__ __forceinline__ void simt_grad_token(int i, bool correct, const float* sZ,
-                                                const float* sAkk, float* sG,
-                                                const float* sV, const float* sGam,
-                                                const float* sBet, float eps, int lnjac,
-                                                int no_ln, int lane) {
-  constexpr int EPL = (D + 31) / 32;
-  float z[EPL], vv[EPL], G[EPL];
+template <int N>
+__device__ __forceinline__ void butterfly(float (&v)[N]) {
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const int f = lane + 32 * e;
-    float zz = 0.f, v = 0.f;
-    if (f < D) {
-      zz = sZ[i * D + f];
-      if (correct) {
-        for (int j = 0; j < i; ++j) zz -= sAkk[i * kSimtCMax + j] * sG[j * D + f];
-      }
-      v = sV[i * D + f];
-    }
-    z[e] = zz;
-    vv[e] = v;
+  for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
   }
-  if (no_ln) {
+}
+
+// Gradient chain of one chunk (one warp). GM: 0 = simplified (G = err),
+// 1 = through the LayerNorm Jacobian, 2 = no LayerNorm (G = z - v).
+// Reads Zpre (z before in-chunk corrections), A (eta_j k_m.k_j, j < m), V,
+// mu0 (mean of each Zpre row); writes G and, for GM 0, the mean of each G row.
+template <int D, typename InT, bool MINIB, int GM>
+__device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
+                                            const float* __restrict__ A,
+                                            const unsigned char* __restrict__ V,
+                                            const float* __restrict__ mu0, float* __restrict__ Gout,
+                                            float* __restrict__ mGout, float eps,
+                                            const float (&gam)[(D + 31) / 32],
+                                            const float (&bet)[(D + 31) / 32], float Sgb, float Sb,
+                                            int lane) {
+  using L = PipeLayout<D, InT>;
+  constexpr int EPL = (D + 31) / 32;
+  const float inv_d = 1.0f / (float)D;
+  float zr[kC][EPL];
+  float mup[kC];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) G[e] = z[e] - vv[e];
-  } else {
-    const float inv_d = 1.0f / (float)D;
-    float s1 = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) s1 += z[e];  // lanes past D hold 0
-    const float mu = warp_sum(s1) * inv_d;
-    float s2 = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const float dz = (lane + 32 * e < D) ? z[e] - mu : 0.f;
-      s2 += dz * dz;
-    }
-    const float var = warp_sum(s2) * inv_d;
-    const float s = sqrtf(var + eps);
-    float xh[EPL], gg[EPL];
-    float sg = 0.f, sgx = 0.f;
+  for (int i = 0; i < kC; ++i) {
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       const int f = lane + 32 * e;
-      const bool ok = f < D;
-      const float gam = ok ? sGam[f] : 0.f;
-      const float bet = ok ? sBet[f] : 0.f;
-      xh[e] = ok ? (z[e] - mu) / s : 0.f;
-      const float err = ok ? gam * xh[e] + bet - vv[e] : 0.f;
-      G[e] = err;
-      gg[e] = gam * err;
-      sg += gg[e];
-      sgx += gg[e] * xh[e];
+      zr[i][e] = (i < n && f < D) ? Z[i * D + f] : 0.f;
     }
-    if (lnjac) {
-      const float mg = warp_sum(sg) * inv_d;
-      const float mgx = warp_sum(sgx) * inv_d;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) G[e] = (gg[e] - mg - xh[e] * mgx) / s;
-    }
+    mup[i] = (i < n) ? mu0[i] : 0.f;
   }
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const int f = lane + 32 * e;
-    if (f < D) sG[i * D + f] = G[e];
+  for (int i = 0; i < kC; ++i) {
+    if (i >= n) break;
+    float v[EPL], G[EPL];
+    float mG = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      v[e] = (f < D) ? lds1(V + i * L::ROWB + f * L::ELT, InT()) : 0.f;
+    }
+    if (GM == 2) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) G[e] = zr[i][e] - v[e];
+    } else {
+      float y[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) y[e] = (lane + 32 * e < D) ? zr[i][e] - mup[i] : 0.f;
+      if (GM == 1) {
+        // moments of y: sum y^2, sum g2 y, sum g2 y^2, sum w y, sum gamma v
+        float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+        float w[EPL], g2[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          g2[e] = gam[e] * gam[e];
+          w[e] = gam[e] * (bet[e] - v[e]);
+          m[0] = fmaf(y[e], y[e], m[0]);
+          m[1] = fmaf(g2[e], y[e], m[1]);
+          m[2] = fmaf(g2[e] * y[e], y[e], m[2]);
+          m[3] = fmaf(w[e], y[e], m[3]);
+          m[4] = fmaf(gam[e], v[e], m[4]);
+        }
+        butterfly<5>(m);
+        const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+        const float mg = (rs * m[1] + Sgb - m[4]) * inv_d;
+        const float mgx = rs * (rs * m[2] + m[3]) * inv_d;
+        const float rs2 = rs * rs;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) G[e] = rs2 * (g2[e] - mgx) * y[e] + rs * (w[e] - mg);
+      } else {
+        float m[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          m[0] = fmaf(y[e], y[e], m[0]);
+          m[1] = fmaf(gam[e], y[e], m[1]);
+          m[2] += v[e];
+        }
+        butterfly<3>(m);
+        const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) G[e] = gam[e] * rs * y[e] + bet[e] - v[e];
+        mG = (rs * m[1] + Sb - m[2]) * inv_d;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      if (f < D) Gout[i * D + f] = G[e];
+    }
+    if (GM == 0 && lane == 0) mGout[i] = mG;
+    if (!MINIB) {
+#pragma unroll
+      for (int m2 = i + 1; m2 < kC; ++m2) {
+        const float a = A[m2 * kC + i];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) zr[m2][e] = fmaf(-a, G[e], zr[m2][e]);
+        if (GM == 0) mup[m2] = fmaf(-a, mG, mup[m2]);
+      }
+    }
+  }
+  if (GM != 0 && lane < kC) mGout[lane] = 0.f;
+}
+
+// Partial products of a bulk thread: acc[i] = sum over its column half of
+// W[r][k] * rows[i][k], for up to two sets of 16 rows.
+template <int D, typename InT>
+__device__ __forceinline__ void bulk_products(const float (&Wr)[D / 2], const unsigned char* R0,
+                                              const unsigned char* R1, float* PP, int r, int kq) {
+  using L = PipeLayout<D, InT>;
+  constexpr int KH = L::KH;
+  const int koff = kq * KH * L::ELT;
+  float* out = PP + kq * (2 * kC * D);
+#pragma unroll 1
+  for (int i0 = 0; i0 < 2 * kC; i0 += 4) {
+    const unsigned char* R = (i0 < kC) ? R0 : R1;
+    if (R == nullptr) continue;
+    const unsigned char* row = R + (i0 & (kC - 1)) * L::ROWB + koff;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < KH; k += 8) {
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        float x[8];
+        lds8(row + u4 * L::ROWB + k * L::ELT, x, InT());
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u4] = fmaf(Wr[k + u], x[u], acc[u4]);
+      }
+    }
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4) out[(i0 + u4) * D + r] = acc[u4];
   }
 }
 
-template <int D, typename InT, typename OutT>
-__global__ void __launch_bounds__(4 * D) scan_simt_kernel(const ScanParams p) {
-  using L = SimtLayout<D>;
-  constexpr int NT = L::NT;
-  constexpr int KP = L::KP;
-  extern __shared__ float smem[];
-  float* sW = smem + L::oW;
-  float* sK = smem + L::oK;
-  float* sQ = smem + L::oQ;
-  float* sV = smem + L::oV;
-  float* sZ = smem + L::oZ;
-  float* sQ0 = smem + L::oQ0;
-  float* sG = smem + L::oG;
-  float* sAkk = smem + L::oAkk;
-  float* sAqk = smem + L::oAqk;
-  float* sEta = smem + L::oEta;
-  float* sGate = smem + L::oGate;
-  float* sGam = smem + L::oGam;
-  float* sBet = smem + L::oBet;
+// Dot products of left rows with one right row per lane pair (16 rows x 2
+// column halves); returns eta-weighted entries through `emit(i, j, dot)`.
+template <int D, typename InT, typename Emit>
+__device__ __forceinline__ void bulk_gram(const unsigned char* right, const unsigned char* left0,
+                                          const unsigned char* left1, int nleft, int tid,
+                                          Emit emit) {
+  using L = PipeLayout<D, InT>;
+  constexpr int KH = L::KH;
+  const int j = tid & 15;
+  const int kq = (tid >> 4) & 1;
+  const int grp = tid >> 5;
+  float rk[KH];
+#pragma unroll
+  for (int k = 0; k < KH; k += 8) {
+    float x[8];
+    lds8(right + j * L::ROWB + (kq * KH + k) * L::ELT, x, InT());
+#pragma unroll
+    for (int u = 0; u < 8; ++u) rk[k + u] = x[u];
+  }
+  // rows s = grp, grp + NG, ... taken two at a time (nleft / NG is even)
+  for (int s = grp; s < nleft; s += 2 * L::NG) {
+    const int s2 = s + L::NG;
+    const unsigned char* row0 = (s < kC ? left0 : left1) + (s & (kC - 1)) * L::ROWB +
+                                kq * KH * L::ELT;
+    const unsigned char* row1 = (s2 < kC ? left0 : left1) + (s2 & (kC - 1)) * L::ROWB +
+                                kq * KH * L::ELT;
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < KH; k += 8) {
+      float x[8], y[8];
+      lds8(row0 + k * L::ELT, x, InT());
+      lds8(row1 + k * L::ELT, y, InT());
+#pragma unroll
+      for (int u = 0; u < 8; u += 2) {
+        a0 = fmaf(rk[k + u], x[u], a0);
+        a1 = fmaf(rk[k + u + 1], x[u + 1], a1);
+        b0 = fmaf(rk[k + u], y[u], b0);
+        b1 = fmaf(rk[k + u + 1], y[u + 1], b1);
+      }
+    }
+    float acc = a0 + a1, acc2 = b0 + b1;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+    acc2 += __shfl_xor_sync(0xffffffffu, acc2, 16);
+    if (kq == 0) {
+      emit(s, j, acc);
+      emit(s2, j, acc2);
+    }
+  }
+}
+
+// mean of each of the kC rows of a [kC][D] fp32 tile: 8 lanes per row,
+// each summing a strided eighth (conflict-free), then a 3-level shuffle.
+template <int D>
+__device__ __forceinline__ void row_means(const float* Z, float* out, int tid, int nthreads) {
+  for (int base = 0; base < kC * 8; base += nthreads) {
+    const int idx = base + tid;
+    const int m = idx >> 3;
+    const int part = idx & 7;
+    float s = 0.f;
+    if (m < kC) {
+#pragma unroll
+      for (int f = part; f < D; f += 8) s += Z[m * D + f];
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if (m < kC && part == 0) out[m] = s * (1.0f / (float)D);
+  }
+}
+
+template <int D, typename InT, typename OutT, bool MINIB, int GM>
+__global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams p) {
+  using L = PipeLayout<D, InT>;
+  constexpr int NBT = L::NBT;
+  constexpr int KH = L::KH;
+  constexpr int EPL = (D + 31) / 32;
+  extern __shared__ __align__(16) unsigned char smem[];
+  unsigned char* sK = smem + L::oK;
+  unsigned char* sQ = smem + L::oQ;
+  unsigned char* sV = smem + L::oV;
+  float* sZ = reinterpret_cast<float*>(smem + L::oZ);
+  float* sG = reinterpret_cast<float*>(smem + L::oG);
+  float* sQ0 = reinterpret_cast<float*>(smem + L::oQ0);
+  float* sPP = reinterpret_cast<float*>(smem + L::oPP);
+  float* sA = reinterpret_cast<float*>(smem + L::oA);
+  float* sS = reinterpret_cast<float*>(smem + L::oS);
+  float* sX = reinterpret_cast<float*>(smem + L::oX);
+  float* sEta = reinterpret_cast<float*>(smem + L::oEta);
+  float* sGate = reinterpret_cast<float*>(smem + L::oGate);
+  float* sMu = reinterpret_cast<float*>(smem + L::oMu);
+  float* sMG = reinterpret_cast<float*>(smem + L::oMG);
+  int* sFlag = reinterpret_cast<int*>(smem + L::oFlag);
 
   const int tid = threadIdx.x;
+  const bool chain = tid >= NBT;
   const int lane = tid & 31;
-  const int warp = tid >> 5;
   const long long bh = blockIdx.x;
   const int bi = (int)(bh / p.H);
   const int h = (int)(bh - (long long)bi * p.H);
-  const size_t tok0 = (size_t)bh * p.T;
-  const InT* __restrict__ gq = static_cast<const InT*>(p.q) + tok0 * D;
-  const InT* __restrict__ gk = static_cast<const InT*>(p.k) + tok0 * D;
-  const InT* __restrict__ gv = static_cast<const InT*>(p.v) + tok0 * D;
-  const InT* __restrict__ gel = static_cast<const InT*>(p.eta_logit) + tok0;
-  const InT* __restrict__ ggl =
-      p.gate_logit ? static_cast<const InT*>(p.gate_logit) + tok0 : nullptr;
-  OutT* __restrict__ go = static_cast<OutT*>(p.o) + tok0 * D;
-  const float* W0 = p.W0 + (size_t)bh * D * D;  // may alias W_T
+  const int T = p.T;
+  const int C = p.C;
+  const int nc = (T + C - 1) / C;
+  const size_t tok0 = (size_t)bh * T;
+  const InT* gq = static_cast<const InT*>(p.q) + tok0 * D;
+  const InT* gk = static_cast<const InT*>(p.k) + tok0 * D;
+  const InT* gv = static_cast<const InT*>(p.v) + tok0 * D;
+  const InT* gel = static_cast<const InT*>(p.eta_logit) + tok0;
+  const InT* ggl = p.gate_logit ? static_cast<const InT*>(p.gate_logit) + tok0 : nullptr;
+  OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
+  const float inv_d = 1.0f / (float)D;
 
-  for (int e = tid; e < D * D; e += NT) sW[(e / D) * KP + (e % D)] = W0[e];
-  if (tid < D) {
-    sGam[tid] = p.no_ln ? 1.f : p.gamma[(size_t)h * D + tid];
-    sBet[tid] = p.no_ln ? 0.f : p.beta[(size_t)h * D + tid];
+  auto chunk_len = [&](int c) { return min(C, T - c * C); };
+  auto tileK = [&](int c) { return sK + (c & 3) * L::TILE; };
+  auto tileQ = [&](int c) { return sQ + (c & 1) * L::TILE; };
+  auto tileV = [&](int c) { return sV + (c & 1) * L::TILE; };
+  // eta (with the mask folded in), gate and the update flag of chunk c: the raw
+  // values are fetched early (issue) and consumed after the bulk work (finish)
+  // so the global-load latency stays off the critical path.
+  struct RawScalars {
+    InT e, g;
+    unsigned char m;
+  };
+  auto issue_scalars = [&](int c) {
+    RawScalars s;
+    s.e = InT();
+    s.g = InT();
+    s.m = 1;
+    if (tid < kC) {
+      const int t0 = c * C;
+      if (p.mask != nullptr) s.m = p.mask[(size_t)bi * p.n_mask_chunks + t0 / p.b];
+      if (tid < chunk_len(c)) {
+        s.e = gel[t0 + tid];
+        if (ggl) s.g = ggl[t0 + tid];
+      }
+    }
+    return s;
+  };
+  auto finish_scalars = [&](int c, const RawScalars& s) {
+    if (tid < kC) {
+      const bool upd = s.m != 0;
+      const bool ok = tid < chunk_len(c);
+      sEta[(c & 3) * kC + tid] = (ok && upd) ? sigmoidf_(to_f32(s.e)) * inv_d : 0.f;
+      sGate[(c & 3) * kC + tid] = (ok && ggl) ? sigmoidf_(to_f32(s.g)) : 1.f;
+      if (tid == 0) sFlag[c & 3] = upd ? 1 : 0;
+    }
+  };
+
+  // ---------------- prologue ----------------
+  float Wr[KH];
+  const int r = tid % D;
+  const int kq = tid / D;  // meaningful for bulk threads
+  float gam[EPL], bet[EPL];
+  float Sgb = 0.f, Sb = 0.f;
+  if (!chain) {
+    const float* W0 = p.W0 + ((size_t)bh * D + r) * D + kq * KH;  // may alias W_T
+#pragma unroll
+    for (int k = 0; k < KH; k += 4) {
+      const float4 w4 = *reinterpret_cast<const float4*>(W0 + k);
+      Wr[k] = w4.x; Wr[k + 1] = w4.y; Wr[k + 2] = w4.z; Wr[k + 3] = w4.w;
+    }
+    if (nc > 0) {
+      tile_load<D>(tileK(0), gk, 0, chunk_len(0), tid, NBT);
+      tile_load<D>(tileQ(0), gq, 0, chunk_len(0), tid, NBT);
+      tile_load<D>(tileV(0), gv, 0, chunk_len(0), tid, NBT);
+      if (nc > 1) tile_load<D>(tileK(1), gk, C, chunk_len(1), tid, NBT);
+      cp_async_commit();
+      finish_scalars(0, issue_scalars(0));
+      if (nc > 1) finish_scalars(1, issue_scalars(1));
+      cp_async_wait_all();
+    }
+  } else {
+    float sgb = 0.f, sb = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      gam[e] = (f < D && !p.no_ln) ? p.gamma[(size_t)h * D + f] : (f < D ? 1.f : 0.f);
+      bet[e] = (f < D && !p.no_ln) ? p.beta[(size_t)h * D + f] : 0.f;
+      sgb = fmaf(gam[e], bet[e], sgb);
+      sb += bet[e];
+    }
+    float s2[2] = {sgb, sb};
+    butterfly<2>(s2);
+    Sgb = s2[0];
+    Sb = s2[1];
+  }
+  __syncthreads();
+  if (!chain && nc > 0) {
+    // P_0 = K_0 W0^T (no correction), its row means, and A_0
+    bulk_products<D, InT>(Wr, nullptr, tileK(0), sPP, r, kq);
+    if (!MINIB) {
+      const int n0 = chunk_len(0);
+      bulk_gram<D, InT>(tileK(0), tileK(0), nullptr, kC, tid, [&](int m, int j, float dot) {
+        sA[m * kC + j] = (j < m && m < n0) ? sEta[j] * dot : 0.f;
+      });
+    }
+    bulk_barrier(NBT);
+    for (int i = kq; i < kC; i += 2) {
+      sZ[i * D + r] = sPP[(kC + i) * D + r] + sPP[2 * kC * D + (kC + i) * D + r];
+    }
+    bulk_barrier(NBT);
+    row_means<D>(sZ, sMu, tid, NBT);
   }
   __syncthreads();
 
-  const float inv_d = 1.0f / (float)D;
-  for (int t0 = 0; t0 < p.T; t0 += p.C) {
-    const int n = min(p.C, p.T - t0);
-    const int mc = t0 / p.b;
-    const bool upd = (p.mask == nullptr) || (p.mask[(size_t)bi * p.n_mask_chunks + mc] != 0);
-    if (Wc && (t0 % p.b) == 0) {
-      float* dst = Wc + (size_t)mc * D * D;
-      for (int e = tid; e < D * D; e += NT) dst[e] = sW[(e / D) * KP + (e % D)];
-    }
-    simt_load_rows<D, NT>(gk + (size_t)t0 * D, n, sK, KP, tid);
-    simt_load_rows<D, NT>(gq + (size_t)t0 * D, n, sQ, KP, tid);
-    simt_load_rows<D, NT>(gv + (size_t)t0 * D, n, sV, D, tid);
-    if (tid < n) {
-      sEta[tid] = upd ? sigmoidf_(to_f32(gel[t0 + tid])) * inv_d : 0.f;
-      sGate[tid] = ggl ? sigmoidf_(to_f32(ggl[t0 + tid])) : 1.f;
-    }
-    __syncthreads();
-
-    // W_s K^T and W_s Q^T: thread owns output feature r for tokens i = g, g + NT/D, ...
-    {
-      const int r = tid % D;
-      for (int i = tid / D; i < n; i += NT / D) {
-        float az = 0.f, aq = 0.f;
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) {
-          const float w = sW[r * KP + c];
-          az = fmaf(w, sK[i * KP + c], az);
-          aq = fmaf(w, sQ[i * KP + c], aq);
-        }
-        sZ[i * D + r] = az;
-        sQ0[i * D + r] = aq;
-      }
-    }
-    // causal Gram terms of the chunk
-    for (int e = tid; e < n * n; e += NT) {
-      const int i = e / n;
-      const int j = e - i * n;
-      float akk = 0.f, aqk = 0.f;
-      if (j <= i) {
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) {
-          const float kj = sK[j * KP + c];
-          akk = fmaf(sK[i * KP + c], kj, akk);
-          aqk = fmaf(sQ[i * KP + c], kj, aqk);
-        }
-      }
-      sAkk[i * kSimtCMax + j] = (j < i) ? sEta[j] * akk : 0.f;
-      sAqk[i * kSimtCMax + j] = (j <= i) ? sEta[j] * aqk : 0.f;
-    }
-    __syncthreads();
-
-    // inner gradients: a sequential chain (per-token) or independent (mini-batch)
-    if (!p.minibatch) {
-      if (warp == 0) {
-        for (int i = 0; i < n; ++i) {
-          simt_grad_token<D>(i, true, sZ, sAkk, sG, sV, sGam, sBet, p.eps, p.lnjac, p.no_ln, lane);
-          __syncwarp();
-        }
+  // ---------------- chunk loop ----------------
+  for (int c = 0; c < nc; ++c) {
+    const int n = chunk_len(c);
+    const bool has_next = c + 1 < nc;
+    if (chain) {
+      // ===== gradient chain of chunk c =====
+      float* Gc = sG + (c & 1) * kC * D;
+      float* mGc = sMG + (c & 1) * kC;
+      if (sFlag[c & 3]) {
+        chain_chunk<D, InT, MINIB, GM>(n, sZ + (c & 1) * kC * D, sA + (c & 1) * kC * kC,
+                                       tileV(c), sMu + (c & 1) * kC, Gc, mGc, p.eps, gam, bet,
+                                       Sgb, Sb, lane);
+      } else {
+        for (int e = lane; e < kC * D; e += 32) Gc[e] = 0.f;
+        if (lane < kC) mGc[lane] = 0.f;
       }
     } else {
-      for (int i = warp; i < n; i += L::NW)
-        simt_grad_token<D>(i, false, sZ, sAkk, sG, sV, sGam, sBet, p.eps, p.lnjac, p.no_ln, lane);
+      // ===== bulk work that does not wait for the chain =====
+      // prefetch: K_{c+2}, Q_{c+1}, V_{c+1}; raw logits of chunk c+2
+      if (c + 2 < nc) tile_load<D>(tileK(c + 2), gk, (c + 2) * C, chunk_len(c + 2), tid, NBT);
+      if (has_next) {
+        tile_load<D>(tileQ(c + 1), gq, (c + 1) * C, chunk_len(c + 1), tid, NBT);
+        tile_load<D>(tileV(c + 1), gv, (c + 1) * C, chunk_len(c + 1), tid, NBT);
+      }
+      cp_async_commit();
+      RawScalars pre{};
+      if (c + 2 < nc) pre = issue_scalars(c + 2);
+
+      // W_{s,c} = W_{s,c-1} - sum_j eta_j G_j k_j^T over chunk c-1
+      if (c >= 1 && sFlag[(c - 1) & 3]) {
+        const unsigned char* Kt = tileK(c - 1);
+        const float* Gp = sG + ((c - 1) & 1) * kC * D;
+        const float* et = sEta + ((c - 1) & 3) * kC;
+        const int np = chunk_len(c - 1);
+        for (int j = 0; j < np; ++j) {
+          const float ge = et[j] * Gp[j * D + r];
+          const unsigned char* row = Kt + j * L::ROWB + kq * KH * L::ELT;
+#pragma unroll
+          for (int k = 0; k < KH; k += 8) {
+            float x[8];
+            lds8(row + k * L::ELT, x, InT());
+#pragma unroll
+            for (int u = 0; u < 8; ++u) Wr[k + u] = fmaf(-ge, x[u], Wr[k + u]);
+          }
+        }
+      }
+      if (Wc && ((c * C) % p.b) == 0) {
+        float* dst = Wc + ((size_t)((c * C) / p.b) * D + r) * D + kq * KH;
+#pragma unroll
+        for (int k = 0; k < KH; k += 4)
+          *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
+      }
+
+      // outputs of chunk c-1
+      if (c >= 1) {
+        const int np = chunk_len(c - 1);
+        const float* Q0p = sQ0 + ((c - 1) & 1) * kC * D;
+        const float* Sp = sS + ((c - 1) & 1) * kC * kC;
+        const float* Gp = sG + ((c - 1) & 1) * kC * D;
+        const float* gt = sGate + ((c - 1) & 3) * kC;
+        const bool upd = sFlag[(c - 1) & 3];
+        OutT* dst = go + (size_t)(c - 1) * C * D;
+        for (int i = kq; i < np; i += 2) {
+          float acc = Q0p[i * D + r], acc2 = 0.f;
+          if (upd) {
+            int j = 0;
+            for (; j + 1 <= i; j += 2) {
+              acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
+              acc2 = fmaf(-Sp[i * kC + j + 1], Gp[(j + 1) * D + r], acc2);
+            }
+            if (j == i) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
+          }
+          dst[(size_t)i * D + r] = from_f32<OutT>(gt[i] * (acc + acc2));
+        }
+      }
+
+      // Grams: S_c (Q_c K_c^T), X_{c+1} (K_{c+1} K_c^T), A_{c+1} (K_{c+1} K_{c+1}^T)
+      {
+        const float* et = sEta + (c & 3) * kC;
+        float* Sc = sS + (c & 1) * kC * kC;
+        const int n1 = has_next ? chunk_len(c + 1) : 0;
+        bulk_gram<D, InT>(tileK(c), tileQ(c), has_next ? tileK(c + 1) : nullptr,
+                          has_next ? 2 * kC : kC, tid, [&](int s, int j, float dot) {
+                            if (s < kC) {
+                              Sc[s * kC + j] = (j <= s && s < n) ? et[j] * dot : 0.f;
+                            } else {
+                              const int m = s - kC;
+                              sX[m * kC + j] = (j < n && m < n1) ? et[j] * dot : 0.f;
+                            }
+                          });
+        if (!MINIB && has_next) {
+          const float* et1 = sEta + ((c + 1) & 3) * kC;
+          float* An = sA + ((c + 1) & 1) * kC * kC;
+          bulk_gram<D, InT>(tileK(c + 1), tileK(c + 1), nullptr, kC, tid,
+                            [&](int m, int j, float dot) {
+                              An[m * kC + j] = (j < m && m < n1) ? et1[j] * dot : 0.f;
+                            });
+        }
+      }
+
+      // Q0_c = Q_c W_{s,c}^T and P_{c+1} = K_{c+1} W_{s,c}^T
+      bulk_products<D, InT>(Wr, tileQ(c), has_next ? tileK(c + 1) : nullptr, sPP, r, kq);
+      bulk_barrier(NBT);
+      {
+        float* Q0c = sQ0 + (c & 1) * kC * D;
+        float* Pn = sZ + ((c + 1) & 1) * kC * D;
+        for (int i = kq; i < 2 * kC; i += 2) {
+          if (i >= kC && !has_next) break;
+          const float val = sPP[i * D + r] + sPP[2 * kC * D + i * D + r];
+          if (i < kC) Q0c[i * D + r] = val;
+          else Pn[(i - kC) * D + r] = val;
+        }
+      }
+      if (has_next) {
+        bulk_barrier(NBT);
+        row_means<D>(sZ + ((c + 1) & 1) * kC * D, sMu + ((c + 1) & 1) * kC, tid, NBT);
+      }
+      if (c + 2 < nc) finish_scalars(c + 2, pre);
+      cp_async_wait_all();
     }
     __syncthreads();
 
-    // W_e = W_s - sum_j eta_j G_j k_j^T (skipped chunks leave W untouched)
-    if (upd) {
-      for (int e = tid; e < D * D; e += NT) {
-        const int r = e / D;
-        const int c = e - r * D;
-        float acc = sW[r * KP + c];
-        for (int j = 0; j < n; ++j) acc -= (sEta[j] * sG[j * D + r]) * sK[j * KP + c];
-        sW[r * KP + c] = acc;
+    // ===== look-ahead correction: Zpre_{c+1} = P_{c+1} - X_{c+1} G_c =====
+    if (!chain && has_next && sFlag[c & 3]) {
+      const int n1 = chunk_len(c + 1);
+      float* Zn = sZ + ((c + 1) & 1) * kC * D;
+      const float* Gc = sG + (c & 1) * kC * D;
+      for (int m = kq; m < n1; m += 2) {
+        float acc = Zn[m * D + r], acc2 = 0.f;
+        int j = 0;
+        for (; j + 1 < n; j += 2) {
+          acc = fmaf(-sX[m * kC + j], Gc[j * D + r], acc);
+          acc2 = fmaf(-sX[m * kC + j + 1], Gc[(j + 1) * D + r], acc2);
+        }
+        if (j < n) acc = fmaf(-sX[m * kC + j], Gc[j * D + r], acc);
+        Zn[m * D + r] = acc + acc2;
+      }
+      if (tid < n1) {
+        const float* mGc = sMG + (c & 1) * kC;
+        float mu = sMu[((c + 1) & 1) * kC + tid];
+        for (int j = 0; j < n; ++j) mu = fmaf(-sX[tid * kC + j], mGc[j], mu);
+        sMu[((c + 1) & 1) * kC + tid] = mu;
       }
     }
-    // o_i = gate_i (W_s q_i - sum_{j<=i} eta_j (k_j . q_i) G_j)
-    for (int e = tid; e < n * D; e += NT) {
-      const int i = e / D;
-      const int r = e - i * D;
-      float acc = sQ0[i * D + r];
-      for (int j = 0; j <= i; ++j) acc -= sAqk[i * kSimtCMax + j] * sG[j * D + r];
-      go[(size_t)(t0 + i) * D + r] = from_f32<OutT>(sGate[i] * acc);
-    }
     __syncthreads();
   }
 
-  if (Wc) {
-    float* dst = Wc + (size_t)p.n_mask_chunks * D * D;
-    for (int e = tid; e < D * D; e += NT) dst[e] = sW[(e / D) * KP + (e % D)];
+  // ---------------- epilogue ----------------
+  if (!chain) {
+    if (nc > 0) {
+      const int c = nc - 1;
+      const int np = chunk_len(c);
+      if (sFlag[c & 3]) {
+        const unsigned char* Kt = tileK(c);
+        const float* Gp = sG + (c & 1) * kC * D;
+        const float* et = sEta + (c & 3) * kC;
+        for (int j = 0; j < np; ++j) {
+          const float ge = et[j] * Gp[j * D + r];
+          const unsigned char* row = Kt + j * L::ROWB + kq * KH * L::ELT;
+#pragma unroll
+          for (int k = 0; k < KH; k += 8) {
+            float x[8];
+            lds8(row + k * L::ELT, x, InT());
+#pragma unroll
+            for (int u = 0; u < 8; ++u) Wr[k + u] = fmaf(-ge, x[u], Wr[k + u]);
+          }
+        }
+      }
+      const float* Q0p = sQ0 + (c & 1) * kC * D;
+      const float* Sp = sS + (c & 1) * kC * kC;
+      const float* Gp = sG + (c & 1) * kC * D;
+      const float* gt = sGate + (c & 3) * kC;
+      const bool upd = sFlag[c & 3];
+      OutT* dst = go + (size_t)c * C * D;
+      for (int i = kq; i < np; i += 2) {
+        float acc = Q0p[i * D + r];
+        if (upd)
+          for (int j = 0; j <= i; ++j) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
+        dst[(size_t)i * D + r] = from_f32<OutT>(gt[i] * acc);
+      }
+    }
+    if (Wc) {
+      float* dst = Wc + ((size_t)p.n_mask_chunks * D + r) * D + kq * KH;
+#pragma unroll
+      for (int k = 0; k < KH; k += 4)
+        *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
+    }
+    float* WT = p.W_T + ((size_t)bh * D + r) * D + kq * KH;
+#pragma unroll
+    for (int k = 0; k < KH; k += 4)
+      *reinterpret_cast<float4*>(WT + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
   }
-  float* WT = p.W_T + (size_t)bh * D * D;
-  for (int e = tid; e < D * D; e += NT) WT[e] = sW[(e / D) * KP + (e % D)];
 }
 
 }  // namespace ttt

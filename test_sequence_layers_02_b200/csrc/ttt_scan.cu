@@ -35,10 +35,10 @@ int largest_divisor_upto(int b, int cap) {
   return 1;
 }
 
-template <int D, typename InT, typename OutT>
+template <int D, typename InT, typename OutT, bool MINIB, int GM>
 int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
-  using L = ttt::SimtLayout<D>;
-  auto kernel = ttt::scan_simt_kernel<D, InT, OutT>;
+  using L = ttt::PipeLayout<D, InT>;
+  auto kernel = ttt::scan_simt_kernel<D, InT, OutT, MINIB, GM>;
   if (L::bytes > 48 * 1024) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L::bytes) != cudaSuccess)
@@ -48,13 +48,26 @@ int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
+template <int D, typename InT, typename OutT>
+int dispatch_simt_mode(const ttt::ScanParams& p, cudaStream_t s) {
+  const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
+  if (p.minibatch) {
+    if (gm == 0) return launch_simt<D, InT, OutT, true, 0>(p, s);
+    if (gm == 1) return launch_simt<D, InT, OutT, true, 1>(p, s);
+    return launch_simt<D, InT, OutT, true, 2>(p, s);
+  }
+  if (gm == 0) return launch_simt<D, InT, OutT, false, 0>(p, s);
+  if (gm == 1) return launch_simt<D, InT, OutT, false, 1>(p, s);
+  return launch_simt<D, InT, OutT, false, 2>(p, s);
+}
+
 template <int D>
 int dispatch_simt_dtypes(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
   const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
-  if (in_bf16 && out_bf16) return launch_simt<D, __nv_bfloat16, __nv_bfloat16>(p, s);
-  if (in_bf16) return launch_simt<D, __nv_bfloat16, float>(p, s);
-  if (out_bf16) return launch_simt<D, float, __nv_bfloat16>(p, s);
-  return launch_simt<D, float, float>(p, s);
+  if (in_bf16 && out_bf16) return dispatch_simt_mode<D, __nv_bfloat16, __nv_bfloat16>(p, s);
+  if (in_bf16) return dispatch_simt_mode<D, __nv_bfloat16, float>(p, s);
+  if (out_bf16) return dispatch_simt_mode<D, float, __nv_bfloat16>(p, s);
+  return dispatch_simt_mode<D, float, float>(p, s);
 }
 
 }  // namespace
@@ -154,11 +167,11 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   if (p.minibatch) {
-    if (b > ttt::kSimtCMax) return TTT_ERR_UNSUPPORTED;
+    if (b > ttt::kC) return TTT_ERR_UNSUPPORTED;
     p.C = b;
   } else {
     // chunks must not straddle a mask / snapshot boundary when either is asked for
-    p.C = (mask || W_chunks) ? largest_divisor_upto(b, ttt::kSimtCMax) : ttt::kSimtCMax;
+    p.C = (mask || W_chunks) ? largest_divisor_upto(b, ttt::kC) : ttt::kC;
   }
   return d == 64 ? dispatch_simt_dtypes<64>(p, mode, stream)
                  : dispatch_simt_dtypes<16>(p, mode, stream);
