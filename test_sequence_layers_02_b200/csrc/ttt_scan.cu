@@ -8,12 +8,11 @@
 #include "ttt_scan.h"
 #include "common.cuh"
 #include "scan_simt.cuh"
+#include "scan_tc.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace {
-
-// Set to a nonzero code by a kernel whose bounded wait gave up; read and
-// cleared by ttt_check_device_status(). One word per device, no allocation.
-__device__ int g_ttt_status;
 
 long long g_wait_limit = 1LL << 26;
 
@@ -61,6 +60,64 @@ int dispatch_simt_mode(const ttt::ScanParams& p, cudaStream_t s) {
   return launch_simt<D, InT, OutT, false, 2>(p, s);
 }
 
+// ---- tensor-core kernel: tensor maps and launch ----
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [B*H][T][64] bf16 viewed as a 3-D tensor {64, T, B*H}; box {64, 16, 1}.
+bool encode_qkv_map(CUtensorMap* map, const void* base, int T, long long heads, bool swizzle) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
+  const cuuint32_t box[3] = {64, 16, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename OutT, int GM>
+int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
+  ttt::TcMaps maps;
+  const long long heads = (long long)p.B * p.H;
+  if (!encode_qkv_map(&maps.q, p.q, p.T, heads, true) ||
+      !encode_qkv_map(&maps.k, p.k, p.T, heads, true) ||
+      !encode_qkv_map(&maps.v, p.v, p.T, heads, false))
+    return TTT_ERR_CUDA;
+  auto kernel = ttt::scan_tc_kernel<OutT, GM>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ttt::tc::kSmemBytes) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)heads, ttt::tc::NT, ttt::tc::kSmemBytes, stream>>>(p, maps);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int dispatch_tc(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
+  const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
+  if (mode & TTT_OUT_BF16) {
+    if (gm == 0) return launch_tc<__nv_bfloat16, 0>(p, s);
+    if (gm == 1) return launch_tc<__nv_bfloat16, 1>(p, s);
+    return launch_tc<__nv_bfloat16, 2>(p, s);
+  }
+  if (gm == 0) return launch_tc<float, 0>(p, s);
+  if (gm == 1) return launch_tc<float, 1>(p, s);
+  return launch_tc<float, 2>(p, s);
+}
+
 template <int D>
 int dispatch_simt_dtypes(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
   const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
@@ -95,10 +152,10 @@ int ttt_check_device_status(void* cuda_stream) {
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return TTT_ERR_CUDA;
   int h = 0;
-  if (cudaMemcpyFromSymbol(&h, g_ttt_status, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&h, ttt::g_ttt_status, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
   if (h != 0) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_ttt_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+    if (cudaMemcpyToSymbol(ttt::g_ttt_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
     return TTT_ERR_DEVICE_TIMEOUT;
   }
   return TTT_OK;
@@ -166,6 +223,9 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   p.minibatch = (mode & TTT_MODE_MINIBATCH) ? 1 : 0;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const bool tc_ok = p.minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
+                     !(mode & TTT_KERNEL_SIMT) && T > 0;
+  if (tc_ok) return dispatch_tc(p, mode, stream);
   if (p.minibatch) {
     if (b > ttt::kC) return TTT_ERR_UNSUPPORTED;
     p.C = b;
