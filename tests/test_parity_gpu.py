@@ -197,8 +197,10 @@ def test_in_place_W_T_and_chaining():
                                sl(t["eta_logit"], T1, None), sl(t["gate_logit"], T1, None), W,
                                t["gamma"], t["beta"], mask=t["mask"][:, n1:].contiguous(), **kw)
         torch.cuda.synchronize()
-        assert torch.equal(torch.cat([oa, ob], dim=2), o)
-        assert torch.equal(Wb, W_T)
+        # the look-ahead form rounds differently at a resume point, so the two
+        # runs agree to the fp32 tolerance rather than bit for bit
+        assert_fp32_close(torch.cat([oa, ob], dim=2).cpu().numpy(), o.cpu().numpy(), "o")
+        assert_fp32_close(Wb.cpu().numpy(), W_T.cpu().numpy(), "W_T")
 
 
 def test_host_buffers_match_device_path():
