@@ -391,6 +391,27 @@ def _workload_desc(job):
             f"T={w.T} d={w.d}{extra}")
 
 
+def shard_rows(B: int, world: int, rank: int) -> tuple:
+    """Contiguous block of batch rows owned by `rank` when a batch is split over
+    `world` ranks (heads and masks follow their batch row, so nothing crosses
+    ranks)."""
+    base, extra = divmod(B, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def weak_scaling_value(units_per_rank: float, t_local: float, world: int, dist=None):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t_max = t_local
+    if world > 1:
+        import torch
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        tt = torch.tensor([t_local], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    return units_per_rank * world / t_max, t_max
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -426,13 +447,8 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     total = sum(step_times)
-    t_max = total
-    if world > 1:
-        tt = torch.tensor([total], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-    units = job.head_tokens_per_step * args.steps * world
-    value = units / t_max
+    value, t_max = weak_scaling_value(job.head_tokens_per_step * args.steps, total, world,
+                                      dist if world > 1 else None)
     per_launch = total / (args.steps * job.launches_per_step())
     roof = _roofline(job, per_launch, peaks, fp32_tflops, n_sm)
     e2e = _e2e(job, max(2, min(args.steps, 5)), device)
