@@ -99,7 +99,7 @@ const char* ttt_status_string(int status);
 
 /*
  * Upper bound on the number of polls of each bounded in-kernel wait, for all
- * later launches of this process (default 2^26). A value of 0 makes every such wait give up at
+ * later launches of this process (default 2^20). A value of 0 makes every such wait give up at
  * once, which exercises the timeout path without hanging; waits that only
  * drain work already in flight keep their own bound. Returns TTT_OK or
  * TTT_ERR_CUDA.

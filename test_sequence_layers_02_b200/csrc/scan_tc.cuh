@@ -404,6 +404,19 @@ __global__ void __launch_bounds__(tc::NT, 3)
     for (int k = 0; k < nc; ++k) {
       const int n = chunk_len(k);
       const bool upd = sFlag[k & (kSR - 1)] != 0;
+      // operands that do not depend on Z_k, fetched before waiting for it
+      float v[8], gam[8], bet[8];
+      {
+        const unsigned char* Vt = tV(k) + tm_m * D * 2;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int f = tm_p + 8 * u;
+          v[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Vt + f * 2));
+          gam[u] = sGam[f];
+          bet[u] = sBet[f];
+        }
+      }
+      const float eta = (tm_m < n) ? sEta[(k & (kSR - 1)) * CB + tm_m] : 0.f;
       bool ok;
       if (k == 0) ok = mbar_wait_bounded(bar_pro, 0, lim);
       else ok = mbar_wait_bounded(&bar_z[k & 1], (uint32_t)(((k - 1) >> 1) & 1), lim);
@@ -425,27 +438,20 @@ __global__ void __launch_bounds__(tc::NT, 3)
       if (upd) {
         // token-major LayerNorm + gradient: token tm_m, features tm_p + 8u
         const float* Zk = sZ + (k & 1) * CB * kZS + tm_m * kZS;
-        const unsigned char* Vt = tV(k) + tm_m * D * 2;
-        float z[8], v[8], G[8];
+        float z[8], G[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int f = tm_p + 8 * u;
-          z[u] = Zk[f];
-          v[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Vt + f * 2));
-        }
+        for (int u = 0; u < 8; ++u) z[u] = Zk[tm_p + 8 * u];
         if (GM == 2) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) G[u] = z[u] - v[u];
         } else {
           // shift by one element of the token, then all moments in one round
           const float c0 = __shfl_sync(0xffffffffu, z[0], lane & ~7);
-          float y[8], gam[8], w[8];
+          float y[8], w[8];
           float m[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int f = tm_p + 8 * u;
-            gam[u] = sGam[f];
-            w[u] = gam[u] * (sBet[f] - v[u]);   // gamma (beta - v)
+            w[u] = gam[u] * (bet[u] - v[u]);    // gamma (beta - v)
             y[u] = z[u] - c0;
             m[0] += y[u];
             m[1] = fmaf(y[u], y[u], m[1]);
@@ -481,14 +487,10 @@ __global__ void __launch_bounds__(tc::NT, 3)
             }
           } else {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int f = tm_p + 8 * u;
-              G[u] = fmaf(gam[u] * rs, y[u] - mu1, sBet[f]) - v[u];
-            }
+            for (int u = 0; u < 8; ++u) G[u] = fmaf(gam[u] * rs, y[u] - mu1, bet[u]) - v[u];
           }
           (void)sgb;
         }
-        const float eta = (tm_m < n) ? sEta[(k & (kSR - 1)) * CB + tm_m] : 0.f;
         unsigned char* An = aneg(k);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -517,28 +519,26 @@ __global__ void __launch_bounds__(tc::NT, 3)
       // ---- W_{s,c+1} (fp32 TMEM) -> bf16 operand; snapshot ----
       const int row = wq * 32 + lane;
       if (upd) {
+        float w[64];
+        tmem_ld32(tmem + tlane + kColW, *reinterpret_cast<float(*)[32]>(&w[0]));
+        tmem_ld32(tmem + tlane + kColW + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+        tmem_wait_ld();
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float w[32];
-          tmem_ld32(tmem + tlane + kColW + 32 * hf, w);
-          tmem_wait_ld();
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint4 u;
-            u.x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
-            u.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
-            u.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
-            u.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
-            *reinterpret_cast<uint4*>(sWb + sw128_off(row, 4 * hf + ch)) = u;
-          }
-          if (Wc && row < 64) {
-            float* dst = Wc + ((size_t)(c + 1) * D + row) * D + 32 * hf;
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-              *reinterpret_cast<float4*>(dst + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
-          }
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 u;
+          u.x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
+          u.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
+          u.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
+          u.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
+          *reinterpret_cast<uint4*>(sWb + sw128_off(row, ch)) = u;
         }
         fence_proxy_async_smem();
+        if (Wc && row < 64) {
+          float* dst = Wc + ((size_t)(c + 1) * D + row) * D;
+#pragma unroll
+          for (int k = 0; k < 64; k += 4)
+            *reinterpret_cast<float4*>(dst + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+        }
       } else if (Wc && row < 64) {
         const float* srcw = Wc + ((size_t)c * D + row) * D;  // W unchanged: repeat the snapshot
         float* dst = Wc + ((size_t)(c + 1) * D + row) * D;
@@ -605,6 +605,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
       if (c + 1 < nc) mma_commit(&bar_z[(c + 1) & 1]);
       mma_commit(bar_w);
       ++w_issued;
+
       if (c + 1 < nc) {
         // W_{s,c+1} in bf16 and the tiles of stage c+2 = {K_{c+2}, Q_{c+1}}
         ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) &&
@@ -618,13 +619,10 @@ __global__ void __launch_bounds__(tc::NT, 3)
         mma_commit(bar_gram);
         mma_ws(tmem + col_p((c + 2) & 1), tKQ(c + 2), 32);          // [P_{c+2} | Q0_{c+1}]
       }
-      // refill: stage c % NST (K_c read by MMA3 of this chunk) with load c + NST
+      // refill stage c % NST with load c + NST. Its K_c was last read by MMA3 of
+      // this chunk, which completed before the bulk warps signalled bar_wb
+      // (c + NST <= nc implies c + 1 < nc, so that wait happened above).
       if (c + NST <= nc) {
-        ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
-        if (!ok || *sAbort) {
-          fail();
-          break;
-        }
         fence_proxy_async_smem();
         issue_tma(c + NST);
       }

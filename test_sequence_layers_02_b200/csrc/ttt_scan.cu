@@ -14,7 +14,7 @@
 
 namespace {
 
-long long g_wait_limit = 1LL << 26;
+long long g_wait_limit = 1LL << 20;
 
 constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
                                  TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT;

@@ -89,7 +89,7 @@ def test_tc_wait_timeout_reports_and_recovers():
         ttt_scan.scan(*args, eps=1e-6, b=16, minibatch=True, lnjac=True)
         assert ttt_scan.check_device_status() == ttt_scan.TTT_ERR_DEVICE_TIMEOUT
     finally:
-        ttt_scan.set_wait_limit(1 << 26)
+        ttt_scan.set_wait_limit(1 << 20)
     assert ttt_scan.check_device_status() == ttt_scan.TTT_OK   # cleared by the read
     o, W_T = ttt_scan.scan(*args, eps=1e-6, b=16, minibatch=True, lnjac=True)
     torch.cuda.synchronize()
