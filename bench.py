@@ -209,63 +209,74 @@ def _time_job(job, steps, warmup, flush_buf):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    few milliseconds while the timed region runs (read-only queries)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+    }
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.dev = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._nvml = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            props = torch.cuda.get_device_properties(self.dev)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self):
+        import pynvml
+        h = self._h
+        bits = {nm: getattr(pynvml, attr, 0) for nm, attr in self.REASONS.items()}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for nm, bit in bits.items():
+                    if bit and (r & bit):
+                        self.reasons.add(nm)
+            except Exception:
+                break
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            self._h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
-        except (FileNotFoundError, OSError):
-            self.proc = None
+        except Exception:
+            self._h = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if getattr(self, "thread", None) is not None:
             self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.lines:
+        if not self.samples:
             return None
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "sm_mhz_min": min(self.samples), "source": "NVML, 2 ms polling"}
 
 
 def _fp32_peak(device):
@@ -546,6 +557,46 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_CASES = {
+    # kernel -> (make_inputs kwargs, scan kwargs)
+    "tc": (dict(B=4, H=16, T=8192, d=64, seed=7, random_affine=True, in_bf16=True),
+           dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
+    "simt": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
+             dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
+}
+
+
+def run_profile_case(name: str):
+    """One warm-up launch and one more launch of a scan kernel on a fixed
+    case, for profiler captures (no timing)."""
+    import torch
+    from test_sequence_layers_02_b200 import build, ttt_scan
+    from test_sequence_layers_02_b200.workloads import make_inputs
+    build.build()
+    mk, kw = PROFILE_CASES[name]
+    inp = make_inputs(**mk)
+    bf = mk.get("in_bf16", False)
+
+    def dev(key):
+        a = inp.get(key)
+        if a is None:
+            return None
+        if bf and key in ("q", "k", "v", "eta_logit", "gate_logit"):
+            return torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
+    kw = dict(kw)
+    out_dtype = torch.bfloat16 if kw.pop("out_bf16") else torch.float32
+    for _ in range(2):
+        ttt_scan.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"],
+                      t["beta"], out_dtype=out_dtype, **kw)
+    rc = ttt_scan.check_device_status()
+    print(f"profile case {name}: status {ttt_scan.status_string(rc)}")
+    if rc != ttt_scan.TTT_OK:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -557,7 +608,12 @@ def main():
                     help="other workloads measured on one GPU (by_workload)")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one kernel on a fixed case for a profiler capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         print("note: at least 3 warm-up steps are required; using 3", file=sys.stderr)
         args.warmup = 3

@@ -35,11 +35,16 @@ namespace ttt {
 
 constexpr int kC = 16;  // largest chunk of the CUDA-core kernel
 
-template <int D, typename InT>
+// IH = 2 splits W's columns in quarters instead of halves (8 bulk warps at
+// d = 64), so every SM sub-partition runs two bulk warps; used when heads are
+// few.
+template <int D, typename InT, int IH = 1>
 struct PipeLayout {
-  static constexpr int NBT = 2 * D;          // bulk threads
+  static constexpr int NBT = 2 * D * IH;     // bulk threads
   static constexpr int NT = NBT + 32;        // + the chain warp
-  static constexpr int KH = D / 2;           // columns of W per bulk thread
+  static constexpr int KH = D / 2;           // Gram column half
+  static constexpr int NKQ = 2 * IH;         // column groups of W
+  static constexpr int KW = D / NKQ;         // columns of W per bulk thread
   static constexpr int NG = NBT / 32;        // bulk warps
   static constexpr int ELT = (int)sizeof(InT);
   static constexpr int ROWB = D * ELT + 16;  // padded row of an input tile (bytes)
@@ -51,8 +56,8 @@ struct PipeLayout {
   static constexpr int oZ = oV + 2 * TILE;             // P / Zpre   [2][kC][D] f32
   static constexpr int oG = oZ + 2 * kC * D * 4;       // G          [2][kC][D]
   static constexpr int oQ0 = oG + 2 * kC * D * 4;      // Q0         [2][kC][D]
-  static constexpr int oPP = oQ0 + 2 * kC * D * 4;     // partial products [2][2kC][D]
-  static constexpr int oA = oPP + 2 * 2 * kC * D * 4;  // in-chunk K Gram [2][kC][kC]
+  static constexpr int oPP = oQ0 + 2 * kC * D * 4;     // partial products [NKQ][2kC][D]
+  static constexpr int oA = oPP + NKQ * 2 * kC * D * 4;  // in-chunk K Gram [2][kC][kC]
   static constexpr int oS = oA + 2 * kC * kC * 4;      // Q K Gram   [2][kC][kC]
   static constexpr int oX = oS + 2 * kC * kC * 4;      // cross Gram [kC][kC]
   static constexpr int oEta = oX + kC * kC * 4;        // eta        [4][kC]
@@ -104,7 +109,7 @@ __device__ __forceinline__ float lds1(const unsigned char* p, __nv_bfloat16) {
 template <int D, typename InT>
 __device__ __forceinline__ void tile_load(unsigned char* tile, const InT* src, int t0, int n,
                                           int tid, int nthreads) {
-  using L = PipeLayout<D, InT>;
+  using L = PipeLayout<D, InT, 1>;
   constexpr int CPR = D * L::ELT / 16;  // 16-byte pieces per row
   for (int idx = tid; idx < kC * CPR; idx += nthreads) {
     const int row = idx / CPR;
@@ -223,13 +228,14 @@ __device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
   if (GM != 0 && lane < kC) mGout[lane] = 0.f;
 }
 
-// Partial products of a bulk thread: acc[i] = sum over its column half of
+// Partial products of a bulk thread: acc[i] = sum over its column group of
 // W[r][k] * rows[i][k], for up to two sets of 16 rows.
-template <int D, typename InT>
-__device__ __forceinline__ void bulk_products(const float (&Wr)[D / 2], const unsigned char* R0,
-                                              const unsigned char* R1, float* PP, int r, int kq) {
-  using L = PipeLayout<D, InT>;
-  constexpr int KH = L::KH;
+template <int D, typename InT, int IH>
+__device__ __forceinline__ void bulk_products(const float (&Wr)[PipeLayout<D, InT, IH>::KW],
+                                              const unsigned char* R0, const unsigned char* R1,
+                                              float* PP, int r, int kq) {
+  using L = PipeLayout<D, InT, IH>;
+  constexpr int KH = L::KW;
   const int koff = kq * KH * L::ELT;
   float* out = PP + kq * (2 * kC * D);
 #pragma unroll 1
@@ -255,11 +261,11 @@ __device__ __forceinline__ void bulk_products(const float (&Wr)[D / 2], const un
 
 // Dot products of left rows with one right row per lane pair (16 rows x 2
 // column halves); returns eta-weighted entries through `emit(i, j, dot)`.
-template <int D, typename InT, typename Emit>
+template <int D, typename InT, int IH, typename Emit>
 __device__ __forceinline__ void bulk_gram(const unsigned char* right, const unsigned char* left0,
                                           const unsigned char* left1, int nleft, int tid,
                                           Emit emit) {
-  using L = PipeLayout<D, InT>;
+  using L = PipeLayout<D, InT, IH>;
   constexpr int KH = L::KH;
   const int j = tid & 15;
   const int kq = (tid >> 4) & 1;
@@ -323,11 +329,12 @@ __device__ __forceinline__ void row_means(const float* Z, float* out, int tid, i
   }
 }
 
-template <int D, typename InT, typename OutT, bool MINIB, int GM>
-__global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams p) {
-  using L = PipeLayout<D, InT>;
+template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
+__global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanParams p) {
+  using L = PipeLayout<D, InT, IH>;
   constexpr int NBT = L::NBT;
-  constexpr int KH = L::KH;
+  constexpr int KW = L::KW;
+  constexpr int NKQ = L::NKQ;
   constexpr int EPL = (D + 31) / 32;
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char* sK = smem + L::oK;
@@ -402,15 +409,16 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
   };
 
   // ---------------- prologue ----------------
-  float Wr[KH];
+  float Wr[KW];
   const int r = tid % D;
-  const int kq = tid / D;  // meaningful for bulk threads
+  const int part = tid / D;  // bulk threads: 0 .. NKQ - 1
+  const int kq = part;       // column group of W held
   float gam[EPL], bet[EPL];
   float Sgb = 0.f, Sb = 0.f;
   if (!chain) {
-    const float* W0 = p.W0 + ((size_t)bh * D + r) * D + kq * KH;  // may alias W_T
+    const float* W0 = p.W0 + ((size_t)bh * D + r) * D + kq * KW;  // may alias W_T
 #pragma unroll
-    for (int k = 0; k < KH; k += 4) {
+    for (int k = 0; k < KW; k += 4) {
       const float4 w4 = *reinterpret_cast<const float4*>(W0 + k);
       Wr[k] = w4.x; Wr[k + 1] = w4.y; Wr[k + 2] = w4.z; Wr[k + 3] = w4.w;
     }
@@ -442,16 +450,19 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
   __syncthreads();
   if (!chain && nc > 0) {
     // P_0 = K_0 W0^T (no correction), its row means, and A_0
-    bulk_products<D, InT>(Wr, nullptr, tileK(0), sPP, r, kq);
+    bulk_products<D, InT, IH>(Wr, nullptr, tileK(0), sPP, r, kq);
     if (!MINIB) {
       const int n0 = chunk_len(0);
-      bulk_gram<D, InT>(tileK(0), tileK(0), nullptr, kC, tid, [&](int m, int j, float dot) {
+      bulk_gram<D, InT, IH>(tileK(0), tileK(0), nullptr, kC, tid, [&](int m, int j, float dot) {
         sA[m * kC + j] = (j < m && m < n0) ? sEta[j] * dot : 0.f;
       });
     }
     bulk_barrier(NBT);
-    for (int i = kq; i < kC; i += 2) {
-      sZ[i * D + r] = sPP[(kC + i) * D + r] + sPP[2 * kC * D + (kC + i) * D + r];
+    for (int i = part; i < kC; i += NKQ) {
+      float acc = 0.f;
+#pragma unroll
+      for (int g = 0; g < NKQ; ++g) acc += sPP[g * 2 * kC * D + (kC + i) * D + r];
+      sZ[i * D + r] = acc;
     }
     bulk_barrier(NBT);
     row_means<D>(sZ, sMu, tid, NBT);
@@ -494,9 +505,9 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         const int np = chunk_len(c - 1);
         for (int j = 0; j < np; ++j) {
           const float ge = et[j] * Gp[j * D + r];
-          const unsigned char* row = Kt + j * L::ROWB + kq * KH * L::ELT;
+          const unsigned char* row = Kt + j * L::ROWB + kq * KW * L::ELT;
 #pragma unroll
-          for (int k = 0; k < KH; k += 8) {
+          for (int k = 0; k < KW; k += 8) {
             float x[8];
             lds8(row + k * L::ELT, x, InT());
 #pragma unroll
@@ -505,9 +516,9 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         }
       }
       if (Wc && ((c * C) % p.b) == 0) {
-        float* dst = Wc + ((size_t)((c * C) / p.b) * D + r) * D + kq * KH;
+        float* dst = Wc + ((size_t)((c * C) / p.b) * D + r) * D + kq * KW;
 #pragma unroll
-        for (int k = 0; k < KH; k += 4)
+        for (int k = 0; k < KW; k += 4)
           *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
       }
 
@@ -520,7 +531,7 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         const float* gt = sGate + ((c - 1) & 3) * kC;
         const bool upd = sFlag[(c - 1) & 3];
         OutT* dst = go + (size_t)(c - 1) * C * D;
-        for (int i = kq; i < np; i += 2) {
+        for (int i = part; i < np; i += 2 * IH) {
           float acc = Q0p[i * D + r], acc2 = 0.f;
           if (upd) {
             int j = 0;
@@ -539,7 +550,7 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         const float* et = sEta + (c & 3) * kC;
         float* Sc = sS + (c & 1) * kC * kC;
         const int n1 = has_next ? chunk_len(c + 1) : 0;
-        bulk_gram<D, InT>(tileK(c), tileQ(c), has_next ? tileK(c + 1) : nullptr,
+        bulk_gram<D, InT, IH>(tileK(c), tileQ(c), has_next ? tileK(c + 1) : nullptr,
                           has_next ? 2 * kC : kC, tid, [&](int s, int j, float dot) {
                             if (s < kC) {
                               Sc[s * kC + j] = (j <= s && s < n) ? et[j] * dot : 0.f;
@@ -551,7 +562,7 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         if (!MINIB && has_next) {
           const float* et1 = sEta + ((c + 1) & 3) * kC;
           float* An = sA + ((c + 1) & 1) * kC * kC;
-          bulk_gram<D, InT>(tileK(c + 1), tileK(c + 1), nullptr, kC, tid,
+          bulk_gram<D, InT, IH>(tileK(c + 1), tileK(c + 1), nullptr, kC, tid,
                             [&](int m, int j, float dot) {
                               An[m * kC + j] = (j < m && m < n1) ? et1[j] * dot : 0.f;
                             });
@@ -559,14 +570,16 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
       }
 
       // Q0_c = Q_c W_{s,c}^T and P_{c+1} = K_{c+1} W_{s,c}^T
-      bulk_products<D, InT>(Wr, tileQ(c), has_next ? tileK(c + 1) : nullptr, sPP, r, kq);
+      bulk_products<D, InT, IH>(Wr, tileQ(c), has_next ? tileK(c + 1) : nullptr, sPP, r, kq);
       bulk_barrier(NBT);
       {
         float* Q0c = sQ0 + (c & 1) * kC * D;
         float* Pn = sZ + ((c + 1) & 1) * kC * D;
-        for (int i = kq; i < 2 * kC; i += 2) {
+        for (int i = part; i < 2 * kC; i += NKQ) {
           if (i >= kC && !has_next) break;
-          const float val = sPP[i * D + r] + sPP[2 * kC * D + i * D + r];
+          float val = 0.f;
+#pragma unroll
+          for (int g = 0; g < NKQ; ++g) val += sPP[g * 2 * kC * D + i * D + r];
           if (i < kC) Q0c[i * D + r] = val;
           else Pn[(i - kC) * D + r] = val;
         }
@@ -585,7 +598,7 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
       const int n1 = chunk_len(c + 1);
       float* Zn = sZ + ((c + 1) & 1) * kC * D;
       const float* Gc = sG + (c & 1) * kC * D;
-      for (int m = kq; m < n1; m += 2) {
+      for (int m = part; m < n1; m += 2 * IH) {
         float acc = Zn[m * D + r], acc2 = 0.f;
         int j = 0;
         for (; j + 1 < n; j += 2) {
@@ -616,9 +629,9 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
         const float* et = sEta + (c & 3) * kC;
         for (int j = 0; j < np; ++j) {
           const float ge = et[j] * Gp[j * D + r];
-          const unsigned char* row = Kt + j * L::ROWB + kq * KH * L::ELT;
+          const unsigned char* row = Kt + j * L::ROWB + kq * KW * L::ELT;
 #pragma unroll
-          for (int k = 0; k < KH; k += 8) {
+          for (int k = 0; k < KW; k += 8) {
             float x[8];
             lds8(row + k * L::ELT, x, InT());
 #pragma unroll
@@ -632,7 +645,7 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
       const float* gt = sGate + (c & 3) * kC;
       const bool upd = sFlag[c & 3];
       OutT* dst = go + (size_t)c * C * D;
-      for (int i = kq; i < np; i += 2) {
+      for (int i = part; i < np; i += 2 * IH) {
         float acc = Q0p[i * D + r];
         if (upd)
           for (int j = 0; j <= i; ++j) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
@@ -640,14 +653,14 @@ __global__ void __launch_bounds__(2 * D + 32) scan_simt_kernel(const ScanParams 
       }
     }
     if (Wc) {
-      float* dst = Wc + ((size_t)p.n_mask_chunks * D + r) * D + kq * KH;
+      float* dst = Wc + ((size_t)p.n_mask_chunks * D + r) * D + kq * KW;
 #pragma unroll
-      for (int k = 0; k < KH; k += 4)
+      for (int k = 0; k < KW; k += 4)
         *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
     }
-    float* WT = p.W_T + ((size_t)bh * D + r) * D + kq * KH;
+    float* WT = p.W_T + ((size_t)bh * D + r) * D + kq * KW;
 #pragma unroll
-    for (int k = 0; k < KH; k += 4)
+    for (int k = 0; k < KW; k += 4)
       *reinterpret_cast<float4*>(WT + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
   }
 }

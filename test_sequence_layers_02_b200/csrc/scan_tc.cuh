@@ -404,16 +404,27 @@ __global__ void __launch_bounds__(tc::NT, 3)
     for (int k = 0; k < nc; ++k) {
       const int n = chunk_len(k);
       const bool upd = sFlag[k & (kSR - 1)] != 0;
-      // operands that do not depend on Z_k, fetched before waiting for it
-      float v[8], gam[8], bet[8];
+      // per-feature coefficients that do not depend on Z_k, formed before
+      // waiting for it: LNJAC a = gamma^2, c = gamma (beta - v);
+      // simplified a = gamma, c = beta - v; no LayerNorm c = -v
+      float a8[8], c8[8];
       {
         const unsigned char* Vt = tV(k) + tm_m * D * 2;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int f = tm_p + 8 * u;
-          v[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Vt + f * 2));
-          gam[u] = sGam[f];
-          bet[u] = sBet[f];
+          const float v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Vt + f * 2));
+          const float g = sGam[f];
+          if (GM == 1) {
+            a8[u] = g * g;
+            c8[u] = g * (sBet[f] - v);
+          } else if (GM == 0) {
+            a8[u] = g;
+            c8[u] = sBet[f] - v;
+          } else {
+            a8[u] = 0.f;
+            c8[u] = -v;
+          }
         }
       }
       const float eta = (tm_m < n) ? sEta[(k & (kSR - 1)) * CB + tm_m] : 0.f;
@@ -439,41 +450,42 @@ __global__ void __launch_bounds__(tc::NT, 3)
         // token-major LayerNorm + gradient: token tm_m, features tm_p + 8u
         const float* Zk = sZ + (k & 1) * CB * kZS + tm_m * kZS;
         float z[8], G[8];
+        (void)sgb;
 #pragma unroll
         for (int u = 0; u < 8; ++u) z[u] = Zk[tm_p + 8 * u];
         if (GM == 2) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) G[u] = z[u] - v[u];
+          for (int u = 0; u < 8; ++u) G[u] = z[u] + c8[u];
         } else {
           // shift by one element of the token, then all moments in one round
           const float c0 = __shfl_sync(0xffffffffu, z[0], lane & ~7);
-          float y[8], w[8];
           float m[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            w[u] = gam[u] * (bet[u] - v[u]);    // gamma (beta - v)
-            y[u] = z[u] - c0;
-            m[0] += y[u];
-            m[1] = fmaf(y[u], y[u], m[1]);
+            const float y = z[u] - c0;
+            z[u] = y;
+            m[0] += y;
+            m[1] = fmaf(y, y, m[1]);
             if (GM == 1) {
-              const float g2y = gam[u] * gam[u] * y[u];
-              m[2] += g2y;
-              m[3] = fmaf(g2y, y[u], m[3]);
-              m[4] = fmaf(w[u], y[u], m[4]);
-              m[5] += w[u];
+              const float ay = a8[u] * y;
+              m[2] += ay;
+              m[3] = fmaf(ay, y, m[3]);
+              m[4] = fmaf(c8[u], y, m[4]);
+              m[5] += c8[u];
             }
           }
 #pragma unroll
           for (int off = 1; off < 8; off <<= 1) {
 #pragma unroll
-            for (int i = 0; i < 6; ++i) m[i] += __shfl_xor_sync(0xffffffffu, m[i], off);
+            for (int i = 0; i < (GM == 1 ? 6 : 2); ++i)
+              m[i] += __shfl_xor_sync(0xffffffffu, m[i], off);
           }
           const float inv_d = 1.0f / D;
-          const float mu1 = m[0] * inv_d;                    // mean of y (shifted)
+          const float mu1 = m[0] * inv_d;                    // mean of the shifted values
           const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
           const float rs = rsqrtf(var + p.eps);
           if (GM == 1) {
-            // moments of the centred y - mu1
+            // moments of the centred values y - mu1
             const float sg2y = m[2] - mu1 * sg2;
             const float sg2yy = m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sg2;
             const float swy = m[4] - mu1 * m[5];
@@ -481,15 +493,12 @@ __global__ void __launch_bounds__(tc::NT, 3)
             const float mgx = rs * (rs * sg2yy + swy) * inv_d;
             const float rs2 = rs * rs;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float yc = y[u] - mu1;
-              G[u] = rs2 * (gam[u] * gam[u] - mgx) * yc + rs * (w[u] - mg);
-            }
+            for (int u = 0; u < 8; ++u)
+              G[u] = rs2 * (a8[u] - mgx) * (z[u] - mu1) + rs * (c8[u] - mg);
           } else {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) G[u] = fmaf(gam[u] * rs, y[u] - mu1, bet[u]) - v[u];
+            for (int u = 0; u < 8; ++u) G[u] = fmaf(a8[u] * rs, z[u] - mu1, c8[u]);
           }
-          (void)sgb;
         }
         unsigned char* An = aneg(k);
 #pragma unroll
@@ -519,26 +528,37 @@ __global__ void __launch_bounds__(tc::NT, 3)
       // ---- W_{s,c+1} (fp32 TMEM) -> bf16 operand; snapshot ----
       const int row = wq * 32 + lane;
       if (upd) {
-        float w[64];
-        tmem_ld32(tmem + tlane + kColW, *reinterpret_cast<float(*)[32]>(&w[0]));
-        tmem_ld32(tmem + tlane + kColW + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
-        tmem_wait_ld();
+        // two 32-column TMEM loads; the second is in flight while the first
+        // half is packed to bf16 and stored
+        float w[32];
+        uint4 packed[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 u;
-          u.x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
-          u.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
-          u.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
-          u.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
-          *reinterpret_cast<uint4*>(sWb + sw128_off(row, ch)) = u;
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tmem + tlane + kColW + 32 * hf, w);
+          if (hf == 1) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+              *reinterpret_cast<uint4*>(sWb + sw128_off(row, ch)) = packed[ch];
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            packed[ch].x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
+            packed[ch].y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
+            packed[ch].z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
+            packed[ch].w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
+          }
+          if (Wc && row < 64) {
+            float* dst = Wc + ((size_t)(c + 1) * D + row) * D + 32 * hf;
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<float4*>(dst + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+          }
         }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          *reinterpret_cast<uint4*>(sWb + sw128_off(row, 4 + ch)) = packed[ch];
         fence_proxy_async_smem();
-        if (Wc && row < 64) {
-          float* dst = Wc + ((size_t)(c + 1) * D + row) * D;
-#pragma unroll
-          for (int k = 0; k < 64; k += 4)
-            *reinterpret_cast<float4*>(dst + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
-        }
       } else if (Wc && row < 64) {
         const float* srcw = Wc + ((size_t)c * D + row) * D;  // W unchanged: repeat the snapshot
         float* dst = Wc + ((size_t)(c + 1) * D + row) * D;

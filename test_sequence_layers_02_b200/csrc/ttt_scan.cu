@@ -34,10 +34,10 @@ int largest_divisor_upto(int b, int cap) {
   return 1;
 }
 
-template <int D, typename InT, typename OutT, bool MINIB, int GM>
-int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
-  using L = ttt::PipeLayout<D, InT>;
-  auto kernel = ttt::scan_simt_kernel<D, InT, OutT, MINIB, GM>;
+template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
+int launch_simt_ih(const ttt::ScanParams& p, cudaStream_t stream) {
+  using L = ttt::PipeLayout<D, InT, IH>;
+  auto kernel = ttt::scan_simt_kernel<D, InT, OutT, MINIB, GM, IH>;
   if (L::bytes > 48 * 1024) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L::bytes) != cudaSuccess)
@@ -45,6 +45,15 @@ int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
   }
   kernel<<<(unsigned)(p.B * p.H), L::NT, L::bytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+// Few heads (at most one CTA per SM): 8 bulk warps per CTA; otherwise 4, so
+// that several CTAs share an SM.
+template <int D, typename InT, typename OutT, bool MINIB, int GM>
+int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
+  if (D == 64 && (long long)p.B * p.H <= 148)
+    return launch_simt_ih<D, InT, OutT, MINIB, GM, 2>(p, stream);
+  return launch_simt_ih<D, InT, OutT, MINIB, GM, 1>(p, stream);
 }
 
 template <int D, typename InT, typename OutT>
