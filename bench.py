@@ -60,15 +60,19 @@ def _csrc_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def _traffic(kernel_key: str):
-    """DRAM bytes per launch from the committed ncu capture, if the kernels are unchanged."""
+def _traffic(kernel_key: str, head_tokens_per_launch: int):
+    """DRAM bytes (read + write) per launch from the committed ncu capture of
+    that kernel, scaled from its case by head-tokens; None if the kernel
+    sources changed since the capture."""
     if not PROFILE_TRAFFIC.exists():
         return None
     d = json.loads(PROFILE_TRAFFIC.read_text())
     if d.get("csrc_hash") != _csrc_hash():
         return None
     e = d.get("kernels", {}).get(kernel_key)
-    return None if e is None else e.get("bytes_per_launch_full")
+    if e is None:
+        return None
+    return round(e["bytes_per_head_token"] * head_tokens_per_launch)
 
 
 # ---------------------------------------------------------------------------
@@ -307,7 +311,8 @@ def _roofline(job, per_launch_s, peaks, fp32_meas_tflops, n_sm):
         peak = n_sm * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
         return {"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 2),
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": _traffic(job.kernel_key()),
+                "traffic": _traffic(job.kernel_key(), job.w.head_tokens),
+                "algorithmic_flops_per_launch": flops,
                 "peak_basis": f"{n_sm} SM x 128 FP32 lanes x 2 x {peaks['sm_max_mhz']:.0f} MHz",
                 "fp32_probe_tflops": round(fp32_meas_tflops, 2),
                 "frac_of_probe": round(achieved / fp32_meas_tflops, 4),
@@ -316,7 +321,8 @@ def _roofline(job, per_launch_s, peaks, fp32_meas_tflops, n_sm):
     achieved = byts / per_launch_s / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": _traffic(job.kernel_key()), "kernel": job.kernel_key(),
+            "traffic": _traffic(job.kernel_key(), job.w.head_tokens), "kernel": job.kernel_key(),
+            "algorithmic_bytes_per_launch": round(byts),
             "peak_basis": f"{peaks['source']} HBM copy bandwidth"}
 
 
