@@ -40,6 +40,10 @@
 //     eps inside the square root: s = sqrt(mean((z - mu)^2) + eps).
 //   * W is stored row-major as W[out][in] so that z = W k.
 //   * gate_logit == NULL means no output gate (sigmoid replaced by 1).
+//   * The gate is one scalar per token by default. With the per-channel gate
+//     option it is a d-vector per token, o_t[r] = sigmoid(gate_t[r]) (W_t q_t)[r]:
+//     the elementwise reading of "Sigmoid gate on output (like SwiGLU)"
+//     ("Edifice.Recurrent.TTT", section "Paper-Faithful Implementation", item 4).
 //   * mask == NULL means every chunk updates.
 //   * NO_LN removes the LayerNorm: pred = z and G = z - v (the delta rule of the
 //     section "Key Innovations").
@@ -64,6 +68,7 @@ namespace {
 constexpr unsigned kMiniBatch = 1u << 0;
 constexpr unsigned kLnJacobian = 1u << 1;
 constexpr unsigned kNoLayerNorm = 1u << 2;
+constexpr unsigned kGateChannel = 1u << 6;
 
 template <typename S>
 S sigmoid(S x) {
@@ -132,6 +137,14 @@ S dot(const S* a, const S* b, int d) {
   return acc;
 }
 
+// Output gate of feature r of token t: scalar per token, or one per feature.
+template <typename S>
+S gate_of(const S* gate_logit, unsigned mode, int t, int d, int r) {
+  if (!gate_logit) return S(1);
+  if (mode & kGateChannel) return sigmoid(gate_logit[(size_t)t * d + r]);
+  return sigmoid(gate_logit[t]);
+}
+
 // One (batch row, head) recurrence over all T tokens.
 template <typename S>
 void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
@@ -161,8 +174,8 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
         for (int r = 0; r < d; ++r)
           for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];
         matvec(W.data(), qt, d, Wq.data());
-        const S gate = gate_logit ? sigmoid(gate_logit[t]) : S(1);
-        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];
+        for (int r = 0; r < d; ++r)
+          o[(size_t)t * d + r] = gate_of(gate_logit, mode, t, d, r) * Wq[r];
       }
     } else {
       // Mini-batch (dual form): all gradients of the chunk at W_s.
@@ -183,8 +196,8 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
           const S a = etas[j] * dot(k + (size_t)(t0 + j) * d, qt, d);
           for (int r = 0; r < d; ++r) Wq[r] -= a * Gs[(size_t)j * d + r];
         }
-        const S gate = gate_logit ? sigmoid(gate_logit[t]) : S(1);
-        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];
+        for (int r = 0; r < d; ++r)
+          o[(size_t)t * d + r] = gate_of(gate_logit, mode, t, d, r) * Wq[r];
       }
       for (int j = 0; j < n; ++j) {
         const S* kj = k + (size_t)(t0 + j) * d;
@@ -218,7 +231,8 @@ int forward(const S* q, const S* k, const S* v, const S* eta_logit,
     const int h = (int)(bh % H);
     const size_t tok = (size_t)bh * T;
     scan_one_head<S>(q + tok * d, k + tok * d, v + tok * d, eta_logit + tok,
-                     gate_logit ? gate_logit + tok : nullptr,
+                     gate_logit ? gate_logit + ((mode & kGateChannel) ? tok * d : tok)
+                                : nullptr,
                      W0 + (size_t)bh * d * d,
                      gamma ? gamma + (size_t)h * d : nullptr,
                      beta ? beta + (size_t)h * d : nullptr, T, d, eps, mode, b,
@@ -235,7 +249,8 @@ int forward(const S* q, const S* k, const S* v, const S* eta_logit,
 extern "C" {
 
 // Full scan. All arrays are host, contiguous, row-major:
-//   q, k, v, o: [B, H, T, d];  eta_logit, gate_logit: [B, H, T];
+//   q, k, v, o: [B, H, T, d];  eta_logit: [B, H, T];
+//   gate_logit: [B, H, T], or [B, H, T, d] with mode bit 1 << 6 (per-channel gate);
 //   W0, W_T: [B, H, d, d] with z = W k;  gamma, beta: [H, d];
 //   mask: [B, ceil(T/b)] bytes, 1 = UPDATE, 0 = SKIP;
 //   W_chunks: [B, H, ceil(T/b) + 1, d, d], W before each chunk and after the last.

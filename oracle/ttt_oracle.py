@@ -29,6 +29,7 @@ _LIB = _HERE / "libttt_oracle.so"
 MINIBATCH = 1 << 0
 GRAD_LNJAC = 1 << 1
 NO_LN = 1 << 2
+GATE_CHANNEL = 1 << 6
 
 _lib = None
 
@@ -91,8 +92,9 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
             nthreads: int = 0, dtype=np.float64):
     """Run the oracle scan.
 
-    Shapes: q, k, v [B, H, T, d]; eta_logit, gate_logit [B, H, T] (gate may be
-    None); W0 [B, H, d, d] with z = W k; gamma, beta [H, d] (ignored with NO_LN);
+    Shapes: q, k, v [B, H, T, d]; eta_logit [B, H, T]; gate_logit [B, H, T], or
+    [B, H, T, d] with GATE_CHANNEL in ``mode``, or None; W0 [B, H, d, d] with
+    z = W k; gamma, beta [H, d] (ignored with NO_LN);
     mask [B, ceil(T/b)] uint8 (1 = UPDATE) or None.
 
     Returns ``(o, W_T)`` or ``(o, W_T, W_chunks)`` when ``want_chunks``; W_chunks
@@ -112,6 +114,10 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
     gamma, beta = cvt(gamma), cvt(beta)
     if b <= 0:
         raise ValueError(f"chunk size b must be positive, got {b}")
+    if gate_logit is not None:
+        gshape = (B, H, T, d) if mode & GATE_CHANNEL else (B, H, T)
+        if gate_logit.shape != gshape:
+            raise ValueError(f"gate_logit: expected shape {gshape}, got {gate_logit.shape}")
     n_chunks = -(-T // b)
     if mask is not None:
         mask = np.ascontiguousarray(mask, dtype=np.uint8)
@@ -127,6 +133,24 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     return (o, W_T, W_chunks) if want_chunks else (o, W_T)
+
+
+def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float,
+                mode: int, update=None, dtype=np.float64):
+    """One streaming step: the per-token recurrence for a single token.
+
+    q, k, v [B, H, d]; eta_logit [B, H]; gate_logit [B, H] (or [B, H, d] with
+    GATE_CHANNEL, or None); W [B, H, d, d]; update [B] uint8 (0 = SKIP) or None.
+    Returns ``(o [B, H, d], W_new [B, H, d, d])``. This is ``forward`` with
+    T = 1 and a one-token mask chunk; it adds no arithmetic of its own.
+    """
+    if mode & MINIBATCH:
+        raise ValueError("a single-token step has no mini-batch form")
+    ex = lambda a: None if a is None else np.asarray(a)[:, :, None]
+    m = None if update is None else np.asarray(update, dtype=np.uint8).reshape(-1, 1)
+    o, W_new = forward(ex(q), ex(k), ex(v), ex(eta_logit), ex(gate_logit), W, gamma, beta,
+                       eps=eps, mode=mode, b=1, mask=m, dtype=dtype)
+    return o[:, :, 0], W_new
 
 
 def lngrad(z, v, gamma, beta, *, eps: float, mode: int):

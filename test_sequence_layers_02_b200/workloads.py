@@ -7,7 +7,8 @@ their inputs from it.
 Recipe (numpy PCG64, seed = workload id, draws in the order q, k, v, eta_logit,
 gate_logit, W0, gamma, beta, mask; each draw is float32):
 
-* q, k, v, eta_logit, gate_logit ~ N(0, 1).
+* q, k, v, eta_logit, gate_logit ~ N(0, 1); the gate is [B, H, T], or
+  [B, H, T, d] for the per-channel gate.
 * W0 ~ N(0, 0.02^2) -- the small initialisation of "Edifice.Recurrent.TTT",
   section "Paper-Faithful Implementation" (0.02 read as the standard deviation).
 * gamma = 1, beta = 0, or per head gamma ~ N(1, 0.1^2), beta ~ N(0, 0.1^2).
@@ -95,16 +96,25 @@ WORKLOADS = {
 }
 
 
+# Streaming decode: one token for every (batch row, head), W carried in place.
+# 16384 heads of d = 64 hold 256 MB of fp32 state, twice the L2.
+DECODE_WORKLOADS = {
+    "dec": Workload("dec", B=512, H=32, T=1, d=64, b=1, eps=1e-6, minibatch=False,
+                    lnjac=True, in_bf16=True, out_bf16=True, random_affine=True, seed=7),
+}
+
+
 def make_inputs(B: int, H: int, T: int, d: int, *, seed: int, b: int = 16,
                 qk_l2norm: bool = False, random_affine: bool = False,
                 in_bf16: bool = False, mask_p: Optional[float] = None,
-                gate: bool = True, w0_std: float = 0.02) -> dict:
+                gate: bool = True, w0_std: float = 0.02, gate_channel: bool = False) -> dict:
     """Draw one seeded problem.
 
     Returns a dict of host arrays. q, k, v, eta_logit, gate_logit, W0, gamma,
     beta are float32 (for bf16 inputs they hold the bf16 values exactly, and
     ``*_bf16`` keys hold the uint16 bits of q, k, v, eta_logit, gate_logit);
-    ``mask`` is uint8 [B, ceil(T/b)] or None.
+    ``mask`` is uint8 [B, ceil(T/b)] or None. ``gate_channel`` draws one gate
+    logit per feature, [B, H, T, d], instead of one per token.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     shp = (B, H, T, d)
@@ -112,7 +122,8 @@ def make_inputs(B: int, H: int, T: int, d: int, *, seed: int, b: int = 16,
     k = rng.standard_normal(shp, dtype=np.float32)
     v = rng.standard_normal(shp, dtype=np.float32)
     eta = rng.standard_normal((B, H, T), dtype=np.float32)
-    gl = rng.standard_normal((B, H, T), dtype=np.float32) if gate else None
+    gshape = (B, H, T, d) if gate_channel else (B, H, T)
+    gl = rng.standard_normal(gshape, dtype=np.float32) if gate else None
     W0 = (rng.standard_normal((B, H, d, d), dtype=np.float32) * np.float32(w0_std))
     if random_affine:
         gamma = (np.float32(1) + np.float32(0.1) * rng.standard_normal((H, d), dtype=np.float32))

@@ -35,8 +35,13 @@ MUTATIONS = [
     ("eps_outside_sqrt", "const S s = std::sqrt(var + eps);", "const S s = std::sqrt(var) + eps;"),
     ("unbiased_variance", "var /= S(d);", "var /= S(d - 1);"),
     ("drop_beta", "pred[f] = gamma[f] * xhat[f] + beta[f];", "pred[f] = gamma[f] * xhat[f];"),
-    ("no_gate_per_token", "const S gate = gate_logit ? sigmoid(gate_logit[t]) : S(1);\n        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];\n      }\n    } else {",
-     "const S gate = S(1);\n        for (int r = 0; r < d; ++r) o[(size_t)t * d + r] = gate * Wq[r];\n      }\n    } else {"),
+    ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
+    ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
+     "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),
+    ("gate_channel_read_as_scalar", "if (mode & kGateChannel) return sigmoid(gate_logit[(size_t)t * d + r]);",
+     "if (mode & kGateChannel) return sigmoid(gate_logit[t]);"),
+    ("gate_channel_wrong_head_offset", "gate_logit + ((mode & kGateChannel) ? tok * d : tok)",
+     "gate_logit + tok"),
     ("minibatch_exclusive_prefix", "for (int j = 0; j <= i; ++j) {", "for (int j = 0; j < i; ++j) {"),
     ("minibatch_wrong_key_index", "const S a = etas[j] * dot(k + (size_t)(t0 + j) * d, qt, d);",
      "const S a = etas[j] * dot(k + (size_t)(t0 + i) * d, qt, d);"),

@@ -16,14 +16,18 @@ at least one of them:
 * cancellation of the prediction-derived gradient term as eps -> 0;
 * mini-batch with b = 1, or with keys orthogonal inside each chunk, equals the
   per-token recurrence; mini-batch with b = T as one vectorised expression;
-* chaining (resume from W_T), mask == eta forced to 0 on the same chunks.
+* chaining (resume from W_T), mask == eta forced to 0 on the same chunks;
+* the per-channel output gate is elementwise: it leaves W alone, scales each
+  feature of the ungated output by its own sigmoid, and a gate that is the same
+  on every feature reproduces the scalar gate;
+* a chain of single-token steps is the per-token scan with a one-token mask.
 """
 
 import numpy as np
 import pytest
 
 import oracle
-from oracle import GRAD_LNJAC, MINIBATCH, NO_LN
+from oracle import GATE_CHANNEL, GRAD_LNJAC, MINIBATCH, NO_LN
 from test_sequence_layers_02_b200.workloads import make_inputs
 from tests.conftest import load_golden
 
@@ -389,6 +393,63 @@ def test_no_gate_means_unit_gate():
     o2, W2 = run(inp2, mode=GRAD_LNJAC)
     np.testing.assert_array_equal(W1, W2)
     np.testing.assert_allclose(o1, sig(inp["gate_logit"])[..., None] * o2, rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------
+# Per-channel output gate: the elementwise reading of the sigmoid output gate
+# ("Edifice.Recurrent.TTT", "Paper-Faithful Implementation", item 4).
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [GRAD_LNJAC, MINIBATCH | GRAD_LNJAC, 0])
+def test_gate_channel_is_elementwise_and_leaves_W_alone(mode):
+    B, H, T, d = 2, 3, 21, 16
+    inp = f64(make_inputs(B, H, T, d, seed=35, random_affine=True, gate_channel=True))
+    assert inp["gate_logit"].shape == (B, H, T, d)
+    o_g, W_g = run(inp, mode=mode | GATE_CHANNEL, b=8)
+    o_n, W_n = run(dict(inp, gate_logit=None), mode=mode | GATE_CHANNEL, b=8)
+    np.testing.assert_array_equal(W_g, W_n)
+    np.testing.assert_allclose(o_g, sig(inp["gate_logit"]) * o_n, rtol=1e-14, atol=1e-300)
+
+
+@pytest.mark.parametrize("mode", [GRAD_LNJAC, MINIBATCH])
+def test_gate_channel_constant_over_features_equals_scalar_gate(mode):
+    B, H, T, d = 2, 2, 13, 16
+    inp = f64(make_inputs(B, H, T, d, seed=36, random_affine=True))
+    o_s, W_s = run(inp, mode=mode, b=4)
+    wide = np.repeat(inp["gate_logit"][..., None], d, axis=-1)
+    o_c, W_c = run(dict(inp, gate_logit=wide), mode=mode | GATE_CHANNEL, b=4)
+    np.testing.assert_array_equal(o_c, o_s)
+    np.testing.assert_array_equal(W_c, W_s)
+
+
+def test_gate_shape_must_match_mode():
+    inp = f64(make_inputs(1, 1, 4, 16, seed=37))
+    with pytest.raises(ValueError):
+        run(inp, mode=GATE_CHANNEL)
+
+
+# ----------------------------------------------------------------------------
+# Streaming decode: one token at a time, W carried between calls.
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [0, GRAD_LNJAC, NO_LN, GRAD_LNJAC | GATE_CHANNEL])
+def test_decode_steps_chain_to_the_per_token_scan(mode):
+    B, H, T, d = 2, 3, 9, 16
+    inp = f64(make_inputs(B, H, T, d, seed=38, random_affine=True, mask_p=0.6, b=1,
+                          gate_channel=bool(mode & GATE_CHANNEL)))
+    o_ref, W_ref = run(inp, mode=mode, b=1)
+    W = inp["W0"]
+    for t in range(T):
+        o_t, W = oracle.decode_step(inp["q"][:, :, t], inp["k"][:, :, t], inp["v"][:, :, t],
+                                    inp["eta_logit"][:, :, t], inp["gate_logit"][:, :, t],
+                                    W, inp["gamma"], inp["beta"], eps=1e-5, mode=mode,
+                                    update=inp["mask"][:, t])
+        np.testing.assert_array_equal(o_t, o_ref[:, :, t])
+    np.testing.assert_array_equal(W, W_ref)
+    with pytest.raises(ValueError):
+        oracle.decode_step(inp["q"][:, :, 0], inp["k"][:, :, 0], inp["v"][:, :, 0],
+                           inp["eta_logit"][:, :, 0], None, W, inp["gamma"], inp["beta"],
+                           eps=1e-5, mode=MINIBATCH)
 
 
 def test_float_twin_close_to_double():
