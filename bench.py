@@ -6,8 +6,9 @@ L2-normalised, eps = 1e-6); one step is one pass with the simplified gradient
 plus one pass with the LayerNorm-Jacobian gradient over the same inputs.
 The metric is head-tokens per second (B*H*T per pass) and the fraction of the
 binding roofline of the dominant kernel. On one GPU the other d = 64 workloads
-(mini-batch bf16 at three shapes, and the per-token bf16-input pass) are
-measured too and reported under ``by_workload``.
+(mini-batch bf16 at three shapes, the per-token bf16-input pass, and the
+streaming decode step over 16384 heads) are measured too and reported under
+``by_workload``.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -181,6 +182,67 @@ class Job:
 
     def kernel_key(self) -> str:
         return "scan_tc" if self.w.minibatch else "scan_simt"
+
+
+class DecodeJob:
+    """The streaming decode step over many heads, W updated in place each step."""
+
+    def __init__(self, name: str, device):
+        import torch
+        from test_sequence_layers_02_b200 import ttt_scan
+        from test_sequence_layers_02_b200.workloads import DECODE_WORKLOADS, make_workload
+        self.w = w = DECODE_WORKLOADS[name]
+        self.name = name
+        self.passes = [dict(lnjac=w.lnjac)]
+        inp = make_workload(w)
+        self.inp = inp
+        self.mask_np = None
+
+        def dev(key):
+            a = inp.get(key)
+            if a is None:
+                return None
+            if w.in_bf16 and key in ("q", "k", "v", "eta_logit", "gate_logit"):
+                a = torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16)
+            else:
+                a = torch.from_numpy(np.ascontiguousarray(a))
+            if key in ("q", "k", "v", "eta_logit", "gate_logit"):
+                a = a[:, :, 0].contiguous()
+            return a.to(device)
+
+        self.t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
+        self.out_dtype = torch.bfloat16 if w.out_bf16 else torch.float32
+        self.o = torch.empty(self.t["q"].shape, dtype=self.out_dtype, device=device)
+        self.step_fn = ttt_scan.decode_step
+
+    @property
+    def head_tokens_per_step(self) -> int:
+        return self.w.heads
+
+    def step(self):
+        t, w = self.t, self.w
+        self.step_fn(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"],
+                     t["beta"], eps=w.eps, lnjac=w.lnjac, out_dtype=self.out_dtype, o=self.o)
+
+    def launches_per_step(self) -> int:
+        return 1
+
+    def flops_per_step(self) -> float:
+        return 6.0 * self.w.d * self.w.d * self.w.heads
+
+    def bytes_per_step(self) -> float:
+        w = self.w
+        d = w.d
+        ie = 2 if w.in_bf16 else 4
+        oe = 2 if w.out_bf16 else 4
+        per_head = 2 * d * d * 4 + 3 * d * ie + 2 * ie + d * oe
+        return float(per_head * w.heads + 2 * w.H * d * 4)
+
+    def bound(self):
+        return "hbm"
+
+    def kernel_key(self) -> str:
+        return "decode_step"
 
 
 def _flush(buf):
@@ -399,6 +461,10 @@ def _e2e(job, steps, device):
 
 def _workload_desc(job):
     w = job.w
+    if isinstance(job, DecodeJob):
+        return (f"TTT-Linear decode step {job.name}: one token per head, W [B,H,d,d] fp32 "
+                f"updated in place, LN-Jacobian gradient, bf16 in, bf16 out, B={w.B} H={w.H} "
+                f"d={w.d}")
     mode = "mini-batch b=%d" % w.b if w.minibatch else "per-token"
     grad = "simplified + LN-Jacobian gradients" if len(job.passes) == 2 else (
         "LN-Jacobian gradient" if w.lnjac else "simplified gradient")
@@ -476,7 +542,7 @@ def run_ours(args):
     by_workload = {}
     if world == 1 and not args.headline_only:
         for name in args.extra:
-            ej = Job(name, device)
+            ej = DecodeJob(name, device) if name == "dec" else Job(name, device)
             ts = _time_job(ej, max(3, min(args.steps, 10)), args.warmup, flush_buf)
             tot = sum(ts)
             pl = tot / (len(ts) * ej.launches_per_step())
@@ -569,6 +635,7 @@ PROFILE_CASES = {
            dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
     "simt": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
              dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
+    "decode": (None, None),
 }
 
 
@@ -579,6 +646,15 @@ def run_profile_case(name: str):
     from test_sequence_layers_02_b200 import build, ttt_scan
     from test_sequence_layers_02_b200.workloads import make_inputs
     build.build()
+    if name == "decode":
+        job = DecodeJob("dec", torch.device("cuda"))
+        for _ in range(2):
+            job.step()
+        rc = ttt_scan.check_device_status()
+        print(f"profile case {name}: status {ttt_scan.status_string(rc)}")
+        if rc != ttt_scan.TTT_OK:
+            raise SystemExit(1)
+        return
     mk, kw = PROFILE_CASES[name]
     inp = make_inputs(**mk)
     bf = mk.get("in_bf16", False)
@@ -610,7 +686,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="2", help="headline workload id (default 2)")
-    ap.add_argument("--extra", nargs="*", default=["3", "4", "4pt", "5"],
+    ap.add_argument("--extra", nargs="*", default=["3", "4", "4pt", "5", "dec"],
                     help="other workloads measured on one GPU (by_workload)")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -50,7 +50,9 @@ enum {
   TTT_NO_LN = 1u << 2,          /* no LayerNorm: pred = z, G = z - v (delta rule); gamma/beta unused */
   TTT_IN_BF16 = 1u << 3,        /* q, k, v, eta_logit, gate_logit are bf16; else fp32 */
   TTT_OUT_BF16 = 1u << 4,       /* o is bf16; else fp32 */
-  TTT_KERNEL_SIMT = 1u << 5     /* run the CUDA-core kernel even where the tensor-core kernel applies */
+  TTT_KERNEL_SIMT = 1u << 5,    /* run the CUDA-core kernel even where the tensor-core kernel applies */
+  TTT_GATE_CHANNEL = 1u << 6    /* gate_logit holds one logit per feature (d per token), applied
+                                   elementwise; else one per token */
 };
 
 /*
@@ -63,7 +65,9 @@ enum {
  * elements, e.g. q..o when T == 0, everything when B*H == 0):
  *   q, k, v      [B, H, T, d]   fp32, or bf16 with TTT_IN_BF16
  *   eta_logit    [B, H, T]      same dtype as q
- *   gate_logit   [B, H, T]      same dtype as q; NULL = no output gate (factor 1)
+ *   gate_logit   [B, H, T]      same dtype as q; NULL = no output gate (factor 1).
+ *                TTT_GATE_CHANNEL (a per-feature gate) is implemented by
+ *                ttt_decode_step only; here it returns TTT_ERR_UNSUPPORTED
  *   W0           [B, H, d, d]   fp32 initial fast weights, z = W k
  *   gamma, beta  [H, d]         fp32 inner-LayerNorm affine; may be NULL with TTT_NO_LN
  *   mask         [B, ceil(T/b)] bytes, nonzero = UPDATE, 0 = SKIP; NULL = all UPDATE
@@ -86,6 +90,44 @@ int ttt_scan_forward(const void* q, const void* k, const void* v,
                      int B, int H, int T, int d, float eps, unsigned mode, int b,
                      const unsigned char* mask, void* o, float* W_T,
                      float* W_chunks, void* cuda_stream);
+
+/*
+ * One streaming decode step: the per-token recurrence above for a single token
+ * of every (batch row, head), with the fast weights carried between calls and
+ * updated IN PLACE (the state-in, state-out step of cortex_rust
+ * src/layers/ttt.rs, forward_update). For each head
+ *
+ *     eta = sigmoid(eta_logit) / d        (0 when update[b] == 0)
+ *     G   = inner gradient at z = W k     (as selected by mode)
+ *     W  <- W - eta * G k^T               (W is not written at all when eta == 0)
+ *     o   = (W q) * sigmoid(gate_logit)   (with the updated W)
+ *
+ * so a chain of T calls equals ttt_scan_forward in per-token mode over those
+ * T tokens (up to fp32 rounding order). Arithmetic is fp32.
+ *
+ * Enqueue-only on `cuda_stream`. All pointers are DEVICE pointers owned by the
+ * caller, 16-byte aligned, contiguous row-major; NULL only where the tensor
+ * has no elements (B*H == 0) or where noted:
+ *   q, k, v      [B, H, d]      fp32, or bf16 with TTT_IN_BF16
+ *   eta_logit    [B, H]         same dtype as q
+ *   gate_logit   [B, H], or [B, H, d] with TTT_GATE_CHANNEL; same dtype as q;
+ *                NULL = no output gate (factor 1)
+ *   W            [B, H, d, d]   fp32 fast weights (z = W k), read and overwritten
+ *   gamma, beta  [H, d]         fp32 inner-LayerNorm affine; may be NULL with TTT_NO_LN
+ *   update       [B] bytes, nonzero = UPDATE, 0 = SKIP (W left bit for bit); NULL = all UPDATE
+ *   o            [B, H, d]      out: fp32, or bf16 with TTT_OUT_BF16
+ * No output may overlap an input, and W may overlap nothing else.
+ * mode: TTT_GRAD_LNJAC, TTT_NO_LN, TTT_IN_BF16, TTT_OUT_BF16, TTT_GATE_CHANNEL.
+ *   TTT_MODE_MINIBATCH returns TTT_ERR_UNSUPPORTED (a one-token step has no
+ *   chunk); TTT_KERNEL_SIMT is accepted and ignored.
+ * Sizes: B, H >= 0, d in {16, 64}, eps >= 0 (finite). Returns TTT_OK or an error
+ * code before launching anything. Allocates no device memory.
+ */
+int ttt_decode_step(const void* q, const void* k, const void* v,
+                    const void* eta_logit, const void* gate_logit, float* W,
+                    const float* gamma, const float* beta, int B, int H, int d,
+                    float eps, unsigned mode, const unsigned char* update, void* o,
+                    void* cuda_stream);
 
 /*
  * Synchronise `cuda_stream`, then report and clear the device status word that

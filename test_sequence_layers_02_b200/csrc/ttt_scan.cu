@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "scan_simt.cuh"
 #include "scan_tc.cuh"
+#include "decode.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -17,7 +18,8 @@ namespace {
 long long g_wait_limit = 1LL << 20;
 
 constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
-                                 TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT;
+                                 TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT |
+                                 TTT_GATE_CHANNEL;
 
 bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
@@ -127,6 +129,23 @@ int dispatch_tc(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
   return launch_tc<float, 2>(p, s);
 }
 
+template <int D, typename InT, typename OutT>
+int launch_decode(const ttt::DecodeParams& p, cudaStream_t stream) {
+  using S = ttt::DecodeShape<D>;
+  const long long blocks = (p.heads + S::HPB - 1) / S::HPB;
+  ttt::decode_step_kernel<D, InT, OutT><<<(unsigned)blocks, S::NT, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+template <int D>
+int dispatch_decode(const ttt::DecodeParams& p, unsigned mode, cudaStream_t s) {
+  const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
+  if (in_bf16 && out_bf16) return launch_decode<D, __nv_bfloat16, __nv_bfloat16>(p, s);
+  if (in_bf16) return launch_decode<D, __nv_bfloat16, float>(p, s);
+  if (out_bf16) return launch_decode<D, float, __nv_bfloat16>(p, s);
+  return launch_decode<D, float, float>(p, s);
+}
+
 template <int D>
 int dispatch_simt_dtypes(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
   const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
@@ -190,6 +209,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
     if (misaligned(p)) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
 
   const size_t heads = (size_t)B * H;
   const int n_mask_chunks = (T + b - 1) / b;
@@ -244,6 +264,58 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   }
   return d == 64 ? dispatch_simt_dtypes<64>(p, mode, stream)
                  : dispatch_simt_dtypes<16>(p, mode, stream);
+}
+
+int ttt_decode_step(const void* q, const void* k, const void* v, const void* eta_logit,
+                    const void* gate_logit, float* W, const float* gamma, const float* beta,
+                    int B, int H, int d, float eps, unsigned mode, const unsigned char* update,
+                    void* o, void* cuda_stream) {
+  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || d <= 0) return TTT_ERR_INVALID_ARG;
+  const bool no_ln = mode & TTT_NO_LN;
+  const bool has_heads = (long long)B * H > 0;
+  if (has_heads && (!q || !k || !v || !eta_logit || !W || !o)) return TTT_ERR_INVALID_ARG;
+  if (has_heads && !no_ln && (!gamma || !beta)) return TTT_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, eta_logit, gate_logit, W, gamma, beta, update, o};
+  for (const void* p : ptrs)
+    if (misaligned(p)) return TTT_ERR_INVALID_ARG;
+  if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
+  if (mode & TTT_MODE_MINIBATCH) return TTT_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+
+  const size_t heads = (size_t)B * H;
+  const size_t in_elt = (mode & TTT_IN_BF16) ? 2 : 4;
+  const size_t out_elt = (mode & TTT_OUT_BF16) ? 2 : 4;
+  const size_t vec_bytes = heads * d * in_elt;
+  const size_t scal_bytes = heads * in_elt;
+  const size_t gate_bytes = (mode & TTT_GATE_CHANNEL) ? vec_bytes : scal_bytes;
+  const size_t o_bytes = heads * d * out_elt;
+  const size_t w_bytes = heads * (size_t)d * d * sizeof(float);
+  const size_t gb_bytes = (size_t)H * d * sizeof(float);
+  struct Span { const void* p; size_t n; };
+  const Span inputs[] = {{q, vec_bytes}, {k, vec_bytes}, {v, vec_bytes},
+                         {eta_logit, scal_bytes}, {gate_logit, gate_bytes},
+                         {gamma, no_ln ? 0 : gb_bytes}, {beta, no_ln ? 0 : gb_bytes},
+                         {update, update ? (size_t)B : 0}};
+  for (const Span& in : inputs) {
+    if (overlaps(o, o_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+    if (overlaps(W, w_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+  }
+  if (overlaps(o, o_bytes, W, w_bytes)) return TTT_ERR_INVALID_ARG;
+  if (heads == 0) return TTT_OK;
+
+  ttt::DecodeParams p{};
+  p.q = q; p.k = k; p.v = v; p.eta_logit = eta_logit; p.gate_logit = gate_logit;
+  p.W = W; p.gamma = gamma; p.beta = beta; p.update = update; p.o = o;
+  p.heads = (long long)heads;
+  p.H = H;
+  p.eps = eps;
+  p.lnjac = (mode & TTT_GRAD_LNJAC) ? 1 : 0;
+  p.no_ln = no_ln ? 1 : 0;
+  p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  return d == 64 ? dispatch_decode<64>(p, mode, stream) : dispatch_decode<16>(p, mode, stream);
 }
 
 }  // extern "C"

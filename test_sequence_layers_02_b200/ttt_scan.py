@@ -2,7 +2,8 @@
 
 Every step of the scan runs in the library's CUDA kernels; this module checks
 shapes and dtypes, allocates outputs with torch, and passes raw device pointers
-and the current CUDA stream to ``ttt_scan_forward`` (include/ttt_scan.h). There
+and the current CUDA stream to ``ttt_scan_forward`` and ``ttt_decode_step``
+(include/ttt_scan.h). There
 is no CPU fallback: if the library cannot be loaded, the first call raises.
 """
 
@@ -23,6 +24,7 @@ NO_LN = 1 << 2
 IN_BF16 = 1 << 3
 OUT_BF16 = 1 << 4
 KERNEL_SIMT = 1 << 5
+GATE_CHANNEL = 1 << 6
 
 TTT_OK = 0
 TTT_ERR_INVALID_ARG = -1
@@ -53,6 +55,9 @@ def lib() -> ctypes.CDLL:
         L.ttt_scan_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
                                        ctypes.c_float, u, i, vp, vp, vp, vp, vp]
         L.ttt_scan_forward.restype = i
+        L.ttt_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i,
+                                      ctypes.c_float, u, vp, vp, vp]
+        L.ttt_decode_step.restype = i
         L.ttt_check_device_status.argtypes = [vp]
         L.ttt_check_device_status.restype = i
         L.ttt_status_string.argtypes = [i]
@@ -167,6 +172,78 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     if want_chunks:
         return o_dev, wt_dev, wc
     return o_dev, wt_dev
+
+
+def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 1e-6,
+                lnjac: bool = False, no_ln: bool = False, update=None,
+                out_dtype: Optional[torch.dtype] = None, o: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None):
+    """One streaming step ``o = decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta)``.
+
+    q, k, v: [B, H, d] fp32 or bf16; eta_logit: [B, H] (same dtype); gate_logit:
+    [B, H], or [B, H, d] for a per-feature gate, or None; W: [B, H, d, d] fp32,
+    UPDATED IN PLACE; gamma, beta: [H, d] fp32 (may be None with ``no_ln``);
+    update: [B] uint8 (0 = SKIP) or None. Returns o [B, H, d] (``out_dtype``,
+    default the input dtype).
+
+    CUDA tensors run on ``stream`` without synchronising. CPU tensors take the
+    end-to-end path: inputs and W go to the current CUDA device, the step runs
+    there, and o and the new W come back (W is overwritten in host memory).
+    """
+    host = not q.is_cuda
+    W_host = None
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+        W_host = W
+        q, k, v, eta_logit, gate_logit, W, gamma, beta, update = map(
+            mv, (q, k, v, eta_logit, gate_logit, W, gamma, beta, update))
+        o_dev = None
+    else:
+        o_dev = o
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, d]")
+    B, H, d = q.shape
+    in_dtype = q.dtype
+    if in_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("inputs must be float32 or bfloat16")
+    channel = gate_logit is not None and gate_logit.dim() == 3
+    for name, t, shp in (("k", k, (B, H, d)), ("v", v, (B, H, d)), ("eta_logit", eta_logit, (B, H)),
+                         ("gate_logit", gate_logit, (B, H, d) if channel else (B, H))):
+        if t is None and name == "gate_logit":
+            continue
+        if tuple(t.shape) != shp or t.dtype != in_dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous {shp} {in_dtype}")
+    if tuple(W.shape) != (B, H, d, d) or W.dtype != torch.float32 or not W.is_contiguous():
+        raise ValueError("W: expected contiguous [B, H, d, d] float32")
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if t is not None and (tuple(t.shape) != (H, d) or t.dtype != torch.float32
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name}: expected contiguous [H, d] float32")
+    if update is not None and (tuple(update.shape) != (B,) or update.dtype != torch.uint8):
+        raise ValueError("update: expected [B] uint8")
+    out_dtype = out_dtype or in_dtype
+    mode = ((GRAD_LNJAC if lnjac else 0) | (NO_LN if no_ln else 0) |
+            (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
+            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (GATE_CHANNEL if channel else 0))
+    if o_dev is None:
+        o_dev = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib().ttt_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W), _ptr(gamma),
+        _ptr(beta), B, H, d, float(eps), mode, _ptr(update), _ptr(o_dev),
+        ctypes.c_void_p(s.cuda_stream))
+    if rc != TTT_OK:
+        raise TTTScanError(rc, "ttt_decode_step")
+    if host:
+        o_h = o if o is not None else torch.empty(o_dev.shape, dtype=o_dev.dtype, pin_memory=True)
+        o_h.copy_(o_dev, non_blocking=True)
+        W_host.copy_(W, non_blocking=True)
+        rc = check_device_status(s)
+        if rc != TTT_OK:
+            raise TTTScanError(rc, "device")
+        return o_h
+    return o_dev
 
 
 def probe_ffma(blocks: int, threads: int, iters: int, sink: torch.Tensor,

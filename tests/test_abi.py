@@ -29,8 +29,8 @@ def declared_functions():
 
 def test_headers_declare_the_boundary():
     names = declared_functions()
-    for must in ("ttt_scan_forward", "ttt_check_device_status", "ttt_status_string",
-                 "ttt_set_wait_limit", "ttt_probe_ffma"):
+    for must in ("ttt_scan_forward", "ttt_decode_step", "ttt_check_device_status",
+                 "ttt_status_string", "ttt_set_wait_limit", "ttt_probe_ffma"):
         assert must in names
 
 
@@ -78,7 +78,7 @@ INVALID, UNSUPPORTED = -1, -2
     dict(q=addr(0, 4)), dict(o=addr(8, 8)), dict(mask=addr(10, 1)), dict(W_chunks=addr(11, 2)),
     dict(B=-1), dict(H=-1), dict(T=-1), dict(b=0), dict(b=-3), dict(d=0), dict(d=-64),
     dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")),
-    dict(mode=1 << 6), dict(mode=1 << 31),
+    dict(mode=1 << 7), dict(mode=1 << 31),
     dict(o=addr(0)),                      # output over an input
     dict(o=addr(2, 1 << 12)),             # output inside v
     dict(W_T=addr(5, 256)),               # W_T partially overlapping W0
@@ -90,7 +90,8 @@ def test_invalid_arguments_rejected(lib, over):
 
 
 @pytest.mark.parametrize("over", [dict(d=32), dict(d=128), dict(d=17),
-                                  dict(mode=1, b=17), dict(mode=1 | 32, b=32)])
+                                  dict(mode=1, b=17), dict(mode=1 | 32, b=32),
+                                  dict(mode=1 << 6)])
 def test_unsupported_shapes(lib, over):
     assert call(lib, **over) == UNSUPPORTED
 
@@ -104,6 +105,42 @@ def test_no_ln_needs_no_affine_and_empty_batch_is_noop(lib):
 
 def test_in_place_W_T_is_accepted_by_the_checks(lib):
     assert call(lib, B=0, W_T=addr(5)) == 0
+
+
+def dcall(lib, **over):
+    a = dict(q=addr(0), k=addr(1), v=addr(2), eta=addr(3), gate=addr(4), W=addr(5),
+             gamma=addr(6), beta=addr(7), B=2, H=3, d=64, eps=1e-6, mode=0, update=None,
+             o=addr(8))
+    a.update(over)
+    return lib.ttt_decode_step(a["q"], a["k"], a["v"], a["eta"], a["gate"], a["W"], a["gamma"],
+                               a["beta"], a["B"], a["H"], a["d"], a["eps"], a["mode"],
+                               a["update"], a["o"], None)
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(k=None), dict(v=None), dict(eta=None), dict(W=None), dict(o=None),
+    dict(gamma=None), dict(beta=None),
+    dict(q=addr(0, 4)), dict(W=addr(5, 8)), dict(update=addr(10, 1)), dict(o=addr(8, 2)),
+    dict(B=-1), dict(H=-1), dict(d=0), dict(eps=-1.0), dict(eps=float("nan")),
+    dict(mode=1 << 7),
+    dict(o=addr(1)),                      # output over an input
+    dict(W=addr(8)),                      # state over the output
+    dict(W=addr(2, 64)),                  # state inside v
+    dict(gate=addr(8, 64), mode=64),      # per-feature gate inside the output
+], ids=lambda o: ",".join(f"{k}" for k in o))
+def test_decode_invalid_arguments_rejected(lib, over):
+    assert dcall(lib, **over) == INVALID
+
+
+@pytest.mark.parametrize("over", [dict(d=32), dict(d=17), dict(mode=1), dict(mode=1 | 2)])
+def test_decode_unsupported(lib, over):
+    assert dcall(lib, **over) == UNSUPPORTED
+
+
+def test_decode_empty_and_no_ln(lib):
+    assert dcall(lib, B=0) == 0
+    assert dcall(lib, H=0, gamma=None, beta=None, mode=4) == 0
+    assert dcall(lib, B=0, q=None, k=None, v=None, eta=None, W=None, o=None) == 0
 
 
 def test_wait_limit(lib):
