@@ -181,7 +181,13 @@ class Job:
         return "hbm" if self.w.minibatch else "alu"
 
     def kernel_key(self) -> str:
-        return "scan_tc" if self.w.minibatch else "scan_simt"
+        from test_sequence_layers_02_b200 import ttt_scan
+        w = self.w
+        k = ttt_scan.kernel_choice(w.B, w.H, w.T, w.d, minibatch=w.minibatch, lnjac=w.lnjac,
+                                   in_bf16=w.in_bf16, out_bf16=w.out_bf16, b=w.b)
+        return {ttt_scan.KERNEL_CUDA_CORE: "scan_simt",
+                ttt_scan.KERNEL_CUDA_CORE_CLUSTER: "scan_cluster",
+                ttt_scan.KERNEL_TENSOR_CORE: "scan_tc"}[k]
 
 
 class DecodeJob:
@@ -634,7 +640,9 @@ PROFILE_CASES = {
     "tc": (dict(B=4, H=16, T=8192, d=64, seed=7, random_affine=True, in_bf16=True),
            dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
     "simt": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
-             dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
+             dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False, single_cta=True)),
+    "cluster": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
+                dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
     "decode": (None, None),
 }
 

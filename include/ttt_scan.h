@@ -51,8 +51,19 @@ enum {
   TTT_IN_BF16 = 1u << 3,        /* q, k, v, eta_logit, gate_logit are bf16; else fp32 */
   TTT_OUT_BF16 = 1u << 4,       /* o is bf16; else fp32 */
   TTT_KERNEL_SIMT = 1u << 5,    /* run the CUDA-core kernel even where the tensor-core kernel applies */
-  TTT_GATE_CHANNEL = 1u << 6    /* gate_logit holds one logit per feature (d per token), applied
+  TTT_GATE_CHANNEL = 1u << 6,   /* gate_logit holds one logit per feature (d per token), applied
                                    elementwise; else one per token */
+  TTT_KERNEL_SINGLE_CTA = 1u << 7 /* per-token mode: keep every head on one CTA even when the
+                                     heads are few enough to spread each over a cluster */
+};
+
+/* Kernel identifiers returned by ttt_scan_kernel_choice(). */
+enum {
+  TTT_KERNEL_NONE = 0,                  /* nothing to launch (B*H == 0) */
+  TTT_KERNEL_ID_CUDA_CORE = 1,          /* CUDA cores, one CTA per head */
+  TTT_KERNEL_ID_CUDA_CORE_CLUSTER = 2,  /* CUDA cores, each head's rows of W split over a
+                                           cluster of 4 CTAs (per-token, d = 64, few heads) */
+  TTT_KERNEL_ID_TENSOR_CORE = 3         /* tcgen05 mini-batch kernel */
 };
 
 /*
@@ -78,8 +89,11 @@ enum {
  *                and, in the last slot, W after the last token (a debugging aid)
  * Sizes: B, H, T >= 0 (B*H == 0 launches nothing; T == 0 copies W0 to W_T),
  *   d in {16, 64}, b >= 1, eps >= 0 (finite).
- * Kernels: per-token mode runs the CUDA-core kernel for any b. Mini-batch mode
- *   runs the tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs, and
+ * Kernels: per-token mode runs a CUDA-core kernel for any b: at d = 64, when
+ *   the B*H heads fit on the device as clusters of 4 CTAs (one per SM), each
+ *   head's rows of W are split over such a cluster; otherwise (or with
+ *   TTT_KERNEL_SINGLE_CTA) one CTA runs each head. Mini-batch mode runs the
+ *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs, and
  *   otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which takes b <= 16.
  *   Other combinations return TTT_ERR_UNSUPPORTED.
  * The library allocates no device memory per call.
@@ -90,6 +104,14 @@ int ttt_scan_forward(const void* q, const void* k, const void* v,
                      int B, int H, int T, int d, float eps, unsigned mode, int b,
                      const unsigned char* mask, void* o, float* W_T,
                      float* W_chunks, void* cuda_stream);
+
+/*
+ * The kernel ttt_scan_forward would run for these sizes and mode bits on the
+ * current CUDA device: one of the TTT_KERNEL_* identifiers above, or a negative
+ * status (TTT_ERR_INVALID_ARG / TTT_ERR_UNSUPPORTED for arguments the scan
+ * rejects). Launches nothing.
+ */
+int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b);
 
 /*
  * One streaming decode step: the per-token recurrence above for a single token
@@ -119,7 +141,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v,
  * No output may overlap an input, and W may overlap nothing else.
  * mode: TTT_GRAD_LNJAC, TTT_NO_LN, TTT_IN_BF16, TTT_OUT_BF16, TTT_GATE_CHANNEL.
  *   TTT_MODE_MINIBATCH returns TTT_ERR_UNSUPPORTED (a one-token step has no
- *   chunk); TTT_KERNEL_SIMT is accepted and ignored.
+ *   chunk); TTT_KERNEL_SIMT and TTT_KERNEL_SINGLE_CTA are accepted and ignored.
  * Sizes: B, H >= 0, d in {16, 64}, eps >= 0 (finite). Returns TTT_OK or an error
  * code before launching anything. Allocates no device memory.
  */

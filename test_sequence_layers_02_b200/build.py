@@ -11,13 +11,15 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libttt_scan.so"
-SOURCES = [CSRC / "ttt_scan.cu", CSRC / "probe.cu"]
-HEADERS = sorted(CSRC.glob("*.cuh")) + sorted((ROOT / "include").glob("*.h"))
+# Translation units, compiled in parallel and linked into one shared library.
+SOURCES = [CSRC / "ttt_scan.cu", CSRC / "simt_f32.cu", CSRC / "simt_bf16.cu",
+           CSRC / "cluster.cu", CSRC / "probe.cu"]
+HEADERS = sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.h")) + sorted((ROOT / "include").glob("*.h"))
 
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    *ARCH, "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
     "-I", str(ROOT / "include"), "-I", str(CSRC),
 ]
@@ -40,12 +42,29 @@ def stale() -> bool:
 def build(force: bool = False, verbose: bool = False, extra=()) -> Path:
     if not force and not stale():
         return LIB
-    tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, *map(str, SOURCES), "-o", str(tmp)]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    tag = f"{os.getpid()}"
+    objs, procs = [], []
+    try:
+        for src in SOURCES:
+            obj = LIB.parent / f".{src.stem}.{tag}.o"
+            cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-c", str(src), "-o", str(obj)]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            objs.append(obj)
+            procs.append((src, subprocess.Popen(cmd)))
+        failed = [src.name for src, pr in procs if pr.wait() != 0]
+        if failed:
+            raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
+        tmp = LIB.with_suffix(f".so.tmp{tag}")
+        link = [_nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *map(str, objs), "-o", str(tmp)]
+        if verbose:
+            print(" ".join(link), file=sys.stderr)
+        subprocess.run(link, check=True)
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if obj.exists():
+                obj.unlink()
     return LIB
 
 

@@ -36,11 +36,6 @@ struct ScanParams {
 
 enum : int { kStatusOk = 0, kStatusTimeout = 1 };
 
-// Set to a nonzero code by a kernel whose bounded wait gave up; read and
-// cleared by ttt_check_device_status(). One word per device, allocated with
-// the module (this header is compiled into a single translation unit).
-__device__ int g_ttt_status;
-
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

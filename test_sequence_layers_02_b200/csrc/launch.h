@@ -1,0 +1,27 @@
+// Host-side launchers of the CUDA-core kernels, each compiled in its own
+// translation unit (simt_f32.cu, simt_bf16.cu, cluster.cu) so the library
+// builds in parallel. Arguments are already checked by the C-ABI entry points;
+// every function returns a ttt_status code.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ttt {
+
+// One CTA per head: fp32 inputs / bf16 inputs (output dtype, mode and d from
+// the arguments).
+int launch_simt_f32in(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+int launch_simt_bf16in(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+
+// Per-token d = 64, each head over a cluster of CTAs. gm: 0 simplified,
+// 1 LN-Jacobian, 2 no LayerNorm gradient.
+int launch_cluster(const ScanParams& p, unsigned mode, int gm, cudaStream_t stream);
+// Clusters of that kernel that fit on the current device at once (0 if unknown).
+int cluster_capacity(unsigned mode, int gm);
+// Read and clear that kernel's device status word: 0 clean, > 0 a bounded wait
+// gave up, < 0 the copy failed.
+int cluster_status_take();
+
+}  // namespace ttt

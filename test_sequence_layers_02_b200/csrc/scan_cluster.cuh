@@ -1,0 +1,736 @@
+// CUDA-core (fp32) per-token scan with one head spread over a cluster of CS
+// CTAs, for the case of few heads (fewer than the SMs / CS).
+//
+// Same exact chunk identity as scan_simt.cuh ("Edifice.Recurrent.TTT",
+// Equations (TTT-Linear)): with W_s the state at the start of chunk c and
+// eta-weighted Grams A (in-chunk, j < m), X (next chunk against this one) and
+// S (queries against keys, j <= i),
+//
+//     z_{c,m}   = P_{c,m} - sum_{j<m} A_mj G_{c,j},        P_c = K_c W_{s,c-1}^T - X_c G_{c-1}
+//     o_{c,i}   = Q0_{c,i} - sum_{j<=i} S_ij G_{c,j},      Q0_c = Q_c W_{s,c}^T
+//     W_{s,c+1} = W_{s,c} - sum_j eta_j G_{c,j} k_{c,j}^T .
+//
+// Work split. CTA q of the cluster owns rows [q RS, (q+1) RS) of W (RS = 64 / CS)
+// in the registers of its four bulk warps (thread = one row x 8 columns). Per
+// chunk period the bulk warps apply the rank-C update to their rows, compute
+// their rows of Q0_c and of K_{c+1} W_{s,c}^T (the latter sent to EVERY CTA of
+// the cluster), form the chunk Grams, write this CTA's rows of the outputs of
+// chunk c-1 and prefetch the next tiles and scalars.
+// Warp 0 of every CTA runs the same sequential gradient chain over the full 64
+// features (replicated, so G never crosses CTAs); besides the in-chunk
+// right-looking update it applies each G_{c,j} to the NEXT chunk's z's (the
+// -X G_c term above), so the next chunk starts from P + that correction with
+// no separate correction phase.
+//
+// Hand-off. Within a CTA, one block barrier ends every chunk period (buffers
+// written in period c are read in period c+1 and are double-buffered). Across
+// the cluster only P moves: each CTA keeps four P slots, each with an
+// mbarrier that expects the slot's 4096 bytes; producers write with
+// asynchronous remote stores that complete those bytes on the consumer's
+// barrier, the chain waits (bounded) for the slot and re-arms it for its next
+// use. The chain waits for every chunk, so no CTA runs more than two periods
+// ahead of another and four slots are enough for a slot never to be rewritten
+// while it is read. A slot holds P transposed, [feature][token] with a padded
+// token stride, so the chain reads its two features' 16 tokens with
+// conflict-free 16-byte loads.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "scan_simt.cuh"
+
+namespace ttt {
+
+template <typename InT, int CS>
+struct ClusterLayout {
+  static constexpr int D = 64;
+  static constexpr int RS = D / CS;         // rows of W per CTA
+  static constexpr int NW = 128;            // bulk threads (warps 0-3)
+  static constexpr int NT = NW + 32;        // + the chain warp (warp 4)
+  static constexpr int G = NW / RS;         // threads per row of W
+  static constexpr int KW = D / G;          // columns of W per thread
+  static constexpr int ELT = (int)sizeof(InT);
+  static constexpr int ROWB = D * ELT + 16; // padded tile row (bytes), as scan_simt.cuh
+  static constexpr int TILE = kC * ROWB;
+  static constexpr int oK = 0;                        // K tiles, ring of 8
+  static constexpr int oQ = oK + 8 * TILE;            // Q tiles, ring of 2
+  static constexpr int oV = oQ + 2 * TILE;            // V tiles, ring of 2
+  static constexpr int NPS = 4;                       // P slots
+  static constexpr int PTS = kC + 4;                  // padded token stride of a P slot
+  static constexpr int PSLOT = D * PTS;               // floats per P slot
+  static constexpr int oP = oV + 2 * TILE;            // P^T of the chain's chunk [NPS][D][PTS]
+  static constexpr int oG = oP + NPS * PSLOT * 4;     // G                     [2][kC][D]
+  static constexpr int oQ0 = oG + 2 * kC * D * 4;     // own rows of Q0        [2][kC][RS]
+  static constexpr int oS = oQ0 + 2 * kC * RS * 4;    // S[i][j]               [2][kC][kC]
+  static constexpr int oAT = oS + 2 * kC * kC * 4;    // A^T[j][m]             [2][kC][kC]
+  static constexpr int oXT = oAT + 2 * kC * kC * 4;   // X^T[j][m]             [2][kC][kC]
+  static constexpr int oEta = oXT + 2 * kC * kC * 4;  // eta  [4][kC]
+  static constexpr int oGate = oEta + 4 * kC * 4;     // gate [4][kC]
+  static constexpr int oFlag = oGate + 4 * kC * 4;    // chunk updates? [4]
+  static constexpr int oBar = oFlag + 16;              // P-slot mbarriers [NPS]
+  static constexpr int bytes = oBar + NPS * 8;
+  static constexpr uint32_t kSlotBytes = kC * D * 4;   // one P delivery, all CTAs together
+  // Requested dynamic shared memory: more than half an SM's, so that one CTA
+  // of a cluster runs per SM.
+  static constexpr int launch_bytes = bytes > 120 * 1024 ? bytes : 120 * 1024;
+  static_assert(KW == 8, "a W thread holds two 4-element units of its row");
+};
+
+// Four consecutive elements of a shared-memory tile row (16 bytes of fp32 or
+// 8 bytes of bf16), widened to two fp32 pairs.
+template <typename InT>
+struct Unit;
+template <>
+struct Unit<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = make_float2(a.x, a.y);
+    x[1] = make_float2(a.z, a.w);
+  }
+};
+template <>
+struct Unit<__nv_bfloat16> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    x[0] = make_float2(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u));
+    x[1] = make_float2(__uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u));
+  }
+};
+
+__device__ __forceinline__ float2 dup2(float x) { return make_float2(x, x); }
+
+// Warp-wide sums of five values; the adds run as pairs.
+__device__ __forceinline__ void butterfly5(float (&m)[5]) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float r[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) r[i] = __shfl_xor_sync(0xffffffffu, m[i], off);
+    const float2 a = __fadd2_rn(make_float2(m[0], m[1]), make_float2(r[0], r[1]));
+    const float2 b = __fadd2_rn(make_float2(m[2], m[3]), make_float2(r[2], r[3]));
+    m[0] = a.x; m[1] = a.y; m[2] = b.x; m[3] = b.y;
+    m[4] += r[4];
+  }
+}
+
+// Set when a bounded wait of this kernel gave up; read and cleared by
+// ttt_check_device_status(). One word per device in this module.
+__device__ int g_cluster_status;
+
+// Polls of the second, fixed bound a chain wait keeps using after the caller's
+// limit ran out (the flag is then already set): it keeps the P slots'
+// barrier bookkeeping in step, so no delivery is still in flight at exit.
+constexpr long long kDrainPolls = 1LL << 24;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ void pbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void pbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// The one expected arrival of a slot phase, announcing its byte count.
+__device__ __forceinline__ void pbar_arm(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool pbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Asynchronous 16-byte store into another CTA's shared memory; its completion
+// counts 16 bytes on that CTA's barrier (both addresses in the cluster window).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_dst, float a, float b, float c,
+                                            float d, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(remote_dst),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
+}
+
+// Reduce-scatter of V partial sums over the G lanes of one row group (lane
+// bits 0 .. log2 G - 1): each step exchanges half of the values still held
+// (S of them) across lane bit B. Afterwards lane g holds the full sums of
+// values g (V/G) .. g (V/G) + V/G - 1 in a[0 .. V/G).
+template <int V, int S, int B>
+__device__ __forceinline__ void reduce_scatter_step(float (&a)[V], int g) {
+  if constexpr (B >= 1) {
+    const bool up = g & B;
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      const float send = up ? a[j] : a[j + S];
+      const float keep = up ? a[j + S] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, B);
+    }
+    reduce_scatter_step<V, S / 2, B / 2>(a, g);
+  }
+}
+template <int V, int G>
+__device__ __forceinline__ void reduce_scatter_lanes(float (&a)[V], int g) {
+  reduce_scatter_step<V, V / 2, G / 2>(a, g);
+}
+
+template <typename InT, typename OutT, int GM, int CS>
+__global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
+    scan_cluster_kernel(const ScanParams p) {
+  namespace cg = cooperative_groups;
+  using L = ClusterLayout<InT, CS>;
+  constexpr int D = 64;
+  constexpr int RS = L::RS, G = L::G, KW = L::KW;
+  constexpr int EPL = 2;                // features per chain lane
+  constexpr int NP = kC / 2;            // token pairs of a chunk
+  extern __shared__ __align__(16) unsigned char smem[];
+  unsigned char* sK = smem + L::oK;
+  unsigned char* sQ = smem + L::oQ;
+  unsigned char* sV = smem + L::oV;
+  float* sP = reinterpret_cast<float*>(smem + L::oP);
+  float* sG = reinterpret_cast<float*>(smem + L::oG);
+  float* sQ0 = reinterpret_cast<float*>(smem + L::oQ0);
+  float* sS = reinterpret_cast<float*>(smem + L::oS);
+  float* sAT = reinterpret_cast<float*>(smem + L::oAT);
+  float* sXT = reinterpret_cast<float*>(smem + L::oXT);
+  float* sEta = reinterpret_cast<float*>(smem + L::oEta);
+  float* sGate = reinterpret_cast<float*>(smem + L::oGate);
+  int* sFlag = reinterpret_cast<int*>(smem + L::oFlag);
+  uint64_t* pbar = reinterpret_cast<uint64_t*>(smem + L::oBar);
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int q = (int)cluster.block_rank();
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const bool chain = tid >= L::NW;
+  const long long bh = blockIdx.x / CS;
+  const int bi = (int)(bh / p.H);
+  const int h = (int)(bh - (long long)bi * p.H);
+  const int T = p.T;
+  const int C = p.C;
+  const int nc = (T + C - 1) / C;
+  const size_t tok0 = (size_t)bh * T;
+  const InT* gq = static_cast<const InT*>(p.q) + tok0 * D;
+  const InT* gk = static_cast<const InT*>(p.k) + tok0 * D;
+  const InT* gv = static_cast<const InT*>(p.v) + tok0 * D;
+  const InT* gel = static_cast<const InT*>(p.eta_logit) + tok0;
+  const InT* ggl = p.gate_logit ? static_cast<const InT*>(p.gate_logit) + tok0 : nullptr;
+  OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
+  float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
+  const float inv_d = 1.0f / (float)D;
+
+  auto chunk_len = [&](int c) { return (c < nc) ? min(C, T - c * C) : 0; };
+  auto tileK = [&](int c) { return sK + (c & 7) * L::TILE; };
+  auto tileQ = [&](int c) { return sQ + (c & 1) * L::TILE; };
+  auto tileV = [&](int c) { return sV + (c & 1) * L::TILE; };
+
+  const int at = tid;  // bulk thread index for prefetch, scalars and outputs
+  struct RawScalars {
+    InT e, g;
+    unsigned char m;
+  };
+  auto issue_scalars = [&](int c) {
+    RawScalars s;
+    s.e = InT();
+    s.g = InT();
+    s.m = 1;
+    if (at < kC) {
+      const int t0 = c * C;
+      if (p.mask != nullptr) s.m = p.mask[(size_t)bi * p.n_mask_chunks + t0 / p.b];
+      if (at < chunk_len(c)) {
+        s.e = gel[t0 + at];
+        if (ggl) s.g = ggl[t0 + at];
+      }
+    }
+    return s;
+  };
+  auto finish_scalars = [&](int c, const RawScalars& s) {
+    if (at < kC) {
+      const bool upd = s.m != 0;
+      const bool ok = at < chunk_len(c);
+      sEta[(c & 3) * kC + at] = (ok && upd) ? sigmoidf_(to_f32(s.e)) * inv_d : 0.f;
+      sGate[(c & 3) * kC + at] = (ok && ggl) ? sigmoidf_(to_f32(s.g)) : 1.f;
+      if (at == 0) sFlag[c & 3] = upd ? 1 : 0;
+    }
+  };
+
+  // ---- bulk thread wt = 0..127 holds W[grow][8 g .. 8 g + 7] ----
+  const int wt = tid;
+  const int rl = wt / G;
+  const int g = wt % G;
+  const int grow = q * RS + rl;
+  // fp32 tiles: the upper half of the column groups takes its two 4-column
+  // units in swapped order, so the 8 broadcast addresses of one load hit
+  // disjoint banks
+  const int swap = (L::ELT == 4 && g >= G / 2) ? 1 : 0;
+  auto ucol = [&](int u) { return g * KW + 4 * (u ^ swap); };  // first column of unit u
+  float2 W2[4];  // unit u: W2[2 u], W2[2 u + 1] = columns ucol(u) .. + 3
+
+  // W_{s} -= sum_j eta_j G_j[grow] k_j^T over the kC rows of tile Kt (rows past
+  // the chunk have eta = 0 and G = 0). All scales are loaded first; keys go in
+  // groups of 4 so the loads of a group overlap the FMAs of the previous one.
+  auto rank_update = [&](const unsigned char* Kt, const float* Gp, const float* et) {
+    float nge[kC];
+#pragma unroll
+    for (int j = 0; j < kC; ++j) nge[j] = -et[j] * Gp[j * D + grow];
+#pragma unroll
+    for (int j0 = 0; j0 < kC; j0 += 4) {
+      float2 x[4][2][2];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) Unit<InT>::ld(Kt + (j0 + b) * L::ROWB + ucol(u) * L::ELT, x[b][u]);
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          W2[2 * u] = __ffma2_rn(dup2(nge[j0 + b]), x[b][u][0], W2[2 * u]);
+          W2[2 * u + 1] = __ffma2_rn(dup2(nge[j0 + b]), x[b][u][1], W2[2 * u + 1]);
+        }
+    }
+  };
+  // Rows [0, kC) of Q0 from rowsA (may be null) and of P from rowsB (may be
+  // null), for this CTA's rows; P goes to slot `pslot` of every CTA of the cluster.
+  auto products = [&](const unsigned char* rowsA, const unsigned char* rowsB, float* q0dst,
+                      int pslot) {
+    float acc[2 * kC];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const unsigned char* R = half == 0 ? rowsA : rowsB;
+      if (R != nullptr) {
+#pragma unroll
+        for (int t0 = 0; t0 < kC; t0 += 4) {
+          float2 x[4][2][2];
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) Unit<InT>::ld(R + (t0 + b) * L::ROWB + ucol(u) * L::ELT, x[b][u]);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            float2 a0 = __fmul2_rn(W2[0], x[b][0][0]);
+            float2 a1 = __fmul2_rn(W2[1], x[b][0][1]);
+            a0 = __ffma2_rn(W2[2], x[b][1][0], a0);
+            a1 = __ffma2_rn(W2[3], x[b][1][1], a1);
+            const float2 a = __fadd2_rn(a0, a1);
+            acc[half * kC + t0 + b] = a.x + a.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < kC; ++t) acc[half * kC + t] = 0.f;
+      }
+    }
+    reduce_scatter_lanes<2 * kC, G>(acc, g);
+    constexpr int PER = 2 * kC / G;
+    static_assert(PER == 4, "four tokens per thread after the reduce-scatter");
+    const int t0 = g * PER;
+    if (t0 < kC) {
+      if (q0dst != nullptr) {
+#pragma unroll
+        for (int v = 0; v < PER; ++v) q0dst[(t0 + v) * RS + rl] = acc[v];
+      }
+    } else if (pslot >= 0) {
+      // tokens t0 - kC .. + 3 of row grow, into P^T of every CTA
+      const uint32_t dst = smem_addr(sP + pslot * L::PSLOT + grow * L::PTS + (t0 - kC));
+      const uint32_t bar = smem_addr(pbar + pslot);
+#pragma unroll
+      for (int rk = 0; rk < CS; ++rk)
+        st_async_v4(cluster_addr(dst, rk), acc[0], acc[1], acc[2], acc[3], cluster_addr(bar, rk));
+    }
+  };
+  const int gt = tid;
+  // Dot products of NL left rows (left0 rows, then left1 rows) with the kC rows
+  // of `right`: Gram thread (j, half) holds right row j's half in registers; the
+  // result of (left row s, right row j) goes to emit(s, j, dot).
+  auto gram = [&](auto nl_tag, const unsigned char* right, const unsigned char* left0,
+                  const unsigned char* left1, auto emit) {
+    constexpr int NL = decltype(nl_tag)::value;
+    constexpr int NG = L::NW / 32;  // bulk warps
+    static_assert(NL % (2 * NG) == 0, "left rows go two per warp at a time");
+    const int j = gt & 15, kq = (gt >> 4) & 1, grp = gt >> 5;
+    float2 rk[D / 4];
+#pragma unroll
+    for (int u = 0; u < (D / 2) / 4; ++u) {
+      float2 x[2];
+      Unit<InT>::ld(right + j * L::ROWB + (kq * (D / 2) + u * 4) * L::ELT, x);
+      rk[2 * u] = x[0];
+      rk[2 * u + 1] = x[1];
+    }
+    // two left rows at a time, each with two accumulator chains
+#pragma unroll
+    for (int it = 0; it < NL / NG; it += 2) {
+      int s[2];
+      const unsigned char* row[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        s[r] = grp + NG * (it + r);
+        row[r] = (s[r] < kC ? left0 + s[r] * L::ROWB : left1 + (s[r] - kC) * L::ROWB) +
+                 kq * (D / 2) * L::ELT;
+      }
+      float2 acc[2][2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < (D / 2) / 4; ++u) {
+        float2 x[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) Unit<InT>::ld(row[r] + u * 4 * L::ELT, x[r]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          acc[r][0] = __ffma2_rn(rk[2 * u], x[r][0], acc[r][0]);
+          acc[r][1] = __ffma2_rn(rk[2 * u + 1], x[r][1], acc[r][1]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float2 a = __fadd2_rn(acc[r][0], acc[r][1]);
+        float dot = a.x + a.y;
+        dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+        if (kq == 0) emit(s[r], j, dot);
+      }
+    }
+  };
+  // eta-weighted Grams feeding the chain of chunk c: A^T_c and X^T_{c+1} into slot c & 1
+  auto chain_grams = [&](int c) {
+    const float* et = sEta + (c & 3) * kC;
+    const int n0 = chunk_len(c), n1 = chunk_len(c + 1);
+    float* AT = sAT + (c & 1) * kC * kC;
+    float* XT = sXT + (c & 1) * kC * kC;
+    gram(std::integral_constant<int, 2 * kC>(), tileK(c), tileK(c), tileK(c + 1),
+         [&](int s, int j, float dot) {
+           if (s < kC) {
+             AT[j * kC + s] = (j < s && s < n0) ? et[j] * dot : 0.f;
+           } else {
+             const int m = s - kC;
+             XT[j * kC + m] = (j < n0 && m < n1) ? et[j] * dot : 0.f;
+           }
+         });
+  };
+  auto store_W = [&](float* dst_row) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      *reinterpret_cast<float4*>(dst_row + ucol(u)) =
+          make_float4(W2[2 * u].x, W2[2 * u].y, W2[2 * u + 1].x, W2[2 * u + 1].y);
+  };
+
+  // ---- outputs of chunk c, this CTA's rows ----
+  auto outputs = [&](int c) {
+    const int np = chunk_len(c);
+    const float* Q0p = sQ0 + (c & 1) * kC * RS;
+    const float* Sp = sS + (c & 1) * kC * kC;
+    const float* Gp = sG + (c & 1) * kC * D + q * RS;
+    const float* gt = sGate + (c & 3) * kC;
+    const bool upd = sFlag[c & 3];
+    OutT* dst = go + (size_t)c * C * D + q * RS;
+#pragma unroll
+    for (int k = 0; k < (kC * RS) / L::NW; ++k) {
+      const int idx = at + L::NW * k;
+      const int i = idx / RS, rr = idx % RS;
+      float acc = Q0p[i * RS + rr], acc2 = 0.f;
+      if (upd) {
+        const float4* srow = reinterpret_cast<const float4*>(Sp + i * kC);
+#pragma unroll
+        for (int j4 = 0; j4 < kC / 4; ++j4) {
+          const float4 s4 = srow[j4];
+          acc = fmaf(-s4.x, Gp[(4 * j4) * D + rr], acc);
+          acc2 = fmaf(-s4.y, Gp[(4 * j4 + 1) * D + rr], acc2);
+          acc = fmaf(-s4.z, Gp[(4 * j4 + 2) * D + rr], acc);
+          acc2 = fmaf(-s4.w, Gp[(4 * j4 + 3) * D + rr], acc2);
+        }
+      }
+      if (i < np) dst[(size_t)i * D + rr] = from_f32<OutT>(gt[i] * (acc + acc2));
+    }
+  };
+
+  // ---- chain state (warp 4) ----
+  float gam[EPL], bet[EPL], g2c[EPL], gbc[EPL];
+  float Sgb = 0.f, Sb = 0.f;
+  float2 cpr[NP][EPL];  // correction of the next chunk's z (token pairs) by this chunk's G
+  unsigned dead = 0;    // P slots whose bookkeeping was lost after a failed drain
+#pragma unroll
+  for (int pp = 0; pp < NP; ++pp)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+
+  // ---------------- prologue ----------------
+  if (chain) {
+    if (lane == 0) {
+#pragma unroll
+      for (int sl = 0; sl < L::NPS; ++sl) {
+        pbar_init(pbar + sl, 1);
+        if (sl < nc) pbar_arm(pbar + sl, L::kSlotBytes);  // deliveries of chunks 0..3
+      }
+      pbar_init_fence();
+    }
+    float sgb = 0.f, sb = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      gam[e] = p.no_ln ? 1.f : p.gamma[(size_t)h * D + f];
+      bet[e] = p.no_ln ? 0.f : p.beta[(size_t)h * D + f];
+      g2c[e] = gam[e] * gam[e];
+      gbc[e] = gam[e] * bet[e];
+      sgb = fmaf(gam[e], bet[e], sgb);
+      sb += bet[e];
+    }
+    float s2[2] = {sgb, sb};
+    butterfly<2>(s2);
+    Sgb = s2[0];
+    Sb = s2[1];
+  } else {
+    const float* W0 = p.W0 + ((size_t)bh * D + grow) * D;  // may alias W_T
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float4 w4 = *reinterpret_cast<const float4*>(W0 + ucol(u));
+      W2[2 * u] = make_float2(w4.x, w4.y);
+      W2[2 * u + 1] = make_float2(w4.z, w4.w);
+    }
+    if (nc > 0) {
+      tile_load<D>(tileK(0), gk, 0, chunk_len(0), at, L::NW);
+      tile_load<D>(tileQ(0), gq, 0, chunk_len(0), at, L::NW);
+      tile_load<D>(tileV(0), gv, 0, chunk_len(0), at, L::NW);
+      if (nc > 1) tile_load<D>(tileK(1), gk, C, chunk_len(1), at, L::NW);
+      if (nc > 2) tile_load<D>(tileK(2), gk, 2 * C, chunk_len(2), at, L::NW);
+      cp_async_commit();
+      finish_scalars(0, issue_scalars(0));
+      if (nc > 1) finish_scalars(1, issue_scalars(1));
+      cp_async_wait_all();
+    }
+  }
+  // every CTA has started and armed its barriers before any remote access
+  cluster.sync();
+  if (!chain && nc > 0) {
+    products(nullptr, tileK(0), nullptr, 0);  // P_0 = K_0 W0^T, into slot 0 everywhere
+    chain_grams(0);                           // A_0, X_1
+  }
+  __syncthreads();
+
+  // ---------------- chunk loop ----------------
+  for (int c = 0; c < nc; ++c) {
+    const int n = chunk_len(c);
+    const bool has_next = c + 1 < nc;
+    if (chain) {
+      // ===== gradient chain of chunk c =====
+      // P_c from every CTA of the cluster, waited for even on a SKIP chunk
+      // (that keeps the CTAs paced), then the slot is re-armed for chunk c + 4
+      const int sl = c % L::NPS;
+      if (!((dead >> sl) & 1u)) {
+        const uint32_t parity = (uint32_t)((c / L::NPS) & 1);
+        bool ok = false;
+        for (long long it = 0; it < p.wait_limit && !ok; ++it) ok = pbar_try_wait(pbar + sl, parity);
+        if (!ok) {
+          if (lane == 0) atomicExch(&g_cluster_status, (int)kStatusTimeout);
+          for (long long it = 0; it < kDrainPolls && !ok; ++it) ok = pbar_try_wait(pbar + sl, parity);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) dead |= 1u << sl;
+        else if (lane == 0 && c + L::NPS < nc) pbar_arm(pbar + sl, L::kSlotBytes);
+      }
+      if (!sFlag[c & 3]) {
+        // SKIP: no gradient is needed, and the next chunk takes no correction
+        // from this one (its X is zero)
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+      } else {
+        const float* PT = sP + sl * L::PSLOT;
+        const float* AT = sAT + (c & 1) * kC * kC;
+        const float* XT = sXT + (c & 1) * kC * kC;
+        const unsigned char* Vt = tileV(c);
+        float* Gc = sG + (c & 1) * kC * D;
+        float2 zp[NP][EPL];  // z of token pairs (2 pp, 2 pp + 1), feature lane + 32 e
+        float2 mp[NP];       // their LayerNorm shift (the feature mean)
+        // z = P + the correction from the previous chunk
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const float4* row = reinterpret_cast<const float4*>(PT + (lane + 32 * e) * L::PTS);
+#pragma unroll
+          for (int m4 = 0; m4 < kC / 4; ++m4) {
+            const float4 x = row[m4];
+            zp[2 * m4][e] = __fadd2_rn(make_float2(x.x, x.y), cpr[2 * m4][e]);
+            zp[2 * m4 + 1][e] = __fadd2_rn(make_float2(x.z, x.w), cpr[2 * m4 + 1][e]);
+          }
+        }
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+        if (GM != 2) {
+          // feature means of the 16 rows of z: reduce-scatter over the lanes,
+          // after which lanes 2m and 2m + 1 hold token m's sum
+          float sm[kC];
+#pragma unroll
+          for (int pp = 0; pp < NP; ++pp) {
+            const float2 t = __fadd2_rn(zp[pp][0], zp[pp][1]);
+            sm[2 * pp] = t.x;
+            sm[2 * pp + 1] = t.y;
+          }
+          reduce_scatter_step<kC, kC / 2, 16>(sm, lane);
+          const float mrow = (sm[0] + __shfl_xor_sync(0xffffffffu, sm[0], 1)) * inv_d;
+#pragma unroll
+          for (int pp = 0; pp < NP; ++pp)
+            mp[pp] = make_float2(__shfl_sync(0xffffffffu, mrow, 4 * pp),
+                                 __shfl_sync(0xffffffffu, mrow, 4 * pp + 2));
+        }
+        // No branch inside: tokens past the chunk's end compute finite values
+        // (their P rows are zero) that a select turns into G = 0.
+#pragma unroll
+        for (int i = 0; i < kC; ++i) {
+          const int pi = i / 2;
+          const bool hi = i & 1;
+          float v[EPL], Gv[EPL], zi[EPL];
+          float mG = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            v[e] = lds1(Vt + i * L::ROWB + (lane + 32 * e) * L::ELT, InT());
+            zi[e] = hi ? zp[pi][e].y : zp[pi][e].x;
+          }
+          if (GM == 2) {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) Gv[e] = zi[e] - v[e];
+          } else {
+            const float mu = hi ? mp[pi].y : mp[pi].x;
+            float y[EPL];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) y[e] = zi[e] - mu;
+            if (GM == 1) {
+              // moments of y: sum y^2, sum g2 y, sum g2 y^2, sum w y, sum gamma v
+              float m5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+              float w[EPL];
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) {
+                w[e] = fmaf(-gam[e], v[e], gbc[e]);
+                const float gy = g2c[e] * y[e];
+                m5[0] = fmaf(y[e], y[e], m5[0]);
+                m5[1] += gy;
+                m5[2] = fmaf(gy, y[e], m5[2]);
+                m5[3] = fmaf(w[e], y[e], m5[3]);
+                m5[4] = fmaf(gam[e], v[e], m5[4]);
+              }
+              butterfly5(m5);
+              const float rs = rsqrtf(fmaf(m5[0], inv_d, p.eps));
+              const float mg = (rs * m5[1] + Sgb - m5[4]) * inv_d;
+              const float mgx = rs * (rs * m5[2] + m5[3]) * inv_d;
+              const float rs2 = rs * rs;
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) Gv[e] = rs2 * (g2c[e] - mgx) * y[e] + rs * (w[e] - mg);
+            } else {
+              float m3[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) {
+                m3[0] = fmaf(y[e], y[e], m3[0]);
+                m3[1] = fmaf(gam[e], y[e], m3[1]);
+                m3[2] += v[e];
+              }
+              butterfly<3>(m3);
+              const float rs = rsqrtf(fmaf(m3[0], inv_d, p.eps));
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) Gv[e] = gam[e] * rs * y[e] + bet[e] - v[e];
+              mG = (rs * m3[1] + Sb - m3[2]) * inv_d;
+            }
+          }
+          const bool valid = i < n;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            Gv[e] = valid ? Gv[e] : 0.f;
+            Gc[i * D + lane + 32 * e] = Gv[e];
+          }
+          mG = valid ? mG : 0.f;
+          // this token's G into the later tokens of chunk c (A, zero for m <= i)
+          // and into every token of chunk c+1 (X)
+          float2 nG[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) nG[e] = dup2(-Gv[e]);
+          // (a row of A or X is read four pairs at a time to keep registers low)
+#pragma unroll
+          for (int m4 = (i + 1) / 4; m4 < kC / 4; ++m4) {
+            const float4 a4 = reinterpret_cast<const float4*>(AT + i * kC)[m4];
+            const float2 a2[2] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w)};
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int pp = 2 * m4 + h2;
+              if (pp < (i + 1) / 2) continue;
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) zp[pp][e] = __ffma2_rn(a2[h2], nG[e], zp[pp][e]);
+              if (GM == 0) mp[pp] = __ffma2_rn(a2[h2], dup2(-mG), mp[pp]);
+            }
+          }
+#pragma unroll
+          for (int m4 = 0; m4 < kC / 4; ++m4) {
+            const float4 x4 = reinterpret_cast<const float4*>(XT + i * kC)[m4];
+            const float2 x2[2] = {make_float2(x4.x, x4.y), make_float2(x4.z, x4.w)};
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+              for (int e = 0; e < EPL; ++e)
+                cpr[2 * m4 + h2][e] = __ffma2_rn(x2[h2], nG[e], cpr[2 * m4 + h2][e]);
+          }
+        }
+      }
+    } else {
+      // ===== bulk work of period c =====
+      if (c + 3 < nc) tile_load<D>(tileK(c + 3), gk, (c + 3) * C, chunk_len(c + 3), at, L::NW);
+      if (has_next) {
+        tile_load<D>(tileQ(c + 1), gq, (c + 1) * C, chunk_len(c + 1), at, L::NW);
+        tile_load<D>(tileV(c + 1), gv, (c + 1) * C, chunk_len(c + 1), at, L::NW);
+      }
+      cp_async_commit();
+      RawScalars pre{};
+      if (c + 2 < nc) pre = issue_scalars(c + 2);
+      // W_{s,c} = W_{s,c-1} - sum_j eta_j G_{c-1,j} k_{c-1,j}^T on this CTA's rows
+      if (c >= 1 && sFlag[(c - 1) & 3])
+        rank_update(tileK(c - 1), sG + ((c - 1) & 1) * kC * D, sEta + ((c - 1) & 3) * kC);
+      if (Wc && ((c * C) % p.b) == 0) store_W(Wc + ((size_t)((c * C) / p.b) * D + grow) * D);
+      // Q0_c (own rows) and K_{c+1} W_{s,c}^T (own rows, to every CTA)
+      products(tileQ(c), has_next ? tileK(c + 1) : nullptr, sQ0 + (c & 1) * kC * RS,
+               has_next ? ((c + 1) % L::NPS) : -1);
+      // the Grams of the chain of chunk c+1, then S_c
+      if (has_next) chain_grams(c + 1);
+      {
+        const float* et = sEta + (c & 3) * kC;
+        float* Sc = sS + (c & 1) * kC * kC;
+        gram(std::integral_constant<int, kC>(), tileK(c), tileQ(c), nullptr,
+             [&](int s, int j, float dot) {
+               Sc[s * kC + j] = (j <= s && s < n) ? et[j] * dot : 0.f;
+             });
+      }
+      if (c >= 1) outputs(c - 1);
+      if (c + 2 < nc) finish_scalars(c + 2, pre);
+      cp_async_wait_all();
+    }
+    __syncthreads();
+  }
+
+  // ---------------- epilogue ----------------
+  if (nc > 0) {
+    const int c = nc - 1;
+    if (!chain && sFlag[c & 3]) rank_update(tileK(c), sG + (c & 1) * kC * D, sEta + (c & 3) * kC);
+    if (!chain) outputs(c);
+  }
+  if (!chain) {
+    if (Wc) store_W(Wc + ((size_t)p.n_mask_chunks * D + grow) * D);
+    store_W(p.W_T + ((size_t)bh * D + grow) * D);
+  }
+  cluster.sync();  // no CTA leaves while a peer could still address its shared memory
+}
+
+}  // namespace ttt

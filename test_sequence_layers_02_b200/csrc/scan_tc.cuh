@@ -40,6 +40,11 @@
 
 namespace ttt {
 
+// Set to a nonzero code by a kernel whose bounded wait gave up; read and
+// cleared by ttt_check_device_status(). One word per device, allocated with
+// the module of the one translation unit that includes this header.
+__device__ int g_ttt_status;
+
 struct TcMaps {
   CUtensorMap q, k, v;  // [B*H][T][64] bf16 as {64, T, B*H}, box {64, 16, 1}
 };

@@ -7,9 +7,10 @@
 
 #include "ttt_scan.h"
 #include "common.cuh"
-#include "scan_simt.cuh"
+#include "scan_simt.cuh"  // chunk limit kC (the kernels themselves are instantiated elsewhere)
 #include "scan_tc.cuh"
 #include "decode.cuh"
+#include "launch.h"
 
 #include <cudaTypedefs.h>
 
@@ -19,7 +20,7 @@ long long g_wait_limit = 1LL << 20;
 
 constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
                                  TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT |
-                                 TTT_GATE_CHANNEL;
+                                 TTT_GATE_CHANNEL | TTT_KERNEL_SINGLE_CTA;
 
 bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
@@ -36,39 +37,18 @@ int largest_divisor_upto(int b, int cap) {
   return 1;
 }
 
-template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
-int launch_simt_ih(const ttt::ScanParams& p, cudaStream_t stream) {
-  using L = ttt::PipeLayout<D, InT, IH>;
-  auto kernel = ttt::scan_simt_kernel<D, InT, OutT, MINIB, GM, IH>;
-  if (L::bytes > 48 * 1024) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)L::bytes) != cudaSuccess)
-      return TTT_ERR_CUDA;
+// Which kernel a valid call runs (see ttt_scan_kernel_choice in the header).
+int choose_kernel(long long heads, int T, int d, unsigned mode, int b) {
+  if (heads == 0) return TTT_KERNEL_NONE;
+  const bool minibatch = mode & TTT_MODE_MINIBATCH;
+  if (minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
+      !(mode & TTT_KERNEL_SIMT) && T > 0)
+    return TTT_KERNEL_ID_TENSOR_CORE;
+  if (!minibatch && d == 64 && !(mode & TTT_KERNEL_SINGLE_CTA) && T > 0) {
+    const int gm = (mode & TTT_NO_LN) ? 2 : ((mode & TTT_GRAD_LNJAC) ? 1 : 0);
+    if (heads <= ttt::cluster_capacity(mode, gm)) return TTT_KERNEL_ID_CUDA_CORE_CLUSTER;
   }
-  kernel<<<(unsigned)(p.B * p.H), L::NT, L::bytes, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
-}
-
-// Few heads (at most one CTA per SM): 8 bulk warps per CTA; otherwise 4, so
-// that several CTAs share an SM.
-template <int D, typename InT, typename OutT, bool MINIB, int GM>
-int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
-  if (D == 64 && (long long)p.B * p.H <= 148)
-    return launch_simt_ih<D, InT, OutT, MINIB, GM, 2>(p, stream);
-  return launch_simt_ih<D, InT, OutT, MINIB, GM, 1>(p, stream);
-}
-
-template <int D, typename InT, typename OutT>
-int dispatch_simt_mode(const ttt::ScanParams& p, cudaStream_t s) {
-  const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
-  if (p.minibatch) {
-    if (gm == 0) return launch_simt<D, InT, OutT, true, 0>(p, s);
-    if (gm == 1) return launch_simt<D, InT, OutT, true, 1>(p, s);
-    return launch_simt<D, InT, OutT, true, 2>(p, s);
-  }
-  if (gm == 0) return launch_simt<D, InT, OutT, false, 0>(p, s);
-  if (gm == 1) return launch_simt<D, InT, OutT, false, 1>(p, s);
-  return launch_simt<D, InT, OutT, false, 2>(p, s);
+  return TTT_KERNEL_ID_CUDA_CORE;
 }
 
 // ---- tensor-core kernel: tensor maps and launch ----
@@ -146,15 +126,6 @@ int dispatch_decode(const ttt::DecodeParams& p, unsigned mode, cudaStream_t s) {
   return launch_decode<D, float, float>(p, s);
 }
 
-template <int D>
-int dispatch_simt_dtypes(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
-  const bool in_bf16 = mode & TTT_IN_BF16, out_bf16 = mode & TTT_OUT_BF16;
-  if (in_bf16 && out_bf16) return dispatch_simt_mode<D, __nv_bfloat16, __nv_bfloat16>(p, s);
-  if (in_bf16) return dispatch_simt_mode<D, __nv_bfloat16, float>(p, s);
-  if (out_bf16) return dispatch_simt_mode<D, float, __nv_bfloat16>(p, s);
-  return dispatch_simt_mode<D, float, float>(p, s);
-}
-
 }  // namespace
 
 extern "C" {
@@ -184,9 +155,10 @@ int ttt_check_device_status(void* cuda_stream) {
   if (h != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(ttt::g_ttt_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
-    return TTT_ERR_DEVICE_TIMEOUT;
   }
-  return TTT_OK;
+  const int hc = ttt::cluster_status_take();
+  if (hc < 0) return TTT_ERR_CUDA;
+  return (h != 0 || hc != 0) ? TTT_ERR_DEVICE_TIMEOUT : TTT_OK;
 }
 
 int ttt_scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
@@ -252,9 +224,8 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   p.minibatch = (mode & TTT_MODE_MINIBATCH) ? 1 : 0;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  const bool tc_ok = p.minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
-                     !(mode & TTT_KERNEL_SIMT) && T > 0;
-  if (tc_ok) return dispatch_tc(p, mode, stream);
+  const int which = choose_kernel((long long)heads, T, d, mode, b);
+  if (which == TTT_KERNEL_ID_TENSOR_CORE) return dispatch_tc(p, mode, stream);
   if (p.minibatch) {
     if (b > ttt::kC) return TTT_ERR_UNSUPPORTED;
     p.C = b;
@@ -262,8 +233,24 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
     // chunks must not straddle a mask / snapshot boundary when either is asked for
     p.C = (mask || W_chunks) ? largest_divisor_upto(b, ttt::kC) : ttt::kC;
   }
-  return d == 64 ? dispatch_simt_dtypes<64>(p, mode, stream)
-                 : dispatch_simt_dtypes<16>(p, mode, stream);
+  if (which == TTT_KERNEL_ID_CUDA_CORE_CLUSTER) {
+    const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
+    return ttt::launch_cluster(p, mode, gm, stream);
+  }
+  return (mode & TTT_IN_BF16) ? ttt::launch_simt_bf16in(p, mode, d, stream)
+                              : ttt::launch_simt_f32in(p, mode, d, stream);
+}
+
+int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b) {
+  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
+  if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
+  const int which = choose_kernel((long long)B * H, T, d, mode, b);
+  if (which == TTT_KERNEL_ID_CUDA_CORE && (mode & TTT_MODE_MINIBATCH) && b > ttt::kC)
+    return TTT_ERR_UNSUPPORTED;
+  return which;
 }
 
 int ttt_decode_step(const void* q, const void* k, const void* v, const void* eta_logit,

@@ -25,6 +25,10 @@ IN_BF16 = 1 << 3
 OUT_BF16 = 1 << 4
 KERNEL_SIMT = 1 << 5
 GATE_CHANNEL = 1 << 6
+KERNEL_SINGLE_CTA = 1 << 7
+
+# Kernel identifiers of ttt_scan_kernel_choice.
+KERNEL_NONE, KERNEL_CUDA_CORE, KERNEL_CUDA_CORE_CLUSTER, KERNEL_TENSOR_CORE = 0, 1, 2, 3
 
 TTT_OK = 0
 TTT_ERR_INVALID_ARG = -1
@@ -58,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i,
                                       ctypes.c_float, u, vp, vp, vp]
         L.ttt_decode_step.restype = i
+        L.ttt_scan_kernel_choice.argtypes = [i, i, i, i, u, i]
+        L.ttt_scan_kernel_choice.restype = i
         L.ttt_check_device_status.argtypes = [vp]
         L.ttt_check_device_status.restype = i
         L.ttt_status_string.argtypes = [i]
@@ -93,7 +99,7 @@ def _ptr(t: Optional[torch.Tensor]):
 def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
          minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
          b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
-         force_simt: bool = False, want_chunks: bool = False,
+         force_simt: bool = False, single_cta: bool = False, want_chunks: bool = False,
          o: Optional[torch.Tensor] = None, W_T: Optional[torch.Tensor] = None,
          stream: Optional[torch.cuda.Stream] = None):
     """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
@@ -101,7 +107,9 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     q, k, v: [B, H, T, d] fp32 or bf16; eta_logit, gate_logit: [B, H, T] with
     the same dtype (gate may be None); W0: [B, H, d, d] fp32 (z = W k);
     gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
-    uint8 or None. ``out_dtype`` defaults to the input dtype.
+    uint8 or None. ``out_dtype`` defaults to the input dtype. ``force_simt``
+    keeps mini-batch mode on the CUDA-core kernel; ``single_cta`` keeps
+    per-token mode on one CTA per head (see ``kernel_choice``).
 
     CUDA tensors run on ``stream`` (default: the current stream) and return
     without synchronising. CPU tensors take the end-to-end path: inputs are
@@ -143,7 +151,8 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     out_dtype = out_dtype or in_dtype
     mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
-            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0))
+            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0) |
+            (KERNEL_SINGLE_CTA if single_cta else 0))
     if o_dev is None:
         o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
     if wt_dev is None:
@@ -172,6 +181,20 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     if want_chunks:
         return o_dev, wt_dev, wc
     return o_dev, wt_dev
+
+
+def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
+                  lnjac: bool = False, no_ln: bool = False, in_bf16: bool = False,
+                  out_bf16: bool = False, b: int = 16, force_simt: bool = False,
+                  single_cta: bool = False) -> int:
+    """The KERNEL_* identifier ``scan`` would run for these sizes (launches nothing)."""
+    mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
+            (NO_LN if no_ln else 0) | (IN_BF16 if in_bf16 else 0) | (OUT_BF16 if out_bf16 else 0) |
+            (KERNEL_SIMT if force_simt else 0) | (KERNEL_SINGLE_CTA if single_cta else 0))
+    rc = lib().ttt_scan_kernel_choice(B, H, T, d, mode, b)
+    if rc < 0:
+        raise TTTScanError(rc, "ttt_scan_kernel_choice")
+    return rc
 
 
 def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 1e-6,

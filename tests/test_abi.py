@@ -29,7 +29,8 @@ def declared_functions():
 
 def test_headers_declare_the_boundary():
     names = declared_functions()
-    for must in ("ttt_scan_forward", "ttt_decode_step", "ttt_check_device_status",
+    for must in ("ttt_scan_forward", "ttt_decode_step", "ttt_scan_kernel_choice",
+                 "ttt_check_device_status",
                  "ttt_status_string", "ttt_set_wait_limit", "ttt_probe_ffma"):
         assert must in names
 
@@ -78,7 +79,7 @@ INVALID, UNSUPPORTED = -1, -2
     dict(q=addr(0, 4)), dict(o=addr(8, 8)), dict(mask=addr(10, 1)), dict(W_chunks=addr(11, 2)),
     dict(B=-1), dict(H=-1), dict(T=-1), dict(b=0), dict(b=-3), dict(d=0), dict(d=-64),
     dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")),
-    dict(mode=1 << 7), dict(mode=1 << 31),
+    dict(mode=1 << 8), dict(mode=1 << 31),
     dict(o=addr(0)),                      # output over an input
     dict(o=addr(2, 1 << 12)),             # output inside v
     dict(W_T=addr(5, 256)),               # W_T partially overlapping W0
@@ -122,7 +123,7 @@ def dcall(lib, **over):
     dict(gamma=None), dict(beta=None),
     dict(q=addr(0, 4)), dict(W=addr(5, 8)), dict(update=addr(10, 1)), dict(o=addr(8, 2)),
     dict(B=-1), dict(H=-1), dict(d=0), dict(eps=-1.0), dict(eps=float("nan")),
-    dict(mode=1 << 7),
+    dict(mode=1 << 8),
     dict(o=addr(1)),                      # output over an input
     dict(W=addr(8)),                      # state over the output
     dict(W=addr(2, 64)),                  # state inside v
@@ -141,6 +142,23 @@ def test_decode_empty_and_no_ln(lib):
     assert dcall(lib, B=0) == 0
     assert dcall(lib, H=0, gamma=None, beta=None, mode=4) == 0
     assert dcall(lib, B=0, q=None, k=None, v=None, eta=None, W=None, o=None) == 0
+
+
+def test_kernel_choice_without_launching(lib):
+    f = lib.ttt_scan_kernel_choice
+    MINIB, LNJAC, BF16 = 1, 2, 8
+    assert f(2, 3, 40, 64, MINIB | LNJAC | BF16, 16) == 3            # tensor cores
+    assert f(2, 3, 40, 64, MINIB | LNJAC | BF16 | 32, 16) == 1       # forced CUDA cores
+    assert f(2, 3, 40, 16, 0, 16) == 1                               # d = 16: one CTA per head
+    assert f(2, 3, 40, 64, 1 << 7, 16) == 1                          # single CTA asked for
+    assert f(0, 3, 40, 64, 0, 16) == 0                               # nothing to launch
+    assert f(2, 3, 40, 64, 1 << 8, 16) == INVALID
+    assert f(2, 3, 40, 64, 0, 0) == INVALID
+    assert f(2, 3, 40, 32, 0, 16) == UNSUPPORTED
+    assert f(2, 3, 40, 64, MINIB, 17) == UNSUPPORTED
+    assert f(2, 3, 40, 64, 1 << 6, 16) == UNSUPPORTED
+    # per-token d = 64 picks the cluster kernel only where clusters fit on a device
+    assert f(2, 3, 40, 64, LNJAC, 16) in (1, 2)
 
 
 def test_wait_limit(lib):

@@ -34,11 +34,19 @@ def _cuda():
 # The named workloads at their full sizes.
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("single_cta", [False, True], ids=["auto", "single_cta"])
 @pytest.mark.parametrize("name", ["1", "2s", "2j"])
-def test_workload_fp32_full(name):
+def test_workload_fp32_full(name, single_cta):
+    from test_sequence_layers_02_b200 import ttt_scan
     w = WORKLOADS[name]
+    if single_cta and w.d != 64:
+        pytest.skip("d = 16 always runs one CTA per head")
+    if w.d == 64:
+        want = ttt_scan.KERNEL_CUDA_CORE if single_cta else ttt_scan.KERNEL_CUDA_CORE_CLUSTER
+        assert ttt_scan.kernel_choice(w.B, w.H, w.T, w.d, lnjac=w.lnjac,
+                                      single_cta=single_cta) == want
     inp = make_workload(w)
-    o, W_T = gpu_scan(inp, in_bf16=False, eps=w.eps, lnjac=w.lnjac, b=w.b)
+    o, W_T = gpu_scan(inp, in_bf16=False, eps=w.eps, lnjac=w.lnjac, b=w.b, single_cta=single_cta)
     ro, rW = oracle_scan(inp, eps=w.eps, mode=_mode(w), b=w.b)
     assert_fp32_close(o, ro, f"{name} o")
     assert_fp32_close(W_T, rW, f"{name} W_T")
@@ -105,17 +113,29 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("single_cta", [False, True], ids=["auto", "single_cta"])
 @pytest.mark.parametrize("with_mask", [False, True])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}H{c[1]}T{c[2]}d{c[3]}m{c[4]}b{c[5]}"
                          f"{'i16' if c[6] else ''}{'o16' if c[7] else ''}")
-def test_small_cases(case, with_mask):
+def test_small_cases(case, with_mask, single_cta):
+    """Per-token d = 64 cases run on the cluster kernel ("auto": few heads) and on
+    the one-CTA-per-head kernel ("single_cta"); the rest on their only kernel."""
     B, H, T, d, mode, b, in_bf16, out_bf16 = case
+    per_token64 = d == 64 and not (mode & MINIB)
+    if single_cta and not per_token64:
+        pytest.skip("same kernel as the auto case")
+    if per_token64:
+        from test_sequence_layers_02_b200 import ttt_scan
+        got = ttt_scan.kernel_choice(B, H, T, d, lnjac=bool(mode & LNJAC), no_ln=bool(mode & NO_LN),
+                                     in_bf16=in_bf16, out_bf16=out_bf16, b=b, single_cta=single_cta)
+        assert got == (ttt_scan.KERNEL_CUDA_CORE if single_cta else ttt_scan.KERNEL_CUDA_CORE_CLUSTER)
     inp = make_inputs(B, H, T, d, seed=100 + T + d + mode + b, random_affine=True,
                       in_bf16=in_bf16, mask_p=0.5 if with_mask else None, b=b)
     eps = 1e-6
     o, W_T, Wc = gpu_scan(inp, in_bf16=in_bf16, out_bf16=out_bf16, eps=eps, b=b,
                           lnjac=bool(mode & LNJAC), minibatch=bool(mode & MINIB),
-                          no_ln=bool(mode & NO_LN), force_simt=True, want_chunks=True)
+                          no_ln=bool(mode & NO_LN), force_simt=True, want_chunks=True,
+                          single_cta=single_cta)
     ro, rW, rWc = oracle_scan(inp, eps=eps, mode=mode, b=b, want_chunks=True)
     if out_bf16:
         assert_rrms(o, ro, "o", tol=1e-2)
@@ -228,3 +248,29 @@ def test_binding_rejects_bad_shapes():
         ttt_scan.scan(q, q, q, torch.zeros((1, 1, 8), device="cuda"), None,
                       torch.zeros((1, 1, 64, 64), device="cuda"), None, None)   # LN needs gamma
     assert e.value.status == ttt_scan.TTT_ERR_INVALID_ARG
+
+
+def test_cluster_wait_timeout_reports_and_recovers():
+    """With a wait limit of 0 the cluster kernel's bounded waits for its peers'
+    P give up at once: the call must report TTT_ERR_DEVICE_TIMEOUT (no hang, no
+    trap) and the context must stay usable for a normal call afterwards."""
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    from tests.helpers import to_torch
+    inp = make_inputs(1, 2, 80, 64, seed=13, random_affine=True)
+    assert ttt_scan.kernel_choice(1, 2, 80, 64, lnjac=True) == ttt_scan.KERNEL_CUDA_CORE_CLUSTER
+    t = to_torch(inp, "cuda", False)
+    args = (t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"], t["beta"])
+    ttt_scan.set_wait_limit(0)
+    try:
+        ttt_scan.scan(*args, eps=1e-6, lnjac=True)
+        assert ttt_scan.check_device_status() == ttt_scan.TTT_ERR_DEVICE_TIMEOUT
+    finally:
+        ttt_scan.set_wait_limit(1 << 20)
+    assert ttt_scan.check_device_status() == ttt_scan.TTT_OK
+    o, W_T = ttt_scan.scan(*args, eps=1e-6, lnjac=True)
+    torch.cuda.synchronize()
+    assert ttt_scan.check_device_status() == ttt_scan.TTT_OK
+    ro, rW = oracle_scan(inp, eps=1e-6, mode=LNJAC, b=16)
+    assert_fp32_close(o.cpu().numpy(), ro, "o")
+    assert_fp32_close(W_T.cpu().numpy(), rW, "W_T")
