@@ -13,9 +13,10 @@
 // Work split. CTA q of the cluster owns rows [q RS, (q+1) RS) of W (RS = 64 / CS)
 // in the registers of its four bulk warps (thread = one row x 8 columns). Per
 // chunk period the bulk warps apply the rank-C update to their rows, compute
-// their rows of Q0_c and of K_{c+1} W_{s,c}^T (the latter sent to EVERY CTA of
-// the cluster), form the chunk Grams, write this CTA's rows of the outputs of
-// chunk c-1 and prefetch the next tiles and scalars.
+// their rows of Q0_c and of K_{c+1} W_{s,c}^T, and rows [4q, 4q+4) of the
+// Grams A_{c+1} and X_{c+2} (those three sent to EVERY CTA of the cluster),
+// form S_c, write this CTA's rows of the outputs of chunk c-1 and prefetch
+// the next tiles and scalars.
 // Warp 0 of every CTA runs the same sequential gradient chain over the full 64
 // features (replicated, so G never crosses CTAs); besides the in-chunk
 // right-looking update it applies each G_{c,j} to the NEXT chunk's z's (the
@@ -24,8 +25,9 @@
 //
 // Hand-off. Within a CTA, one block barrier ends every chunk period (buffers
 // written in period c are read in period c+1 and are double-buffered). Across
-// the cluster only P moves: each CTA keeps four P slots, each with an
-// mbarrier that expects the slot's 4096 bytes; producers write with
+// the cluster the chain's inputs move: each CTA keeps four delivery slots
+// (P^T, A^T, X^T of one chunk), each with an mbarrier that expects the slot's
+// 6144 bytes; producers write with
 // asynchronous remote stores that complete those bytes on the consumer's
 // barrier, the chain waits (bounded) for the slot and re-arms it for its next
 // use. The chain waits for every chunk, so no CTA runs more than two periods
@@ -60,19 +62,21 @@ struct ClusterLayout {
   static constexpr int oV = oQ + 2 * TILE;            // V tiles, ring of 2
   static constexpr int NPS = 4;                       // P slots
   static constexpr int PTS = kC + 4;                  // padded token stride of a P slot
-  static constexpr int PSLOT = D * PTS;               // floats per P slot
-  static constexpr int oP = oV + 2 * TILE;            // P^T of the chain's chunk [NPS][D][PTS]
+  static constexpr int SAT = D * PTS;                 // offset of A^T[j][m] in a slot (floats)
+  static constexpr int SXT = SAT + kC * kC;           // offset of X^T[j][m]
+  static constexpr int PSLOT = SXT + kC * kC;         // floats per delivery slot
+  static constexpr int oP = oV + 2 * TILE;            // delivery slots [NPS][PSLOT]
   static constexpr int oG = oP + NPS * PSLOT * 4;     // G                     [2][kC][D]
   static constexpr int oQ0 = oG + 2 * kC * D * 4;     // own rows of Q0        [2][kC][RS]
   static constexpr int oS = oQ0 + 2 * kC * RS * 4;    // S[i][j]               [2][kC][kC]
-  static constexpr int oAT = oS + 2 * kC * kC * 4;    // A^T[j][m]             [2][kC][kC]
-  static constexpr int oXT = oAT + 2 * kC * kC * 4;   // X^T[j][m]             [2][kC][kC]
-  static constexpr int oEta = oXT + 2 * kC * kC * 4;  // eta  [4][kC]
+  static constexpr int oEta = oS + 2 * kC * kC * 4;   // eta  [4][kC]
   static constexpr int oGate = oEta + 4 * kC * 4;     // gate [4][kC]
   static constexpr int oFlag = oGate + 4 * kC * 4;    // chunk updates? [4]
   static constexpr int oBar = oFlag + 16;              // P-slot mbarriers [NPS]
   static constexpr int bytes = oBar + NPS * 8;
-  static constexpr uint32_t kSlotBytes = kC * D * 4;   // one P delivery, all CTAs together
+  // one delivery, all CTAs together: P (kC x D) and the two Grams (kC x kC each)
+  static constexpr uint32_t kSlotBytes = (kC * D + 2 * kC * kC) * 4;
+  static_assert(RS == 16 && NW == 128, "each CTA computes four Gram rows with two threads per dot");
   // Requested dynamic shared memory: more than half an SM's, so that one CTA
   // of a cluster runs per SM.
   static constexpr int launch_bytes = bytes > 120 * 1024 ? bytes : 120 * 1024;
@@ -209,8 +213,6 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   float* sG = reinterpret_cast<float*>(smem + L::oG);
   float* sQ0 = reinterpret_cast<float*>(smem + L::oQ0);
   float* sS = reinterpret_cast<float*>(smem + L::oS);
-  float* sAT = reinterpret_cast<float*>(smem + L::oAT);
-  float* sXT = reinterpret_cast<float*>(smem + L::oXT);
   float* sEta = reinterpret_cast<float*>(smem + L::oEta);
   float* sGate = reinterpret_cast<float*>(smem + L::oGate);
   int* sFlag = reinterpret_cast<int*>(smem + L::oFlag);
@@ -408,21 +410,60 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
       }
     }
   };
-  // eta-weighted Grams feeding the chain of chunk c: A^T_c and X^T_{c+1} into slot c & 1
-  auto chain_grams = [&](int c) {
+  // Rows [4q, 4q+4) of the eta-weighted Grams feeding the chain of chunk c,
+  // A_c (K_c against K_c) and X_{c+1} (K_{c+1} against K_c), sent transposed
+  // into delivery slot c % NPS of every CTA. Thread (j, r, half): right row j,
+  // left row 4q + r, half the features; four threads' values per j travel as
+  // one 16-byte store.
+  auto split_grams = [&](int c) {
+    const int pr = wt >> 1, kq = wt & 1;
+    const int j = pr >> 2, r = pr & 3, Lrow = 4 * q + r;
     const float* et = sEta + (c & 3) * kC;
     const int n0 = chunk_len(c), n1 = chunk_len(c + 1);
-    float* AT = sAT + (c & 1) * kC * kC;
-    float* XT = sXT + (c & 1) * kC * kC;
-    gram(std::integral_constant<int, 2 * kC>(), tileK(c), tileK(c), tileK(c + 1),
-         [&](int s, int j, float dot) {
-           if (s < kC) {
-             AT[j * kC + s] = (j < s && s < n0) ? et[j] * dot : 0.f;
-           } else {
-             const int m = s - kC;
-             XT[j * kC + m] = (j < n0 && m < n1) ? et[j] * dot : 0.f;
-           }
-         });
+    const unsigned char* right = tileK(c) + j * L::ROWB + kq * (D / 2) * L::ELT;
+    const unsigned char* la = tileK(c) + Lrow * L::ROWB + kq * (D / 2) * L::ELT;
+    const unsigned char* lx = tileK(c + 1) + Lrow * L::ROWB + kq * (D / 2) * L::ELT;
+    float2 aa[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 ax[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int u = 0; u < (D / 2) / 4; ++u) {
+      float2 xr[2], xa[2], xx[2];
+      Unit<InT>::ld(right + u * 4 * L::ELT, xr);
+      Unit<InT>::ld(la + u * 4 * L::ELT, xa);
+      Unit<InT>::ld(lx + u * 4 * L::ELT, xx);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        aa[t] = __ffma2_rn(xr[t], xa[t], aa[t]);
+        ax[t] = __ffma2_rn(xr[t], xx[t], ax[t]);
+      }
+    }
+    const float2 sa = __fadd2_rn(aa[0], aa[1]), sx = __fadd2_rn(ax[0], ax[1]);
+    float da = sa.x + sa.y, dx = sx.x + sx.y;
+    da += __shfl_xor_sync(0xffffffffu, da, 1);
+    dx += __shfl_xor_sync(0xffffffffu, dx, 1);
+    da = (j < Lrow && Lrow < n0) ? et[j] * da : 0.f;
+    dx = (j < n0 && Lrow < n1) ? et[j] * dx : 0.f;
+    // lanes 8 j' + 2 r hold r = 0..3 of one j: gather them on lane 8 j'
+    float va[4], vx[4];
+    va[0] = da;
+    vx[0] = dx;
+#pragma unroll
+    for (int k = 1; k < 4; ++k) {
+      va[k] = __shfl_down_sync(0xffffffffu, da, 2 * k);
+      vx[k] = __shfl_down_sync(0xffffffffu, dx, 2 * k);
+    }
+    if ((lane & 7) == 0) {
+      float* slot = sP + (c % L::NPS) * L::PSLOT;
+      const uint32_t dA = smem_addr(slot + L::SAT + j * kC + 4 * q);
+      const uint32_t dX = smem_addr(slot + L::SXT + j * kC + 4 * q);
+      const uint32_t bar = smem_addr(pbar + (c % L::NPS));
+#pragma unroll
+      for (int rk = 0; rk < CS; ++rk) {
+        const uint32_t rb = cluster_addr(bar, rk);
+        st_async_v4(cluster_addr(dA, rk), va[0], va[1], va[2], va[3], rb);
+        st_async_v4(cluster_addr(dX, rk), vx[0], vx[1], vx[2], vx[3], rb);
+      }
+    }
   };
   auto store_W = [&](float* dst_row) {
 #pragma unroll
@@ -519,7 +560,7 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   cluster.sync();
   if (!chain && nc > 0) {
     products(nullptr, tileK(0), nullptr, 0);  // P_0 = K_0 W0^T, into slot 0 everywhere
-    chain_grams(0);                           // A_0, X_1
+    split_grams(0);                           // A_0, X_1
   }
   __syncthreads();
 
@@ -553,8 +594,8 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
           for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
       } else {
         const float* PT = sP + sl * L::PSLOT;
-        const float* AT = sAT + (c & 1) * kC * kC;
-        const float* XT = sXT + (c & 1) * kC * kC;
+        const float* AT = PT + L::SAT;
+        const float* XT = PT + L::SXT;
         const unsigned char* Vt = tileV(c);
         float* Gc = sG + (c & 1) * kC * D;
         float2 zp[NP][EPL];  // z of token pairs (2 pp, 2 pp + 1), feature lane + 32 e
@@ -703,8 +744,8 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
       // Q0_c (own rows) and K_{c+1} W_{s,c}^T (own rows, to every CTA)
       products(tileQ(c), has_next ? tileK(c + 1) : nullptr, sQ0 + (c & 1) * kC * RS,
                has_next ? ((c + 1) % L::NPS) : -1);
-      // the Grams of the chain of chunk c+1, then S_c
-      if (has_next) chain_grams(c + 1);
+      // this CTA's rows of the Grams of the chain of chunk c+1, then S_c
+      if (has_next) split_grams(c + 1);
       {
         const float* et = sEta + (c & 3) * kC;
         float* Sc = sS + (c & 1) * kC * kC;
