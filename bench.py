@@ -578,7 +578,9 @@ def run_ours(args):
                                   if len(job.passes) == 2 else "one launch"),
                        "parallelism": f"heads sharded across {world} rank(s), no collective"},
             "roofline": roof,
-            "chain_step_ns": round(per_launch / w.T * 1e9, 2),
+            # the passes of a step run concurrently, so one chain step takes the
+            # step time over the sequence length
+            "chain_step_ns": round(t_max / args.steps / w.T * 1e9, 2),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": job.launches_per_step() * args.steps,
