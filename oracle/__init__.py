@@ -4,5 +4,6 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package. It shares no code with the CUDA path.
 """
 
-from .ttt_oracle import (GATE_CHANNEL, GRAD_LNJAC, MINIBATCH, NO_LN, build,  # noqa: F401
-                         decode_step, forward, forward_heads, lngrad, max_threads)
+from .ttt_oracle import (GATE_CHANNEL, GRAD_ABLATE, GRAD_LNJAC, GRAD_NORM_MATCH,  # noqa: F401
+                         MINIBATCH, NO_LN, build, decode_step, forward, forward_heads,
+                         lngrad, max_threads)

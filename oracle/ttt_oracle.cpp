@@ -47,6 +47,12 @@
 //   * mask == NULL means every chunk updates.
 //   * NO_LN removes the LayerNorm: pred = z and G = z - v (the delta rule of the
 //     section "Key Innovations").
+//   * The ablation gradient ("Error Correction in Trained TTT Layers", Abstract:
+//     the full normalised prediction's contribution removed, the LayerNorm
+//     Jacobian retained) is the Jacobian form with the whole prediction
+//     gamma * xhat + beta dropped from the error: g = -gamma * v. With per-token
+//     norm matching it is rescaled to the L2 norm of the full Jacobian-form
+//     gradient of the same token (and is 0 where its own norm is 0).
 //
 // Arithmetic runs in the template scalar type: double is the oracle; the float
 // instantiation exists only to measure how much plain fp32 rounding alone moves
@@ -69,6 +75,8 @@ constexpr unsigned kMiniBatch = 1u << 0;
 constexpr unsigned kLnJacobian = 1u << 1;
 constexpr unsigned kNoLayerNorm = 1u << 2;
 constexpr unsigned kGateChannel = 1u << 6;
+constexpr unsigned kGradAblate = 1u << 8;
+constexpr unsigned kNormMatch = 1u << 9;
 
 template <typename S>
 S sigmoid(S x) {
@@ -99,17 +107,36 @@ void ln_and_grad(const S* z, const S* v, const S* gamma, const S* beta, int d,
       xhat[f] = (z[f] - mu) / s;
       pred[f] = gamma[f] * xhat[f] + beta[f];
     }
-    if (mode & kLnJacobian) {
-      std::vector<S> g(d);
-      S mean_g = 0, mean_gx = 0;
-      for (int f = 0; f < d; ++f) {
-        g[f] = gamma[f] * (pred[f] - v[f]);
-        mean_g += g[f];
-        mean_gx += g[f] * xhat[f];
+    if (mode & (kLnJacobian | kGradAblate)) {
+      // back through the LayerNorm: G = J^T g with g the gradient at its output
+      auto jacobian_t = [&](const std::vector<S>& g, S* out) {
+        S mean_g = 0, mean_gx = 0;
+        for (int f = 0; f < d; ++f) {
+          mean_g += g[f];
+          mean_gx += g[f] * xhat[f];
+        }
+        mean_g /= S(d);
+        mean_gx /= S(d);
+        for (int f = 0; f < d; ++f) out[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;
+      };
+      std::vector<S> g(d), full(d);
+      for (int f = 0; f < d; ++f) g[f] = gamma[f] * (pred[f] - v[f]);
+      jacobian_t(g, full.data());
+      if (mode & kGradAblate) {
+        for (int f = 0; f < d; ++f) g[f] = gamma[f] * (-v[f]);
+        jacobian_t(g, G);
+        if (mode & kNormMatch) {
+          S n_full = 0, n_abl = 0;
+          for (int f = 0; f < d; ++f) {
+            n_full += full[f] * full[f];
+            n_abl += G[f] * G[f];
+          }
+          const S scale = n_abl > S(0) ? std::sqrt(n_full / n_abl) : S(0);
+          for (int f = 0; f < d; ++f) G[f] *= scale;
+        }
+      } else {
+        for (int f = 0; f < d; ++f) G[f] = full[f];
       }
-      mean_g /= S(d);
-      mean_gx /= S(d);
-      for (int f = 0; f < d; ++f) G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;
     } else {
       for (int f = 0; f < d; ++f) G[f] = pred[f] - v[f];
     }
@@ -218,6 +245,8 @@ int forward(const S* q, const S* k, const S* v, const S* eta_logit,
             int B, int H, int T, int d, S eps, unsigned mode, int b,
             const unsigned char* mask, S* o, S* W_T, S* W_chunks, int nthreads) {
   if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return -1;
+  if ((mode & kGradAblate) && (mode & kNoLayerNorm)) return -1;
+  if ((mode & kNormMatch) && !(mode & kGradAblate)) return -1;
   if (!q || !k || !v || !eta_logit || !W0 || !o || !W_T) return -1;
   if (!(mode & kNoLayerNorm) && (!gamma || !beta)) return -1;
   const int n_chunks = (T + b - 1) / b;
@@ -283,6 +312,8 @@ int ttt_oracle_lngrad_f64(const double* z, const double* v, const double* gamma,
                           const double* beta, int d, double eps, unsigned mode,
                           double* pred, double* G, double* xhat) {
   if (!z || !v || !G || d <= 0) return -1;
+  if ((mode & kGradAblate) && (mode & kNoLayerNorm)) return -1;
+  if ((mode & kNormMatch) && !(mode & kGradAblate)) return -1;
   if (!(mode & kNoLayerNorm) && (!gamma || !beta)) return -1;
   ln_and_grad<double>(z, v, gamma, beta, d, eps, mode, pred, G, xhat);
   return 0;

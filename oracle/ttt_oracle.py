@@ -30,6 +30,8 @@ MINIBATCH = 1 << 0
 GRAD_LNJAC = 1 << 1
 NO_LN = 1 << 2
 GATE_CHANNEL = 1 << 6
+GRAD_ABLATE = 1 << 8
+GRAD_NORM_MATCH = 1 << 9
 
 _lib = None
 
@@ -157,6 +159,9 @@ def lngrad(z, v, gamma, beta, *, eps: float, mode: int):
     """One inner LayerNorm + gradient on a single d-vector.
 
     Returns ``(pred, G, xhat)``; with NO_LN, pred = xhat = z and G = z - v.
+    GRAD_ABLATE gives the ablation gradient (prediction removed, LayerNorm
+    Jacobian kept), GRAD_NORM_MATCH additionally rescales it to the norm of the
+    full Jacobian-form gradient.
     """
     lib = _load()
     z = np.ascontiguousarray(z, dtype=np.float64)

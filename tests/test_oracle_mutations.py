@@ -28,13 +28,18 @@ MUTATIONS = [
      "        matvec(W.data(), qt, d, Wq.data());",
      "matvec(W.data(), qt, d, Wq.data());\n        for (int r = 0; r < d; ++r)\n"
      "          for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];"),
-    ("lnjac_drop_mean_g", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - xhat[f] * mean_gx) / s;"),
-    ("lnjac_drop_xhat_term", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - mean_g) / s;"),
+    ("lnjac_drop_mean_g", "out[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "out[f] = (g[f] - xhat[f] * mean_gx) / s;"),
+    ("lnjac_drop_xhat_term", "out[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "out[f] = (g[f] - mean_g) / s;"),
     ("lnjac_drop_gamma", "g[f] = gamma[f] * (pred[f] - v[f]);", "g[f] = (pred[f] - v[f]);"),
-    ("lnjac_no_1_over_s", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "G[f] = (g[f] - mean_g - xhat[f] * mean_gx);"),
+    ("lnjac_no_1_over_s", "out[f] = (g[f] - mean_g - xhat[f] * mean_gx) / s;", "out[f] = (g[f] - mean_g - xhat[f] * mean_gx);"),
     ("eps_outside_sqrt", "const S s = std::sqrt(var + eps);", "const S s = std::sqrt(var) + eps;"),
     ("unbiased_variance", "var /= S(d);", "var /= S(d - 1);"),
     ("drop_beta", "pred[f] = gamma[f] * xhat[f] + beta[f];", "pred[f] = gamma[f] * xhat[f];"),
+    ("ablation_keeps_beta", "for (int f = 0; f < d; ++f) g[f] = gamma[f] * (-v[f]);",
+     "for (int f = 0; f < d; ++f) g[f] = gamma[f] * (beta[f] - v[f]);"),
+    ("ablation_without_jacobian", "        jacobian_t(g, G);\n        if (mode & kNormMatch) {",
+     "        for (int f = 0; f < d; ++f) G[f] = g[f];\n        if (mode & kNormMatch) {"),
+    ("norm_match_without_sqrt", "std::sqrt(n_full / n_abl)", "(n_full / n_abl)"),
     ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
     ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
      "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),

@@ -20,14 +20,18 @@ at least one of them:
 * the per-channel output gate is elementwise: it leaves W alone, scales each
   feature of the ungated output by its own sigmoid, and a gate that is the same
   on every feature reproduces the scalar gate;
-* a chain of single-token steps is the per-token scan with a one-token mask.
+* a chain of single-token steps is the per-token scan with a one-token mask;
+* the ablation gradient is the full Jacobian-form gradient minus its
+  prediction-derived part (the P8 closed form at gamma = 1, beta = 0), is
+  linear in v and vanishes at v = 0; norm matching gives the full gradient's
+  norm in the ablation's direction.
 """
 
 import numpy as np
 import pytest
 
 import oracle
-from oracle import GATE_CHANNEL, GRAD_LNJAC, MINIBATCH, NO_LN
+from oracle import GATE_CHANNEL, GRAD_ABLATE, GRAD_LNJAC, GRAD_NORM_MATCH, MINIBATCH, NO_LN
 from test_sequence_layers_02_b200.workloads import make_inputs
 from tests.conftest import load_golden
 
@@ -304,6 +308,71 @@ def test_p8_prediction_term_cancels_as_eps_to_zero():
     G = lambda v: oracle.lngrad(z, v, None, None, eps=1e-6, mode=GRAD_LNJAC)[1]
     np.testing.assert_allclose(G(v1 + v2) - G(np.zeros(d)), (G(v1) - G(np.zeros(d))) + (G(v2) - G(np.zeros(d))),
                                rtol=1e-9, atol=1e-9)
+
+
+# ----------------------------------------------------------------------------
+# Ablation gradient ("Error Correction in Trained TTT Layers", Abstract: the
+# prediction's contribution removed, the LayerNorm Jacobian retained).
+# ----------------------------------------------------------------------------
+
+def test_ablation_differs_from_full_by_the_prediction_term():
+    """gamma = 1, beta = 0: G_full - G_ablation is the prediction part alone,
+    xhat * eps / (s (var + eps)) (the same closed form as P8)."""
+    rng = np.random.default_rng(28)
+    d = 16
+    z = rng.normal(size=d) * 0.05 + 0.01
+    v = rng.normal(size=d)
+    var = np.var(z)
+    for eps in (1e-2, 1e-4, 1e-6):
+        _, Gf, xhat = oracle.lngrad(z, v, None, None, eps=eps, mode=GRAD_LNJAC)
+        _, Ga, _ = oracle.lngrad(z, v, None, None, eps=eps, mode=GRAD_ABLATE)
+        s = np.sqrt(var + eps)
+        np.testing.assert_allclose(Gf - Ga, xhat * eps / (s * (var + eps)), rtol=1e-9, atol=1e-13)
+
+
+def test_ablation_with_affine_is_the_v_part_of_the_full_gradient():
+    """Any gamma, beta: G_ablation(z, v) = G_full(z, v) - G_full(z, 0), is linear
+    in v and is 0 at v = 0 (the prediction, beta included, no longer enters)."""
+    rng = np.random.default_rng(29)
+    d = 24
+    z = rng.normal(size=d) * 0.3
+    gam = 1.0 + 0.2 * rng.normal(size=d)
+    bet = 0.3 * rng.normal(size=d)
+    v1, v2 = rng.normal(size=d), rng.normal(size=d)
+    full = lambda v: oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_LNJAC)[1]
+    abl = lambda v: oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_ABLATE)[1]
+    np.testing.assert_allclose(abl(v1), full(v1) - full(np.zeros(d)), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(abl(v1 + 2.5 * v2), abl(v1) + 2.5 * abl(v2), rtol=1e-9, atol=1e-12)
+    np.testing.assert_array_equal(abl(np.zeros(d)), np.zeros(d))
+
+
+def test_norm_matching_keeps_direction_and_takes_the_full_norm():
+    rng = np.random.default_rng(30)
+    d = 32
+    z = rng.normal(size=d) * 0.2
+    gam = 1.0 + 0.1 * rng.normal(size=d)
+    bet = 0.1 * rng.normal(size=d)
+    v = rng.normal(size=d)
+    Gf = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_LNJAC)[1]
+    Ga = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_ABLATE)[1]
+    Gn = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_ABLATE | GRAD_NORM_MATCH)[1]
+    np.testing.assert_allclose(np.linalg.norm(Gn), np.linalg.norm(Gf), rtol=1e-12)
+    lam = np.dot(Gn, Ga) / np.dot(Ga, Ga)
+    assert lam > 0
+    np.testing.assert_allclose(Gn, lam * Ga, rtol=1e-12, atol=1e-15)
+    # zero ablation gradient (v = 0) stays zero
+    G0 = oracle.lngrad(z, np.zeros(d), gam, bet, eps=1e-6, mode=GRAD_ABLATE | GRAD_NORM_MATCH)[1]
+    np.testing.assert_array_equal(G0, np.zeros(d))
+
+
+def test_ablation_mode_combinations():
+    inp = f64(make_inputs(1, 1, 8, 16, seed=39))
+    with pytest.raises(ValueError):
+        run(inp, mode=GRAD_ABLATE | NO_LN)
+    with pytest.raises(ValueError):
+        run(inp, mode=GRAD_NORM_MATCH)
+    o, W = run(inp, mode=GRAD_ABLATE | GRAD_NORM_MATCH)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(W))
 
 
 # ----------------------------------------------------------------------------
