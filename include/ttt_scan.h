@@ -53,8 +53,15 @@ enum {
   TTT_KERNEL_SIMT = 1u << 5,    /* run the CUDA-core kernel even where the tensor-core kernel applies */
   TTT_GATE_CHANNEL = 1u << 6,   /* gate_logit holds one logit per feature (d per token), applied
                                    elementwise; else one per token */
-  TTT_KERNEL_SINGLE_CTA = 1u << 7 /* per-token mode: keep every head on one CTA even when the
-                                     heads are few enough to spread each over a cluster */
+  TTT_KERNEL_SINGLE_CTA = 1u << 7, /* per-token mode: keep every head on one CTA even when the
+                                      heads are few enough to spread each over a cluster */
+  TTT_GRAD_ABLATE = 1u << 8,      /* ablation gradient: the LayerNorm Jacobian applied to
+                                     -gamma*v, i.e. the prediction's contribution removed
+                                     ("Error Correction in Trained TTT Layers", Abstract);
+                                     per-token mode only; invalid with TTT_NO_LN */
+  TTT_GRAD_NORM_MATCH = 1u << 9   /* with TTT_GRAD_ABLATE: rescale each token's gradient to the
+                                     L2 norm of its full LN-Jacobian gradient (0 where the
+                                     ablated gradient is 0); invalid without TTT_GRAD_ABLATE */
 };
 
 /* Kernel identifiers returned by ttt_scan_kernel_choice(). */
@@ -92,7 +99,7 @@ enum {
  * Kernels: per-token mode runs a CUDA-core kernel for any b: at d = 64, when
  *   the B*H heads fit on the device as clusters of 4 CTAs (one per SM), each
  *   head's rows of W are split over such a cluster; otherwise (or with
- *   TTT_KERNEL_SINGLE_CTA) one CTA runs each head. Mini-batch mode runs the
+ *   TTT_KERNEL_SINGLE_CTA, or the ablation gradient) one CTA runs each head. Mini-batch mode runs the
  *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs, and
  *   otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which takes b <= 16.
  *   Other combinations return TTT_ERR_UNSUPPORTED.
@@ -139,7 +146,8 @@ int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b);
  *   update       [B] bytes, nonzero = UPDATE, 0 = SKIP (W left bit for bit); NULL = all UPDATE
  *   o            [B, H, d]      out: fp32, or bf16 with TTT_OUT_BF16
  * No output may overlap an input, and W may overlap nothing else.
- * mode: TTT_GRAD_LNJAC, TTT_NO_LN, TTT_IN_BF16, TTT_OUT_BF16, TTT_GATE_CHANNEL.
+ * mode: TTT_GRAD_LNJAC, TTT_NO_LN, TTT_IN_BF16, TTT_OUT_BF16, TTT_GATE_CHANNEL,
+ *   TTT_GRAD_ABLATE, TTT_GRAD_NORM_MATCH (as for the scan).
  *   TTT_MODE_MINIBATCH returns TTT_ERR_UNSUPPORTED (a one-token step has no
  *   chunk); TTT_KERNEL_SIMT and TTT_KERNEL_SINGLE_CTA are accepted and ignored.
  * Sizes: B, H >= 0, d in {16, 64}, eps >= 0 (finite). Returns TTT_OK or an error

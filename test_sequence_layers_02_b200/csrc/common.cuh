@@ -32,7 +32,17 @@ struct ScanParams {
   int lnjac;
   int no_ln;
   int minibatch;
+  int ablate;              // ablation gradient (prediction removed, Jacobian kept)
+  int norm_match;          // ... rescaled per token to the full gradient's norm
 };
+
+// Gradient variant of the CUDA-core chain: 0 simplified, 1 LN Jacobian, 2 no
+// LayerNorm, 3 ablation, 4 ablation with per-token norm matching.
+inline int grad_variant(const ScanParams& p) {
+  if (p.no_ln) return 2;
+  if (p.ablate) return p.norm_match ? 4 : 3;
+  return p.lnjac ? 1 : 0;
+}
 
 enum : int { kStatusOk = 0, kStatusTimeout = 1 };
 

@@ -6,7 +6,8 @@
 //
 // Per head, from ONE read of W:
 //   z = W k and W q (both from the same registers),
-//   LayerNorm + gradient G (simplified, LN-Jacobian or no LayerNorm),
+//   LayerNorm + gradient G (simplified, LN-Jacobian, no LayerNorm, or the
+//     ablation: the Jacobian applied to -gamma v, optionally norm-matched),
 //   eta = sigmoid(eta_logit) / d, or 0 when the batch row's update flag is 0,
 //   W' = W - eta G k^T, written back in place (not written at all when eta = 0,
 //        so a skipped head keeps its W bit for bit),
@@ -40,6 +41,7 @@ struct DecodeParams {
   int H;
   float eps;
   int lnjac, no_ln, gate_channel;
+  int ablate, norm_match;   // ablation gradient; per-token norm matching
 };
 
 template <int D>
@@ -88,7 +90,7 @@ __device__ __forceinline__ void reduce_scatter(float (&p)[N], int lane) {
 template <int D, typename InT, typename OutT>
 __global__ void __launch_bounds__(DecodeShape<D>::NT) decode_step_kernel(const DecodeParams p) {
   using S = DecodeShape<D>;
-  __shared__ float red[3][S::WPH][2];    // per-warp partials of the three LayerNorm rounds
+  __shared__ float red[5][S::WPH][2];    // per-warp partials of the LayerNorm rounds
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wih = warp % S::WPH;
   const long long bh = (long long)blockIdx.x * S::HPB + warp / S::WPH;
@@ -166,10 +168,22 @@ __global__ void __launch_bounds__(DecodeShape<D>::NT) decode_step_kernel(const D
     const float s = sqrtf(var + p.eps);
     const float xh = y / s;
     const float err = fmaf(gam, xh, bet) - vr;
-    if (p.lnjac) {
-      const float g = gam * err;
-      const float2 m = head_sum(g, g * xh, 2);
-      G = (g - m.x * inv_d - xh * (m.y * inv_d)) / s;
+    // back through the LayerNorm: J^T g = (g - mean g - xhat mean(g xhat)) / s
+    auto jacobian_t = [&](float g, int round) {
+      const float2 m = head_sum(g, g * xh, round);
+      return (g - m.x * inv_d - xh * (m.y * inv_d)) / s;
+    };
+    if (p.ablate) {
+      // the prediction removed, the Jacobian kept; optionally rescaled to the
+      // full gradient's norm
+      G = jacobian_t(-gam * vr, 2);
+      if (p.norm_match) {
+        const float Gf = jacobian_t(gam * err, 3);
+        const float2 n = head_sum(Gf * Gf, G * G, 4);
+        G *= n.y > 0.f ? sqrtf(n.x / n.y) : 0.f;
+      }
+    } else if (p.lnjac) {
+      G = jacobian_t(gam * err, 2);
     } else {
       G = err;
     }

@@ -130,7 +130,11 @@ __device__ __forceinline__ void butterfly(float (&v)[N]) {
 }
 
 // Gradient chain of one chunk (one warp). GM: 0 = simplified (G = err),
-// 1 = through the LayerNorm Jacobian, 2 = no LayerNorm (G = z - v).
+// 1 = through the LayerNorm Jacobian, 2 = no LayerNorm (G = z - v),
+// 3 = the ablation gradient (the Jacobian applied to -gamma * v, the
+// prediction removed; "Error Correction in Trained TTT Layers", Abstract),
+// 4 = the ablation rescaled per token to the norm of the GM 1 gradient.
+// Both Jacobian forms (1, 3, 4) give G a zero feature mean.
 // Reads Zpre (z before in-chunk corrections), A (eta_j k_m.k_j, j < m), V,
 // mu0 (mean of each Zpre row); writes G and, for GM 0, the mean of each G row.
 template <int D, typename InT, bool MINIB, int GM>
@@ -173,7 +177,59 @@ __device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
       float y[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) y[e] = (lane + 32 * e < D) ? zr[i][e] - mup[i] : 0.f;
-      if (GM == 1) {
+      if (GM == 3) {
+        // g = -gamma v: sum y^2, sum gamma v, sum gamma v y
+        float m[3] = {0.f, 0.f, 0.f};
+        float gv[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          gv[e] = gam[e] * v[e];
+          m[0] = fmaf(y[e], y[e], m[0]);
+          m[1] += gv[e];
+          m[2] = fmaf(gv[e], y[e], m[2]);
+        }
+        butterfly<3>(m);
+        const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+        const float a = m[1] * inv_d, bq = rs * rs * rs * m[2] * inv_d;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) G[e] = fmaf(bq, y[e], rs * (a - gv[e]));
+      } else if (GM == 4) {
+        // both forms from one butterfly: the GM 1 moments plus sum gamma v y
+        float m[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float w[EPL], g2[EPL], gv[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          g2[e] = gam[e] * gam[e];
+          w[e] = gam[e] * (bet[e] - v[e]);
+          gv[e] = gam[e] * v[e];
+          m[0] = fmaf(y[e], y[e], m[0]);
+          m[1] = fmaf(g2[e], y[e], m[1]);
+          m[2] = fmaf(g2[e] * y[e], y[e], m[2]);
+          m[3] = fmaf(w[e], y[e], m[3]);
+          m[4] = fmaf(gam[e], v[e], m[4]);
+          m[5] = fmaf(gv[e], y[e], m[5]);
+        }
+        butterfly<6>(m);
+        const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+        const float mg = (rs * m[1] + Sgb - m[4]) * inv_d;
+        const float mgx = rs * (rs * m[2] + m[3]) * inv_d;
+        const float rs2 = rs * rs;
+        const float a = m[4] * inv_d, bq = rs2 * rs * m[5] * inv_d;
+        float Gf[EPL], nrm[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          Gf[e] = rs2 * (g2[e] - mgx) * y[e] + rs * (w[e] - mg);
+          G[e] = fmaf(bq, y[e], rs * (a - gv[e]));
+          if (lane + 32 * e < D) {  // lanes past the features (d = 16) hold no feature
+            nrm[0] = fmaf(Gf[e], Gf[e], nrm[0]);
+            nrm[1] = fmaf(G[e], G[e], nrm[1]);
+          }
+        }
+        butterfly<2>(nrm);
+        const float scale = nrm[1] > 0.f ? sqrtf(nrm[0] / nrm[1]) : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) G[e] *= scale;
+      } else if (GM == 1) {
         // moments of y: sum y^2, sum g2 y, sum g2 y^2, sum w y, sum gamma v
         float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
         float w[EPL], g2[EPL];

@@ -29,7 +29,7 @@ int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
 
 template <int D, typename InT, typename OutT>
 int dispatch_simt_mode(const ttt::ScanParams& p, cudaStream_t s) {
-  const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
+  const int gm = ttt::grad_variant(p);
   if (p.minibatch) {
     if (gm == 0) return launch_simt<D, InT, OutT, true, 0>(p, s);
     if (gm == 1) return launch_simt<D, InT, OutT, true, 1>(p, s);
@@ -37,6 +37,8 @@ int dispatch_simt_mode(const ttt::ScanParams& p, cudaStream_t s) {
   }
   if (gm == 0) return launch_simt<D, InT, OutT, false, 0>(p, s);
   if (gm == 1) return launch_simt<D, InT, OutT, false, 1>(p, s);
+  if (gm == 3) return launch_simt<D, InT, OutT, false, 3>(p, s);
+  if (gm == 4) return launch_simt<D, InT, OutT, false, 4>(p, s);
   return launch_simt<D, InT, OutT, false, 2>(p, s);
 }
 

@@ -20,7 +20,15 @@ long long g_wait_limit = 1LL << 20;
 
 constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
                                  TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT |
-                                 TTT_GATE_CHANNEL | TTT_KERNEL_SINGLE_CTA;
+                                 TTT_GATE_CHANNEL | TTT_KERNEL_SINGLE_CTA | TTT_GRAD_ABLATE |
+                                 TTT_GRAD_NORM_MATCH;
+
+// Gradient-mode combinations that make no sense, whatever the kernel.
+bool bad_grad_mode(unsigned mode) {
+  if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_NO_LN)) return true;
+  if ((mode & TTT_GRAD_NORM_MATCH) && !(mode & TTT_GRAD_ABLATE)) return true;
+  return false;
+}
 
 bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
@@ -44,7 +52,7 @@ int choose_kernel(long long heads, int T, int d, unsigned mode, int b) {
   if (minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
       !(mode & TTT_KERNEL_SIMT) && T > 0)
     return TTT_KERNEL_ID_TENSOR_CORE;
-  if (!minibatch && d == 64 && !(mode & TTT_KERNEL_SINGLE_CTA) && T > 0) {
+  if (!minibatch && d == 64 && !(mode & (TTT_KERNEL_SINGLE_CTA | TTT_GRAD_ABLATE)) && T > 0) {
     const int gm = (mode & TTT_NO_LN) ? 2 : ((mode & TTT_GRAD_LNJAC) ? 1 : 0);
     if (heads <= ttt::cluster_capacity(mode, gm)) return TTT_KERNEL_ID_CUDA_CORE_CLUSTER;
   }
@@ -167,7 +175,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
                      int b, const unsigned char* mask, void* o, float* W_T, float* W_chunks,
                      void* cuda_stream) {
   // ---- argument checks (nothing is launched on failure) ----
-  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if ((mode & ~kKnownModes) || bad_grad_mode(mode)) return TTT_ERR_INVALID_ARG;
   if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
   const bool no_ln = mode & TTT_NO_LN;
   // a pointer may be null only where the tensor it names is empty
@@ -182,6 +190,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
   if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
+  if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
 
   const size_t heads = (size_t)B * H;
   const int n_mask_chunks = (T + b - 1) / b;
@@ -222,6 +231,8 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   p.lnjac = (mode & TTT_GRAD_LNJAC) ? 1 : 0;
   p.no_ln = no_ln ? 1 : 0;
   p.minibatch = (mode & TTT_MODE_MINIBATCH) ? 1 : 0;
+  p.ablate = (mode & TTT_GRAD_ABLATE) ? 1 : 0;
+  p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int which = choose_kernel((long long)heads, T, d, mode, b);
@@ -242,11 +253,12 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
 }
 
 int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b) {
-  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if ((mode & ~kKnownModes) || bad_grad_mode(mode)) return TTT_ERR_INVALID_ARG;
   if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
   if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
+  if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
   const int which = choose_kernel((long long)B * H, T, d, mode, b);
   if (which == TTT_KERNEL_ID_CUDA_CORE && (mode & TTT_MODE_MINIBATCH) && b > ttt::kC)
     return TTT_ERR_UNSUPPORTED;
@@ -257,7 +269,7 @@ int ttt_decode_step(const void* q, const void* k, const void* v, const void* eta
                     const void* gate_logit, float* W, const float* gamma, const float* beta,
                     int B, int H, int d, float eps, unsigned mode, const unsigned char* update,
                     void* o, void* cuda_stream) {
-  if (mode & ~kKnownModes) return TTT_ERR_INVALID_ARG;
+  if ((mode & ~kKnownModes) || bad_grad_mode(mode)) return TTT_ERR_INVALID_ARG;
   if (B < 0 || H < 0 || d <= 0) return TTT_ERR_INVALID_ARG;
   const bool no_ln = mode & TTT_NO_LN;
   const bool has_heads = (long long)B * H > 0;
@@ -301,6 +313,8 @@ int ttt_decode_step(const void* q, const void* k, const void* v, const void* eta
   p.lnjac = (mode & TTT_GRAD_LNJAC) ? 1 : 0;
   p.no_ln = no_ln ? 1 : 0;
   p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
+  p.ablate = (mode & TTT_GRAD_ABLATE) ? 1 : 0;
+  p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   return d == 64 ? dispatch_decode<64>(p, mode, stream) : dispatch_decode<16>(p, mode, stream);
 }

@@ -26,6 +26,8 @@ OUT_BF16 = 1 << 4
 KERNEL_SIMT = 1 << 5
 GATE_CHANNEL = 1 << 6
 KERNEL_SINGLE_CTA = 1 << 7
+GRAD_ABLATE = 1 << 8
+GRAD_NORM_MATCH = 1 << 9
 
 # Kernel identifiers of ttt_scan_kernel_choice.
 KERNEL_NONE, KERNEL_CUDA_CORE, KERNEL_CUDA_CORE_CLUSTER, KERNEL_TENSOR_CORE = 0, 1, 2, 3
@@ -99,7 +101,8 @@ def _ptr(t: Optional[torch.Tensor]):
 def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
          minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
          b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
-         force_simt: bool = False, single_cta: bool = False, want_chunks: bool = False,
+         force_simt: bool = False, single_cta: bool = False, ablate: bool = False,
+         norm_match: bool = False, want_chunks: bool = False,
          o: Optional[torch.Tensor] = None, W_T: Optional[torch.Tensor] = None,
          stream: Optional[torch.cuda.Stream] = None):
     """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
@@ -109,7 +112,9 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
     uint8 or None. ``out_dtype`` defaults to the input dtype. ``force_simt``
     keeps mini-batch mode on the CUDA-core kernel; ``single_cta`` keeps
-    per-token mode on one CTA per head (see ``kernel_choice``).
+    per-token mode on one CTA per head (see ``kernel_choice``). ``ablate``
+    selects the ablation gradient (the LayerNorm Jacobian applied to
+    -gamma * v), ``norm_match`` rescales it per token to the full gradient's norm.
 
     CUDA tensors run on ``stream`` (default: the current stream) and return
     without synchronising. CPU tensors take the end-to-end path: inputs are
@@ -152,7 +157,8 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
             (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0) |
-            (KERNEL_SINGLE_CTA if single_cta else 0))
+            (KERNEL_SINGLE_CTA if single_cta else 0) | (GRAD_ABLATE if ablate else 0) |
+            (GRAD_NORM_MATCH if norm_match else 0))
     if o_dev is None:
         o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
     if wt_dev is None:
@@ -186,11 +192,12 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
 def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
                   lnjac: bool = False, no_ln: bool = False, in_bf16: bool = False,
                   out_bf16: bool = False, b: int = 16, force_simt: bool = False,
-                  single_cta: bool = False) -> int:
+                  single_cta: bool = False, ablate: bool = False, norm_match: bool = False) -> int:
     """The KERNEL_* identifier ``scan`` would run for these sizes (launches nothing)."""
     mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_bf16 else 0) | (OUT_BF16 if out_bf16 else 0) |
-            (KERNEL_SIMT if force_simt else 0) | (KERNEL_SINGLE_CTA if single_cta else 0))
+            (KERNEL_SIMT if force_simt else 0) | (KERNEL_SINGLE_CTA if single_cta else 0) |
+            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0))
     rc = lib().ttt_scan_kernel_choice(B, H, T, d, mode, b)
     if rc < 0:
         raise TTTScanError(rc, "ttt_scan_kernel_choice")
@@ -198,7 +205,8 @@ def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
 
 
 def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 1e-6,
-                lnjac: bool = False, no_ln: bool = False, update=None,
+                lnjac: bool = False, no_ln: bool = False, ablate: bool = False,
+                norm_match: bool = False, update=None,
                 out_dtype: Optional[torch.dtype] = None, o: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None):
     """One streaming step ``o = decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta)``.
@@ -248,7 +256,8 @@ def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 
     out_dtype = out_dtype or in_dtype
     mode = ((GRAD_LNJAC if lnjac else 0) | (NO_LN if no_ln else 0) |
             (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
-            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (GATE_CHANNEL if channel else 0))
+            (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (GATE_CHANNEL if channel else 0) |
+            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0))
     if o_dev is None:
         o_dev = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
     s = stream if stream is not None else torch.cuda.current_stream(q.device)

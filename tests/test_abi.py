@@ -79,7 +79,9 @@ INVALID, UNSUPPORTED = -1, -2
     dict(q=addr(0, 4)), dict(o=addr(8, 8)), dict(mask=addr(10, 1)), dict(W_chunks=addr(11, 2)),
     dict(B=-1), dict(H=-1), dict(T=-1), dict(b=0), dict(b=-3), dict(d=0), dict(d=-64),
     dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")),
-    dict(mode=1 << 8), dict(mode=1 << 31),
+    dict(mode=1 << 10), dict(mode=1 << 31),
+    dict(mode=(1 << 8) | 4),              # ablation without a LayerNorm
+    dict(mode=1 << 9),                    # norm matching without the ablation
     dict(o=addr(0)),                      # output over an input
     dict(o=addr(2, 1 << 12)),             # output inside v
     dict(W_T=addr(5, 256)),               # W_T partially overlapping W0
@@ -92,7 +94,7 @@ def test_invalid_arguments_rejected(lib, over):
 
 @pytest.mark.parametrize("over", [dict(d=32), dict(d=128), dict(d=17),
                                   dict(mode=1, b=17), dict(mode=1 | 32, b=32),
-                                  dict(mode=1 << 6)])
+                                  dict(mode=1 << 6), dict(mode=1 | (1 << 8))])
 def test_unsupported_shapes(lib, over):
     assert call(lib, **over) == UNSUPPORTED
 
@@ -123,7 +125,7 @@ def dcall(lib, **over):
     dict(gamma=None), dict(beta=None),
     dict(q=addr(0, 4)), dict(W=addr(5, 8)), dict(update=addr(10, 1)), dict(o=addr(8, 2)),
     dict(B=-1), dict(H=-1), dict(d=0), dict(eps=-1.0), dict(eps=float("nan")),
-    dict(mode=1 << 8),
+    dict(mode=1 << 10), dict(mode=(1 << 8) | 4), dict(mode=1 << 9),
     dict(o=addr(1)),                      # output over an input
     dict(W=addr(8)),                      # state over the output
     dict(W=addr(2, 64)),                  # state inside v
@@ -152,7 +154,11 @@ def test_kernel_choice_without_launching(lib):
     assert f(2, 3, 40, 16, 0, 16) == 1                               # d = 16: one CTA per head
     assert f(2, 3, 40, 64, 1 << 7, 16) == 1                          # single CTA asked for
     assert f(0, 3, 40, 64, 0, 16) == 0                               # nothing to launch
-    assert f(2, 3, 40, 64, 1 << 8, 16) == INVALID
+    assert f(2, 3, 40, 64, 1 << 10, 16) == INVALID
+    assert f(2, 3, 40, 64, 1 << 9, 16) == INVALID                     # norm match alone
+    assert f(2, 3, 40, 64, (1 << 8) | 4, 16) == INVALID               # ablation without LN
+    assert f(2, 3, 40, 64, 1 | (1 << 8), 16) == UNSUPPORTED           # mini-batch ablation
+    assert f(2, 3, 40, 64, 1 << 8, 16) == 1                           # ablation: one CTA per head
     assert f(2, 3, 40, 64, 0, 0) == INVALID
     assert f(2, 3, 40, 32, 0, 16) == UNSUPPORTED
     assert f(2, 3, 40, 64, MINIB, 17) == UNSUPPORTED

@@ -93,6 +93,25 @@ def test_decode_step_matches_oracle(d, grad, dtypes, gate):
     assert_fp32_close(np64(W), rW, "W")
 
 
+@pytest.mark.parametrize("norm_match", [False, True], ids=["ablate", "ablate_nm"])
+@pytest.mark.parametrize("d", [16, 64])
+def test_decode_ablation_gradient(d, norm_match):
+    B, H = 3, 5
+    inp = step_inputs(B, H, d, seed=540 + d, in_bf16=False, update_p=0.7)
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    t = to_torch(inp, "cuda", False)
+    W = t["W0"].clone()
+    o = ttt_scan.decode_step(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], W,
+                             t["gamma"], t["beta"], eps=1e-6, ablate=True, norm_match=norm_match,
+                             update=torch.from_numpy(inp["update"]).cuda())
+    torch.cuda.synchronize()
+    assert ttt_scan.check_device_status() == ttt_scan.TTT_OK
+    ro, rW = oracle_step(inp, mode=(1 << 8) | ((1 << 9) if norm_match else 0), eps=1e-6)
+    assert_fp32_close(np64(o), ro, "o")
+    assert_fp32_close(np64(W), rW, "W")
+
+
 def test_decode_skip_rows_keep_W_bit_for_bit():
     B, H, d = 6, 4, 64
     inp = step_inputs(B, H, d, seed=510, in_bf16=True, update_p=0.5)

@@ -274,3 +274,59 @@ def test_cluster_wait_timeout_reports_and_recovers():
     ro, rW = oracle_scan(inp, eps=1e-6, mode=LNJAC, b=16)
     assert_fp32_close(o.cpu().numpy(), ro, "o")
     assert_fp32_close(W_T.cpu().numpy(), rW, "W_T")
+
+
+# ---------------------------------------------------------------------------
+# Ablation gradient ("Error Correction in Trained TTT Layers", Abstract): the
+# prediction's contribution removed, the LayerNorm Jacobian kept, optionally
+# rescaled per token to the full gradient's norm. Per-token mode.
+# ---------------------------------------------------------------------------
+
+ABLATE, NORM_MATCH = 1 << 8, 1 << 9
+
+
+@pytest.mark.parametrize("norm_match", [False, True], ids=["ablate", "ablate_nm"])
+@pytest.mark.parametrize("case", [(2, 3, 53, 16, 16, False), (2, 3, 77, 64, 16, False),
+                                  (2, 2, 70, 64, 24, False), (2, 3, 77, 64, 16, True)],
+                         ids=lambda c: f"B{c[0]}H{c[1]}T{c[2]}d{c[3]}b{c[4]}{'i16' if c[5] else ''}")
+@pytest.mark.parametrize("with_mask", [False, True])
+def test_ablation_gradient_small_cases(case, norm_match, with_mask):
+    from test_sequence_layers_02_b200 import ttt_scan
+    B, H, T, d, b, in_bf16 = case
+    assert ttt_scan.kernel_choice(B, H, T, d, ablate=True, norm_match=norm_match,
+                                  in_bf16=in_bf16) == ttt_scan.KERNEL_CUDA_CORE
+    inp = make_inputs(B, H, T, d, seed=600 + T + d + b, random_affine=True, in_bf16=in_bf16,
+                      mask_p=0.5 if with_mask else None, b=b)
+    mode = ABLATE | (NORM_MATCH if norm_match else 0)
+    o, W_T, Wc = gpu_scan(inp, in_bf16=in_bf16, eps=1e-6, b=b, ablate=True,
+                          norm_match=norm_match, want_chunks=True)
+    ro, rW, rWc = oracle_scan(inp, eps=1e-6, mode=mode, b=b, want_chunks=True)
+    assert_fp32_close(o, ro, "o")
+    assert_fp32_close(W_T, rW, "W_T")
+    assert_fp32_close(Wc, rWc, "W_chunks")
+
+
+@pytest.mark.parametrize("norm_match", [False, True], ids=["ablate", "ablate_nm"])
+def test_ablation_gradient_headline_shape(norm_match):
+    w = WORKLOADS["2j"]
+    inp = make_workload(w)
+    mode = ABLATE | (NORM_MATCH if norm_match else 0)
+    o, W_T = gpu_scan(inp, in_bf16=False, eps=w.eps, b=w.b, ablate=True, norm_match=norm_match)
+    ro, rW = oracle_scan(inp, eps=w.eps, mode=mode, b=w.b)
+    assert_fp32_close(o, ro, "o")
+    assert_fp32_close(W_T, rW, "W_T")
+
+
+def test_ablation_rejected_where_not_defined():
+    import torch
+    from test_sequence_layers_02_b200 import ttt_scan
+    inp = make_inputs(1, 2, 32, 64, seed=14, random_affine=True)
+    from tests.helpers import to_torch
+    t = to_torch(inp, "cuda", False)
+    args = (t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"], t["beta"])
+    with pytest.raises(ttt_scan.TTTScanError, match="INVALID"):
+        ttt_scan.scan(*args, ablate=True, no_ln=True)
+    with pytest.raises(ttt_scan.TTTScanError, match="INVALID"):
+        ttt_scan.scan(*args, norm_match=True)
+    with pytest.raises(ttt_scan.TTTScanError, match="UNSUPPORTED"):
+        ttt_scan.scan(*args, ablate=True, minibatch=True)
