@@ -83,31 +83,6 @@ struct ClusterLayout {
   static_assert(KW == 8, "a W thread holds two 4-element units of its row");
 };
 
-// Four consecutive elements of a shared-memory tile row (16 bytes of fp32 or
-// 8 bytes of bf16), widened to two fp32 pairs.
-template <typename InT>
-struct Unit;
-template <>
-struct Unit<float> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    x[0] = make_float2(a.x, a.y);
-    x[1] = make_float2(a.z, a.w);
-  }
-};
-template <>
-struct Unit<__nv_bfloat16> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
-    const uint2 a = *reinterpret_cast<const uint2*>(p);
-    x[0] = make_float2(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u));
-    x[1] = make_float2(__uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u));
-  }
-};
-
-__device__ __forceinline__ float2 dup2(float x) { return make_float2(x, x); }
-
 // Warp-wide sums of five values; the adds run as pairs.
 __device__ __forceinline__ void butterfly5(float (&m)[5]) {
 #pragma unroll
@@ -172,28 +147,6 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_dst, float a, float 
           "r"(remote_dst),
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
       : "memory");
-}
-
-// Reduce-scatter of V partial sums over the G lanes of one row group (lane
-// bits 0 .. log2 G - 1): each step exchanges half of the values still held
-// (S of them) across lane bit B. Afterwards lane g holds the full sums of
-// values g (V/G) .. g (V/G) + V/G - 1 in a[0 .. V/G).
-template <int V, int S, int B>
-__device__ __forceinline__ void reduce_scatter_step(float (&a)[V], int g) {
-  if constexpr (B >= 1) {
-    const bool up = g & B;
-#pragma unroll
-    for (int j = 0; j < S; ++j) {
-      const float send = up ? a[j] : a[j + S];
-      const float keep = up ? a[j + S] : a[j];
-      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, B);
-    }
-    reduce_scatter_step<V, S / 2, B / 2>(a, g);
-  }
-}
-template <int V, int G>
-__device__ __forceinline__ void reduce_scatter_lanes(float (&a)[V], int g) {
-  reduce_scatter_step<V, V / 2, G / 2>(a, g);
 }
 
 template <typename InT, typename OutT, int GM, int CS>

@@ -35,17 +35,24 @@ namespace ttt {
 
 constexpr int kC = 16;  // largest chunk of the CUDA-core kernel
 
-// IH = 2 splits W's columns in quarters instead of halves (8 bulk warps at
-// d = 64), so every SM sub-partition runs two bulk warps; used when heads are
-// few.
+// IH = 2 doubles the bulk warps (8 at d = 64), so every SM sub-partition runs
+// two of them; used when heads are few.
+//
+// W lives in the bulk threads' registers as RB x CBW blocks: thread
+// (row group rg, column group cg) holds rows RB rg .. + RB - 1, columns
+// CBW cg .. + CBW - 1. The CG = D / CBW threads of a row group are consecutive
+// lanes, so a product's partial sums over column groups finish with a lane
+// reduce-scatter, and every input-row segment a thread loads feeds RB rows.
 template <int D, typename InT, int IH = 1>
 struct PipeLayout {
   static constexpr int NBT = 2 * D * IH;     // bulk threads
   static constexpr int NT = NBT + 32;        // + the chain warp
   static constexpr int KH = D / 2;           // Gram column half
-  static constexpr int NKQ = 2 * IH;         // column groups of W
-  static constexpr int KW = D / NKQ;         // columns of W per bulk thread
   static constexpr int NG = NBT / 32;        // bulk warps
+  static constexpr int CBW = D >= 64 ? 8 : 4;          // columns of a W block
+  static constexpr int CG = D / CBW;                   // column groups (lanes per row group)
+  static constexpr int RB = D * D / (NBT * CBW);       // rows of a W block
+  static_assert(RB * CBW * NBT == D * D && RB >= 2 && 32 % CG == 0, "W block geometry");
   static constexpr int ELT = (int)sizeof(InT);
   static constexpr int ROWB = D * ELT + 16;  // padded row of an input tile (bytes)
   static constexpr int TILE = kC * ROWB;
@@ -56,8 +63,7 @@ struct PipeLayout {
   static constexpr int oZ = oV + 2 * TILE;             // P / Zpre   [2][kC][D] f32
   static constexpr int oG = oZ + 2 * kC * D * 4;       // G          [2][kC][D]
   static constexpr int oQ0 = oG + 2 * kC * D * 4;      // Q0         [2][kC][D]
-  static constexpr int oPP = oQ0 + 2 * kC * D * 4;     // partial products [NKQ][2kC][D]
-  static constexpr int oA = oPP + NKQ * 2 * kC * D * 4;  // in-chunk K Gram [2][kC][kC]
+  static constexpr int oA = oQ0 + 2 * kC * D * 4;      // in-chunk K Gram [2][kC][kC]
   static constexpr int oS = oA + 2 * kC * kC * 4;      // Q K Gram   [2][kC][kC]
   static constexpr int oX = oS + 2 * kC * kC * 4;      // cross Gram [kC][kC]
   static constexpr int oEta = oX + kC * kC * 4;        // eta        [4][kC]
@@ -119,6 +125,152 @@ __device__ __forceinline__ void tile_load(unsigned char* tile, const InT* src, i
     cp_async16(tile + row * L::ROWB + piece * 16, g, ok ? 16 : 0);
   }
 }
+
+// Four consecutive elements of a shared-memory tile row (16 bytes of fp32 or
+// 8 bytes of bf16), widened to two fp32 pairs.
+template <typename InT>
+struct Unit;
+template <>
+struct Unit<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = make_float2(a.x, a.y);
+    x[1] = make_float2(a.z, a.w);
+  }
+};
+template <>
+struct Unit<__nv_bfloat16> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void ld(const unsigned char* p, float2 (&x)[2]) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    x[0] = make_float2(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u));
+    x[1] = make_float2(__uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u));
+  }
+};
+
+__device__ __forceinline__ float2 dup2(float x) { return make_float2(x, x); }
+
+// Reduce-scatter of V partial sums over the G lanes of one lane group (lane
+// bits 0 .. log2 G - 1): each step exchanges half of the values still held
+// (S of them) across lane bit B. Afterwards lane g holds the full sums of
+// values g (V/G) .. g (V/G) + V/G - 1 in a[0 .. V/G).
+template <int V, int S, int B>
+__device__ __forceinline__ void reduce_scatter_step(float (&a)[V], int g) {
+  if constexpr (B >= 1) {
+    const bool up = g & B;
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      const float send = up ? a[j] : a[j + S];
+      const float keep = up ? a[j + S] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, B);
+    }
+    reduce_scatter_step<V, S / 2, B / 2>(a, g);
+  }
+}
+template <int V, int G>
+__device__ __forceinline__ void reduce_scatter_lanes(float (&a)[V], int g) {
+  reduce_scatter_step<V, V / 2, G / 2>(a, g);
+}
+
+// A bulk thread's block of W (see PipeLayout) and the work done on it.
+template <int D, typename InT, int IH>
+struct WBlock {
+  using L = PipeLayout<D, InT, IH>;
+  static constexpr int RB = L::RB, CBW = L::CBW, CG = L::CG, NU = CBW / 4;
+  float2 w[RB][CBW / 2];  // w[rb][2 u + t]: columns col(u) + 2 t, + 1 of row row0 + rb
+  int row0, cg, swap;
+
+  __device__ __forceinline__ void init(int tid) {
+    cg = tid % CG;
+    row0 = (tid / CG) * RB;
+    // fp32 tiles with two units per block: the upper half of the column groups
+    // takes its units in swapped order so the broadcast addresses of one load
+    // fall in disjoint banks
+    swap = (L::ELT == 4 && NU == 2 && cg >= CG / 2) ? 1 : 0;
+  }
+  __device__ __forceinline__ int col(int u) const { return cg * CBW + 4 * (u ^ swap); }
+
+  __device__ __forceinline__ void load(const float* Wh) {
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        const float4 x = *reinterpret_cast<const float4*>(Wh + (size_t)(row0 + rb) * D + col(u));
+        w[rb][2 * u] = make_float2(x.x, x.y);
+        w[rb][2 * u + 1] = make_float2(x.z, x.w);
+      }
+  }
+  __device__ __forceinline__ void store(float* Wh) const {
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+      for (int u = 0; u < NU; ++u)
+        *reinterpret_cast<float4*>(Wh + (size_t)(row0 + rb) * D + col(u)) =
+            make_float4(w[rb][2 * u].x, w[rb][2 * u].y, w[rb][2 * u + 1].x, w[rb][2 * u + 1].y);
+  }
+  // W -= sum_{j < n} eta_j G_j k_j^T over the rows of tile Kt (rows of G past
+  // n may hold anything, so their scale is selected away, not multiplied).
+  __device__ __forceinline__ void rank_update(const unsigned char* Kt, const float* Gp,
+                                              const float* et, int n) {
+#pragma unroll
+    for (int j = 0; j < kC; ++j) {
+      float g[RB];
+      if constexpr (RB == 4) {
+        const float4 g4 = *reinterpret_cast<const float4*>(Gp + j * D + row0);
+        g[0] = g4.x; g[1] = g4.y; g[2] = g4.z; g[3] = g4.w;
+      } else {
+        const float2 g2 = *reinterpret_cast<const float2*>(Gp + j * D + row0);
+        g[0] = g2.x; g[1] = g2.y;
+      }
+      const float e = j < n ? -et[j] : 0.f;
+      float2 x[NU][2];
+#pragma unroll
+      for (int u = 0; u < NU; ++u) Unit<InT>::ld(Kt + j * L::ROWB + col(u) * L::ELT, x[u]);
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb) {
+        const float2 s = dup2(j < n ? e * g[rb] : 0.f);
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          w[rb][2 * u] = __ffma2_rn(s, x[u][0], w[rb][2 * u]);
+          w[rb][2 * u + 1] = __ffma2_rn(s, x[u][1], w[rb][2 * u + 1]);
+        }
+      }
+    }
+  }
+  // out[t][row] = (W x_t)_row for the kC rows x_t of tile R, this block's rows,
+  // in batches of 8 tokens finished by a reduce-scatter over the CG lanes.
+  __device__ __forceinline__ void products(const unsigned char* R, float* out) const {
+    constexpr int V = RB * 8, PER = V / CG;
+#pragma unroll
+    for (int t0 = 0; t0 < kC; t0 += 8) {
+      float2 x[8][NU][2];
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+#pragma unroll
+        for (int u = 0; u < NU; ++u) Unit<InT>::ld(R + (t0 + b) * L::ROWB + col(u) * L::ELT, x[b][u]);
+      float acc[V];
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          float2 a = __fmul2_rn(w[rb][0], x[b][0][0]);
+          a = __ffma2_rn(w[rb][1], x[b][0][1], a);
+#pragma unroll
+          for (int u = 1; u < NU; ++u) {
+            a = __ffma2_rn(w[rb][2 * u], x[b][u][0], a);
+            a = __ffma2_rn(w[rb][2 * u + 1], x[b][u][1], a);
+          }
+          acc[rb * 8 + b] = a.x + a.y;
+        }
+      reduce_scatter_lanes<V, CG>(acc, cg);
+      // lane cg now holds values cg * PER .. + PER - 1: one row, PER tokens
+      const int i0 = cg * PER, rb = i0 / 8, tb = i0 % 8;
+#pragma unroll
+      for (int u = 0; u < PER; ++u) out[(t0 + tb + u) * D + row0 + rb] = acc[u];
+    }
+  }
+};
 
 template <int N>
 __device__ __forceinline__ void butterfly(float (&v)[N]) {
@@ -284,37 +436,6 @@ __device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
   if (GM != 0 && lane < kC) mGout[lane] = 0.f;
 }
 
-// Partial products of a bulk thread: acc[i] = sum over its column group of
-// W[r][k] * rows[i][k], for up to two sets of 16 rows.
-template <int D, typename InT, int IH>
-__device__ __forceinline__ void bulk_products(const float (&Wr)[PipeLayout<D, InT, IH>::KW],
-                                              const unsigned char* R0, const unsigned char* R1,
-                                              float* PP, int r, int kq) {
-  using L = PipeLayout<D, InT, IH>;
-  constexpr int KH = L::KW;
-  const int koff = kq * KH * L::ELT;
-  float* out = PP + kq * (2 * kC * D);
-#pragma unroll 1
-  for (int i0 = 0; i0 < 2 * kC; i0 += 4) {
-    const unsigned char* R = (i0 < kC) ? R0 : R1;
-    if (R == nullptr) continue;
-    const unsigned char* row = R + (i0 & (kC - 1)) * L::ROWB + koff;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < KH; k += 8) {
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        float x[8];
-        lds8(row + u4 * L::ROWB + k * L::ELT, x, InT());
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u4] = fmaf(Wr[k + u], x[u], acc[u4]);
-      }
-    }
-#pragma unroll
-    for (int u4 = 0; u4 < 4; ++u4) out[(i0 + u4) * D + r] = acc[u4];
-  }
-}
-
 // Dot products of left rows with one right row per lane pair (16 rows x 2
 // column halves); returns eta-weighted entries through `emit(i, j, dot)`.
 template <int D, typename InT, int IH, typename Emit>
@@ -389,8 +510,6 @@ template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
 __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanParams p) {
   using L = PipeLayout<D, InT, IH>;
   constexpr int NBT = L::NBT;
-  constexpr int KW = L::KW;
-  constexpr int NKQ = L::NKQ;
   constexpr int EPL = (D + 31) / 32;
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char* sK = smem + L::oK;
@@ -399,7 +518,6 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
   float* sZ = reinterpret_cast<float*>(smem + L::oZ);
   float* sG = reinterpret_cast<float*>(smem + L::oG);
   float* sQ0 = reinterpret_cast<float*>(smem + L::oQ0);
-  float* sPP = reinterpret_cast<float*>(smem + L::oPP);
   float* sA = reinterpret_cast<float*>(smem + L::oA);
   float* sS = reinterpret_cast<float*>(smem + L::oS);
   float* sX = reinterpret_cast<float*>(smem + L::oX);
@@ -465,19 +583,15 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
   };
 
   // ---------------- prologue ----------------
-  float Wr[KW];
+  WBlock<D, InT, IH> wb;
+  wb.init(tid);
+  // (token, row) work of the outputs and the look-ahead correction
   const int r = tid % D;
-  const int part = tid / D;  // bulk threads: 0 .. NKQ - 1
-  const int kq = part;       // column group of W held
+  const int part = tid / D;  // 0 .. 2 IH - 1
   float gam[EPL], bet[EPL];
   float Sgb = 0.f, Sb = 0.f;
   if (!chain) {
-    const float* W0 = p.W0 + ((size_t)bh * D + r) * D + kq * KW;  // may alias W_T
-#pragma unroll
-    for (int k = 0; k < KW; k += 4) {
-      const float4 w4 = *reinterpret_cast<const float4*>(W0 + k);
-      Wr[k] = w4.x; Wr[k + 1] = w4.y; Wr[k + 2] = w4.z; Wr[k + 3] = w4.w;
-    }
+    wb.load(p.W0 + (size_t)bh * D * D);  // may alias W_T
     if (nc > 0) {
       tile_load<D>(tileK(0), gk, 0, chunk_len(0), tid, NBT);
       tile_load<D>(tileQ(0), gq, 0, chunk_len(0), tid, NBT);
@@ -506,19 +620,12 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
   __syncthreads();
   if (!chain && nc > 0) {
     // P_0 = K_0 W0^T (no correction), its row means, and A_0
-    bulk_products<D, InT, IH>(Wr, nullptr, tileK(0), sPP, r, kq);
+    wb.products(tileK(0), sZ);
     if (!MINIB) {
       const int n0 = chunk_len(0);
       bulk_gram<D, InT, IH>(tileK(0), tileK(0), nullptr, kC, tid, [&](int m, int j, float dot) {
         sA[m * kC + j] = (j < m && m < n0) ? sEta[j] * dot : 0.f;
       });
-    }
-    bulk_barrier(NBT);
-    for (int i = part; i < kC; i += NKQ) {
-      float acc = 0.f;
-#pragma unroll
-      for (int g = 0; g < NKQ; ++g) acc += sPP[g * 2 * kC * D + (kC + i) * D + r];
-      sZ[i * D + r] = acc;
     }
     bulk_barrier(NBT);
     row_means<D>(sZ, sMu, tid, NBT);
@@ -554,29 +661,10 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
       if (c + 2 < nc) pre = issue_scalars(c + 2);
 
       // W_{s,c} = W_{s,c-1} - sum_j eta_j G_j k_j^T over chunk c-1
-      if (c >= 1 && sFlag[(c - 1) & 3]) {
-        const unsigned char* Kt = tileK(c - 1);
-        const float* Gp = sG + ((c - 1) & 1) * kC * D;
-        const float* et = sEta + ((c - 1) & 3) * kC;
-        const int np = chunk_len(c - 1);
-        for (int j = 0; j < np; ++j) {
-          const float ge = et[j] * Gp[j * D + r];
-          const unsigned char* row = Kt + j * L::ROWB + kq * KW * L::ELT;
-#pragma unroll
-          for (int k = 0; k < KW; k += 8) {
-            float x[8];
-            lds8(row + k * L::ELT, x, InT());
-#pragma unroll
-            for (int u = 0; u < 8; ++u) Wr[k + u] = fmaf(-ge, x[u], Wr[k + u]);
-          }
-        }
-      }
-      if (Wc && ((c * C) % p.b) == 0) {
-        float* dst = Wc + ((size_t)((c * C) / p.b) * D + r) * D + kq * KW;
-#pragma unroll
-        for (int k = 0; k < KW; k += 4)
-          *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
-      }
+      if (c >= 1 && sFlag[(c - 1) & 3])
+        wb.rank_update(tileK(c - 1), sG + ((c - 1) & 1) * kC * D, sEta + ((c - 1) & 3) * kC,
+                       chunk_len(c - 1));
+      if (Wc && ((c * C) % p.b) == 0) wb.store(Wc + (size_t)((c * C) / p.b) * D * D);
 
       // outputs of chunk c-1
       if (c >= 1) {
@@ -626,20 +714,8 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
       }
 
       // Q0_c = Q_c W_{s,c}^T and P_{c+1} = K_{c+1} W_{s,c}^T
-      bulk_products<D, InT, IH>(Wr, tileQ(c), has_next ? tileK(c + 1) : nullptr, sPP, r, kq);
-      bulk_barrier(NBT);
-      {
-        float* Q0c = sQ0 + (c & 1) * kC * D;
-        float* Pn = sZ + ((c + 1) & 1) * kC * D;
-        for (int i = part; i < 2 * kC; i += NKQ) {
-          if (i >= kC && !has_next) break;
-          float val = 0.f;
-#pragma unroll
-          for (int g = 0; g < NKQ; ++g) val += sPP[g * 2 * kC * D + i * D + r];
-          if (i < kC) Q0c[i * D + r] = val;
-          else Pn[(i - kC) * D + r] = val;
-        }
-      }
+      wb.products(tileQ(c), sQ0 + (c & 1) * kC * D);
+      if (has_next) wb.products(tileK(c + 1), sZ + ((c + 1) & 1) * kC * D);
       if (has_next) {
         bulk_barrier(NBT);
         row_means<D>(sZ + ((c + 1) & 1) * kC * D, sMu + ((c + 1) & 1) * kC, tid, NBT);
@@ -679,22 +755,7 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
     if (nc > 0) {
       const int c = nc - 1;
       const int np = chunk_len(c);
-      if (sFlag[c & 3]) {
-        const unsigned char* Kt = tileK(c);
-        const float* Gp = sG + (c & 1) * kC * D;
-        const float* et = sEta + (c & 3) * kC;
-        for (int j = 0; j < np; ++j) {
-          const float ge = et[j] * Gp[j * D + r];
-          const unsigned char* row = Kt + j * L::ROWB + kq * KW * L::ELT;
-#pragma unroll
-          for (int k = 0; k < KW; k += 8) {
-            float x[8];
-            lds8(row + k * L::ELT, x, InT());
-#pragma unroll
-            for (int u = 0; u < 8; ++u) Wr[k + u] = fmaf(-ge, x[u], Wr[k + u]);
-          }
-        }
-      }
+      if (sFlag[c & 3]) wb.rank_update(tileK(c), sG + (c & 1) * kC * D, sEta + (c & 3) * kC, np);
       const float* Q0p = sQ0 + (c & 1) * kC * D;
       const float* Sp = sS + (c & 1) * kC * kC;
       const float* Gp = sG + (c & 1) * kC * D;
@@ -708,16 +769,8 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
         dst[(size_t)i * D + r] = from_f32<OutT>(gt[i] * acc);
       }
     }
-    if (Wc) {
-      float* dst = Wc + ((size_t)p.n_mask_chunks * D + r) * D + kq * KW;
-#pragma unroll
-      for (int k = 0; k < KW; k += 4)
-        *reinterpret_cast<float4*>(dst + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
-    }
-    float* WT = p.W_T + ((size_t)bh * D + r) * D + kq * KW;
-#pragma unroll
-    for (int k = 0; k < KW; k += 4)
-      *reinterpret_cast<float4*>(WT + k) = make_float4(Wr[k], Wr[k + 1], Wr[k + 2], Wr[k + 3]);
+    if (Wc) wb.store(Wc + (size_t)p.n_mask_chunks * D * D);
+    wb.store(p.W_T + (size_t)bh * D * D);
   }
 }
 

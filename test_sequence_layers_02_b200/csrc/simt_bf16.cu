@@ -22,8 +22,9 @@ int launch_simt_ih(const ttt::ScanParams& p, cudaStream_t stream) {
 // that several CTAs share an SM.
 template <int D, typename InT, typename OutT, bool MINIB, int GM>
 int launch_simt(const ttt::ScanParams& p, cudaStream_t stream) {
-  if (D == 64 && (long long)p.B * p.H <= 148)
-    return launch_simt_ih<D, InT, OutT, MINIB, GM, 2>(p, stream);
+  if constexpr (D == 64) {
+    if ((long long)p.B * p.H <= 148) return launch_simt_ih<D, InT, OutT, MINIB, GM, 2>(p, stream);
+  }
   return launch_simt_ih<D, InT, OutT, MINIB, GM, 1>(p, stream);
 }
 
