@@ -83,9 +83,8 @@ enum {
  * elements, e.g. q..o when T == 0, everything when B*H == 0):
  *   q, k, v      [B, H, T, d]   fp32, or bf16 with TTT_IN_BF16
  *   eta_logit    [B, H, T]      same dtype as q
- *   gate_logit   [B, H, T]      same dtype as q; NULL = no output gate (factor 1).
- *                TTT_GATE_CHANNEL (a per-feature gate) is implemented by
- *                ttt_decode_step only; here it returns TTT_ERR_UNSUPPORTED
+ *   gate_logit   [B, H, T], or [B, H, T, d] with TTT_GATE_CHANNEL (o[r] = sigmoid(gate[r]) *
+ *                (W q)[r]); same dtype as q; NULL = no output gate (factor 1)
  *   W0           [B, H, d, d]   fp32 initial fast weights, z = W k
  *   gamma, beta  [H, d]         fp32 inner-LayerNorm affine; may be NULL with TTT_NO_LN
  *   mask         [B, ceil(T/b)] bytes, nonzero = UPDATE, 0 = SKIP; NULL = all UPDATE
@@ -100,8 +99,9 @@ enum {
  *   the B*H heads fit on the device as clusters of 4 CTAs (one per SM), each
  *   head's rows of W are split over such a cluster; otherwise (or with
  *   TTT_KERNEL_SINGLE_CTA, or the ablation gradient) one CTA runs each head. Mini-batch mode runs the
- *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs, and
- *   otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which takes b <= 16.
+ *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs and a per-token
+ *   gate, and otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which
+ *   takes b <= 16.
  *   Other combinations return TTT_ERR_UNSUPPORTED.
  * The library allocates no device memory per call.
  */

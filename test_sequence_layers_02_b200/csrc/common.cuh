@@ -32,6 +32,7 @@ struct ScanParams {
   int lnjac;
   int no_ln;
   int minibatch;
+  int gate_channel;        // gate_logit holds one logit per feature ([B, H, T, d])
   int ablate;              // ablation gradient (prediction removed, Jacobian kept)
   int norm_match;          // ... rescaled per token to the full gradient's norm
 };

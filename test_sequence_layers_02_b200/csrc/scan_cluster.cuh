@@ -187,7 +187,12 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   const InT* gk = static_cast<const InT*>(p.k) + tok0 * D;
   const InT* gv = static_cast<const InT*>(p.v) + tok0 * D;
   const InT* gel = static_cast<const InT*>(p.eta_logit) + tok0;
-  const InT* ggl = p.gate_logit ? static_cast<const InT*>(p.gate_logit) + tok0 : nullptr;
+  // per-token gates (scalars staged with eta) or per-feature gates (read by the
+  // threads that write the outputs)
+  const InT* ggl = (p.gate_logit && !p.gate_channel) ? static_cast<const InT*>(p.gate_logit) + tok0
+                                                      : nullptr;
+  const InT* gch = (p.gate_logit && p.gate_channel)
+                       ? static_cast<const InT*>(p.gate_logit) + tok0 * D : nullptr;
   OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const float inv_d = 1.0f / (float)D;
@@ -426,7 +431,17 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   };
 
   // ---- outputs of chunk c, this CTA's rows ----
-  auto outputs = [&](int c) {
+  constexpr int NOUT = (kC * RS) / L::NW;
+  // per-feature gate logits of this thread's outputs of chunk c
+  auto gate_logits = [&](int c, float (&g)[NOUT]) {
+#pragma unroll
+    for (int k = 0; k < NOUT; ++k) {
+      const int idx = at + L::NW * k;
+      const int i = idx / RS, rr = idx % RS;
+      g[k] = (gch && i < chunk_len(c)) ? to_f32(gch[((size_t)c * C + i) * D + q * RS + rr]) : 0.f;
+    }
+  };
+  auto outputs = [&](int c, const float (&gpre)[NOUT]) {
     const int np = chunk_len(c);
     const float* Q0p = sQ0 + (c & 1) * kC * RS;
     const float* Sp = sS + (c & 1) * kC * kC;
@@ -435,7 +450,7 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
     const bool upd = sFlag[c & 3];
     OutT* dst = go + (size_t)c * C * D + q * RS;
 #pragma unroll
-    for (int k = 0; k < (kC * RS) / L::NW; ++k) {
+    for (int k = 0; k < NOUT; ++k) {
       const int idx = at + L::NW * k;
       const int i = idx / RS, rr = idx % RS;
       float acc = Q0p[i * RS + rr], acc2 = 0.f;
@@ -450,7 +465,8 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
           acc2 = fmaf(-s4.w, Gp[(4 * j4 + 3) * D + rr], acc2);
         }
       }
-      if (i < np) dst[(size_t)i * D + rr] = from_f32<OutT>(gt[i] * (acc + acc2));
+      const float gate = gch ? sigmoidf_(gpre[k]) : gt[i];
+      if (i < np) dst[(size_t)i * D + rr] = from_f32<OutT>(gate * (acc + acc2));
     }
   };
 
@@ -690,6 +706,8 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
       cp_async_commit();
       RawScalars pre{};
       if (c + 2 < nc) pre = issue_scalars(c + 2);
+      float gpre[NOUT];
+      if (c >= 1) gate_logits(c - 1, gpre);
       // W_{s,c} = W_{s,c-1} - sum_j eta_j G_{c-1,j} k_{c-1,j}^T on this CTA's rows
       if (c >= 1 && sFlag[(c - 1) & 3])
         rank_update(tileK(c - 1), sG + ((c - 1) & 1) * kC * D, sEta + ((c - 1) & 3) * kC);
@@ -707,7 +725,7 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
                Sc[s * kC + j] = (j <= s && s < n) ? et[j] * dot : 0.f;
              });
       }
-      if (c >= 1) outputs(c - 1);
+      if (c >= 1) outputs(c - 1, gpre);
       if (c + 2 < nc) finish_scalars(c + 2, pre);
       cp_async_wait_all();
     }
@@ -718,7 +736,11 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   if (nc > 0) {
     const int c = nc - 1;
     if (!chain && sFlag[c & 3]) rank_update(tileK(c), sG + (c & 1) * kC * D, sEta + (c & 3) * kC);
-    if (!chain) outputs(c);
+    if (!chain) {
+      float gpre[NOUT];
+      gate_logits(c, gpre);
+      outputs(c, gpre);
+    }
   }
   if (!chain) {
     if (Wc) store_W(Wc + ((size_t)p.n_mask_chunks * D + grow) * D);

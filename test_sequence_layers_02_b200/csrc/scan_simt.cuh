@@ -541,7 +541,13 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
   const InT* gk = static_cast<const InT*>(p.k) + tok0 * D;
   const InT* gv = static_cast<const InT*>(p.v) + tok0 * D;
   const InT* gel = static_cast<const InT*>(p.eta_logit) + tok0;
-  const InT* ggl = p.gate_logit ? static_cast<const InT*>(p.gate_logit) + tok0 : nullptr;
+  // per-token gates (scalars staged with eta) or per-feature gates (read by the
+  // threads that write the outputs)
+  const InT* ggl = (p.gate_logit && !p.gate_channel) ? static_cast<const InT*>(p.gate_logit) + tok0
+                                                      : nullptr;
+  const InT* gch = (p.gate_logit && p.gate_channel)
+                       ? static_cast<const InT*>(p.gate_logit) + tok0 * D : nullptr;
+  constexpr int NOUT = kC / (2 * IH);  // outputs per thread and chunk: tokens part + 2 IH k
   OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const float inv_d = 1.0f / (float)D;
@@ -659,6 +665,16 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
       cp_async_commit();
       RawScalars pre{};
       if (c + 2 < nc) pre = issue_scalars(c + 2);
+      // per-feature gate logits of this thread's outputs of chunk c-1, fetched
+      // now so the global-load latency overlaps the rank update
+      float gpre[NOUT];
+      if (gch && c >= 1) {
+#pragma unroll
+        for (int k = 0; k < NOUT; ++k) {
+          const int i = part + 2 * IH * k;
+          gpre[k] = i < chunk_len(c - 1) ? to_f32(gch[((size_t)(c - 1) * C + i) * D + r]) : 0.f;
+        }
+      }
 
       // W_{s,c} = W_{s,c-1} - sum_j eta_j G_j k_j^T over chunk c-1
       if (c >= 1 && sFlag[(c - 1) & 3])
@@ -675,7 +691,10 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
         const float* gt = sGate + ((c - 1) & 3) * kC;
         const bool upd = sFlag[(c - 1) & 3];
         OutT* dst = go + (size_t)(c - 1) * C * D;
-        for (int i = part; i < np; i += 2 * IH) {
+#pragma unroll
+        for (int k = 0; k < NOUT; ++k) {
+          const int i = part + 2 * IH * k;
+          if (i >= np) break;
           float acc = Q0p[i * D + r], acc2 = 0.f;
           if (upd) {
             int j = 0;
@@ -685,7 +704,8 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
             }
             if (j == i) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
           }
-          dst[(size_t)i * D + r] = from_f32<OutT>(gt[i] * (acc + acc2));
+          const float gate = gch ? sigmoidf_(gpre[k]) : gt[i];
+          dst[(size_t)i * D + r] = from_f32<OutT>(gate * (acc + acc2));
         }
       }
 
@@ -766,7 +786,8 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
         float acc = Q0p[i * D + r];
         if (upd)
           for (int j = 0; j <= i; ++j) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
-        dst[(size_t)i * D + r] = from_f32<OutT>(gt[i] * acc);
+        const float gate = gch ? sigmoidf_(to_f32(gch[((size_t)c * C + i) * D + r])) : gt[i];
+        dst[(size_t)i * D + r] = from_f32<OutT>(gate * acc);
       }
     }
     if (Wc) wb.store(Wc + (size_t)p.n_mask_chunks * D * D);

@@ -50,7 +50,7 @@ int choose_kernel(long long heads, int T, int d, unsigned mode, int b) {
   if (heads == 0) return TTT_KERNEL_NONE;
   const bool minibatch = mode & TTT_MODE_MINIBATCH;
   if (minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
-      !(mode & TTT_KERNEL_SIMT) && T > 0)
+      !(mode & (TTT_KERNEL_SIMT | TTT_GATE_CHANNEL)) && T > 0)
     return TTT_KERNEL_ID_TENSOR_CORE;
   if (!minibatch && d == 64 && !(mode & (TTT_KERNEL_SINGLE_CTA | TTT_GRAD_ABLATE)) && T > 0) {
     const int gm = (mode & TTT_NO_LN) ? 2 : ((mode & TTT_GRAD_LNJAC) ? 1 : 0);
@@ -189,7 +189,6 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
     if (misaligned(p)) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
-  if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
   if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
 
   const size_t heads = (size_t)B * H;
@@ -204,8 +203,9 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   const size_t mask_bytes = (size_t)B * n_mask_chunks;
   const size_t wc_bytes = heads * (size_t)(n_mask_chunks + 1) * d * d * sizeof(float);
   struct Span { const void* p; size_t n; };
+  const size_t gate_bytes = (mode & TTT_GATE_CHANNEL) ? tok_bytes : scal_bytes;
   const Span inputs[] = {{q, tok_bytes}, {k, tok_bytes}, {v, tok_bytes},
-                         {eta_logit, scal_bytes}, {gate_logit, scal_bytes},
+                         {eta_logit, scal_bytes}, {gate_logit, gate_bytes},
                          {W0, w_bytes}, {gamma, no_ln ? 0 : gb_bytes},
                          {beta, no_ln ? 0 : gb_bytes}, {mask, mask ? mask_bytes : 0}};
   for (const Span& in : inputs) {
@@ -233,6 +233,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   p.minibatch = (mode & TTT_MODE_MINIBATCH) ? 1 : 0;
   p.ablate = (mode & TTT_GRAD_ABLATE) ? 1 : 0;
   p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
+  p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int which = choose_kernel((long long)heads, T, d, mode, b);
@@ -257,7 +258,6 @@ int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b) {
   if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
-  if (mode & TTT_GATE_CHANNEL) return TTT_ERR_UNSUPPORTED;
   if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
   const int which = choose_kernel((long long)B * H, T, d, mode, b);
   if (which == TTT_KERNEL_ID_CUDA_CORE && (mode & TTT_MODE_MINIBATCH) && b > ttt::kC)

@@ -107,8 +107,9 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
          stream: Optional[torch.cuda.Stream] = None):
     """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
 
-    q, k, v: [B, H, T, d] fp32 or bf16; eta_logit, gate_logit: [B, H, T] with
-    the same dtype (gate may be None); W0: [B, H, d, d] fp32 (z = W k);
+    q, k, v: [B, H, T, d] fp32 or bf16; eta_logit: [B, H, T] with the same
+    dtype; gate_logit: [B, H, T], or [B, H, T, d] for a per-feature gate, or
+    None; W0: [B, H, d, d] fp32 (z = W k);
     gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
     uint8 or None. ``out_dtype`` defaults to the input dtype. ``force_simt``
     keeps mini-batch mode on the CUDA-core kernel; ``single_cta`` keeps
@@ -136,8 +137,10 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     in_dtype = q.dtype
     if in_dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("inputs must be float32 or bfloat16")
+    channel = gate_logit is not None and gate_logit.dim() == 4
     for name, t, shp in (("k", k, (B, H, T, d)), ("v", v, (B, H, T, d)),
-                         ("eta_logit", eta_logit, (B, H, T)), ("gate_logit", gate_logit, (B, H, T))):
+                         ("eta_logit", eta_logit, (B, H, T)),
+                         ("gate_logit", gate_logit, (B, H, T, d) if channel else (B, H, T))):
         if t is None and name == "gate_logit":
             continue
         if tuple(t.shape) != shp or t.dtype != in_dtype or not t.is_contiguous():
@@ -158,7 +161,7 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
             (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
             (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0) |
             (KERNEL_SINGLE_CTA if single_cta else 0) | (GRAD_ABLATE if ablate else 0) |
-            (GRAD_NORM_MATCH if norm_match else 0))
+            (GRAD_NORM_MATCH if norm_match else 0) | (GATE_CHANNEL if channel else 0))
     if o_dev is None:
         o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
     if wt_dev is None:

@@ -94,7 +94,7 @@ def test_invalid_arguments_rejected(lib, over):
 
 @pytest.mark.parametrize("over", [dict(d=32), dict(d=128), dict(d=17),
                                   dict(mode=1, b=17), dict(mode=1 | 32, b=32),
-                                  dict(mode=1 << 6), dict(mode=1 | (1 << 8))])
+                                  dict(mode=1 | (1 << 8))])
 def test_unsupported_shapes(lib, over):
     assert call(lib, **over) == UNSUPPORTED
 
@@ -162,7 +162,7 @@ def test_kernel_choice_without_launching(lib):
     assert f(2, 3, 40, 64, 0, 0) == INVALID
     assert f(2, 3, 40, 32, 0, 16) == UNSUPPORTED
     assert f(2, 3, 40, 64, MINIB, 17) == UNSUPPORTED
-    assert f(2, 3, 40, 64, 1 << 6, 16) == UNSUPPORTED
+    assert f(2, 3, 40, 64, MINIB | LNJAC | BF16 | (1 << 6), 16) == 1 # per-feature gate: CUDA cores
     # per-token d = 64 picks the cluster kernel only where clusters fit on a device
     assert f(2, 3, 40, 64, LNJAC, 16) in (1, 2)
 
