@@ -83,20 +83,6 @@ struct ClusterLayout {
   static_assert(KW == 8, "a W thread holds two 4-element units of its row");
 };
 
-// Warp-wide sums of five values; the adds run as pairs.
-__device__ __forceinline__ void butterfly5(float (&m)[5]) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    float r[5];
-#pragma unroll
-    for (int i = 0; i < 5; ++i) r[i] = __shfl_xor_sync(0xffffffffu, m[i], off);
-    const float2 a = __fadd2_rn(make_float2(m[0], m[1]), make_float2(r[0], r[1]));
-    const float2 b = __fadd2_rn(make_float2(m[2], m[3]), make_float2(r[2], r[3]));
-    m[0] = a.x; m[1] = a.y; m[2] = b.x; m[3] = b.y;
-    m[4] += r[4];
-  }
-}
-
 // Set when a bounded wait of this kernel gave up; read and cleared by
 // ttt_check_device_status(). One word per device in this module.
 __device__ int g_cluster_status;
@@ -471,14 +457,8 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   };
 
   // ---- chain state (warp 4) ----
-  float gam[EPL], bet[EPL], g2c[EPL], gbc[EPL];
-  float Sgb = 0.f, Sb = 0.f;
-  float2 cpr[NP][EPL];  // correction of the next chunk's z (token pairs) by this chunk's G
-  unsigned dead = 0;    // P slots whose bookkeeping was lost after a failed drain
-#pragma unroll
-  for (int pp = 0; pp < NP; ++pp)
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+  Chain<D, InT, false, GM, L::PTS> ch;
+  unsigned dead = 0;  // P slots whose bookkeeping was lost after a failed drain
 
   // ---------------- prologue ----------------
   if (chain) {
@@ -490,21 +470,7 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
       }
       pbar_init_fence();
     }
-    float sgb = 0.f, sb = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const int f = lane + 32 * e;
-      gam[e] = p.no_ln ? 1.f : p.gamma[(size_t)h * D + f];
-      bet[e] = p.no_ln ? 0.f : p.beta[(size_t)h * D + f];
-      g2c[e] = gam[e] * gam[e];
-      gbc[e] = gam[e] * bet[e];
-      sgb = fmaf(gam[e], bet[e], sgb);
-      sb += bet[e];
-    }
-    float s2[2] = {sgb, sb};
-    butterfly<2>(s2);
-    Sgb = s2[0];
-    Sb = s2[1];
+    ch.init(p.gamma + (size_t)h * D, p.beta + (size_t)h * D, p.no_ln, lane);
   } else {
     const float* W0 = p.W0 + ((size_t)bh * D + grow) * D;  // may alias W_T
 #pragma unroll
@@ -555,146 +521,10 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
         else if (lane == 0 && c + L::NPS < nc) pbar_arm(pbar + sl, L::kSlotBytes);
       }
       if (!sFlag[c & 3]) {
-        // SKIP: no gradient is needed, and the next chunk takes no correction
-        // from this one (its X is zero)
-#pragma unroll
-        for (int pp = 0; pp < NP; ++pp)
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+        ch.reset();  // a SKIP chunk leaves the next chunk uncorrected (its X is zero)
       } else {
         const float* PT = sP + sl * L::PSLOT;
-        const float* AT = PT + L::SAT;
-        const float* XT = PT + L::SXT;
-        const unsigned char* Vt = tileV(c);
-        float* Gc = sG + (c & 1) * kC * D;
-        float2 zp[NP][EPL];  // z of token pairs (2 pp, 2 pp + 1), feature lane + 32 e
-        float2 mp[NP];       // their LayerNorm shift (the feature mean)
-        // z = P + the correction from the previous chunk
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const float4* row = reinterpret_cast<const float4*>(PT + (lane + 32 * e) * L::PTS);
-#pragma unroll
-          for (int m4 = 0; m4 < kC / 4; ++m4) {
-            const float4 x = row[m4];
-            zp[2 * m4][e] = __fadd2_rn(make_float2(x.x, x.y), cpr[2 * m4][e]);
-            zp[2 * m4 + 1][e] = __fadd2_rn(make_float2(x.z, x.w), cpr[2 * m4 + 1][e]);
-          }
-        }
-#pragma unroll
-        for (int pp = 0; pp < NP; ++pp)
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
-        if (GM != 2) {
-          // feature means of the 16 rows of z: reduce-scatter over the lanes,
-          // after which lanes 2m and 2m + 1 hold token m's sum
-          float sm[kC];
-#pragma unroll
-          for (int pp = 0; pp < NP; ++pp) {
-            const float2 t = __fadd2_rn(zp[pp][0], zp[pp][1]);
-            sm[2 * pp] = t.x;
-            sm[2 * pp + 1] = t.y;
-          }
-          reduce_scatter_step<kC, kC / 2, 16>(sm, lane);
-          const float mrow = (sm[0] + __shfl_xor_sync(0xffffffffu, sm[0], 1)) * inv_d;
-#pragma unroll
-          for (int pp = 0; pp < NP; ++pp)
-            mp[pp] = make_float2(__shfl_sync(0xffffffffu, mrow, 4 * pp),
-                                 __shfl_sync(0xffffffffu, mrow, 4 * pp + 2));
-        }
-        // No branch inside: tokens past the chunk's end compute finite values
-        // (their P rows are zero) that a select turns into G = 0.
-#pragma unroll
-        for (int i = 0; i < kC; ++i) {
-          const int pi = i / 2;
-          const bool hi = i & 1;
-          float v[EPL], Gv[EPL], zi[EPL];
-          float mG = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            v[e] = lds1(Vt + i * L::ROWB + (lane + 32 * e) * L::ELT, InT());
-            zi[e] = hi ? zp[pi][e].y : zp[pi][e].x;
-          }
-          if (GM == 2) {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) Gv[e] = zi[e] - v[e];
-          } else {
-            const float mu = hi ? mp[pi].y : mp[pi].x;
-            float y[EPL];
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) y[e] = zi[e] - mu;
-            if (GM == 1) {
-              // moments of y: sum y^2, sum g2 y, sum g2 y^2, sum w y, sum gamma v
-              float m5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-              float w[EPL];
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) {
-                w[e] = fmaf(-gam[e], v[e], gbc[e]);
-                const float gy = g2c[e] * y[e];
-                m5[0] = fmaf(y[e], y[e], m5[0]);
-                m5[1] += gy;
-                m5[2] = fmaf(gy, y[e], m5[2]);
-                m5[3] = fmaf(w[e], y[e], m5[3]);
-                m5[4] = fmaf(gam[e], v[e], m5[4]);
-              }
-              butterfly5(m5);
-              const float rs = rsqrtf(fmaf(m5[0], inv_d, p.eps));
-              const float mg = (rs * m5[1] + Sgb - m5[4]) * inv_d;
-              const float mgx = rs * (rs * m5[2] + m5[3]) * inv_d;
-              const float rs2 = rs * rs;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) Gv[e] = rs2 * (g2c[e] - mgx) * y[e] + rs * (w[e] - mg);
-            } else {
-              float m3[3] = {0.f, 0.f, 0.f};
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) {
-                m3[0] = fmaf(y[e], y[e], m3[0]);
-                m3[1] = fmaf(gam[e], y[e], m3[1]);
-                m3[2] += v[e];
-              }
-              butterfly<3>(m3);
-              const float rs = rsqrtf(fmaf(m3[0], inv_d, p.eps));
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) Gv[e] = gam[e] * rs * y[e] + bet[e] - v[e];
-              mG = (rs * m3[1] + Sb - m3[2]) * inv_d;
-            }
-          }
-          const bool valid = i < n;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            Gv[e] = valid ? Gv[e] : 0.f;
-            Gc[i * D + lane + 32 * e] = Gv[e];
-          }
-          mG = valid ? mG : 0.f;
-          // this token's G into the later tokens of chunk c (A, zero for m <= i)
-          // and into every token of chunk c+1 (X)
-          float2 nG[EPL];
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) nG[e] = dup2(-Gv[e]);
-          // (a row of A or X is read four pairs at a time to keep registers low)
-#pragma unroll
-          for (int m4 = (i + 1) / 4; m4 < kC / 4; ++m4) {
-            const float4 a4 = reinterpret_cast<const float4*>(AT + i * kC)[m4];
-            const float2 a2[2] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w)};
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int pp = 2 * m4 + h2;
-              if (pp < (i + 1) / 2) continue;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) zp[pp][e] = __ffma2_rn(a2[h2], nG[e], zp[pp][e]);
-              if (GM == 0) mp[pp] = __ffma2_rn(a2[h2], dup2(-mG), mp[pp]);
-            }
-          }
-#pragma unroll
-          for (int m4 = 0; m4 < kC / 4; ++m4) {
-            const float4 x4 = reinterpret_cast<const float4*>(XT + i * kC)[m4];
-            const float2 x2[2] = {make_float2(x4.x, x4.y), make_float2(x4.z, x4.w)};
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-              for (int e = 0; e < EPL; ++e)
-                cpr[2 * m4 + h2][e] = __ffma2_rn(x2[h2], nG[e], cpr[2 * m4 + h2][e]);
-          }
-        }
+        ch.run(n, PT, PT + L::SAT, PT + L::SXT, tileV(c), sG + (c & 1) * kC * D, p.eps, lane);
       }
     } else {
       // ===== bulk work of period c =====

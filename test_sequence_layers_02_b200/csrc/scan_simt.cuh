@@ -238,8 +238,10 @@ struct WBlock {
       }
     }
   }
-  // out[t][row] = (W x_t)_row for the kC rows x_t of tile R, this block's rows,
-  // in batches of 8 tokens finished by a reduce-scatter over the CG lanes.
+  // (W x_t)_row for the kC rows x_t of tile R and this block's rows, in batches
+  // of 8 tokens finished by a reduce-scatter over the CG lanes; stored as
+  // out[t][row] (PTS == 0) or transposed, out[row][t] with token stride PTS.
+  template <int PTS = 0>
   __device__ __forceinline__ void products(const unsigned char* R, float* out) const {
     constexpr int V = RB * 8, PER = V / CG;
 #pragma unroll
@@ -266,8 +268,13 @@ struct WBlock {
       reduce_scatter_lanes<V, CG>(acc, cg);
       // lane cg now holds values cg * PER .. + PER - 1: one row, PER tokens
       const int i0 = cg * PER, rb = i0 / 8, tb = i0 % 8;
+      if constexpr (PTS == 0) {
 #pragma unroll
-      for (int u = 0; u < PER; ++u) out[(t0 + tb + u) * D + row0 + rb] = acc[u];
+        for (int u = 0; u < PER; ++u) out[(t0 + tb + u) * D + row0 + rb] = acc[u];
+      } else {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) out[(row0 + rb) * PTS + t0 + tb + u] = acc[u];
+      }
     }
   }
 };
@@ -281,7 +288,11 @@ __device__ __forceinline__ void butterfly(float (&v)[N]) {
   }
 }
 
-// Gradient chain of one chunk (one warp). GM: 0 = simplified (G = err),
+// Gradient chain of one chunk of the one-CTA-per-head kernel (one warp).
+// (The cluster kernel uses the Chain struct below, which also applies the
+// next chunk's correction; here that stays a separate phase, which keeps this
+// kernel's registers low enough for three CTAs per SM when heads are many.)
+// GM: 0 = simplified (G = err),
 // 1 = through the LayerNorm Jacobian, 2 = no LayerNorm (G = z - v),
 // 3 = the ablation gradient (the Jacobian applied to -gamma * v, the
 // prediction removed; "Error Correction in Trained TTT Layers", Abstract),
@@ -506,6 +517,256 @@ __device__ __forceinline__ void row_means(const float* Z, float* out, int tid, i
   }
 }
 
+// Warp-wide sums of five values; the adds run as pairs.
+__device__ __forceinline__ void butterfly5(float (&m)[5]) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float r[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) r[i] = __shfl_xor_sync(0xffffffffu, m[i], off);
+    const float2 a = __fadd2_rn(make_float2(m[0], m[1]), make_float2(r[0], r[1]));
+    const float2 b = __fadd2_rn(make_float2(m[2], m[3]), make_float2(r[2], r[3]));
+    m[0] = a.x; m[1] = a.y; m[2] = b.x; m[3] = b.y;
+    m[4] += r[4];
+  }
+}
+
+// The sequential gradient chain of one head, shared by the CUDA-core scan
+// kernels: one warp, lane l holding features l + 32 e (e < EPL; at d = 16
+// lanes 16-31 hold none). For chunk c, z of its tokens is P_c (read from
+// PT[feature][token], token stride PTS) plus the correction the previous
+// chunk left in `cpr`. Per token i the LayerNorm gradient G_i (GM: 0
+// simplified, 1 LN Jacobian, 2 no LayerNorm, 3 ablation, 4 ablation with
+// per-token norm matching) goes to Gc[i][feature] and is applied at once to
+// the later tokens of the chunk through A^T (per-token mode only) and to every
+// token of the next chunk through X^T, accumulated in `cpr`. Token pairs are
+// updated with paired FMAs, and tokens past n are masked to G = 0 so the
+// unrolled token loop has no branch. The LayerNorm shift is the feature mean
+// of z at the chunk start (exact for the Jacobian forms, whose G has zero
+// mean; tracked through the chunk for the simplified gradient).
+template <int D, typename InT, bool MINIB, int GM, int PTS>
+struct Chain {
+  static constexpr int EPL = (D + 31) / 32;
+  static constexpr int NP = kC / 2;
+  static constexpr int ROWB = D * (int)sizeof(InT) + 16;  // V tile row, as the kernels' tiles
+  float gam[EPL], bet[EPL], g2c[EPL], gbc[EPL];
+  float Sgb, Sb;
+  float2 cpr[NP][EPL];
+
+  __device__ __forceinline__ void init(const float* gamma_h, const float* beta_h, bool no_ln,
+                                       int lane) {
+    float sgb = 0.f, sb = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      gam[e] = (f < D && !no_ln) ? gamma_h[f] : (f < D ? 1.f : 0.f);
+      bet[e] = (f < D && !no_ln) ? beta_h[f] : 0.f;
+      g2c[e] = gam[e] * gam[e];
+      gbc[e] = gam[e] * bet[e];
+      sgb = fmaf(gam[e], bet[e], sgb);
+      sb += bet[e];
+    }
+    float s2[2] = {sgb, sb};
+    butterfly<2>(s2);
+    Sgb = s2[0];
+    Sb = s2[1];
+    reset();
+  }
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cpr[pp][e] = make_float2(0.f, 0.f);
+  }
+
+  __device__ __forceinline__ void run(int n, const float* PT, const float* AT, const float* XT,
+                                      const unsigned char* Vt, float* Gc, float eps, int lane) {
+    const float inv_d = 1.0f / (float)D;
+    float2 zp[NP][EPL];  // z of token pairs (2 pp, 2 pp + 1)
+    float2 mp[NP];       // their LayerNorm shift
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      const float4* row = reinterpret_cast<const float4*>(PT + (f < D ? f : 0) * PTS);
+#pragma unroll
+      for (int m4 = 0; m4 < kC / 4; ++m4) {
+        float4 x = row[m4];
+        if (f >= D) x = make_float4(0.f, 0.f, 0.f, 0.f);
+        zp[2 * m4][e] = __fadd2_rn(make_float2(x.x, x.y), cpr[2 * m4][e]);
+        zp[2 * m4 + 1][e] = __fadd2_rn(make_float2(x.z, x.w), cpr[2 * m4 + 1][e]);
+      }
+    }
+    reset();
+    if (GM != 2) {
+      // feature means of the kC rows of z: reduce-scatter over the lanes, after
+      // which lanes 2m and 2m + 1 hold token m's sum
+      float sm[kC];
+#pragma unroll
+      for (int pp = 0; pp < NP; ++pp) {
+        float2 t = zp[pp][0];
+#pragma unroll
+        for (int e = 1; e < EPL; ++e) t = __fadd2_rn(t, zp[pp][e]);
+        sm[2 * pp] = t.x;
+        sm[2 * pp + 1] = t.y;
+      }
+      reduce_scatter_step<kC, kC / 2, 16>(sm, lane);
+      const float mrow = (sm[0] + __shfl_xor_sync(0xffffffffu, sm[0], 1)) * inv_d;
+#pragma unroll
+      for (int pp = 0; pp < NP; ++pp)
+        mp[pp] = make_float2(__shfl_sync(0xffffffffu, mrow, 4 * pp),
+                             __shfl_sync(0xffffffffu, mrow, 4 * pp + 2));
+    }
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+      const int pi = i / 2;
+      const bool hi = i & 1;
+      float v[EPL], Gv[EPL], zi[EPL];
+      bool fv[EPL];
+      float mG = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        fv[e] = f < D;
+        v[e] = fv[e] ? lds1(Vt + i * ROWB + f * (int)sizeof(InT), InT()) : 0.f;
+        zi[e] = hi ? zp[pi][e].y : zp[pi][e].x;
+      }
+      if (GM == 2) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) Gv[e] = zi[e] - v[e];
+      } else {
+        const float mu = hi ? mp[pi].y : mp[pi].x;
+        float y[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) y[e] = fv[e] ? zi[e] - mu : 0.f;
+        if (GM == 1) {
+          // moments of y: sum y^2, sum g2 y, sum g2 y^2, sum w y, sum gamma v
+          float m5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+          float w[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            w[e] = fmaf(-gam[e], v[e], gbc[e]);
+            const float gy = g2c[e] * y[e];
+            m5[0] = fmaf(y[e], y[e], m5[0]);
+            m5[1] += gy;
+            m5[2] = fmaf(gy, y[e], m5[2]);
+            m5[3] = fmaf(w[e], y[e], m5[3]);
+            m5[4] = fmaf(gam[e], v[e], m5[4]);
+          }
+          butterfly5(m5);
+          const float rs = rsqrtf(fmaf(m5[0], inv_d, eps));
+          const float mg = (rs * m5[1] + Sgb - m5[4]) * inv_d;
+          const float mgx = rs * (rs * m5[2] + m5[3]) * inv_d;
+          const float rs2 = rs * rs;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) Gv[e] = rs2 * (g2c[e] - mgx) * y[e] + rs * (w[e] - mg);
+        } else if (GM == 3) {
+          // g = -gamma v: sum y^2, sum gamma v, sum gamma v y
+          float m[3] = {0.f, 0.f, 0.f};
+          float gv[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            gv[e] = gam[e] * v[e];
+            m[0] = fmaf(y[e], y[e], m[0]);
+            m[1] += gv[e];
+            m[2] = fmaf(gv[e], y[e], m[2]);
+          }
+          butterfly<3>(m);
+          const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+          const float a = m[1] * inv_d, bq = rs * rs * rs * m[2] * inv_d;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) Gv[e] = fmaf(bq, y[e], rs * (a - gv[e]));
+        } else if (GM == 4) {
+          // both forms from one butterfly (the GM 1 moments and sum gamma v y),
+          // then the two norms
+          float m[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float w[EPL], gv[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            w[e] = fmaf(-gam[e], v[e], gbc[e]);
+            gv[e] = gam[e] * v[e];
+            m[0] = fmaf(y[e], y[e], m[0]);
+            m[1] = fmaf(g2c[e], y[e], m[1]);
+            m[2] = fmaf(g2c[e] * y[e], y[e], m[2]);
+            m[3] = fmaf(w[e], y[e], m[3]);
+            m[4] = fmaf(gam[e], v[e], m[4]);
+            m[5] = fmaf(gv[e], y[e], m[5]);
+          }
+          butterfly<6>(m);
+          const float rs = rsqrtf(fmaf(m[0], inv_d, eps));
+          const float mg = (rs * m[1] + Sgb - m[4]) * inv_d;
+          const float mgx = rs * (rs * m[2] + m[3]) * inv_d;
+          const float rs2 = rs * rs;
+          const float a = m[4] * inv_d, bq = rs2 * rs * m[5] * inv_d;
+          float nrm[2] = {0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const float gf = rs2 * (g2c[e] - mgx) * y[e] + rs * (w[e] - mg);
+            Gv[e] = fmaf(bq, y[e], rs * (a - gv[e]));
+            if (fv[e]) {
+              nrm[0] = fmaf(gf, gf, nrm[0]);
+              nrm[1] = fmaf(Gv[e], Gv[e], nrm[1]);
+            }
+          }
+          butterfly<2>(nrm);
+          const float scale = nrm[1] > 0.f ? sqrtf(nrm[0] / nrm[1]) : 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) Gv[e] *= scale;
+        } else {
+          float m3[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            m3[0] = fmaf(y[e], y[e], m3[0]);
+            m3[1] = fmaf(gam[e], y[e], m3[1]);
+            m3[2] += v[e];
+          }
+          butterfly<3>(m3);
+          const float rs = rsqrtf(fmaf(m3[0], inv_d, eps));
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) Gv[e] = gam[e] * rs * y[e] + bet[e] - v[e];
+          mG = (rs * m3[1] + Sb - m3[2]) * inv_d;
+        }
+      }
+      const bool valid = i < n;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        Gv[e] = (valid && fv[e]) ? Gv[e] : 0.f;
+        if (fv[e]) Gc[i * D + lane + 32 * e] = Gv[e];
+      }
+      mG = valid ? mG : 0.f;
+      float2 nG[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) nG[e] = dup2(-Gv[e]);
+      if (!MINIB) {
+        // into the later tokens of this chunk (A^T row i, zero for m <= i)
+#pragma unroll
+        for (int m4 = (i + 1) / 4; m4 < kC / 4; ++m4) {
+          const float4 a4 = reinterpret_cast<const float4*>(AT + i * kC)[m4];
+          const float2 a2[2] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w)};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int pp = 2 * m4 + h2;
+            if (pp < (i + 1) / 2) continue;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) zp[pp][e] = __ffma2_rn(a2[h2], nG[e], zp[pp][e]);
+            if (GM == 0) mp[pp] = __ffma2_rn(a2[h2], dup2(-mG), mp[pp]);
+          }
+        }
+      }
+      // into every token of the next chunk (X^T row i)
+#pragma unroll
+      for (int m4 = 0; m4 < kC / 4; ++m4) {
+        const float4 x4 = reinterpret_cast<const float4*>(XT + i * kC)[m4];
+        const float2 x2[2] = {make_float2(x4.x, x4.y), make_float2(x4.z, x4.w)};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e)
+            cpr[2 * m4 + h2][e] = __ffma2_rn(x2[h2], nG[e], cpr[2 * m4 + h2][e]);
+      }
+    }
+  }
+};
+
 template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
 __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanParams p) {
   using L = PipeLayout<D, InT, IH>;
@@ -547,7 +808,6 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
                                                       : nullptr;
   const InT* gch = (p.gate_logit && p.gate_channel)
                        ? static_cast<const InT*>(p.gate_logit) + tok0 * D : nullptr;
-  constexpr int NOUT = kC / (2 * IH);  // outputs per thread and chunk: tokens part + 2 IH k
   OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const float inv_d = 1.0f / (float)D;
@@ -665,16 +925,6 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
       cp_async_commit();
       RawScalars pre{};
       if (c + 2 < nc) pre = issue_scalars(c + 2);
-      // per-feature gate logits of this thread's outputs of chunk c-1, fetched
-      // now so the global-load latency overlaps the rank update
-      float gpre[NOUT];
-      if (gch && c >= 1) {
-#pragma unroll
-        for (int k = 0; k < NOUT; ++k) {
-          const int i = part + 2 * IH * k;
-          gpre[k] = i < chunk_len(c - 1) ? to_f32(gch[((size_t)(c - 1) * C + i) * D + r]) : 0.f;
-        }
-      }
 
       // W_{s,c} = W_{s,c-1} - sum_j eta_j G_j k_j^T over chunk c-1
       if (c >= 1 && sFlag[(c - 1) & 3])
@@ -691,10 +941,8 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
         const float* gt = sGate + ((c - 1) & 3) * kC;
         const bool upd = sFlag[(c - 1) & 3];
         OutT* dst = go + (size_t)(c - 1) * C * D;
-#pragma unroll
-        for (int k = 0; k < NOUT; ++k) {
-          const int i = part + 2 * IH * k;
-          if (i >= np) break;
+        // (a rolled loop: unrolling it costs the registers of a third CTA per SM)
+        for (int i = part; i < np; i += 2 * IH) {
           float acc = Q0p[i * D + r], acc2 = 0.f;
           if (upd) {
             int j = 0;
@@ -704,7 +952,7 @@ __global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanPa
             }
             if (j == i) acc = fmaf(-Sp[i * kC + j], Gp[j * D + r], acc);
           }
-          const float gate = gch ? sigmoidf_(gpre[k]) : gt[i];
+          const float gate = gch ? sigmoidf_(to_f32(gch[((size_t)(c - 1) * C + i) * D + r])) : gt[i];
           dst[(size_t)i * D + r] = from_f32<OutT>(gate * (acc + acc2));
         }
       }
