@@ -142,8 +142,6 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
   using L = ClusterLayout<InT, CS>;
   constexpr int D = 64;
   constexpr int RS = L::RS, G = L::G, KW = L::KW;
-  constexpr int EPL = 2;                // features per chain lane
-  constexpr int NP = kC / 2;            // token pairs of a chunk
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char* sK = smem + L::oK;
   unsigned char* sQ = smem + L::oQ;

@@ -18,13 +18,19 @@
 //   chain 0-3   read Z_k^T (TMEM, feature-major), transpose through shared
 //               memory, token-major LayerNorm + gradient (8 lanes per token,
 //               one shuffle round of shifted moments), write Aneg_k (bf16).
-//   bulk 4-7    W (fp32 TMEM) -> bf16 operand W_s; outputs o_c = gate * O_c^T;
-//               Gram products -> bf16 operands Xg_{c+2}, M_{c+1}; per-chunk scalars.
-//   issuer 8    (one thread) every tcgen05.mma and TMA:
-//               MMA2 O_c^T += Aneg_c M_c^T, MMA3 W += Aneg_c K_c (K as an MN-major
-//               operand), MMAc P_{c+1}^T += Aneg_c Xg_{c+1}^T;
-//               Gram [K_{c+2}; Q_{c+1}] K_{c+1}^T and MMA1 [P_{c+2} | Q0_{c+1}]^T =
-//               W_s [K_{c+2}; Q_{c+1}]^T; TMA of chunk x = {K_x, Q_{x-1}, V_x}.
+//   bulk 4-7    W (fp32 TMEM) -> bf16 operand W_s; Gram products two chunks
+//               ahead -> bf16 operand [Xg_{c+3}; M_{c+2}]; outputs o_c = gate * O_c^T;
+//               per-chunk scalars.
+//   issuer 8    (one thread) every tcgen05.mma and TMA, per chunk c in this order:
+//               MMAc [P_{c+1} | O_c]^T += Aneg_c [Xg_{c+1}; M_c]^T (one N = 32 MMA,
+//               committed alone: the chain's next Z waits for nothing else);
+//               MMA3 W += Aneg_c K_c (K as an MN-major operand); the Gram
+//               [K_{c+3}; Q_{c+2}] K_{c+2}^T; once W_s is refreshed, MMA1
+//               [P_{c+2} | Q0_{c+1}]^T = W_s [K_{c+2}; Q_{c+1}]^T; TMA of chunk
+//               x = {K_x, Q_{x-1}, V_x}, NST chunks ahead.
+// One chunk period is then the longer of two loops from MMAc: the chain's
+// (Z -> LayerNorm -> Aneg) and the W refresh's (MMA3 -> bf16 W_s -> MMA1,
+// which must precede the next MMAc); the Grams and the outputs stay off both.
 // M = 128 everywhere: A operands stack two copies of their 64 rows, so TMEM
 // lanes 0-63 and 64-127 hold identical d-row results and every warp quarter
 // reads its own lanes.
@@ -54,12 +60,13 @@ namespace tc {
 constexpr int D = 64;
 constexpr int CB = 16;              // chunk (b)
 constexpr int NT = 288;             // 4 chain + 4 bulk + 1 issuer warps
-constexpr int NST = 4;              // TMA stages
+constexpr int NST = 5;              // TMA stages
 constexpr int kSR = 32;             // scalar ring (chunks)
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kTmemGramCols = 32;
 constexpr uint32_t kColW = 0;       // W accumulator (64 columns)
-// slot s = 0, 1: [P^T | Q0^T / O^T] at 64 + 32 s (16 + 16 columns)
+// slot s = 0, 1: [P^T | Q0^T / O^T] at 64 + 32 s (16 + 16 columns); the Gram
+// of chunk x in columns 16 (x & 1) of the second allocation
 __device__ __forceinline__ uint32_t col_p(int s) { return 64u + 32u * (uint32_t)s; }
 __device__ __forceinline__ uint32_t col_o(int s) { return 80u + 32u * (uint32_t)s; }
 constexpr int kTile = CB * D * 2;   // 2048 bytes
@@ -70,9 +77,8 @@ constexpr int oKQ = 0;                             // [NST][K_x | Q_{x-1}] 128B-
 constexpr int oV = oKQ + NST * 2 * kTile;          // [NST] V_x, row-major
 constexpr int oWb = oV + NST * kTile;              // W_s bf16, 128 rows x 128 B, 128B-swizzled
 constexpr int oAneg = oWb + 128 * 128;             // [2] 128 rows x 16 bf16 (core matrices)
-constexpr int oM = oAneg + 2 * 128 * 32;           // [2] M  16 x 16 bf16 (core matrices)
-constexpr int oXg = oM + 2 * 512;                  // [2] Xg 16 x 16 bf16 (core matrices)
-constexpr int oZ = oXg + 2 * 512;                  // [2][16][kZS] f32
+constexpr int oXM = oAneg + 2 * 128 * 32;          // [2] [Xg_{x+1}; M_x] 32 x 16 bf16 (core matrices)
+constexpr int oZ = oXM + 2 * 1024;                 // [2][16][kZS] f32
 constexpr int oEta = oZ + 2 * CB * kZS * 4;        // [kSR][16] f32 (mask folded in)
 constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
 constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
@@ -85,6 +91,7 @@ constexpr int oAbort = oTmem + 8;
 constexpr int kSmemUsed = oAbort + 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
 static_assert(kSmemBytes <= 75 * 1024, "three CTAs per SM must fit in shared memory");
+static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
 static_assert(3 * (kTmemCols + kTmemGramCols) <= 512, "three CTAs per SM must fit in TMEM");
 // The 128-row A operand of the Gram MMA starts at a stage's K tile and runs
 // 16 KB forward: it must stay inside this CTA's shared memory.
@@ -145,18 +152,17 @@ __global__ void __launch_bounds__(tc::NT, 3)
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + oBar);  // [NST] chunk x -> x % NST
   uint64_t* bar_g = bar_tma + NST;   // [2] Aneg_k written (chain, 128 arrivals)
   uint64_t* bar_z = bar_g + 2;       // [2] Z_k complete in TMEM (commit)
-  uint64_t* bar_xm = bar_z + 2;      // [2] Xg_{x+1}, M_x written (bulk, 128 arrivals)
-  uint64_t* bar_w = bar_xm + 2;      // a chunk's MMA2/3/c complete (commit)
+  uint64_t* bar_xm = bar_z + 2;      // [2] [Xg_{x+1}; M_x] written (bulk, 128 arrivals)
+  uint64_t* bar_w = bar_xm + 2;      // a chunk's MMAc and MMA3 complete (commit)
   uint64_t* bar_wb = bar_w + 1;      // W_s bf16 refreshed (bulk, 128 arrivals)
   uint64_t* bar_gram = bar_wb + 1;   // Gram MMA complete (commit)
   uint64_t* bar_pro = bar_gram + 1;  // prologue MMAs complete (commit)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + oTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + oAbort);
-  auto tKQ = [&](int x) { return smem + oKQ + (x & (NST - 1)) * 2 * kTile; };  // K_x, then Q_{x-1}
-  auto tV = [&](int x) { return smem + oV + (x & (NST - 1)) * kTile; };
+  auto tKQ = [&](int x) { return smem + oKQ + (x % NST) * 2 * kTile; };  // K_x, then Q_{x-1}
+  auto tV = [&](int x) { return smem + oV + (x % NST) * kTile; };
   auto aneg = [&](int c) { return smem + oAneg + (c & 1) * 4096; };
-  auto mmat = [&](int c) { return smem + oM + (c & 1) * 512; };
-  auto xgm = [&](int c) { return smem + oXg + (c & 1) * 512; };
+  auto xm = [&](int x) { return smem + oXM + (x & 1) * 1024; };  // [Xg_{x+1}; M_x]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
   int tma_issued = 0;  // TMA loads [0, tma_issued) issued (chunk x = {K_x, Q_{x-1}, V_x})
   int w_issued = 0;    // commits to bar_w
   auto issue_tma = [&](int x) {
-    uint64_t* bar = &bar_tma[x & (NST - 1)];
+    uint64_t* bar = &bar_tma[x % NST];
     const uint32_t bytes = (x < nc ? 2 * kTile : 0) + (x >= 1 ? kTile : 0);
     mbar_arrive_expect_tx(bar, bytes);
     if (x < nc) {
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
     if (x >= 1) tma_load_3d(tKQ(x) + kTile, &maps.q, bar, 0, (x - 1) * CB, (int)bh);
     tma_issued = x + 1;
   };
-  auto tma_parity = [&](int x) { return (uint32_t)((x >> 2) & 1); };
+  auto tma_parity = [&](int x) { return (uint32_t)((x / NST) & 1); };
   const uint32_t idescN16 = idesc_bf16_f32(128, 16, false, false);
   const uint32_t idescN32 = idesc_bf16_f32(128, 32, false, false);
   const uint32_t idescW = idesc_bf16_f32(128, 64, false, true);
@@ -249,38 +255,36 @@ __global__ void __launch_bounds__(tc::NT, 3)
                   smem_desc(ar + kk * 32, 16, 1024, kLayoutSw128), n == 32 ? idescN32 : idescN16,
                   kk > 0 ? 1u : 0u);
   };
-  // Gram for chunk x: A = [K_{x+1}; Q_x] (stage x+1; the 128-row operand reads
-  // on into the following shared memory, whose rows land in TMEM lanes that
-  // are never read), B = K_x:  lanes 0-15 k_{x+1,m}.k_{x,j}, lanes 16-31 q_{x,i}.k_{x,j}
+  // Gram for chunk x into TMEM columns 16 (x & 1) of the second allocation:
+  // A = [K_{x+1}; Q_x] (stage x+1; the 128-row operand reads on into the
+  // following shared memory, whose rows land in TMEM lanes that are never
+  // read), B = K_x:  lanes 0-15 k_{x+1,m}.k_{x,j}, lanes 16-31 q_{x,i}.k_{x,j}
   auto mma_gram = [&](uint32_t tmem2, int x) {
     const uint32_t a = smem_u32(tKQ(x + 1)), b = smem_u32(tKQ(x));
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ss(tmem2, smem_desc(a + kk * 32, 16, 1024, kLayoutSw128),
+      mma_bf16_ss(tmem2 + 16u * (uint32_t)(x & 1), smem_desc(a + kk * 32, 16, 1024, kLayoutSw128),
                   smem_desc(b + kk * 32, 16, 1024, kLayoutSw128), idescN16, kk > 0 ? 1u : 0u);
   };
-  // bulk warp with TMEM lane quarter 0: Gram rows -> Xg_{x+1} (bf16, rows m,
-  // zero past the chunk lengths) and M_x (bf16, causal, rows i)
+  // bulk warp with TMEM lane quarter 0: Gram rows -> the 32-row operand
+  // [Xg_{x+1}; M_x] (bf16): rows 0-15 Xg_{x+1}[m][j] (zero past the chunk
+  // lengths), rows 16-31 M_x[i][j] (causal), row = lane
   auto gram_extract = [&](uint32_t tmem2, int x) {
     float r[16];
-    tmem_ld16(tmem2, r);
+    tmem_ld16(tmem2 + 16u * (uint32_t)(x & 1), r);
     tmem_wait_ld();
     const int n0 = chunk_len(x);
     float v[16];
-    unsigned char* dst;
-    int row;
-    if (lane < CB) {  // Xg_{x+1}[m][j], m = lane
+    if (lane < CB) {
       const int n1 = (x + 1 < nc) ? chunk_len(x + 1) : 0;
-      row = lane;
 #pragma unroll
-      for (int j = 0; j < CB; ++j) v[j] = (row < n1 && j < n0) ? r[j] : 0.f;
-      dst = xgm(x + 1);
-    } else {  // M_x[i][j], i = lane - 16
-      row = lane - CB;
+      for (int j = 0; j < CB; ++j) v[j] = (lane < n1 && j < n0) ? r[j] : 0.f;
+    } else {
+      const int i = lane - CB;
 #pragma unroll
-      for (int j = 0; j < CB; ++j) v[j] = (j <= row && row < n0) ? r[j] : 0.f;
-      dst = mmat(x);
+      for (int j = 0; j < CB; ++j) v[j] = (j <= i && i < n0) ? r[j] : 0.f;
     }
+    unsigned char* dst = xm(x);
 #pragma unroll
     for (int j0 = 0; j0 < CB; j0 += 8) {
       uint4 u;
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
       u.y = pack_bf16(v[j0 + 2], v[j0 + 3]);
       u.z = pack_bf16(v[j0 + 4], v[j0 + 5]);
       u.w = pack_bf16(v[j0 + 6], v[j0 + 7]);
-      *reinterpret_cast<uint4*>(dst + core_off(row, j0)) = u;
+      *reinterpret_cast<uint4*>(dst + core_off(lane, j0)) = u;
     }
     fence_proxy_async_smem();
   };
@@ -372,30 +376,35 @@ __global__ void __launch_bounds__(tc::NT, 3)
     tmem_wait_st();
     fence_proxy_async_smem();
   }
-  // tiles of chunks 0 and 1 (chunk 1 carries Q_0)
+  // tiles of chunks 0, 1 (chunk 1 carries Q_0) and, for the Gram of chunk 1, 2
   bool bad = false;
   if (!mbar_wait_bounded(&bar_tma[0], 0, lim)) bad = true;
   if (!mbar_wait_bounded(&bar_tma[1], 0, lim)) bad = true;
+  if (nc > 1 && !mbar_wait_bounded(&bar_tma[2], 0, lim)) bad = true;
   tc_fence_before();
   const bool pro_bad = __syncthreads_or(bad);
   tc_fence_after();
   if (pro_bad && tid == 0) fail();
   if (issuer && !pro_bad) {
     mma_gram(tmem2, 0);                        // Xg_1, M_0
-    mma_commit(bar_gram);
+    if (nc > 1) mma_gram(tmem2, 1);            // Xg_2, M_1
     mma_ws(tmem + col_p(0), tKQ(0), 16);       // P_0
     mma_ws(tmem + col_p(1), tKQ(1), 32);       // [P_1 | Q0_0]
     mma_commit(bar_pro);
   }
   if (warp == 4 && !pro_bad) {
-    if (mbar_wait_bounded(bar_gram, 0, lim)) {
+    if (mbar_wait_bounded(bar_pro, 0, lim)) {
       tc_fence_after();
       gram_extract(tmem2, 0);
+      if (nc > 1) gram_extract(tmem2, 1);
     } else if (lane == 0) {
       fail();
     }
   }
-  if (is_bulk && !pro_bad) mbar_arrive(&bar_xm[0]);
+  if (is_bulk && !pro_bad) {
+    mbar_arrive(&bar_xm[0]);
+    mbar_arrive(&bar_xm[1]);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -523,7 +532,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
     for (int c = 0; c < nc; ++c) {
       const bool upd = sFlag[c & (kSR - 1)] != 0;
       if ((c & 7) == 0) pre = fetch_block(c + 16);
-      // ---- MMA2/3/c of chunk c complete ----
+      // ---- MMAc and MMA3 of chunk c complete ----
       bool ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
       if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
         if (gt == 0) fail();
@@ -572,6 +581,24 @@ __global__ void __launch_bounds__(tc::NT, 3)
       }
       tc_fence_before();
       mbar_arrive(bar_wb);
+      // ---- Gram of chunk c+2 -> [Xg_{c+3}; M_{c+2}]. Its buffer held the
+      // operand of chunk c's MMAc, complete since bar_w ----
+      if (c + 2 < nc) {
+        ok = true;
+        if (wq == 0) {
+          ok = mbar_wait_bounded(bar_gram, (uint32_t)(c & 1), lim);
+          if (ok) {
+            tc_fence_after();
+            gram_extract(tmem2, c + 2);
+          }
+        }
+        tc_fence_before();
+        if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
+          if (gt == 0) fail();
+          break;
+        }
+        mbar_arrive(&bar_xm[c & 1]);
+      }
       // ---- outputs o_c = gate * O_c^T ----
       {
         float ov[8];
@@ -586,67 +613,59 @@ __global__ void __launch_bounds__(tc::NT, 3)
           if (t < n) dst[(size_t)t * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
         }
       }
-      // ---- Gram of chunk c+1 -> Xg_{c+2}, M_{c+1} ----
-      if (c + 1 < nc) {
-        ok = true;
-        if (wq == 0) {
-          ok = mbar_wait_bounded(bar_gram, (uint32_t)((c + 1) & 1), lim);
-          if (ok) {
-            tc_fence_after();
-            gram_extract(tmem2, c + 1);
-          }
-        }
-        tc_fence_before();
-        if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
-          if (gt == 0) fail();
-          break;
-        }
-        mbar_arrive(&bar_xm[(c + 1) & 1]);
-      }
       if ((c & 7) == 4) store_block(c + 12, pre);
     }
   } else if (issuer && run) {
     // =========================== issuer ===========================
     for (int c = 0; c < nc; ++c) {
       const bool upd = sFlag[c & (kSR - 1)] != 0;
-      // Aneg_c, and the operands Xg_{c+1}, M_c
-      bool ok = mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim) &&
-                mbar_wait_bounded(&bar_xm[c & 1], (uint32_t)((c >> 1) & 1), lim);
+      const bool next = c + 1 < nc;
+      // the operand [Xg_{c+1}; M_c] (its Gram has left TMEM slot c & 1), Aneg_c
+      bool ok = mbar_wait_bounded(&bar_xm[c & 1], (uint32_t)((c >> 1) & 1), lim) &&
+                mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim);
       if (!ok || *sAbort) {
         fail();
         break;
       }
       tc_fence_after();
-      if (upd) {
-        const uint64_t da = smem_desc(smem_u32(aneg(c)), 128, 256, kLayoutNone);
-        mma_bf16_ss(tmem + col_o((c + 1) & 1), da,
-                    smem_desc(smem_u32(mmat(c)), 128, 256, kLayoutNone), idescN16, 1u);
-        if (c + 1 < nc)
-          mma_bf16_ss(tmem + col_p((c + 1) & 1), da,
-                      smem_desc(smem_u32(xgm(c + 1)), 128, 256, kLayoutNone), idescN16, 1u);
+      const uint64_t da = smem_desc(smem_u32(aneg(c)), 128, 256, kLayoutNone);
+      if (upd)
+        mma_bf16_ss(tmem + col_p((c + 1) & 1), da,
+                    smem_desc(smem_u32(xm(c)), 128, 256, kLayoutNone), idescN32, 1u);
+      if (next) mma_commit(&bar_z[(c + 1) & 1]);
+      if (upd)
         mma_bf16_ss(tmem + kColW, da, smem_desc(smem_u32(tKQ(c)), 2048, 1024, kLayoutSw128),
                     idescW, 1u);
-      }
-      if (c + 1 < nc) mma_commit(&bar_z[(c + 1) & 1]);
       mma_commit(bar_w);
       ++w_issued;
 
-      if (c + 1 < nc) {
-        // W_{s,c+1} in bf16 and the tiles of stage c+2 = {K_{c+2}, Q_{c+1}}
-        ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) &&
-             mbar_wait_bounded(&bar_tma[(c + 2) & (NST - 1)], tma_parity(c + 2), lim);
+      if (c + 2 < nc) {
+        // Gram of chunk c+2 (stages c+2, c+3) into TMEM slot c & 1
+        ok = mbar_wait_bounded(&bar_tma[(c + 2) % NST], tma_parity(c + 2), lim) &&
+             mbar_wait_bounded(&bar_tma[(c + 3) % NST], tma_parity(c + 3), lim);
         if (!ok || *sAbort) {
           fail();
           break;
         }
         tc_fence_after();
-        mma_gram(tmem2, c + 1);                                     // Xg_{c+2}, M_{c+1}
+        mma_gram(tmem2, c + 2);
         mma_commit(bar_gram);
-        mma_ws(tmem + col_p((c + 2) & 1), tKQ(c + 2), 32);          // [P_{c+2} | Q0_{c+1}]
+      }
+      if (next) {
+        // W_{s,c+1} in bf16, then [P_{c+2} | Q0_{c+1}] = W_{s,c+1} [K_{c+2}; Q_{c+1}]^T
+        ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) &&
+             mbar_wait_bounded(&bar_tma[(c + 2) % NST], tma_parity(c + 2), lim);
+        if (!ok || *sAbort) {
+          fail();
+          break;
+        }
+        tc_fence_after();
+        mma_ws(tmem + col_p((c + 2) & 1), tKQ(c + 2), 32);
       }
       // refill stage c % NST with load c + NST. Its K_c was last read by MMA3 of
       // this chunk, which completed before the bulk warps signalled bar_wb
-      // (c + NST <= nc implies c + 1 < nc, so that wait happened above).
+      // (c + NST <= nc implies c + 1 < nc, so that wait happened above), and by
+      // the Gram of chunk c, extracted before bar_xm of this chunk.
       if (c + NST <= nc) {
         fence_proxy_async_smem();
         issue_tma(c + NST);
@@ -666,7 +685,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
       if (w_issued > 0) mbar_wait_bounded(bar_w, (uint32_t)((w_issued - 1) & 1), drain_lim);
       mbar_wait_bounded(bar_w, (uint32_t)(w_issued & 1), drain_lim);
       for (int x = (tma_issued > NST ? tma_issued - NST : 0); x < tma_issued; ++x)
-        mbar_wait_bounded(&bar_tma[x & (NST - 1)], tma_parity(x), drain_lim);
+        mbar_wait_bounded(&bar_tma[x % NST], tma_parity(x), drain_lim);
     }
   } else if (is_bulk && wq < 2) {
     const int row = wq * 32 + lane;  // W_T from the rows of copy 0
