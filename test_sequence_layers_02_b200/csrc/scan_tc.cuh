@@ -20,14 +20,14 @@
 //               one shuffle round of shifted moments), write Aneg_k (bf16).
 //   bulk 4-7    W (fp32 TMEM) -> bf16 operand W_s; Gram products two chunks
 //               ahead -> bf16 operand [Xg_{c+3}; M_{c+2}]; outputs o_c = gate * O_c^T;
-//               per-chunk scalars.
-//   issuer 8    (one thread) every tcgen05.mma and TMA, per chunk c in this order:
+//               per-chunk scalars; one thread issues every TMA load of chunk
+//               x = {K_x, Q_{x-1}, V_x}, NST chunks ahead.
+//   issuer 8    (one thread) every tcgen05.mma, per chunk c in this order:
 //               MMAc [P_{c+1} | O_c]^T += Aneg_c [Xg_{c+1}; M_c]^T (one N = 32 MMA,
 //               committed alone: the chain's next Z waits for nothing else);
 //               MMA3 W += Aneg_c K_c (K as an MN-major operand); the Gram
 //               [K_{c+3}; Q_{c+2}] K_{c+2}^T; once W_s is refreshed, MMA1
-//               [P_{c+2} | Q0_{c+1}]^T = W_s [K_{c+2}; Q_{c+1}]^T; TMA of chunk
-//               x = {K_x, Q_{x-1}, V_x}, NST chunks ahead.
+//               [P_{c+2} | Q0_{c+1}]^T = W_s [K_{c+2}; Q_{c+1}]^T.
 // One chunk period is then the longer of two loops from MMAc: the chain's
 // (Z -> LayerNorm -> Aneg) and the W refresh's (MMA3 -> bf16 W_s -> MMA1,
 // which must precede the next MMAc); the Grams and the outputs stay off both.
@@ -38,7 +38,7 @@
 // Handoffs are mbarriers in rings of two (a producer can never run two phases
 // ahead of its consumer). Every wait is bounded: on expiry the CTA records the
 // timeout status, all warps leave their loops, the issuer drains its MMAs and
-// copies (with a bound of its own) and TMEM is freed.
+// the TMA thread its copies (each with a bound of its own) and TMEM is freed.
 #pragma once
 
 #include "common.cuh"
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + oBar);  // [NST] chunk x -> x % NST
   uint64_t* bar_g = bar_tma + NST;   // [2] Aneg_k written (chain, 128 arrivals)
   uint64_t* bar_z = bar_g + 2;       // [2] Z_k complete in TMEM (commit)
-  uint64_t* bar_xm = bar_z + 2;      // [2] [Xg_{x+1}; M_x] written (bulk, 128 arrivals)
+  uint64_t* bar_xm = bar_z + 2;      // [2] [Xg_{x+1}; M_x] written (bulk warp 4, 32 arrivals)
   uint64_t* bar_w = bar_xm + 2;      // a chunk's MMAc and MMA3 complete (commit)
   uint64_t* bar_wb = bar_w + 1;      // W_s bf16 refreshed (bulk, 128 arrivals)
   uint64_t* bar_gram = bar_wb + 1;   // Gram MMA complete (commit)
@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
   const bool is_chain = warp < 4;
   const bool is_bulk = warp >= 4 && warp < 8;
   const bool issuer = (tid == 256);
+  const bool tma_thread = (tid == 224);        // bulk warp 7, lane 0
   const int wq = warp & 3;                     // TMEM lane quarter of this warp
   const uint32_t tlane = (uint32_t)(wq * 32) << 16;
   const int fm = (wq & 1) * 32 + lane;         // feature-major role: feature
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_g[s], 128);
       mbar_init(&bar_z[s], 1);
-      mbar_init(&bar_xm[s], 128);
+      mbar_init(&bar_xm[s], 32);
     }
     mbar_init(bar_w, 1);
     mbar_init(bar_wb, 128);
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
   tc_fence_after();
   const uint32_t tmem = sTmem[0];
   const uint32_t tmem2 = sTmem[1];
-  if (issuer) {
+  if (tma_thread) {
     prefetch_tensormap(&maps.q);
     prefetch_tensormap(&maps.k);
     prefetch_tensormap(&maps.v);
@@ -401,7 +402,7 @@ __global__ void __launch_bounds__(tc::NT, 3)
       fail();
     }
   }
-  if (is_bulk && !pro_bad) {
+  if (warp == 4 && !pro_bad) {
     mbar_arrive(&bar_xm[0]);
     mbar_arrive(&bar_xm[1]);
   }
@@ -581,23 +582,25 @@ __global__ void __launch_bounds__(tc::NT, 3)
       }
       tc_fence_before();
       mbar_arrive(bar_wb);
+      // refill stage c % NST with load c + NST: every reader of its tiles (MMA1
+      // and the Grams of chunks c-1 and c, MMA3 of chunk c, the chain's V_c)
+      // completed before bar_w of this chunk
+      if (tma_thread && c + NST <= nc) {
+        fence_proxy_async_smem();
+        issue_tma(c + NST);
+      }
       // ---- Gram of chunk c+2 -> [Xg_{c+3}; M_{c+2}]. Its buffer held the
       // operand of chunk c's MMAc, complete since bar_w ----
-      if (c + 2 < nc) {
-        ok = true;
-        if (wq == 0) {
-          ok = mbar_wait_bounded(bar_gram, (uint32_t)(c & 1), lim);
-          if (ok) {
-            tc_fence_after();
-            gram_extract(tmem2, c + 2);
-          }
+      // (warp 4 alone: the other bulk warps go on to the outputs; a failed
+      // wait is seen by all at the next bar_any)
+      if (c + 2 < nc && wq == 0) {
+        if (mbar_wait_bounded(bar_gram, (uint32_t)(c & 1), lim)) {
+          tc_fence_after();
+          gram_extract(tmem2, c + 2);
+          mbar_arrive(&bar_xm[c & 1]);
+        } else if (lane == 0) {
+          fail();
         }
-        tc_fence_before();
-        if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
-          if (gt == 0) fail();
-          break;
-        }
-        mbar_arrive(&bar_xm[c & 1]);
       }
       // ---- outputs o_c = gate * O_c^T ----
       {
@@ -662,14 +665,6 @@ __global__ void __launch_bounds__(tc::NT, 3)
         tc_fence_after();
         mma_ws(tmem + col_p((c + 2) & 1), tKQ(c + 2), 32);
       }
-      // refill stage c % NST with load c + NST. Its K_c was last read by MMA3 of
-      // this chunk, which completed before the bulk warps signalled bar_wb
-      // (c + NST <= nc implies c + 1 < nc, so that wait happened above), and by
-      // the Gram of chunk c, extracted before bar_xm of this chunk.
-      if (c + NST <= nc) {
-        fence_proxy_async_smem();
-        issue_tma(c + NST);
-      }
     }
   }
 
@@ -679,11 +674,12 @@ __global__ void __launch_bounds__(tc::NT, 3)
   tc_fence_after();
   if (*sAbort) {
     if (issuer) {
-      // all MMAs this thread issued (one commit tracks them all), then every
-      // TMA stage that may still be loading; each wait has its own bound
+      // all MMAs this thread issued (one commit tracks them all)
       mma_commit(bar_w);
       if (w_issued > 0) mbar_wait_bounded(bar_w, (uint32_t)((w_issued - 1) & 1), drain_lim);
       mbar_wait_bounded(bar_w, (uint32_t)(w_issued & 1), drain_lim);
+    } else if (tma_thread) {
+      // every TMA stage that may still be loading
       for (int x = (tma_issued > NST ? tma_issued - NST : 0); x < tma_issued; ++x)
         mbar_wait_bounded(&bar_tma[x % NST], tma_parity(x), drain_lim);
     }
