@@ -135,8 +135,11 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_dst, float a, float 
       : "memory");
 }
 
+// One CTA per SM, as the shared memory request already forces: the explicit
+// minimum in the launch bounds lets the compiler give every thread up to 255
+// registers.
 template <typename InT, typename OutT, int GM, int CS>
-__global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT)
+__global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT, 1)
     scan_cluster_kernel(const ScanParams p) {
   namespace cg = cooperative_groups;
   using L = ClusterLayout<InT, CS>;

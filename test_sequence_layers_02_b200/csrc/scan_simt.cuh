@@ -767,8 +767,11 @@ struct Chain {
   }
 };
 
+// IH = 1 runs three CTAs per SM when heads are many (the bound caps registers
+// accordingly); IH = 2 is the few-heads form, one CTA per SM.
 template <int D, typename InT, typename OutT, bool MINIB, int GM, int IH>
-__global__ void __launch_bounds__(2 * D * IH + 32) scan_simt_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(2 * D * IH + 32, IH == 1 ? 3 : 1)
+    scan_simt_kernel(const ScanParams p) {
   using L = PipeLayout<D, InT, IH>;
   constexpr int NBT = L::NBT;
   constexpr int EPL = (D + 31) / 32;
