@@ -133,8 +133,10 @@ constexpr int kBarBulk = 3;
 
 }  // namespace tc
 
-template <typename OutT, int GM>
-__global__ void __launch_bounds__(tc::NT, 3)
+// MINB = 3: three CTAs share an SM (heads above the SM count; 72 registers);
+// MINB = 1: one CTA per SM, for up to one head per SM (more registers).
+template <typename OutT, int GM, int MINB>
+__global__ void __launch_bounds__(tc::NT, MINB)
     scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps) {
   using namespace tc;
   using namespace sm100;

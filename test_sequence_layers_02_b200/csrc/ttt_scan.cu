@@ -89,6 +89,18 @@ bool encode_qkv_map(CUtensorMap* map, const void* base, int T, long long heads, 
   return r == CUDA_SUCCESS;
 }
 
+// SMs of the current device (0 if the query fails).
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
 template <typename OutT, int GM>
 int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   ttt::TcMaps maps;
@@ -97,7 +109,10 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
       !encode_qkv_map(&maps.k, p.k, p.T, heads, true) ||
       !encode_qkv_map(&maps.v, p.v, p.T, heads, false))
     return TTT_ERR_CUDA;
-  auto kernel = ttt::scan_tc_kernel<OutT, GM>;
+  // up to one head per SM: the one-CTA-per-SM build (more registers per
+  // thread); beyond that, three CTAs share an SM
+  auto kernel = heads <= device_sm_count() ? ttt::scan_tc_kernel<OutT, GM, 1>
+                                           : ttt::scan_tc_kernel<OutT, GM, 3>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ttt::tc::kSmemBytes) != cudaSuccess)
     return TTT_ERR_CUDA;

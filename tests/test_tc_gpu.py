@@ -35,6 +35,22 @@ def test_tc_matches_oracle(grad, out_bf16, T):
     assert_rrms(W_T, rW, "W_T")
 
 
+@pytest.mark.parametrize("grad", [LNJAC, 0, NO_LN], ids=["lnjac", "simple", "no_ln"])
+@pytest.mark.parametrize("BH", [(4, 37), (10, 15)], ids=["148heads", "150heads"])
+def test_tc_both_occupancy_builds(grad, BH):
+    """Up to one head per SM runs the one-CTA-per-SM build, more heads the
+    three-CTAs-per-SM build (B200: 148 SMs); both against the oracle, with a
+    ragged tail and a SKIP/UPDATE mask."""
+    B, H = BH
+    inp = make_inputs(B, H, 40, 64, seed=250 + grad + B, random_affine=True, in_bf16=True,
+                      mask_p=0.7, b=16)
+    o, W_T = gpu_scan(inp, in_bf16=True, out_bf16=True, eps=1e-6, b=16, minibatch=True,
+                      lnjac=bool(grad & LNJAC), no_ln=bool(grad & NO_LN))
+    ro, rW = oracle_scan(inp, eps=1e-6, mode=MINIB | grad, b=16)
+    assert_rrms(o, ro, "o")
+    assert_rrms(W_T, rW, "W_T")
+
+
 @pytest.mark.parametrize("T", [64, 77])
 def test_tc_mask_is_bit_exact_on_skipped_chunks(T):
     B, H, b = 2, 3, 16
