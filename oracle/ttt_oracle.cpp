@@ -84,10 +84,14 @@ S sigmoid(S x) {
 }
 
 // Inner LayerNorm forward and the inner gradient with respect to z.
-// Writes pred (may be null), G, and xhat (may be null).
+// Writes pred (may be null), G, and xhat (may be null). With the ablation
+// gradient, norms (may be null) receives the L2 norms of the full
+// Jacobian-form gradient and of the ablated gradient before any norm matching
+// (their ratio is the gradient norm ratio of "Error Correction in Trained TTT
+// Layers", Abstract).
 template <typename S>
 void ln_and_grad(const S* z, const S* v, const S* gamma, const S* beta, int d,
-                 S eps, unsigned mode, S* pred_out, S* G, S* xhat_out) {
+                 S eps, unsigned mode, S* pred_out, S* G, S* xhat_out, S* norms = nullptr) {
   std::vector<S> pred(d), xhat(d);
   if (mode & kNoLayerNorm) {
     for (int f = 0; f < d; ++f) {
@@ -125,12 +129,16 @@ void ln_and_grad(const S* z, const S* v, const S* gamma, const S* beta, int d,
       if (mode & kGradAblate) {
         for (int f = 0; f < d; ++f) g[f] = gamma[f] * (-v[f]);
         jacobian_t(g, G);
+        S n_full = 0, n_abl = 0;
+        for (int f = 0; f < d; ++f) {
+          n_full += full[f] * full[f];
+          n_abl += G[f] * G[f];
+        }
+        if (norms) {
+          norms[0] = std::sqrt(n_full);
+          norms[1] = std::sqrt(n_abl);
+        }
         if (mode & kNormMatch) {
-          S n_full = 0, n_abl = 0;
-          for (int f = 0; f < d; ++f) {
-            n_full += full[f] * full[f];
-            n_abl += G[f] * G[f];
-          }
           const S scale = n_abl > S(0) ? std::sqrt(n_full / n_abl) : S(0);
           for (int f = 0; f < d; ++f) G[f] *= scale;
         }
@@ -177,7 +185,8 @@ template <typename S>
 void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
                    const S* gate_logit, const S* W0, const S* gamma,
                    const S* beta, int T, int d, S eps, unsigned mode, int b,
-                   const unsigned char* mask_row, S* o, S* W_T, S* W_chunks) {
+                   const unsigned char* mask_row, S* o, S* W_T, S* W_chunks,
+                   S* gnorms) {
   const int n_chunks = (T + b - 1) / b;
   std::vector<S> W(W0, W0 + (size_t)d * d);
   std::vector<S> z(d), G(d), Wq(d);
@@ -197,7 +206,7 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
         const S eta = update ? sigmoid(eta_logit[t]) / S(d) : S(0);
         matvec(W.data(), kt, d, z.data());
         ln_and_grad(z.data(), vt, gamma, beta, d, eps, mode, (S*)nullptr,
-                    G.data(), (S*)nullptr);
+                    G.data(), (S*)nullptr, gnorms ? gnorms + (size_t)t * 2 : (S*)nullptr);
         for (int r = 0; r < d; ++r)
           for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];
         matvec(W.data(), qt, d, Wq.data());
@@ -213,7 +222,8 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
         etas[i] = update ? sigmoid(eta_logit[t]) / S(d) : S(0);
         matvec(W.data(), k + (size_t)t * d, d, z.data());
         ln_and_grad(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode,
-                    (S*)nullptr, Gs.data() + (size_t)i * d, (S*)nullptr);
+                    (S*)nullptr, Gs.data() + (size_t)i * d, (S*)nullptr,
+                    gnorms ? gnorms + (size_t)t * 2 : (S*)nullptr);
       }
       for (int i = 0; i < n; ++i) {
         const int t = t0 + i;
@@ -243,8 +253,10 @@ template <typename S>
 int forward(const S* q, const S* k, const S* v, const S* eta_logit,
             const S* gate_logit, const S* W0, const S* gamma, const S* beta,
             int B, int H, int T, int d, S eps, unsigned mode, int b,
-            const unsigned char* mask, S* o, S* W_T, S* W_chunks, int nthreads) {
+            const unsigned char* mask, S* o, S* W_T, S* W_chunks, S* grad_norms,
+            int nthreads) {
   if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return -1;
+  if (grad_norms && !(mode & kGradAblate)) return -1;
   if ((mode & kGradAblate) && (mode & kNoLayerNorm)) return -1;
   if ((mode & kNormMatch) && !(mode & kGradAblate)) return -1;
   if (!q || !k || !v || !eta_logit || !W0 || !o || !W_T) return -1;
@@ -268,7 +280,8 @@ int forward(const S* q, const S* k, const S* v, const S* eta_logit,
                      mask ? mask + (size_t)bi * n_chunks : nullptr,
                      o + tok * d, W_T + (size_t)bh * d * d,
                      W_chunks ? W_chunks + (size_t)bh * (n_chunks + 1) * d * d
-                              : nullptr);
+                              : nullptr,
+                     grad_norms ? grad_norms + tok * 2 : nullptr);
   }
   return 0;
 }
@@ -282,7 +295,10 @@ extern "C" {
 //   gate_logit: [B, H, T], or [B, H, T, d] with mode bit 1 << 6 (per-channel gate);
 //   W0, W_T: [B, H, d, d] with z = W k;  gamma, beta: [H, d];
 //   mask: [B, ceil(T/b)] bytes, 1 = UPDATE, 0 = SKIP;
-//   W_chunks: [B, H, ceil(T/b) + 1, d, d], W before each chunk and after the last.
+//   W_chunks: [B, H, ceil(T/b) + 1, d, d], W before each chunk and after the last;
+//   grad_norms: [B, H, T, 2] (ablation gradient only, may be null): per token the
+//     L2 norm of the full Jacobian-form gradient and of the ablated gradient
+//     before any norm matching.
 // Returns 0, or -1 on an invalid argument. nthreads <= 0 keeps the OpenMP default.
 int ttt_oracle_forward_f64(const double* q, const double* k, const double* v,
                            const double* eta_logit, const double* gate_logit,
@@ -290,9 +306,9 @@ int ttt_oracle_forward_f64(const double* q, const double* k, const double* v,
                            const double* beta, int B, int H, int T, int d,
                            double eps, unsigned mode, int b,
                            const unsigned char* mask, double* o, double* W_T,
-                           double* W_chunks, int nthreads) {
+                           double* W_chunks, double* grad_norms, int nthreads) {
   return forward<double>(q, k, v, eta_logit, gate_logit, W0, gamma, beta, B, H,
-                         T, d, eps, mode, b, mask, o, W_T, W_chunks, nthreads);
+                         T, d, eps, mode, b, mask, o, W_T, W_chunks, grad_norms, nthreads);
 }
 
 // The same definition evaluated in float (conditioning-floor measurement only).
@@ -302,20 +318,22 @@ int ttt_oracle_forward_f32(const float* q, const float* k, const float* v,
                            const float* beta, int B, int H, int T, int d,
                            float eps, unsigned mode, int b,
                            const unsigned char* mask, float* o, float* W_T,
-                           float* W_chunks, int nthreads) {
+                           float* W_chunks, float* grad_norms, int nthreads) {
   return forward<float>(q, k, v, eta_logit, gate_logit, W0, gamma, beta, B, H,
-                        T, d, eps, mode, b, mask, o, W_T, W_chunks, nthreads);
+                        T, d, eps, mode, b, mask, o, W_T, W_chunks, grad_norms, nthreads);
 }
 
-// One inner LayerNorm + gradient evaluation on a single d-vector z (for pins).
+// One inner LayerNorm + gradient evaluation on a single d-vector z (for pins);
+// norms (may be null, ablation gradient only) as for grad_norms above.
 int ttt_oracle_lngrad_f64(const double* z, const double* v, const double* gamma,
                           const double* beta, int d, double eps, unsigned mode,
-                          double* pred, double* G, double* xhat) {
+                          double* pred, double* G, double* xhat, double* norms) {
   if (!z || !v || !G || d <= 0) return -1;
+  if (norms && !(mode & kGradAblate)) return -1;
   if ((mode & kGradAblate) && (mode & kNoLayerNorm)) return -1;
   if ((mode & kNormMatch) && !(mode & kGradAblate)) return -1;
   if (!(mode & kNoLayerNorm) && (!gamma || !beta)) return -1;
-  ln_and_grad<double>(z, v, gamma, beta, d, eps, mode, pred, G, xhat);
+  ln_and_grad<double>(z, v, gamma, beta, d, eps, mode, pred, G, xhat, norms);
   return 0;
 }
 

@@ -64,14 +64,14 @@ def _load():
         i = ctypes.c_int
         lib.ttt_oracle_forward_f64.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i,
                                                ctypes.c_double, ctypes.c_uint, i, u8p,
-                                               dp, dp, dp, i]
+                                               dp, dp, dp, dp, i]
         lib.ttt_oracle_forward_f64.restype = i
         lib.ttt_oracle_forward_f32.argtypes = [fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i,
                                                ctypes.c_float, ctypes.c_uint, i, u8p,
-                                               fp, fp, fp, i]
+                                               fp, fp, fp, fp, i]
         lib.ttt_oracle_forward_f32.restype = i
         lib.ttt_oracle_lngrad_f64.argtypes = [dp, dp, dp, dp, i, ctypes.c_double,
-                                              ctypes.c_uint, dp, dp, dp]
+                                              ctypes.c_uint, dp, dp, dp, dp]
         lib.ttt_oracle_lngrad_f64.restype = i
         lib.ttt_oracle_max_threads.argtypes = []
         lib.ttt_oracle_max_threads.restype = i
@@ -91,7 +91,7 @@ def max_threads() -> int:
 
 def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
             mode: int, b: int = 16, mask=None, want_chunks: bool = False,
-            nthreads: int = 0, dtype=np.float64):
+            want_grad_norms: bool = False, nthreads: int = 0, dtype=np.float64):
     """Run the oracle scan.
 
     Shapes: q, k, v [B, H, T, d]; eta_logit [B, H, T]; gate_logit [B, H, T], or
@@ -101,7 +101,10 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
 
     Returns ``(o, W_T)`` or ``(o, W_T, W_chunks)`` when ``want_chunks``; W_chunks
     has shape [B, H, ceil(T/b) + 1, d, d] and holds W before every chunk and
-    after the last one. ``dtype=np.float32`` runs the float twin.
+    after the last one. ``want_grad_norms`` (GRAD_ABLATE only) appends
+    ``grad_norms`` [B, H, T, 2]: per token the L2 norm of the full
+    Jacobian-form gradient and of the ablated gradient before any norm
+    matching. ``dtype=np.float32`` runs the float twin.
     """
     lib = _load()
     f64 = np.dtype(dtype) == np.float64
@@ -127,14 +130,16 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
     o = np.empty((B, H, T, d), dtype=dtype)
     W_T = np.empty((B, H, d, d), dtype=dtype)
     W_chunks = np.empty((B, H, n_chunks + 1, d, d), dtype=dtype) if want_chunks else None
+    gnorms = np.empty((B, H, T, 2), dtype=dtype) if want_grad_norms else None
     fn = lib.ttt_oracle_forward_f64 if f64 else lib.ttt_oracle_forward_f32
     rc = fn(_ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(eta_logit, ct),
             _ptr(gate_logit, ct), _ptr(W0, ct), _ptr(gamma, ct), _ptr(beta, ct),
             B, H, T, d, eps, mode, b, _ptr(mask, ctypes.c_ubyte),
-            _ptr(o, ct), _ptr(W_T, ct), _ptr(W_chunks, ct), nthreads)
+            _ptr(o, ct), _ptr(W_T, ct), _ptr(W_chunks, ct), _ptr(gnorms, ct), nthreads)
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
-    return (o, W_T, W_chunks) if want_chunks else (o, W_T)
+    out = (o, W_T) + ((W_chunks,) if want_chunks else ()) + ((gnorms,) if want_grad_norms else ())
+    return out
 
 
 def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float,
@@ -155,13 +160,14 @@ def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float,
     return o[:, :, 0], W_new
 
 
-def lngrad(z, v, gamma, beta, *, eps: float, mode: int):
+def lngrad(z, v, gamma, beta, *, eps: float, mode: int, want_norms: bool = False):
     """One inner LayerNorm + gradient on a single d-vector.
 
     Returns ``(pred, G, xhat)``; with NO_LN, pred = xhat = z and G = z - v.
     GRAD_ABLATE gives the ablation gradient (prediction removed, LayerNorm
     Jacobian kept), GRAD_NORM_MATCH additionally rescales it to the norm of the
-    full Jacobian-form gradient.
+    full Jacobian-form gradient. ``want_norms`` (GRAD_ABLATE only) appends the
+    pair (norm of the full gradient, norm of the ablated one before matching).
     """
     lib = _load()
     z = np.ascontiguousarray(z, dtype=np.float64)
@@ -170,12 +176,14 @@ def lngrad(z, v, gamma, beta, *, eps: float, mode: int):
     gamma = np.ones(d) if gamma is None else np.ascontiguousarray(gamma, dtype=np.float64)
     beta = np.zeros(d) if beta is None else np.ascontiguousarray(beta, dtype=np.float64)
     pred, G, xhat = np.empty(d), np.empty(d), np.empty(d)
+    norms = np.empty(2) if want_norms else None
     dp = ctypes.c_double
     rc = lib.ttt_oracle_lngrad_f64(_ptr(z, dp), _ptr(v, dp), _ptr(gamma, dp), _ptr(beta, dp),
-                                   d, eps, mode, _ptr(pred, dp), _ptr(G, dp), _ptr(xhat, dp))
+                                   d, eps, mode, _ptr(pred, dp), _ptr(G, dp), _ptr(xhat, dp),
+                                   _ptr(norms, dp))
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
-    return pred, G, xhat
+    return (pred, G, xhat, norms) if want_norms else (pred, G, xhat)
 
 
 def forward_heads(inputs: dict, heads, *, eps: float, mode: int, b: int,

@@ -37,9 +37,11 @@ MUTATIONS = [
     ("drop_beta", "pred[f] = gamma[f] * xhat[f] + beta[f];", "pred[f] = gamma[f] * xhat[f];"),
     ("ablation_keeps_beta", "for (int f = 0; f < d; ++f) g[f] = gamma[f] * (-v[f]);",
      "for (int f = 0; f < d; ++f) g[f] = gamma[f] * (beta[f] - v[f]);"),
-    ("ablation_without_jacobian", "        jacobian_t(g, G);\n        if (mode & kNormMatch) {",
-     "        for (int f = 0; f < d; ++f) G[f] = g[f];\n        if (mode & kNormMatch) {"),
+    ("ablation_without_jacobian", "        jacobian_t(g, G);\n        S n_full = 0, n_abl = 0;",
+     "        for (int f = 0; f < d; ++f) G[f] = g[f];\n        S n_full = 0, n_abl = 0;"),
     ("norm_match_without_sqrt", "std::sqrt(n_full / n_abl)", "(n_full / n_abl)"),
+    ("grad_norms_both_full", "norms[1] = std::sqrt(n_abl);", "norms[1] = std::sqrt(n_full);"),
+    ("grad_norms_squared", "norms[0] = std::sqrt(n_full);", "norms[0] = n_full;"),
     ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
     ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
      "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),

@@ -365,6 +365,69 @@ def test_norm_matching_keeps_direction_and_takes_the_full_norm():
     np.testing.assert_array_equal(G0, np.zeros(d))
 
 
+def test_grad_norms_are_the_norms_of_the_two_gradients():
+    """The norms output is (||G_full||, ||G_ablation||), the latter before any
+    norm matching; each gradient comes from its own (separately pinned) mode."""
+    rng = np.random.default_rng(31)
+    d = 32
+    z = rng.normal(size=d) * 0.2
+    gam = 1.0 + 0.1 * rng.normal(size=d)
+    bet = 0.1 * rng.normal(size=d)
+    v = rng.normal(size=d)
+    Gf = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_LNJAC)[1]
+    Ga = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_ABLATE)[1]
+    for nm in (0, GRAD_NORM_MATCH):
+        n = oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_ABLATE | nm, want_norms=True)[3]
+        np.testing.assert_allclose(n, [np.linalg.norm(Gf), np.linalg.norm(Ga)], rtol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.lngrad(z, v, gam, bet, eps=1e-6, mode=GRAD_LNJAC, want_norms=True)
+
+
+def test_grad_norm_ratio_is_one_at_released_init_in_the_zero_eps_limit():
+    """gamma = 1, beta = 0: the prediction-derived part cancels as eps -> 0
+    ("Error Correction in Trained TTT Layers", Abstract), so the ratio
+    ||G_ablation|| / ||G_full|| is 1 at eps = 0; for eps > 0 it differs from 1
+    by at most ||xhat eps / (s (var + eps))|| / ||G_full|| (triangle inequality
+    on the closed-form difference)."""
+    rng = np.random.default_rng(32)
+    d = 64
+    z = rng.normal(size=d) * 0.1 + 0.02
+    v = rng.normal(size=d)
+    n0 = oracle.lngrad(z, v, None, None, eps=0.0, mode=GRAD_ABLATE, want_norms=True)[3]
+    np.testing.assert_allclose(n0[1] / n0[0], 1.0, rtol=1e-12)
+    var = np.var(z)
+    for eps in (1e-2, 1e-4):
+        n = oracle.lngrad(z, v, None, None, eps=eps, mode=GRAD_ABLATE, want_norms=True)[3]
+        xhat = (z - z.mean()) / np.sqrt(var + eps)
+        gap = np.linalg.norm(xhat) * eps / (np.sqrt(var + eps) * (var + eps))
+        assert abs(n[1] - n[0]) <= gap * (1 + 1e-9) + 1e-15
+        assert abs(n[1] / n[0] - 1.0) > 1e-6   # the bound is not vacuous here
+
+
+@pytest.mark.parametrize("nm", [0, GRAD_NORM_MATCH], ids=["ablate", "ablate_nm"])
+def test_scan_grad_norms_follow_the_state_trajectory(nm):
+    """Per-token norms of the scan equal the single-vector norms at
+    z_t = W_{t-1} k_t, with W_{t-1} read from the per-token state snapshots
+    (b = 1) and the matvec done here in numpy."""
+    inp = f64(make_inputs(1, 2, 20, 16, seed=33, random_affine=True, mask_p=0.7, b=1))
+    mode = GRAD_ABLATE | nm
+    o, W_T, Wc, gn = oracle.forward(inp["q"], inp["k"], inp["v"], inp["eta_logit"],
+                                    inp["gate_logit"], inp["W0"], inp["gamma"], inp["beta"],
+                                    eps=1e-6, mode=mode, b=1, mask=inp["mask"], want_chunks=True,
+                                    want_grad_norms=True)
+    assert gn.shape == (1, 2, 20, 2)
+    for h in range(2):
+        for t in range(20):
+            z = Wc[0, h, t] @ inp["k"][0, h, t]
+            n = oracle.lngrad(z, inp["v"][0, h, t], inp["gamma"][h], inp["beta"][h], eps=1e-6,
+                              mode=mode, want_norms=True)[3]
+            np.testing.assert_allclose(gn[0, h, t], n, rtol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["eta_logit"], inp["gate_logit"],
+                       inp["W0"], inp["gamma"], inp["beta"], eps=1e-6, mode=GRAD_LNJAC, b=1,
+                       want_grad_norms=True)
+
+
 def test_ablation_mode_combinations():
     inp = f64(make_inputs(1, 1, 8, 16, seed=39))
     with pytest.raises(ValueError):
