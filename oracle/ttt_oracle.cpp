@@ -207,6 +207,8 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
         matvec(W.data(), kt, d, z.data());
         ln_and_grad(z.data(), vt, gamma, beta, d, eps, mode, (S*)nullptr,
                     G.data(), (S*)nullptr, gnorms ? gnorms + (size_t)t * 2 : (S*)nullptr);
+        // a SKIP chunk takes no gradient: its tokens report zero norms
+        if (gnorms && !update) gnorms[(size_t)t * 2] = gnorms[(size_t)t * 2 + 1] = S(0);
         for (int r = 0; r < d; ++r)
           for (int cc = 0; cc < d; ++cc) W[r * d + cc] -= eta * G[r] * kt[cc];
         matvec(W.data(), qt, d, Wq.data());
@@ -224,6 +226,7 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
         ln_and_grad(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode,
                     (S*)nullptr, Gs.data() + (size_t)i * d, (S*)nullptr,
                     gnorms ? gnorms + (size_t)t * 2 : (S*)nullptr);
+        if (gnorms && !update) gnorms[(size_t)t * 2] = gnorms[(size_t)t * 2 + 1] = S(0);
       }
       for (int i = 0; i < n; ++i) {
         const int t = t0 + i;
@@ -298,7 +301,8 @@ extern "C" {
 //   W_chunks: [B, H, ceil(T/b) + 1, d, d], W before each chunk and after the last;
 //   grad_norms: [B, H, T, 2] (ablation gradient only, may be null): per token the
 //     L2 norm of the full Jacobian-form gradient and of the ablated gradient
-//     before any norm matching.
+//     before any norm matching; zeros on the tokens of SKIP chunks, which take
+//     no gradient.
 // Returns 0, or -1 on an invalid argument. nthreads <= 0 keeps the OpenMP default.
 int ttt_oracle_forward_f64(const double* q, const double* k, const double* v,
                            const double* eta_logit, const double* gate_logit,

@@ -104,7 +104,8 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
     after the last one. ``want_grad_norms`` (GRAD_ABLATE only) appends
     ``grad_norms`` [B, H, T, 2]: per token the L2 norm of the full
     Jacobian-form gradient and of the ablated gradient before any norm
-    matching. ``dtype=np.float32`` runs the float twin.
+    matching (zeros on SKIP chunks, which take no gradient).
+    ``dtype=np.float32`` runs the float twin.
     """
     lib = _load()
     f64 = np.dtype(dtype) == np.float64

@@ -408,7 +408,8 @@ def test_grad_norm_ratio_is_one_at_released_init_in_the_zero_eps_limit():
 def test_scan_grad_norms_follow_the_state_trajectory(nm):
     """Per-token norms of the scan equal the single-vector norms at
     z_t = W_{t-1} k_t, with W_{t-1} read from the per-token state snapshots
-    (b = 1) and the matvec done here in numpy."""
+    (b = 1) and the matvec done here in numpy; SKIP tokens take no gradient
+    and report zeros."""
     inp = f64(make_inputs(1, 2, 20, 16, seed=33, random_affine=True, mask_p=0.7, b=1))
     mode = GRAD_ABLATE | nm
     o, W_T, Wc, gn = oracle.forward(inp["q"], inp["k"], inp["v"], inp["eta_logit"],
@@ -416,8 +417,13 @@ def test_scan_grad_norms_follow_the_state_trajectory(nm):
                                     eps=1e-6, mode=mode, b=1, mask=inp["mask"], want_chunks=True,
                                     want_grad_norms=True)
     assert gn.shape == (1, 2, 20, 2)
+    m = inp["mask"][0]
+    assert 0 < m.sum() < 20
     for h in range(2):
         for t in range(20):
+            if not m[t]:
+                np.testing.assert_array_equal(gn[0, h, t], [0.0, 0.0])
+                continue
             z = Wc[0, h, t] @ inp["k"][0, h, t]
             n = oracle.lngrad(z, inp["v"][0, h, t], inp["gamma"][h], inp["beta"][h], eps=1e-6,
                               mode=mode, want_norms=True)[3]
