@@ -113,6 +113,28 @@ int ttt_scan_forward(const void* q, const void* k, const void* v,
                      float* W_chunks, void* cuda_stream);
 
 /*
+ * ttt_scan_forward, plus the per-token inner-gradient norms of the ablation
+ * study ("Error Correction in Trained TTT Layers", Abstract: the mean ratio of
+ * the ablated gradient's norm to the full gradient's norm). Needs
+ * TTT_GRAD_ABLATE in per-token mode (else TTT_ERR_INVALID_ARG / _UNSUPPORTED
+ * as for the scan); the outputs o, W_T and W_chunks are those of
+ * ttt_scan_forward with the same arguments.
+ *   grad_norms  device, [B, H, T, 2] fp32, written: per head-token the L2 norm
+ *               of the full LayerNorm-Jacobian gradient J^T(gamma*(pred - v))
+ *               and of the ablated gradient J^T(-gamma*v) before any norm
+ *               matching, both at that token's state W_{t-1}; zeros on the
+ *               tokens of SKIP chunks, which take no gradient. Must not
+ *               overlap any other argument; null only when B*H*T == 0.
+ * The call costs one more warp reduction per token on the gradient chain.
+ */
+int ttt_scan_forward_grad_norms(const void* q, const void* k, const void* v,
+                                const void* eta_logit, const void* gate_logit,
+                                const float* W0, const float* gamma, const float* beta,
+                                int B, int H, int T, int d, float eps, unsigned mode, int b,
+                                const unsigned char* mask, void* o, float* W_T,
+                                float* W_chunks, float* grad_norms, void* cuda_stream);
+
+/*
  * The kernel ttt_scan_forward would run for these sizes and mode bits on the
  * current CUDA device: one of the TTT_KERNEL_* identifiers above, or a negative
  * status (TTT_ERR_INVALID_ARG / TTT_ERR_UNSUPPORTED for arguments the scan

@@ -35,13 +35,15 @@ struct ScanParams {
   int gate_channel;        // gate_logit holds one logit per feature ([B, H, T, d])
   int ablate;              // ablation gradient (prediction removed, Jacobian kept)
   int norm_match;          // ... rescaled per token to the full gradient's norm
+  float* grad_norms;       // [B, H, T, 2] per-token gradient norms (ablation), may be null
 };
 
 // Gradient variant of the CUDA-core chain: 0 simplified, 1 LN Jacobian, 2 no
-// LayerNorm, 3 ablation, 4 ablation with per-token norm matching.
+// LayerNorm, 3 ablation, 4 ablation that also forms the full gradient's norm
+// (per-token norm matching, or the gradient norms asked for).
 inline int grad_variant(const ScanParams& p) {
   if (p.no_ln) return 2;
-  if (p.ablate) return p.norm_match ? 4 : 3;
+  if (p.ablate) return (p.norm_match || p.grad_norms) ? 4 : 3;
   return p.lnjac ? 1 : 0;
 }
 

@@ -296,7 +296,9 @@ __device__ __forceinline__ void butterfly(float (&v)[N]) {
 // 1 = through the LayerNorm Jacobian, 2 = no LayerNorm (G = z - v),
 // 3 = the ablation gradient (the Jacobian applied to -gamma * v, the
 // prediction removed; "Error Correction in Trained TTT Layers", Abstract),
-// 4 = the ablation rescaled per token to the norm of the GM 1 gradient.
+// 4 = the ablation together with the norm of the GM 1 gradient: rescaled per
+// token to that norm when nmatch, and both norms (full, ablated before any
+// rescaling) written to gnorm[2 i], gnorm[2 i + 1] when gnorm is not null.
 // Both Jacobian forms (1, 3, 4) give G a zero feature mean.
 // Reads Zpre (z before in-chunk corrections), A (eta_j k_m.k_j, j < m), V,
 // mu0 (mean of each Zpre row); writes G and, for GM 0, the mean of each G row.
@@ -308,7 +310,8 @@ __device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
                                             float* __restrict__ mGout, float eps,
                                             const float (&gam)[(D + 31) / 32],
                                             const float (&bet)[(D + 31) / 32], float Sgb, float Sb,
-                                            int lane) {
+                                            int lane, float* __restrict__ gnorm = nullptr,
+                                            bool nmatch = true) {
   using L = PipeLayout<D, InT>;
   constexpr int EPL = (D + 31) / 32;
   const float inv_d = 1.0f / (float)D;
@@ -389,7 +392,11 @@ __device__ __forceinline__ void chain_chunk(int n, const float* __restrict__ Z,
           }
         }
         butterfly<2>(nrm);
-        const float scale = nrm[1] > 0.f ? sqrtf(nrm[0] / nrm[1]) : 0.f;
+        if (gnorm != nullptr && lane == 0) {
+          gnorm[2 * i] = sqrtf(nrm[0]);
+          gnorm[2 * i + 1] = sqrtf(nrm[1]);
+        }
+        const float scale = !nmatch ? 1.f : (nrm[1] > 0.f ? sqrtf(nrm[0] / nrm[1]) : 0.f);
 #pragma unroll
         for (int e = 0; e < EPL; ++e) G[e] *= scale;
       } else if (GM == 1) {
@@ -816,6 +823,10 @@ __global__ void __launch_bounds__(2 * D * IH + 32, IH == 1 ? 3 : 1)
   const float inv_d = 1.0f / (float)D;
 
   auto chunk_len = [&](int c) { return min(C, T - c * C); };
+  // per-token gradient norms of chunk c ([n][2]), or null
+  auto gnorm_of = [&](int c) -> float* {
+    return p.grad_norms ? p.grad_norms + (tok0 + (size_t)c * C) * 2 : nullptr;
+  };
   auto tileK = [&](int c) { return sK + (c & 3) * L::TILE; };
   auto tileQ = [&](int c) { return sQ + (c & 1) * L::TILE; };
   auto tileV = [&](int c) { return sV + (c & 1) * L::TILE; };
@@ -912,10 +923,12 @@ __global__ void __launch_bounds__(2 * D * IH + 32, IH == 1 ? 3 : 1)
       if (sFlag[c & 3]) {
         chain_chunk<D, InT, MINIB, GM>(n, sZ + (c & 1) * kC * D, sA + (c & 1) * kC * kC,
                                        tileV(c), sMu + (c & 1) * kC, Gc, mGc, p.eps, gam, bet,
-                                       Sgb, Sb, lane);
+                                       Sgb, Sb, lane, gnorm_of(c), p.norm_match != 0);
       } else {
         for (int e = lane; e < kC * D; e += 32) Gc[e] = 0.f;
         if (lane < kC) mGc[lane] = 0.f;
+        // a SKIP chunk takes no gradient: zero norms for its tokens
+        if (float* gn = gnorm_of(c); gn != nullptr && lane < 2 * n) gn[lane] = 0.f;
       }
     } else {
       // ===== bulk work that does not wait for the chain =====

@@ -184,13 +184,14 @@ int ttt_check_device_status(void* cuda_stream) {
   return (h != 0 || hc != 0) ? TTT_ERR_DEVICE_TIMEOUT : TTT_OK;
 }
 
-int ttt_scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
-                     const void* gate_logit, const float* W0, const float* gamma,
-                     const float* beta, int B, int H, int T, int d, float eps, unsigned mode,
-                     int b, const unsigned char* mask, void* o, float* W_T, float* W_chunks,
-                     void* cuda_stream) {
+static int scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
+                        const void* gate_logit, const float* W0, const float* gamma,
+                        const float* beta, int B, int H, int T, int d, float eps, unsigned mode,
+                        int b, const unsigned char* mask, void* o, float* W_T, float* W_chunks,
+                        float* grad_norms, void* cuda_stream) {
   // ---- argument checks (nothing is launched on failure) ----
   if ((mode & ~kKnownModes) || bad_grad_mode(mode)) return TTT_ERR_INVALID_ARG;
+  if (grad_norms && !(mode & TTT_GRAD_ABLATE)) return TTT_ERR_INVALID_ARG;
   if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
   const bool no_ln = mode & TTT_NO_LN;
   // a pointer may be null only where the tensor it names is empty
@@ -199,7 +200,8 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   if (has_heads && (!W0 || !W_T)) return TTT_ERR_INVALID_ARG;
   if (has_heads && !no_ln && (!gamma || !beta)) return TTT_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) || !std::isfinite(eps)) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask, o, W_T, W_chunks};
+  const void* ptrs[] = {q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask, o, W_T, W_chunks,
+                        grad_norms};
   for (const void* p : ptrs)
     if (misaligned(p)) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
@@ -233,6 +235,14 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   if (W_chunks && (overlaps(W_chunks, wc_bytes, o, o_bytes) ||
                    overlaps(W_chunks, wc_bytes, W_T, w_bytes)))
     return TTT_ERR_INVALID_ARG;
+  if (grad_norms) {
+    const size_t gn_bytes = heads * (size_t)T * 2 * sizeof(float);
+    for (const Span& in : inputs)
+      if (overlaps(grad_norms, gn_bytes, in.p, in.n)) return TTT_ERR_INVALID_ARG;
+    if (overlaps(grad_norms, gn_bytes, o, o_bytes) || overlaps(grad_norms, gn_bytes, W_T, w_bytes) ||
+        (W_chunks && overlaps(grad_norms, gn_bytes, W_chunks, wc_bytes)))
+      return TTT_ERR_INVALID_ARG;
+  }
   if (heads == 0) return TTT_OK;
 
   ttt::ScanParams p{};
@@ -249,6 +259,7 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   p.ablate = (mode & TTT_GRAD_ABLATE) ? 1 : 0;
   p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
   p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
+  p.grad_norms = grad_norms;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int which = choose_kernel((long long)heads, T, d, mode, b);
@@ -266,6 +277,26 @@ int ttt_scan_forward(const void* q, const void* k, const void* v, const void* et
   }
   return (mode & TTT_IN_BF16) ? ttt::launch_simt_bf16in(p, mode, d, stream)
                               : ttt::launch_simt_f32in(p, mode, d, stream);
+}
+
+int ttt_scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
+                     const void* gate_logit, const float* W0, const float* gamma,
+                     const float* beta, int B, int H, int T, int d, float eps, unsigned mode,
+                     int b, const unsigned char* mask, void* o, float* W_T, float* W_chunks,
+                     void* cuda_stream) {
+  return scan_forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, B, H, T, d, eps, mode, b,
+                      mask, o, W_T, W_chunks, nullptr, cuda_stream);
+}
+
+int ttt_scan_forward_grad_norms(const void* q, const void* k, const void* v,
+                                const void* eta_logit, const void* gate_logit, const float* W0,
+                                const float* gamma, const float* beta, int B, int H, int T,
+                                int d, float eps, unsigned mode, int b,
+                                const unsigned char* mask, void* o, float* W_T, float* W_chunks,
+                                float* grad_norms, void* cuda_stream) {
+  if (!grad_norms && (long long)B * H * T > 0) return TTT_ERR_INVALID_ARG;
+  return scan_forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, B, H, T, d, eps, mode, b,
+                      mask, o, W_T, W_chunks, grad_norms, cuda_stream);
 }
 
 int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b) {

@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
         L.ttt_scan_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
                                        ctypes.c_float, u, i, vp, vp, vp, vp, vp]
         L.ttt_scan_forward.restype = i
+        L.ttt_scan_forward_grad_norms.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                                  ctypes.c_float, u, i, vp, vp, vp, vp, vp, vp]
+        L.ttt_scan_forward_grad_norms.restype = i
         L.ttt_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i,
                                       ctypes.c_float, u, vp, vp, vp]
         L.ttt_decode_step.restype = i
@@ -102,7 +105,7 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
          minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
          b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
          force_simt: bool = False, single_cta: bool = False, ablate: bool = False,
-         norm_match: bool = False, want_chunks: bool = False,
+         norm_match: bool = False, want_chunks: bool = False, want_grad_norms: bool = False,
          o: Optional[torch.Tensor] = None, W_T: Optional[torch.Tensor] = None,
          stream: Optional[torch.cuda.Stream] = None):
     """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
@@ -116,6 +119,9 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     per-token mode on one CTA per head (see ``kernel_choice``). ``ablate``
     selects the ablation gradient (the LayerNorm Jacobian applied to
     -gamma * v), ``norm_match`` rescales it per token to the full gradient's norm.
+    ``want_grad_norms`` (with ``ablate``, per-token) also returns [B, H, T, 2]
+    fp32: per token the norms of the full and of the ablated gradient (zeros
+    on SKIP chunks), after W_T (and the chunk snapshots, if asked for).
 
     CUDA tensors run on ``stream`` (default: the current stream) and return
     without synchronising. CPU tensors take the end-to-end path: inputs are
@@ -168,11 +174,16 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
         wt_dev = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
     wc = (torch.empty((B, H, n_chunks + 1, d, d), dtype=torch.float32, device=q.device)
           if want_chunks else None)
+    gn = (torch.empty((B, H, T, 2), dtype=torch.float32, device=q.device)
+          if want_grad_norms else None)
     s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = lib().ttt_scan_forward(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W0), _ptr(gamma),
-        _ptr(beta), B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(o_dev), _ptr(wt_dev),
-        _ptr(wc), ctypes.c_void_p(s.cuda_stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W0), _ptr(gamma),
+            _ptr(beta), B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(o_dev),
+            _ptr(wt_dev), _ptr(wc))
+    if want_grad_norms:
+        rc = lib().ttt_scan_forward_grad_norms(*args, _ptr(gn), ctypes.c_void_p(s.cuda_stream))
+    else:
+        rc = lib().ttt_scan_forward(*args, ctypes.c_void_p(s.cuda_stream))
     if rc != TTT_OK:
         raise TTTScanError(rc)
     if host:
@@ -184,12 +195,10 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
         rc = check_device_status(s)
         if rc != TTT_OK:
             raise TTTScanError(rc, "device")
-        if want_chunks:
-            return o_h, wt_h, wc.cpu()
-        return o_h, wt_h
-    if want_chunks:
-        return o_dev, wt_dev, wc
-    return o_dev, wt_dev
+        extra = ((wc.cpu(),) if want_chunks else ()) + ((gn.cpu(),) if want_grad_norms else ())
+        return (o_h, wt_h) + extra
+    extra = ((wc,) if want_chunks else ()) + ((gn,) if want_grad_norms else ())
+    return (o_dev, wt_dev) + extra
 
 
 def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,

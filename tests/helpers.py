@@ -40,14 +40,16 @@ def gpu_scan(inp: dict, *, in_bf16: bool, out_bf16: bool = False, device="cuda",
     return tuple(None if x is None else x.float().cpu().numpy().astype(np.float64) for x in res)
 
 
-def oracle_scan(inp: dict, *, eps, mode, b, want_chunks=False, mask="inp"):
+def oracle_scan(inp: dict, *, eps, mode, b, want_chunks=False, mask="inp",
+                want_grad_norms=False):
     import oracle
 
     m = inp.get("mask") if isinstance(mask, str) else mask
     f = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
     return oracle.forward(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["eta_logit"]),
                           f(inp["gate_logit"]), f(inp["W0"]), f(inp["gamma"]), f(inp["beta"]),
-                          eps=eps, mode=mode, b=b, mask=m, want_chunks=want_chunks)
+                          eps=eps, mode=mode, b=b, mask=m, want_chunks=want_chunks,
+                          want_grad_norms=want_grad_norms)
 
 
 def assert_fp32_close(got, ref, what=""):

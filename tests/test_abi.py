@@ -29,7 +29,8 @@ def declared_functions():
 
 def test_headers_declare_the_boundary():
     names = declared_functions()
-    for must in ("ttt_scan_forward", "ttt_decode_step", "ttt_scan_kernel_choice",
+    for must in ("ttt_scan_forward", "ttt_scan_forward_grad_norms", "ttt_decode_step",
+                 "ttt_scan_kernel_choice",
                  "ttt_check_device_status",
                  "ttt_status_string", "ttt_set_wait_limit", "ttt_probe_ffma"):
         assert must in names
@@ -97,6 +98,36 @@ def test_invalid_arguments_rejected(lib, over):
                                   dict(mode=1 | (1 << 8))])
 def test_unsupported_shapes(lib, over):
     assert call(lib, **over) == UNSUPPORTED
+
+
+def call_gn(lib, **over):
+    """ttt_scan_forward_grad_norms with the same fake arguments as call()."""
+    a = dict(q=addr(0), k=addr(1), v=addr(2), eta=addr(3), gate=addr(4), W0=addr(5),
+             gamma=addr(6), beta=addr(7), B=2, H=3, T=40, d=64, eps=1e-6, mode=(1 << 8) | 2,
+             b=16, mask=None, o=addr(8), W_T=addr(9), W_chunks=None, gn=addr(12))
+    a.update(over)
+    fn = lib.ttt_scan_forward_grad_norms
+    fn.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_uint,
+                                                                 ctypes.c_int] + [ctypes.c_void_p] * 6
+    return fn(a["q"], a["k"], a["v"], a["eta"], a["gate"], a["W0"], a["gamma"], a["beta"],
+              a["B"], a["H"], a["T"], a["d"], a["eps"], a["mode"], a["b"], a["mask"], a["o"],
+              a["W_T"], a["W_chunks"], a["gn"], None)
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(mode=2), INVALID),                       # norms need the ablation gradient
+    (dict(mode=0), INVALID),
+    (dict(gn=None), INVALID),                      # no output for a non-empty problem
+    (dict(gn=addr(12, 4)), INVALID),               # misaligned
+    (dict(gn=addr(8)), INVALID),                   # over o
+    (dict(gn=addr(9)), INVALID),                   # over W_T
+    (dict(gn=addr(2, 1 << 10)), INVALID),          # inside v
+    (dict(mode=(1 << 8) | 1), UNSUPPORTED),        # mini-batch has no ablation form
+    (dict(d=32), UNSUPPORTED),
+    (dict(B=0), 0), (dict(B=0, gn=None), 0), (dict(T=0, B=0), 0),   # empty: nothing launched
+], ids=lambda x: ",".join(x) if isinstance(x, dict) else str(x))
+def test_grad_norms_entry_checks(lib, over, want):
+    assert call_gn(lib, **over) == want
 
 
 def test_no_ln_needs_no_affine_and_empty_batch_is_noop(lib):

@@ -317,6 +317,45 @@ def test_ablation_gradient_headline_shape(norm_match):
     assert_fp32_close(W_T, rW, "W_T")
 
 
+@pytest.mark.parametrize("case", [
+    # (B, H, T, d, b, in_bf16)
+    (2, 3, 77, 64, 16, False),
+    (2, 3, 53, 16, 16, False),
+    (2, 2, 70, 64, 24, True),     # internal chunk 12, bf16 inputs
+], ids=["d64", "d16", "d64_b24_bf16"])
+@pytest.mark.parametrize("norm_match", [False, True], ids=["ablate", "ablate_nm"])
+@pytest.mark.parametrize("with_mask", [False, True], ids=["nomask", "mask"])
+def test_ablation_grad_norms(case, norm_match, with_mask):
+    """Per-token (||G_full||, ||G_ablation||) against the oracle (fp32 bound),
+    exact zeros on SKIP chunks, and the scan's outputs unchanged by asking."""
+    B, H, T, d, b, in_bf16 = case
+    inp = make_inputs(B, H, T, d, seed=650 + T + d + b, random_affine=True, in_bf16=in_bf16,
+                      mask_p=0.5 if with_mask else None, b=b)
+    mode = ABLATE | (NORM_MATCH if norm_match else 0)
+    o, W_T, gn = gpu_scan(inp, in_bf16=in_bf16, eps=1e-6, b=b, ablate=True, norm_match=norm_match,
+                          want_grad_norms=True)
+    ro, rW, rgn = oracle_scan(inp, eps=1e-6, mode=mode, b=b, want_grad_norms=True)
+    assert_fp32_close(o, ro, "o")
+    assert_fp32_close(W_T, rW, "W_T")
+    assert_fp32_close(gn, rgn, "grad_norms")
+    if with_mask:
+        skip = np.repeat(inp["mask"] == 0, b, axis=1)[:, :T]          # [B, T]
+        assert skip.any()
+        assert np.all(gn[skip[:, None, :, None].repeat(H, 1).repeat(2, 3)] == 0.0)
+
+
+def test_ablation_grad_norm_ratio_headline_shape():
+    """The mean gradient norm ratio over the headline workload's tokens, GPU
+    against the oracle."""
+    w = WORKLOADS["2j"]
+    inp = make_workload(w)
+    o, W_T, gn = gpu_scan(inp, in_bf16=False, eps=w.eps, b=w.b, ablate=True, want_grad_norms=True)
+    ro, rW, rgn = oracle_scan(inp, eps=w.eps, mode=ABLATE, b=w.b, want_grad_norms=True)
+    assert_fp32_close(gn, rgn, "grad_norms")
+    ratio, rratio = (gn[..., 1] / gn[..., 0]).mean(), (rgn[..., 1] / rgn[..., 0]).mean()
+    assert abs(ratio - rratio) <= 2e-4 * rratio, (ratio, rratio)
+
+
 def test_ablation_rejected_where_not_defined():
     import torch
     from test_sequence_layers_02_b200 import ttt_scan
@@ -330,6 +369,8 @@ def test_ablation_rejected_where_not_defined():
         ttt_scan.scan(*args, norm_match=True)
     with pytest.raises(ttt_scan.TTTScanError, match="UNSUPPORTED"):
         ttt_scan.scan(*args, ablate=True, minibatch=True)
+    with pytest.raises(ttt_scan.TTTScanError, match="INVALID"):
+        ttt_scan.scan(*args, lnjac=True, want_grad_norms=True)
 
 
 # ---------------------------------------------------------------------------
