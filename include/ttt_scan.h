@@ -38,7 +38,7 @@ extern "C" {
 typedef enum {
   TTT_OK = 0,
   TTT_ERR_INVALID_ARG = -1,    /* null/misaligned pointer, bad size, aliasing, unknown mode bit */
-  TTT_ERR_UNSUPPORTED = -2,    /* valid arguments the library does not implement (d, b, dtype mix) */
+  TTT_ERR_UNSUPPORTED = -2,    /* valid arguments this build does not implement (d, b, dtype mix) */
   TTT_ERR_CUDA = -3,           /* a CUDA runtime call or a launch failed */
   TTT_ERR_DEVICE_TIMEOUT = -4  /* a bounded in-kernel wait gave up; outputs are not valid */
 } ttt_status;
