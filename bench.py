@@ -435,23 +435,46 @@ def _cpu_baseline(job, min_seconds=8.0):
 
 
 def _e2e(job, steps, device):
-    """Same metric through the public API with pinned host buffers (copies inside)."""
+    """Same metric through the public API, end to end. Every step copies that
+    step's inputs from pinned host memory to the device (once: the passes share
+    them), runs the passes on their own streams as the device-timed step does,
+    copies every pass's results (o, W_T) back to pinned host memory as soon as
+    that pass ends, and waits for them on the host."""
     import torch
     from test_sequence_layers_02_b200 import ttt_scan
     t = job.t
-    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
-    o_h = torch.empty(t["q"].shape, dtype=job.out_dtype).pin_memory()
-    wt_h = torch.empty(t["W0"].shape, dtype=torch.float32).pin_memory()
     w = job.w
-    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None) * len(job.passes)
-    d2h = (o_h.numel() * o_h.element_size() + wt_h.numel() * 4) * len(job.passes)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
+    dev = {k: (None if v is None else torch.empty_like(v)) for k, v in t.items()}
+    n = len(job.passes)
+    o_h = [torch.empty(t["q"].shape, dtype=job.out_dtype).pin_memory() for _ in range(n)]
+    wt_h = [torch.empty(t["W0"].shape, dtype=torch.float32).pin_memory() for _ in range(n)]
+    o_d = [torch.empty_like(t["q"], dtype=job.out_dtype) for _ in range(n)]
+    wt_d = [torch.empty_like(t["W0"]) for _ in range(n)]
+    streams = [torch.cuda.Stream(device) for _ in range(n)]
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = sum(o.numel() * o.element_size() + x.numel() * x.element_size()
+              for o, x in zip(o_h, wt_h))
 
     def step():
-        for ps in job.passes:
-            ttt_scan.scan(host["q"], host["k"], host["v"], host["eta_logit"], host["gate_logit"],
-                          host["W0"], host["gamma"], host["beta"], eps=w.eps,
-                          minibatch=w.minibatch, b=w.b, mask=host["mask"],
-                          out_dtype=job.out_dtype, o=o_h, W_T=wt_h, **ps)
+        main = torch.cuda.current_stream(device)
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        for i, ps in enumerate(job.passes):
+            st = streams[i]
+            st.wait_stream(main)
+            ttt_scan.scan(dev["q"], dev["k"], dev["v"], dev["eta_logit"], dev["gate_logit"],
+                          dev["W0"], dev["gamma"], dev["beta"], eps=w.eps,
+                          minibatch=w.minibatch, b=w.b, mask=dev["mask"],
+                          out_dtype=job.out_dtype, o=o_d[i], W_T=wt_d[i], stream=st, **ps)
+            with torch.cuda.stream(st):
+                o_h[i].copy_(o_d[i], non_blocking=True)
+                wt_h[i].copy_(wt_d[i], non_blocking=True)
+            main.wait_stream(st)
+        rc = ttt_scan.check_device_status(main)   # synchronises: the results are on the host
+        if rc != ttt_scan.TTT_OK:
+            raise ttt_scan.TTTScanError(rc, "device")
 
     step()
     torch.cuda.synchronize()
