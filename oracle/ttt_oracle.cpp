@@ -77,10 +77,20 @@ constexpr unsigned kNoLayerNorm = 1u << 2;
 constexpr unsigned kGateChannel = 1u << 6;
 constexpr unsigned kGradAblate = 1u << 8;
 constexpr unsigned kNormMatch = 1u << 9;
+// The `:mlp` variant ("Edifice.Recurrent.TTT", `build` options, `:variant`):
+// SiLU applied to the keys and the queries before the inner model. Oracle
+// only for now; the bit is reserved for the scan's interface.
+constexpr unsigned kKqSilu = 1u << 10;
 
 template <typename S>
 S sigmoid(S x) {
   return S(1) / (S(1) + std::exp(-x));
+}
+
+// SiLU(x) = x * sigmoid(x).
+template <typename S>
+S silu(S x) {
+  return x * sigmoid(x);
 }
 
 // Inner LayerNorm forward and the inner gradient with respect to z.
@@ -190,6 +200,18 @@ void scan_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
   const int n_chunks = (T + b - 1) / b;
   std::vector<S> W(W0, W0 + (size_t)d * d);
   std::vector<S> z(d), G(d), Wq(d);
+  // the `:mlp` variant feeds SiLU(k), SiLU(q) to the inner model
+  std::vector<S> ks, qs;
+  if (mode & kKqSilu) {
+    ks.resize((size_t)T * d);
+    qs.resize((size_t)T * d);
+    for (size_t i = 0; i < (size_t)T * d; ++i) {
+      ks[i] = silu(k[i]);
+      qs[i] = silu(q[i]);
+    }
+    k = ks.data();
+    q = qs.data();
+  }
 
   for (int c = 0; c < n_chunks; ++c) {
     const int t0 = c * b;

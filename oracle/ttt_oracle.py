@@ -32,6 +32,9 @@ NO_LN = 1 << 2
 GATE_CHANNEL = 1 << 6
 GRAD_ABLATE = 1 << 8
 GRAD_NORM_MATCH = 1 << 9
+# The `:mlp` variant: SiLU on keys and queries before the inner model (oracle
+# only for now; the bit is reserved for the scan's interface).
+KQ_SILU = 1 << 10
 
 _lib = None
 

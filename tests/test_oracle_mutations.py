@@ -42,6 +42,8 @@ MUTATIONS = [
     ("norm_match_without_sqrt", "std::sqrt(n_full / n_abl)", "(n_full / n_abl)"),
     ("grad_norms_both_full", "norms[1] = std::sqrt(n_abl);", "norms[1] = std::sqrt(n_full);"),
     ("grad_norms_squared", "norms[0] = std::sqrt(n_full);", "norms[0] = n_full;"),
+    ("kq_silu_keys_only", "      qs[i] = silu(q[i]);", "      qs[i] = q[i];"),
+    ("kq_silu_as_sigmoid", "  return x * sigmoid(x);", "  return sigmoid(x);"),
     ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
     ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
      "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),

@@ -31,7 +31,8 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import GATE_CHANNEL, GRAD_ABLATE, GRAD_LNJAC, GRAD_NORM_MATCH, MINIBATCH, NO_LN
+from oracle import (GATE_CHANNEL, GRAD_ABLATE, GRAD_LNJAC, GRAD_NORM_MATCH, KQ_SILU, MINIBATCH,
+                    NO_LN)
 from test_sequence_layers_02_b200.workloads import make_inputs
 from tests.conftest import load_golden
 
@@ -442,6 +443,49 @@ def test_ablation_mode_combinations():
         run(inp, mode=GRAD_NORM_MATCH)
     o, W = run(inp, mode=GRAD_ABLATE | GRAD_NORM_MATCH)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(W))
+
+
+# ----------------------------------------------------------------------------
+# The `:mlp` variant ("Edifice.Recurrent.TTT", `build` options, `:variant`):
+# SiLU on the keys and the queries before the inner model.
+# ----------------------------------------------------------------------------
+
+def test_kq_silu_known_values():
+    """W0 = I, eta = 0, no gate: o_t = SiLU(q_t) exactly; SiLU(1) = e / (1 + e),
+    SiLU(-1) = 1 / (1 + e) - 1 ... written from the constants, not the oracle."""
+    d, T = 4, 3
+    q = np.array([[0.0, 1.0, -1.0, 2.0], [20.0, -20.0, 0.5, -0.5], [3.0, -3.0, 1e-3, -1e-3]])
+    k = np.ones((T, d))
+    e = np.e
+    want = np.array([
+        [0.0, e / (1 + e), -1.0 / (1 + e), 2.0 * e * e / (1 + e * e)],
+        [20.0 / (1 + np.exp(-20.0)), -20.0 * np.exp(-20.0) / (1 + np.exp(-20.0)),
+         0.5 / (1 + np.exp(-0.5)), -0.5 / (1 + np.exp(0.5))],
+        [3.0 / (1 + np.exp(-3.0)), -3.0 / (1 + np.exp(3.0)),
+         1e-3 / (1 + np.exp(-1e-3)), -1e-3 / (1 + np.exp(1e-3))]])
+    sh = lambda a: a.reshape(1, 1, *a.shape)
+    o, W_T = oracle.forward(sh(q), sh(k), sh(np.zeros((T, d))), np.full((1, 1, T), -1e4), None,
+                            np.eye(d).reshape(1, 1, d, d), np.ones((1, d)), np.zeros((1, d)),
+                            eps=1e-6, mode=KQ_SILU | GRAD_LNJAC, b=1)
+    np.testing.assert_allclose(o[0, 0], want, rtol=1e-14, atol=1e-300)
+    np.testing.assert_array_equal(W_T[0, 0], np.eye(d))
+
+
+@pytest.mark.parametrize("grad", [0, GRAD_LNJAC, NO_LN], ids=["simple", "lnjac", "no_ln"])
+@pytest.mark.parametrize("minib", [0, MINIBATCH], ids=["per_token", "minibatch"])
+def test_kq_silu_is_the_linear_scan_on_silu_features(grad, minib):
+    """The variant equals the linear scan run on SiLU(k), SiLU(q) computed here
+    in numpy (v, the logits and the state untouched), with a mask and a ragged
+    tail."""
+    inp = f64(make_inputs(2, 3, 37, 16, seed=41, random_affine=True, mask_p=0.6, b=8))
+    silu = lambda x: x / (1.0 + np.exp(-x))
+    lin = dict(inp, q=silu(inp["q"]), k=silu(inp["k"]))
+    o1, W1 = run(inp, mode=grad | minib | KQ_SILU, b=8, eps=1e-6)
+    o2, W2 = run(lin, mode=grad | minib, b=8, eps=1e-6)
+    np.testing.assert_allclose(o1, o2, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(W1, W2, rtol=1e-11, atol=1e-13)
+    o3, _ = run(inp, mode=grad | minib, b=8, eps=1e-6)
+    assert not np.allclose(o1, o3)      # the variant does change the result
 
 
 # ----------------------------------------------------------------------------
