@@ -5,5 +5,5 @@ leg may import this package. It shares no code with the CUDA path.
 """
 
 from .ttt_oracle import (GATE_CHANNEL, GRAD_ABLATE, GRAD_LNJAC, GRAD_NORM_MATCH,  # noqa: F401
-                         KQ_SILU, MINIBATCH, NO_LN, build, decode_step, forward,
+                         KQ_SILU, MINIBATCH, NO_LN, backward, build, decode_step, forward,
                          forward_heads, lngrad, max_threads)

@@ -311,9 +311,229 @@ int forward(const S* q, const S* k, const S* v, const S* eta_logit,
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Backward of the per-token recurrence (reverse mode through every token).
+// No page gives this; it is the chain rule applied, in reverse order, to the
+// forward steps above: z = W k, the LayerNorm and its gradient G, the update
+// W' = W - eta G k^T, the output o = gate * (W' q). Given dO (= dL/do) and
+// dW_T (= dL/dW_T) it returns dL/d of every input.
+// ---------------------------------------------------------------------------
+
+// dz, and the contributions to dv, dgamma, dbeta, of dG through G(z, v).
+template <typename S>
+void lngrad_backward(const S* z, const S* v, const S* gamma, const S* beta, int d, S eps,
+                     unsigned mode, const S* dG, S* dz, S* dv, S* dgamma, S* dbeta) {
+  if (mode & kNoLayerNorm) {  // G = z - v
+    for (int f = 0; f < d; ++f) {
+      dz[f] = dG[f];
+      dv[f] -= dG[f];
+    }
+    return;
+  }
+  S mu = 0;
+  for (int f = 0; f < d; ++f) mu += z[f];
+  mu /= S(d);
+  S var = 0;
+  for (int f = 0; f < d; ++f) var += (z[f] - mu) * (z[f] - mu);
+  var /= S(d);
+  const S s = std::sqrt(var + eps);
+  std::vector<S> xhat(d), err(d), dxhat(d, S(0));
+  for (int f = 0; f < d; ++f) {
+    xhat[f] = (z[f] - mu) / s;
+    err[f] = gamma[f] * xhat[f] + beta[f] - v[f];
+  }
+  S ds = 0;  // dL/ds through G's explicit 1/s (LN-Jacobian form only)
+  std::vector<S> derr(d);
+  if (mode & kLnJacobian) {
+    // G = (g - mean g - xhat mean(g xhat)) / s, g = gamma err
+    std::vector<S> g(d), G(d);
+    S a = 0, c = 0, mdG = 0, mdGx = 0;
+    for (int f = 0; f < d; ++f) {
+      g[f] = gamma[f] * err[f];
+      a += g[f];
+      c += g[f] * xhat[f];
+      mdG += dG[f];
+      mdGx += dG[f] * xhat[f];
+    }
+    a /= S(d);
+    c /= S(d);
+    mdG /= S(d);
+    mdGx /= S(d);
+    for (int f = 0; f < d; ++f) G[f] = (g[f] - a - xhat[f] * c) / s;
+    for (int f = 0; f < d; ++f) {
+      const S dg = (dG[f] - mdG - xhat[f] * mdGx) / s;       // J^T is symmetric
+      dxhat[f] += (-dG[f] * c - g[f] * mdGx) / s;
+      ds -= dG[f] * G[f] / s;
+      dgamma[f] += dg * err[f];
+      derr[f] = dg * gamma[f];
+    }
+  } else {  // G = err
+    for (int f = 0; f < d; ++f) derr[f] = dG[f];
+  }
+  // err = gamma xhat + beta - v
+  for (int f = 0; f < d; ++f) {
+    dgamma[f] += derr[f] * xhat[f];
+    dbeta[f] += derr[f];
+    dv[f] -= derr[f];
+    dxhat[f] += derr[f] * gamma[f];
+  }
+  // xhat = (z - mu) / s, s = sqrt(var + eps), var = mean((z - mu)^2)
+  S dxx = 0;
+  for (int f = 0; f < d; ++f) dxx += dxhat[f] * xhat[f];
+  const S ds_total = ds - dxx / s;
+  const S dvar = ds_total / (S(2) * s);
+  std::vector<S> dy(d);
+  S mdy = 0;
+  for (int f = 0; f < d; ++f) {
+    dy[f] = dxhat[f] / s + dvar * S(2) * (z[f] - mu) / S(d);
+    mdy += dy[f];
+  }
+  mdy /= S(d);
+  for (int f = 0; f < d; ++f) dz[f] = dy[f] - mdy;
+}
+
+template <typename S>
+void backward_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
+                       const S* gate_logit, const S* W0, const S* gamma, const S* beta,
+                       int T, int d, S eps, unsigned mode, int b,
+                       const unsigned char* mask_row, const S* dO, const S* dW_T,
+                       S* dq, S* dk, S* dv, S* deta, S* dgate, S* dW0, S* dgamma,
+                       S* dbeta) {
+  // forward, keeping the state before every token
+  std::vector<S> Ws((size_t)(T + 1) * d * d);
+  std::memcpy(Ws.data(), W0, sizeof(S) * d * d);
+  std::vector<S> z(d), G(d), y(d), dz(d), dG(d), dy(d), dWk(d);
+  auto upd_of = [&](int t) { return (mask_row == nullptr) || (mask_row[t / b] != 0); };
+  for (int t = 0; t < T; ++t) {
+    const S* W = Ws.data() + (size_t)t * d * d;
+    S* Wn = Ws.data() + (size_t)(t + 1) * d * d;
+    const S* kt = k + (size_t)t * d;
+    const S eta = upd_of(t) ? sigmoid(eta_logit[t]) / S(d) : S(0);
+    matvec(W, kt, d, z.data());
+    ln_and_grad(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode, (S*)nullptr,
+                G.data(), (S*)nullptr);
+    for (int r = 0; r < d; ++r)
+      for (int c = 0; c < d; ++c) Wn[r * d + c] = W[r * d + c] - eta * G[r] * kt[c];
+  }
+  // reverse: dW holds dL/dW_t, starting from dL/dW_T
+  std::vector<S> dW(dW_T, dW_T + (size_t)d * d);
+  for (int t = T - 1; t >= 0; --t) {
+    const S* W = Ws.data() + (size_t)t * d * d;       // W_{t-1}
+    const S* Wn = Ws.data() + (size_t)(t + 1) * d * d; // W_t
+    const S* kt = k + (size_t)t * d;
+    const S* qt = q + (size_t)t * d;
+    const S* dOt = dO + (size_t)t * d;
+    const bool upd = upd_of(t);
+    const S sg = upd ? sigmoid(eta_logit[t]) : S(0);
+    const S eta = sg / S(d);
+    // o = gate * (W_t q)
+    matvec(Wn, qt, d, y.data());
+    if (gate_logit && (mode & kGateChannel)) {
+      for (int r = 0; r < d; ++r) {
+        const S g = sigmoid(gate_logit[(size_t)t * d + r]);
+        dy[r] = g * dOt[r];
+        dgate[(size_t)t * d + r] = dOt[r] * y[r] * g * (S(1) - g);
+      }
+    } else if (gate_logit) {
+      const S g = sigmoid(gate_logit[t]);
+      S acc = 0;
+      for (int r = 0; r < d; ++r) {
+        dy[r] = g * dOt[r];
+        acc += dOt[r] * y[r];
+      }
+      dgate[t] = acc * g * (S(1) - g);
+    } else {
+      for (int r = 0; r < d; ++r) dy[r] = dOt[r];
+    }
+    for (int c = 0; c < d; ++c) {
+      S acc = 0;
+      for (int r = 0; r < d; ++r) acc += Wn[r * d + c] * dy[r];
+      dq[(size_t)t * d + c] = acc;
+    }
+    for (int r = 0; r < d; ++r)
+      for (int c = 0; c < d; ++c) dW[r * d + c] += dy[r] * qt[c];
+    // W_t = W_{t-1} - eta G k^T, G = G(z = W_{t-1} k)
+    matvec(W, kt, d, z.data());
+    ln_and_grad(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode, (S*)nullptr,
+                G.data(), (S*)nullptr);
+    matvec(dW.data(), kt, d, dWk.data());               // dW k
+    S deta_t = 0;
+    for (int r = 0; r < d; ++r) {
+      deta_t -= G[r] * dWk[r];
+      dG[r] = -eta * dWk[r];
+    }
+    for (int c = 0; c < d; ++c) {
+      S acc = 0;
+      for (int r = 0; r < d; ++r) acc += dW[r * d + c] * G[r];
+      dk[(size_t)t * d + c] = -eta * acc;
+    }
+    deta[t] = upd ? deta_t * sg * (S(1) - sg) / S(d) : S(0);
+    lngrad_backward(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode, dG.data(),
+                    dz.data(), dv + (size_t)t * d, dgamma, dbeta);
+    // z = W_{t-1} k
+    for (int c = 0; c < d; ++c) {
+      S acc = 0;
+      for (int r = 0; r < d; ++r) acc += W[r * d + c] * dz[r];
+      dk[(size_t)t * d + c] += acc;
+    }
+    for (int r = 0; r < d; ++r)
+      for (int c = 0; c < d; ++c) dW[r * d + c] += dz[r] * kt[c];
+  }
+  std::memcpy(dW0, dW.data(), sizeof(S) * d * d);
+}
+
 }  // namespace
 
 extern "C" {
+
+// Backward of the per-token scan (SIMPLE, LN-Jacobian or no-LayerNorm
+// gradient; scalar or per-feature gate; mask). Inputs as for the forward scan,
+// plus dO [B, H, T, d] and dW_T [B, H, d, d]. Writes dq, dk, dv [B, H, T, d],
+// deta [B, H, T], dgate (shape of gate_logit; may be null when gate_logit is),
+// dW0 [B, H, d, d], dgamma, dbeta [H, d] (summed over the batch rows; ignored
+// with NO_LN). Returns 0, or -1 on an argument it does not take (mini-batch
+// mode, the ablation gradient).
+int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
+                            const double* eta_logit, const double* gate_logit,
+                            const double* W0, const double* gamma, const double* beta,
+                            int B, int H, int T, int d, double eps, unsigned mode, int b,
+                            const unsigned char* mask, const double* dO, const double* dW_T,
+                            double* dq, double* dk, double* dv, double* deta, double* dgate,
+                            double* dW0, double* dgamma, double* dbeta) {
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return -1;
+  if (mode & (kMiniBatch | kGradAblate | kNormMatch | kKqSilu)) return -1;
+  if (!q || !k || !v || !eta_logit || !W0 || !dO || !dW_T || !dq || !dk || !dv || !deta ||
+      !dW0)
+    return -1;
+  if (gate_logit && !dgate) return -1;
+  const bool no_ln = mode & kNoLayerNorm;
+  if (!no_ln && (!gamma || !beta || !dgamma || !dbeta)) return -1;
+  const int n_chunks = (T + b - 1) / b;
+  std::vector<double> ones((size_t)d, 1.0), zeros((size_t)d, 0.0), sink_g((size_t)d),
+      sink_b((size_t)d);
+  if (!no_ln) {
+    std::memset(dgamma, 0, sizeof(double) * (size_t)H * d);
+    std::memset(dbeta, 0, sizeof(double) * (size_t)H * d);
+  }
+  const size_t gstride = (mode & kGateChannel) ? (size_t)d : 1;
+  std::memset(dv, 0, sizeof(double) * (size_t)B * H * T * d);  // accumulated per token
+  for (long long bh = 0; bh < (long long)B * H; ++bh) {
+    const int bi = (int)(bh / H);
+    const int h = (int)(bh % H);
+    const size_t tok = (size_t)bh * T;
+    backward_one_head<double>(
+        q + tok * d, k + tok * d, v + tok * d, eta_logit + tok,
+        gate_logit ? gate_logit + tok * gstride : nullptr, W0 + (size_t)bh * d * d,
+        no_ln ? ones.data() : gamma + (size_t)h * d, no_ln ? zeros.data() : beta + (size_t)h * d,
+        T, d, eps, mode, b, mask ? mask + (size_t)bi * n_chunks : nullptr, dO + tok * d,
+        dW_T + (size_t)bh * d * d, dq + tok * d, dk + tok * d, dv + tok * d, deta + tok,
+        gate_logit ? dgate + tok * gstride : nullptr, dW0 + (size_t)bh * d * d,
+        no_ln ? sink_g.data() : dgamma + (size_t)h * d,
+        no_ln ? sink_b.data() : dbeta + (size_t)h * d);
+  }
+  return 0;
+}
+
 
 // Full scan. All arrays are host, contiguous, row-major:
 //   q, k, v, o: [B, H, T, d];  eta_logit: [B, H, T];

@@ -76,6 +76,10 @@ def _load():
         lib.ttt_oracle_lngrad_f64.argtypes = [dp, dp, dp, dp, i, ctypes.c_double,
                                               ctypes.c_uint, dp, dp, dp, dp]
         lib.ttt_oracle_lngrad_f64.restype = i
+        lib.ttt_oracle_backward_f64.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i,
+                                                ctypes.c_double, ctypes.c_uint, i, u8p, dp, dp,
+                                                dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.ttt_oracle_backward_f64.restype = i
         lib.ttt_oracle_max_threads.argtypes = []
         lib.ttt_oracle_max_threads.restype = i
         _lib = lib
@@ -143,6 +147,45 @@ def forward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float,
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     out = (o, W_T) + ((W_chunks,) if want_chunks else ()) + ((gnorms,) if want_grad_norms else ())
+    return out
+
+
+def backward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, dO, dW_T, *, eps: float,
+             mode: int, b: int = 16, mask=None):
+    """Backward of the per-token scan: the gradients of L = <dO, o> + <dW_T, W_T>
+    with respect to every input, by reverse mode through the tokens.
+
+    Shapes as for ``forward``; dO [B, H, T, d], dW_T [B, H, d, d]. Returns a dict
+    with dq, dk, dv, deta_logit, dgate_logit (None without a gate), dW0, dgamma,
+    dbeta (summed over the batch rows; None with NO_LN). Per-token mode with
+    the SIMPLE, LN-Jacobian or no-LayerNorm gradient only.
+    """
+    lib = _load()
+    dp = ctypes.c_double
+    cvt = (lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float64))
+    q, k, v, eta_logit, gate_logit, W0, dO, dW_T = map(
+        cvt, (q, k, v, eta_logit, gate_logit, W0, dO, dW_T))
+    B, H, T, d = q.shape
+    no_ln = bool(mode & NO_LN)
+    gamma = np.ones((H, d)) if gamma is None else cvt(gamma)
+    beta = np.zeros((H, d)) if beta is None else cvt(beta)
+    if mask is not None:
+        mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    out = dict(dq=np.empty_like(q), dk=np.empty_like(k), dv=np.empty_like(v),
+               deta_logit=np.empty_like(eta_logit),
+               dgate_logit=None if gate_logit is None else np.empty_like(gate_logit),
+               dW0=np.empty_like(W0), dgamma=np.zeros((H, d)), dbeta=np.zeros((H, d)))
+    rc = lib.ttt_oracle_backward_f64(
+        _ptr(q, dp), _ptr(k, dp), _ptr(v, dp), _ptr(eta_logit, dp), _ptr(gate_logit, dp),
+        _ptr(W0, dp), _ptr(gamma, dp), _ptr(beta, dp), B, H, T, d, eps, mode, b,
+        _ptr(mask, ctypes.c_ubyte), _ptr(dO, dp), _ptr(dW_T, dp), _ptr(out["dq"], dp),
+        _ptr(out["dk"], dp), _ptr(out["dv"], dp), _ptr(out["deta_logit"], dp),
+        _ptr(out["dgate_logit"], dp), _ptr(out["dW0"], dp), _ptr(out["dgamma"], dp),
+        _ptr(out["dbeta"], dp))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (rc={rc})")
+    if no_ln:
+        out["dgamma"] = out["dbeta"] = None
     return out
 
 

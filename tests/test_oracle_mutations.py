@@ -44,6 +44,9 @@ MUTATIONS = [
     ("grad_norms_squared", "norms[0] = std::sqrt(n_full);", "norms[0] = n_full;"),
     ("kq_silu_keys_only", "      qs[i] = silu(q[i]);", "      qs[i] = q[i];"),
     ("kq_silu_as_sigmoid", "  return x * sigmoid(x);", "  return sigmoid(x);"),
+    ("backward_drops_explicit_1_over_s", "      ds -= dG[f] * G[f] / s;", "      ds -= 0 * G[f];"),
+    ("backward_dk_without_update_term", "      dk[(size_t)t * d + c] = -eta * acc;",
+     "      dk[(size_t)t * d + c] = 0;"),
     ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
     ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
      "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),

@@ -489,6 +489,67 @@ def test_kq_silu_is_the_linear_scan_on_silu_features(grad, minib):
 
 
 # ----------------------------------------------------------------------------
+# Backward of the per-token scan (no page gives it: reverse mode through the
+# forward steps), pinned by central finite differences of the forward oracle.
+# ----------------------------------------------------------------------------
+
+def _fd_check_backward(inp, mode, b, eps, seed, tol=1e-7):
+    rng = np.random.default_rng(seed)
+    keys = ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")
+    x = {k_: (None if inp[k_] is None else np.asarray(inp[k_], np.float64)) for k_ in keys}
+    dO = rng.normal(size=x["q"].shape)
+    dWT = rng.normal(size=x["W0"].shape)
+    m = inp.get("mask")
+    g = oracle.backward(**x, dO=dO, dW_T=dWT, eps=eps, mode=mode, b=b, mask=m)
+
+    def loss(xx):
+        o, W = oracle.forward(**xx, eps=eps, mode=mode, b=b, mask=m)
+        return float((dO * o).sum() + (dWT * W).sum())
+
+    names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("eta_logit", "deta_logit"),
+             ("gate_logit", "dgate_logit"), ("W0", "dW0")]
+    if not mode & NO_LN:
+        names += [("gamma", "dgamma"), ("beta", "dbeta")]
+    for key, gk in names:
+        if x[key] is None:
+            assert g[gk] is None
+            continue
+        a = x[key]
+        fd = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            h = 1e-6 * max(1.0, abs(a[idx]))
+            ap, am = a.copy(), a.copy()
+            ap[idx] += h
+            am[idx] -= h
+            fd[idx] = (loss(dict(x, **{key: ap})) - loss(dict(x, **{key: am}))) / (2 * h)
+        scale = np.abs(fd).max() + 1e-12
+        assert np.abs(fd - g[gk]).max() <= tol * scale, (key, np.abs(fd - g[gk]).max() / scale)
+
+
+@pytest.mark.parametrize("grad", [0, GRAD_LNJAC, NO_LN], ids=["simple", "lnjac", "no_ln"])
+def test_backward_matches_finite_differences(grad):
+    inp = make_inputs(1, 2, 7, 4, seed=45 + grad, random_affine=True, mask_p=0.6, b=2)
+    _fd_check_backward(inp, grad, b=2, eps=1e-5, seed=46)
+
+
+def test_backward_per_feature_gate_and_no_gate():
+    inp = make_inputs(1, 1, 5, 4, seed=47, random_affine=True, gate_channel=True)
+    _fd_check_backward(inp, GRAD_LNJAC | GATE_CHANNEL, b=16, eps=1e-5, seed=48)
+    inp = make_inputs(1, 1, 5, 4, seed=49, random_affine=True, gate=False)
+    _fd_check_backward(inp, GRAD_LNJAC, b=16, eps=1e-5, seed=50)
+
+
+def test_backward_rejects_what_it_does_not_take():
+    inp = f64(make_inputs(1, 1, 4, 4, seed=51))
+    z = np.zeros_like(inp["q"])
+    for mode in (MINIBATCH, GRAD_ABLATE, KQ_SILU):
+        with pytest.raises(ValueError):
+            oracle.backward(inp["q"], inp["k"], inp["v"], inp["eta_logit"], inp["gate_logit"],
+                            inp["W0"], inp["gamma"], inp["beta"], z, np.zeros_like(inp["W0"]),
+                            eps=1e-5, mode=mode)
+
+
+# ----------------------------------------------------------------------------
 # Mini-batch (dual form; PonderTTT "Technical Architecture").
 # ----------------------------------------------------------------------------
 
