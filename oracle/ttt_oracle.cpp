@@ -482,6 +482,136 @@ void backward_one_head(const S* q, const S* k, const S* v, const S* eta_logit,
   std::memcpy(dW0, dW.data(), sizeof(S) * d * d);
 }
 
+// Backward of the mini-batch (dual-form) recurrence: per chunk, every
+// gradient at the chunk-start W_s, the inclusive causal readout
+// o_i = gate (W_s q_i - sum_{j<=i} eta_j (k_j.q_i) G_j), one update
+// W_e = W_s - sum_j eta_j G_j k_j^T; reverse mode over the chunks.
+template <typename S>
+void backward_one_head_minibatch(const S* q, const S* k, const S* v, const S* eta_logit,
+                                 const S* gate_logit, const S* W0, const S* gamma,
+                                 const S* beta, int T, int d, S eps, unsigned mode, int b,
+                                 const unsigned char* mask_row, const S* dO, const S* dW_T,
+                                 S* dq, S* dk, S* dv, S* deta, S* dgate, S* dW0, S* dgamma,
+                                 S* dbeta) {
+  const int n_chunks = (T + b - 1) / b;
+  std::vector<S> Ws((size_t)(n_chunks + 1) * d * d);
+  std::memcpy(Ws.data(), W0, sizeof(S) * d * d);
+  std::vector<S> z(d), dz(d), y(d), dy(d), dWk(d);
+  // forward: the chunk-start states
+  for (int c = 0; c < n_chunks; ++c) {
+    const int t0 = c * b, n = std::min(b, T - t0);
+    const bool upd = (mask_row == nullptr) || (mask_row[c] != 0);
+    const S* W = Ws.data() + (size_t)c * d * d;
+    S* Wn = Ws.data() + (size_t)(c + 1) * d * d;
+    std::memcpy(Wn, W, sizeof(S) * d * d);
+    for (int j = 0; j < n; ++j) {
+      const S* kj = k + (size_t)(t0 + j) * d;
+      const S eta = upd ? sigmoid(eta_logit[t0 + j]) / S(d) : S(0);
+      std::vector<S> G(d);
+      matvec(W, kj, d, z.data());
+      ln_and_grad(z.data(), v + (size_t)(t0 + j) * d, gamma, beta, d, eps, mode, (S*)nullptr,
+                  G.data(), (S*)nullptr);
+      for (int r = 0; r < d; ++r)
+        for (int cc = 0; cc < d; ++cc) Wn[r * d + cc] -= eta * G[r] * kj[cc];
+    }
+  }
+  std::vector<S> dW(dW_T, dW_T + (size_t)d * d);  // dL/dW_e of the chunk being undone
+  for (int c = n_chunks - 1; c >= 0; --c) {
+    const int t0 = c * b, n = std::min(b, T - t0);
+    const bool upd = (mask_row == nullptr) || (mask_row[c] != 0);
+    const S* W = Ws.data() + (size_t)c * d * d;
+    std::vector<S> Gs((size_t)n * d), dGs((size_t)n * d, S(0)), etas(n), sgs(n), detas(n, S(0));
+    for (int j = 0; j < n; ++j) {
+      sgs[j] = upd ? sigmoid(eta_logit[t0 + j]) : S(0);
+      etas[j] = sgs[j] / S(d);
+      matvec(W, k + (size_t)(t0 + j) * d, d, z.data());
+      ln_and_grad(z.data(), v + (size_t)(t0 + j) * d, gamma, beta, d, eps, mode, (S*)nullptr,
+                  Gs.data() + (size_t)j * d, (S*)nullptr);
+    }
+    std::vector<S> dWs(dW);  // W_e = W_s - ...: identity part
+    for (int j = 0; j < n; ++j) {
+      const S* kj = k + (size_t)(t0 + j) * d;
+      const S* Gj = Gs.data() + (size_t)j * d;
+      matvec(dW.data(), kj, d, dWk.data());
+      for (int r = 0; r < d; ++r) {
+        detas[j] -= Gj[r] * dWk[r];
+        dGs[(size_t)j * d + r] -= etas[j] * dWk[r];
+      }
+      for (int cc = 0; cc < d; ++cc) {
+        S acc = 0;
+        for (int r = 0; r < d; ++r) acc += dW[r * d + cc] * Gj[r];
+        dk[(size_t)(t0 + j) * d + cc] = -etas[j] * acc;
+      }
+    }
+    // outputs of the chunk
+    for (int i = 0; i < n; ++i) {
+      const int t = t0 + i;
+      const S* qi = q + (size_t)t * d;
+      const S* dOt = dO + (size_t)t * d;
+      matvec(W, qi, d, y.data());
+      for (int j = 0; j <= i; ++j) {
+        const S a = etas[j] * dot(k + (size_t)(t0 + j) * d, qi, d);
+        for (int r = 0; r < d; ++r) y[r] -= a * Gs[(size_t)j * d + r];
+      }
+      if (gate_logit && (mode & kGateChannel)) {
+        for (int r = 0; r < d; ++r) {
+          const S g = sigmoid(gate_logit[(size_t)t * d + r]);
+          dy[r] = g * dOt[r];
+          dgate[(size_t)t * d + r] = dOt[r] * y[r] * g * (S(1) - g);
+        }
+      } else if (gate_logit) {
+        const S g = sigmoid(gate_logit[t]);
+        S acc = 0;
+        for (int r = 0; r < d; ++r) {
+          dy[r] = g * dOt[r];
+          acc += dOt[r] * y[r];
+        }
+        dgate[t] = acc * g * (S(1) - g);
+      } else {
+        for (int r = 0; r < d; ++r) dy[r] = dOt[r];
+      }
+      // y = W_s q_i - sum_{j<=i} eta_j (k_j . q_i) G_j
+      for (int cc = 0; cc < d; ++cc) {
+        S acc = 0;
+        for (int r = 0; r < d; ++r) acc += W[r * d + cc] * dy[r];
+        dq[(size_t)t * d + cc] = acc;
+      }
+      for (int r = 0; r < d; ++r)
+        for (int cc = 0; cc < d; ++cc) dWs[r * d + cc] += dy[r] * qi[cc];
+      for (int j = 0; j <= i; ++j) {
+        const S* kj = k + (size_t)(t0 + j) * d;
+        const S* Gj = Gs.data() + (size_t)j * d;
+        const S kq = dot(kj, qi, d);
+        const S dyG = dot(dy.data(), Gj, d);
+        for (int cc = 0; cc < d; ++cc) {
+          dq[(size_t)t * d + cc] -= etas[j] * dyG * kj[cc];
+          dk[(size_t)(t0 + j) * d + cc] -= etas[j] * dyG * qi[cc];
+        }
+        detas[j] -= kq * dyG;
+        for (int r = 0; r < d; ++r) dGs[(size_t)j * d + r] -= etas[j] * kq * dy[r];
+      }
+    }
+    // G_j = G(z_j), z_j = W_s k_j
+    for (int j = 0; j < n; ++j) {
+      const int t = t0 + j;
+      const S* kj = k + (size_t)t * d;
+      matvec(W, kj, d, z.data());
+      lngrad_backward(z.data(), v + (size_t)t * d, gamma, beta, d, eps, mode,
+                      dGs.data() + (size_t)j * d, dz.data(), dv + (size_t)t * d, dgamma, dbeta);
+      for (int cc = 0; cc < d; ++cc) {
+        S acc = 0;
+        for (int r = 0; r < d; ++r) acc += W[r * d + cc] * dz[r];
+        dk[(size_t)t * d + cc] += acc;
+      }
+      for (int r = 0; r < d; ++r)
+        for (int cc = 0; cc < d; ++cc) dWs[r * d + cc] += dz[r] * kj[cc];
+      deta[t] = upd ? detas[j] * sgs[j] * (S(1) - sgs[j]) / S(d) : S(0);
+    }
+    dW.swap(dWs);
+  }
+  std::memcpy(dW0, dW.data(), sizeof(S) * d * d);
+}
+
 }  // namespace
 
 extern "C" {
@@ -491,8 +621,8 @@ extern "C" {
 // plus dO [B, H, T, d] and dW_T [B, H, d, d]. Writes dq, dk, dv [B, H, T, d],
 // deta [B, H, T], dgate (shape of gate_logit; may be null when gate_logit is),
 // dW0 [B, H, d, d], dgamma, dbeta [H, d] (summed over the batch rows; ignored
-// with NO_LN). Returns 0, or -1 on an argument it does not take (mini-batch
-// mode, the ablation gradient).
+// with NO_LN). Per-token or mini-batch mode. Returns 0, or -1 on an argument
+// it does not take (the ablation gradient, the SiLU variant).
 int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
                             const double* eta_logit, const double* gate_logit,
                             const double* W0, const double* gamma, const double* beta,
@@ -501,7 +631,7 @@ int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
                             double* dq, double* dk, double* dv, double* deta, double* dgate,
                             double* dW0, double* dgamma, double* dbeta) {
   if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return -1;
-  if (mode & (kMiniBatch | kGradAblate | kNormMatch | kKqSilu)) return -1;
+  if (mode & (kGradAblate | kNormMatch | kKqSilu)) return -1;
   if (!q || !k || !v || !eta_logit || !W0 || !dO || !dW_T || !dq || !dk || !dv || !deta ||
       !dW0)
     return -1;
@@ -521,8 +651,9 @@ int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
     const int bi = (int)(bh / H);
     const int h = (int)(bh % H);
     const size_t tok = (size_t)bh * T;
-    backward_one_head<double>(
-        q + tok * d, k + tok * d, v + tok * d, eta_logit + tok,
+    auto one = (mode & kMiniBatch) ? backward_one_head_minibatch<double>
+                                   : backward_one_head<double>;
+    one(q + tok * d, k + tok * d, v + tok * d, eta_logit + tok,
         gate_logit ? gate_logit + tok * gstride : nullptr, W0 + (size_t)bh * d * d,
         no_ln ? ones.data() : gamma + (size_t)h * d, no_ln ? zeros.data() : beta + (size_t)h * d,
         T, d, eps, mode, b, mask ? mask + (size_t)bi * n_chunks : nullptr, dO + tok * d,

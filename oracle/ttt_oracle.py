@@ -157,8 +157,8 @@ def backward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, dO, dW_T, *, eps: 
 
     Shapes as for ``forward``; dO [B, H, T, d], dW_T [B, H, d, d]. Returns a dict
     with dq, dk, dv, deta_logit, dgate_logit (None without a gate), dW0, dgamma,
-    dbeta (summed over the batch rows; None with NO_LN). Per-token mode with
-    the SIMPLE, LN-Jacobian or no-LayerNorm gradient only.
+    dbeta (summed over the batch rows; None with NO_LN). Per-token or
+    mini-batch mode, with the SIMPLE, LN-Jacobian or no-LayerNorm gradient.
     """
     lib = _load()
     dp = ctypes.c_double

@@ -47,6 +47,8 @@ MUTATIONS = [
     ("backward_drops_explicit_1_over_s", "      ds -= dG[f] * G[f] / s;", "      ds -= 0 * G[f];"),
     ("backward_dk_without_update_term", "      dk[(size_t)t * d + c] = -eta * acc;",
      "      dk[(size_t)t * d + c] = 0;"),
+    ("backward_minibatch_without_readout_terms", "const S dyG = dot(dy.data(), Gj, d);",
+     "const S dyG = 0;"),
     ("scalar_gate_ignored", "  return sigmoid(gate_logit[t]);", "  return S(1);"),
     ("gate_channel_wrong_feature", "sigmoid(gate_logit[(size_t)t * d + r])",
      "sigmoid(gate_logit[(size_t)t * d + (d - 1 - r)])"),

@@ -532,6 +532,13 @@ def test_backward_matches_finite_differences(grad):
     _fd_check_backward(inp, grad, b=2, eps=1e-5, seed=46)
 
 
+@pytest.mark.parametrize("grad", [0, GRAD_LNJAC, NO_LN], ids=["simple", "lnjac", "no_ln"])
+def test_backward_minibatch_matches_finite_differences(grad):
+    """Mini-batch mode, b = 3 over T = 8 (ragged tail), with a mask."""
+    inp = make_inputs(1, 2, 8, 4, seed=52 + grad, random_affine=True, mask_p=0.6, b=3)
+    _fd_check_backward(inp, MINIBATCH | grad, b=3, eps=1e-5, seed=53)
+
+
 def test_backward_per_feature_gate_and_no_gate():
     inp = make_inputs(1, 1, 5, 4, seed=47, random_affine=True, gate_channel=True)
     _fd_check_backward(inp, GRAD_LNJAC | GATE_CHANNEL, b=16, eps=1e-5, seed=48)
@@ -542,7 +549,7 @@ def test_backward_per_feature_gate_and_no_gate():
 def test_backward_rejects_what_it_does_not_take():
     inp = f64(make_inputs(1, 1, 4, 4, seed=51))
     z = np.zeros_like(inp["q"])
-    for mode in (MINIBATCH, GRAD_ABLATE, KQ_SILU):
+    for mode in (GRAD_ABLATE, KQ_SILU):
         with pytest.raises(ValueError):
             oracle.backward(inp["q"], inp["k"], inp["v"], inp["eta_logit"], inp["gate_logit"],
                             inp["W0"], inp["gamma"], inp["beta"], z, np.zeros_like(inp["W0"]),
