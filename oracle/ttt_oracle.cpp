@@ -342,14 +342,16 @@ void lngrad_backward(const S* z, const S* v, const S* gamma, const S* beta, int 
     xhat[f] = (z[f] - mu) / s;
     err[f] = gamma[f] * xhat[f] + beta[f] - v[f];
   }
-  S ds = 0;  // dL/ds through G's explicit 1/s (LN-Jacobian form only)
-  std::vector<S> derr(d);
-  if (mode & kLnJacobian) {
-    // G = (g - mean g - xhat mean(g xhat)) / s, g = gamma err
+  S ds = 0;  // dL/ds through G's explicit 1/s (the Jacobian forms only)
+  std::vector<S> derr(d, S(0));
+  const bool ablate = mode & kGradAblate;
+  if (mode & (kLnJacobian | kGradAblate)) {
+    // G = (g - mean g - xhat mean(g xhat)) / s, g = gamma err (ablation:
+    // g = -gamma v, which does not depend on z)
     std::vector<S> g(d), G(d);
     S a = 0, c = 0, mdG = 0, mdGx = 0;
     for (int f = 0; f < d; ++f) {
-      g[f] = gamma[f] * err[f];
+      g[f] = ablate ? -gamma[f] * v[f] : gamma[f] * err[f];
       a += g[f];
       c += g[f] * xhat[f];
       mdG += dG[f];
@@ -364,8 +366,13 @@ void lngrad_backward(const S* z, const S* v, const S* gamma, const S* beta, int 
       const S dg = (dG[f] - mdG - xhat[f] * mdGx) / s;       // J^T is symmetric
       dxhat[f] += (-dG[f] * c - g[f] * mdGx) / s;
       ds -= dG[f] * G[f] / s;
-      dgamma[f] += dg * err[f];
-      derr[f] = dg * gamma[f];
+      if (ablate) {
+        dgamma[f] -= dg * v[f];
+        dv[f] -= dg * gamma[f];
+      } else {
+        dgamma[f] += dg * err[f];
+        derr[f] = dg * gamma[f];
+      }
     }
   } else {  // G = err
     for (int f = 0; f < d; ++f) derr[f] = dG[f];
@@ -621,8 +628,8 @@ extern "C" {
 // plus dO [B, H, T, d] and dW_T [B, H, d, d]. Writes dq, dk, dv [B, H, T, d],
 // deta [B, H, T], dgate (shape of gate_logit; may be null when gate_logit is),
 // dW0 [B, H, d, d], dgamma, dbeta [H, d] (summed over the batch rows; ignored
-// with NO_LN). Per-token or mini-batch mode. Returns 0, or -1 on an argument
-// it does not take (the ablation gradient, the SiLU variant).
+// with NO_LN). Per-token or mini-batch mode, every gradient form but norm
+// matching, the SiLU variant. Returns 0, or -1 on an argument it does not take.
 int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
                             const double* eta_logit, const double* gate_logit,
                             const double* W0, const double* gamma, const double* beta,
@@ -631,7 +638,8 @@ int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
                             double* dq, double* dk, double* dv, double* deta, double* dgate,
                             double* dW0, double* dgamma, double* dbeta) {
   if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return -1;
-  if (mode & (kGradAblate | kNormMatch | kKqSilu)) return -1;
+  if (mode & kNormMatch) return -1;
+  if ((mode & kGradAblate) && (mode & kNoLayerNorm)) return -1;
   if (!q || !k || !v || !eta_logit || !W0 || !dO || !dW_T || !dq || !dk || !dv || !deta ||
       !dW0)
     return -1;
@@ -647,6 +655,21 @@ int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
   }
   const size_t gstride = (mode & kGateChannel) ? (size_t)d : 1;
   std::memset(dv, 0, sizeof(double) * (size_t)B * H * T * d);  // accumulated per token
+  // the SiLU variant: run on SiLU(q), SiLU(k), then chain dq, dk through SiLU
+  const size_t ntok = (size_t)B * H * T * d;
+  std::vector<double> qs, ks;
+  const double* q_in = q;
+  const double* k_in = k;
+  if (mode & kKqSilu) {
+    qs.resize(ntok);
+    ks.resize(ntok);
+    for (size_t i = 0; i < ntok; ++i) {
+      qs[i] = silu(q[i]);
+      ks[i] = silu(k[i]);
+    }
+    q = qs.data();
+    k = ks.data();
+  }
   for (long long bh = 0; bh < (long long)B * H; ++bh) {
     const int bi = (int)(bh / H);
     const int h = (int)(bh % H);
@@ -661,6 +684,14 @@ int ttt_oracle_backward_f64(const double* q, const double* k, const double* v,
         gate_logit ? dgate + tok * gstride : nullptr, dW0 + (size_t)bh * d * d,
         no_ln ? sink_g.data() : dgamma + (size_t)h * d,
         no_ln ? sink_b.data() : dbeta + (size_t)h * d);
+  }
+  if (mode & kKqSilu) {
+    // d SiLU(x) / dx = sigmoid(x) (1 + x (1 - sigmoid(x)))
+    for (size_t i = 0; i < ntok; ++i) {
+      const double sq = sigmoid(q_in[i]), sk = sigmoid(k_in[i]);
+      dq[i] *= sq * (1.0 + q_in[i] * (1.0 - sq));
+      dk[i] *= sk * (1.0 + k_in[i] * (1.0 - sk));
+    }
   }
   return 0;
 }

@@ -158,7 +158,8 @@ def backward(q, k, v, eta_logit, gate_logit, W0, gamma, beta, dO, dW_T, *, eps: 
     Shapes as for ``forward``; dO [B, H, T, d], dW_T [B, H, d, d]. Returns a dict
     with dq, dk, dv, deta_logit, dgate_logit (None without a gate), dW0, dgamma,
     dbeta (summed over the batch rows; None with NO_LN). Per-token or
-    mini-batch mode, with the SIMPLE, LN-Jacobian or no-LayerNorm gradient.
+    mini-batch mode; the SIMPLE, LN-Jacobian, no-LayerNorm or ablation gradient
+    (not norm matching); the SiLU variant (KQ_SILU).
     """
     lib = _load()
     dp = ctypes.c_double

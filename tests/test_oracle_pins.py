@@ -546,10 +546,18 @@ def test_backward_per_feature_gate_and_no_gate():
     _fd_check_backward(inp, GRAD_LNJAC, b=16, eps=1e-5, seed=50)
 
 
+@pytest.mark.parametrize("mode", [GRAD_ABLATE, MINIBATCH | GRAD_ABLATE, KQ_SILU | GRAD_LNJAC,
+                                  MINIBATCH | KQ_SILU],
+                         ids=["ablate", "ablate_minibatch", "silu_lnjac", "silu_minibatch"])
+def test_backward_ablation_and_silu_match_finite_differences(mode):
+    inp = make_inputs(1, 2, 6, 4, seed=54 + mode % 97, random_affine=True, mask_p=0.7, b=2)
+    _fd_check_backward(inp, mode, b=2, eps=1e-5, seed=55)
+
+
 def test_backward_rejects_what_it_does_not_take():
     inp = f64(make_inputs(1, 1, 4, 4, seed=51))
     z = np.zeros_like(inp["q"])
-    for mode in (GRAD_ABLATE, KQ_SILU):
+    for mode in (GRAD_ABLATE | GRAD_NORM_MATCH, GRAD_ABLATE | NO_LN):
         with pytest.raises(ValueError):
             oracle.backward(inp["q"], inp["k"], inp["v"], inp["eta_logit"], inp["gate_logit"],
                             inp["W0"], inp["gamma"], inp["beta"], z, np.zeros_like(inp["W0"]),
