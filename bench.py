@@ -61,17 +61,44 @@ def _csrc_hash() -> str:
     return h.hexdigest()[:16]
 
 
+# The files each kernel's binary is built from: the translation unit that
+# instantiates it and everything that unit includes, plus (for every kernel)
+# the launcher that sets its parameters, the public header and the build flags.
+_KERNEL_SOURCES = {
+    "scan_cluster": ["cluster.cu", "scan_cluster.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
+    "scan_simt": ["simt_f32.cu", "simt_bf16.cu", "scan_simt.cuh", "launch.h", "common.cuh"],
+    # one translation unit holds both
+    "scan_tc": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
+    "decode_step": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h",
+                    "common.cuh"],
+}
+
+
+def _kernel_hash(kernel_key: str) -> str:
+    pkg = ROOT / "test_sequence_layers_02_b200"
+    files = sorted(set(_KERNEL_SOURCES[kernel_key] + ["ttt_scan.cu"]))
+    paths = [pkg / "csrc" / f for f in files] + [pkg / "build.py", ROOT / "include" / "ttt_scan.h"]
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(p.name.encode())
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
 def _traffic(kernel_key: str, head_tokens_per_launch: int):
     """DRAM bytes (read + write) per launch from the committed ncu capture of
-    that kernel, scaled from its case by head-tokens; None if the kernel
+    that kernel, scaled from its case by head-tokens; None if that kernel's
     sources changed since the capture."""
     if not PROFILE_TRAFFIC.exists():
         return None
     d = json.loads(PROFILE_TRAFFIC.read_text())
-    if d.get("csrc_hash") != _csrc_hash():
-        return None
     e = d.get("kernels", {}).get(kernel_key)
     if e is None:
+        return None
+    if "sources_hash" in e:
+        if e["sources_hash"] != _kernel_hash(kernel_key):
+            return None
+    elif d.get("csrc_hash") != _csrc_hash():
         return None
     return round(e["bytes_per_head_token"] * head_tokens_per_launch)
 
