@@ -1,14 +1,15 @@
 #!/usr/bin/env python
 """Throughput of the B200 TTT-Linear scan, as one JSON line.
 
-Headline workload: the per-token fp32 scan at d = 64 (B=4, H=4, T=2048, q and k
-L2-normalised, eps = 1e-6); one step is one pass with the simplified gradient
-plus one pass with the LayerNorm-Jacobian gradient over the same inputs.
-The metric is head-tokens per second (B*H*T per pass) and the fraction of the
-binding roofline of the dominant kernel. On one GPU the other d = 64 workloads
-(mini-batch bf16 at three shapes, the per-token bf16-input pass, and the
-streaming decode step over 16384 heads) are measured too and reported under
-``by_workload``.
+Headline workload: workload 5, the largest single-GPU configuration (the long
+gated mini-batch scan: B=2, H=32, T=32768, d=64, b=16, bf16 inputs, fp32 state,
+a SKIP/UPDATE mask ~ Bernoulli(0.5) per chunk, LN-Jacobian gradient) on the
+tcgen05 kernel. The metric is head-tokens per second (B*H*T per step) and the
+fraction of the binding roofline of the kernel. On one GPU every other
+workload is measured too and reported under ``by_workload`` with its own
+roofline, CPU-oracle baseline and end-to-end figure: 1 (d = 16, per-token),
+2 (per-token fp32, both gradient forms), 3 and 4 (mini-batch on tensor cores),
+4pt (workload 4's per-token pass) and dec (the streaming decode step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -25,7 +26,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -37,6 +37,8 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 METRIC = "TTT-Linear scan head-tokens/sec at d=64 on 1 B200; % of binding roofline"
+HEADLINE = "5"
+EXTRA = ["1", "2", "3", "4", "4pt", "dec"]
 L2_FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PROFILE_TRAFFIC = ROOT / "profiles" / "dram_traffic.json"
 
@@ -52,29 +54,24 @@ def _peaks():
                 sm_max_mhz=1965.0, source="fallback")
 
 
-def _csrc_hash() -> str:
-    h = hashlib.sha256()
-    csrc = ROOT / "test_sequence_layers_02_b200" / "csrc"
-    for p in sorted(csrc.glob("*")) + sorted((ROOT / "include").glob("*.h")):
-        h.update(p.name.encode())
-        h.update(p.read_bytes())
-    return h.hexdigest()[:16]
-
-
 # The files each kernel's binary is built from: the translation unit that
 # instantiates it and everything that unit includes, plus (for every kernel)
 # the launcher that sets its parameters, the public header and the build flags.
 _KERNEL_SOURCES = {
     "scan_cluster": ["cluster.cu", "scan_cluster.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
-    "scan_simt": ["simt_f32.cu", "simt_bf16.cu", "scan_simt.cuh", "launch.h", "common.cuh"],
-    # one translation unit holds both
+    "scan_simt": ["simt.cu", "scan_simt.cuh", "launch.h", "common.cuh"],
+    # one translation unit holds the tensor-core and decode kernels
     "scan_tc": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
     "decode_step": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h",
                     "common.cuh"],
 }
+# Captures: a kernel may have several (e.g. the tensor-core kernel with and
+# without a SKIP/UPDATE mask); each names the kernel whose sources it covers.
+_CAPTURE_KERNEL = {"scan_tc_masked": "scan_tc", "scan_simt_4pt": "scan_simt"}
 
 
 def _kernel_hash(kernel_key: str) -> str:
+    kernel_key = _CAPTURE_KERNEL.get(kernel_key, kernel_key)
     pkg = ROOT / "test_sequence_layers_02_b200"
     files = sorted(set(_KERNEL_SOURCES[kernel_key] + ["ttt_scan.cu"]))
     paths = [pkg / "csrc" / f for f in files] + [pkg / "build.py", ROOT / "include" / "ttt_scan.h"]
@@ -85,20 +82,15 @@ def _kernel_hash(kernel_key: str) -> str:
     return h.hexdigest()[:16]
 
 
-def _traffic(kernel_key: str, head_tokens_per_launch: int):
-    """DRAM bytes (read + write) per launch from the committed ncu capture of
-    that kernel, scaled from its case by head-tokens; None if that kernel's
-    sources changed since the capture."""
+def _traffic(capture_key: str, head_tokens_per_launch: int):
+    """DRAM bytes (read + write) per launch from the committed ncu capture,
+    scaled from its case by head-tokens; None if the kernel's sources changed
+    since the capture (or it was never captured)."""
     if not PROFILE_TRAFFIC.exists():
         return None
     d = json.loads(PROFILE_TRAFFIC.read_text())
-    e = d.get("kernels", {}).get(kernel_key)
-    if e is None:
-        return None
-    if "sources_hash" in e:
-        if e["sources_hash"] != _kernel_hash(kernel_key):
-            return None
-    elif d.get("csrc_hash") != _csrc_hash():
+    e = d.get("kernels", {}).get(capture_key)
+    if e is None or e.get("sources_hash") != _kernel_hash(capture_key):
         return None
     return round(e["bytes_per_head_token"] * head_tokens_per_launch)
 
@@ -107,8 +99,31 @@ def _traffic(kernel_key: str, head_tokens_per_launch: int):
 # Workloads
 # ---------------------------------------------------------------------------
 
+def _dev_inputs(inp, w, device, decode=False):
+    import torch
+
+    def dev(key):
+        a = inp.get(key)
+        if a is None:
+            return None
+        if w.in_bf16 and key in ("q", "k", "v", "eta_logit", "gate_logit"):
+            a = torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16)
+        else:
+            a = torch.from_numpy(np.ascontiguousarray(a))
+        if decode and key in ("q", "k", "v", "eta_logit", "gate_logit"):
+            a = a[:, :, 0].contiguous()
+        return a.to(device)
+
+    t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
+    m = inp.get("mask")
+    t["mask"] = None if m is None else torch.from_numpy(np.ascontiguousarray(m)).to(device)
+    return t
+
+
 class Job:
-    """One workload resident on the device, with its step function."""
+    """One scan workload resident on the device, with its step function."""
+
+    decode = False
 
     def __init__(self, name: str, device, seed_offset: int = 0):
         import torch
@@ -121,49 +136,40 @@ class Job:
         inp = make_workload(w, seed=w.seed + seed_offset) if seed_offset else make_workload(w)
         self.inp = inp
         self.mask_np = inp.get("mask")
-
-        def dev(key):
-            a = inp.get(key)
-            if a is None:
-                return None
-            if w.in_bf16 and key in ("q", "k", "v", "eta_logit", "gate_logit"):
-                return torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16).to(device)
-            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
-
-        self.t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
-        self.t["mask"] = None if self.mask_np is None else torch.from_numpy(self.mask_np).to(device)
+        self.t = _dev_inputs(inp, w, device)
         self.out_dtype = torch.bfloat16 if w.out_bf16 else torch.float32
-        t = self.t
-        self.o = torch.empty(t["q"].shape, dtype=self.out_dtype, device=device)
-        self.W_T = torch.empty(t["W0"].shape, dtype=torch.float32, device=device)
+        self.outs = [(torch.empty(self.t["q"].shape, dtype=self.out_dtype, device=device),
+                      torch.empty(self.t["W0"].shape, dtype=torch.float32, device=device))
+                     for _ in self.passes]
         self.scan = ttt_scan.scan
+        self.streams = None
 
     @property
     def head_tokens_per_step(self) -> int:
         return self.w.head_tokens * len(self.passes)
 
+    def _call(self, t, ps, o, wt, stream=None):
+        w = self.w
+        return self.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"],
+                         t["gamma"], t["beta"], eps=w.eps, minibatch=w.minibatch, b=w.b,
+                         mask=t["mask"], out_dtype=self.out_dtype, o=o, W_T=wt, stream=stream,
+                         **ps)
+
     def step(self):
         """One step: every pass over the resident inputs. Independent passes (the
         two gradient forms of workload 2) run concurrently on their own streams."""
         import torch
-        t, w = self.t, self.w
         if len(self.passes) == 1:
-            self.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"],
-                      t["gamma"], t["beta"], eps=w.eps, minibatch=w.minibatch, b=w.b,
-                      mask=t["mask"], out_dtype=self.out_dtype, o=self.o, W_T=self.W_T,
-                      **self.passes[0])
+            self._call(self.t, self.passes[0], *self.outs[0])
             return
         main = torch.cuda.current_stream()
-        if not hasattr(self, "streams"):
+        if self.streams is None:
             self.streams = [torch.cuda.Stream() for _ in self.passes]
-            self.outs = [(torch.empty_like(self.o), torch.empty_like(self.W_T)) for _ in self.passes]
         start = torch.cuda.Event()
         start.record(main)
         for st, ps, (o, wt) in zip(self.streams, self.passes, self.outs):
             st.wait_event(start)
-            self.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"],
-                      t["gamma"], t["beta"], eps=w.eps, minibatch=w.minibatch, b=w.b,
-                      mask=t["mask"], out_dtype=self.out_dtype, o=o, W_T=wt, stream=st, **ps)
+            self._call(self.t, ps, o, wt, stream=st)
         for st in self.streams:
             ev = torch.cuda.Event()
             ev.record(st)
@@ -172,7 +178,14 @@ class Job:
     def launches_per_step(self) -> int:
         return len(self.passes)
 
+    def steps_per_chain(self) -> int:
+        """Dependent steps of one head's recurrence (chunks, or tokens)."""
+        return self.w.n_chunks if self.w.minibatch else self.w.T
+
     # --- algorithmic work per step -------------------------------------------------
+    def update_fraction(self) -> float:
+        return 1.0 if self.mask_np is None else float(self.mask_np.mean())
+
     def flops_per_step(self) -> float:
         w = self.w
         d, b = w.d, w.b
@@ -180,7 +193,7 @@ class Job:
             return 6.0 * d * d * w.head_tokens * len(self.passes)
         f_upd = 6.0 * d * d + 2.0 * d * (b + 1)
         f_skip = 2.0 * d * d
-        frac = 1.0 if self.mask_np is None else float(self.mask_np.mean())
+        frac = self.update_fraction()
         return w.head_tokens * (frac * f_upd + (1 - frac) * f_skip)
 
     def bytes_per_step(self) -> float:
@@ -205,7 +218,7 @@ class Job:
         return total + state
 
     def bound(self):
-        return "hbm" if self.w.minibatch else "alu"
+        return "hbm" if (self.w.minibatch or self.w.d == 16) else "alu"
 
     def kernel_key(self) -> str:
         from test_sequence_layers_02_b200 import ttt_scan
@@ -216,9 +229,38 @@ class Job:
                 ttt_scan.KERNEL_CUDA_CORE_CLUSTER: "scan_cluster",
                 ttt_scan.KERNEL_TENSOR_CORE: "scan_tc"}[k]
 
+    def capture_key(self) -> str:
+        k = self.kernel_key()
+        if k == "scan_tc" and self.mask_np is not None:
+            return "scan_tc_masked"
+        if k == "scan_simt" and self.name == "4pt":
+            return "scan_simt_4pt"
+        return k
+
+    # --- end to end ------------------------------------------------------------------
+    def e2e_setup(self):
+        """Pinned host copies of the inputs and of every pass's outputs."""
+        import torch
+        self.h_in = {k: (None if v is None else v.cpu().pin_memory()) for k, v in self.t.items()}
+        self.h_out = [(torch.empty(self.t["q"].shape, dtype=self.out_dtype).pin_memory(),
+                       torch.empty(self.t["W0"].shape, dtype=torch.float32).pin_memory())
+                      for _ in self.passes]
+        h2d = sum(v.numel() * v.element_size() for v in self.h_in.values() if v is not None)
+        d2h = sum(o.numel() * o.element_size() + x.numel() * x.element_size()
+                  for o, x in self.h_out)
+        return h2d * len(self.passes), d2h
+
+    def e2e_step(self):
+        """Every pass through the public call with host buffers: the call copies
+        its inputs in, scans and copies o and W_T back before returning."""
+        for ps, (o, wt) in zip(self.passes, self.h_out):
+            self._call(self.h_in, ps, o, wt)
+
 
 class DecodeJob:
     """The streaming decode step over many heads, W updated in place each step."""
+
+    decode = True
 
     def __init__(self, name: str, device):
         import torch
@@ -230,20 +272,7 @@ class DecodeJob:
         inp = make_workload(w)
         self.inp = inp
         self.mask_np = None
-
-        def dev(key):
-            a = inp.get(key)
-            if a is None:
-                return None
-            if w.in_bf16 and key in ("q", "k", "v", "eta_logit", "gate_logit"):
-                a = torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16)
-            else:
-                a = torch.from_numpy(np.ascontiguousarray(a))
-            if key in ("q", "k", "v", "eta_logit", "gate_logit"):
-                a = a[:, :, 0].contiguous()
-            return a.to(device)
-
-        self.t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
+        self.t = _dev_inputs(inp, w, device, decode=True)
         self.out_dtype = torch.bfloat16 if w.out_bf16 else torch.float32
         self.o = torch.empty(self.t["q"].shape, dtype=self.out_dtype, device=device)
         self.step_fn = ttt_scan.decode_step
@@ -252,12 +281,19 @@ class DecodeJob:
     def head_tokens_per_step(self) -> int:
         return self.w.heads
 
+    def _call(self, t, W, o):
+        w = self.w
+        return self.step_fn(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], W,
+                            t["gamma"], t["beta"], eps=w.eps, lnjac=w.lnjac,
+                            out_dtype=self.out_dtype, o=o)
+
     def step(self):
-        t, w = self.t, self.w
-        self.step_fn(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"],
-                     t["beta"], eps=w.eps, lnjac=w.lnjac, out_dtype=self.out_dtype, o=self.o)
+        self._call(self.t, self.t["W0"], self.o)
 
     def launches_per_step(self) -> int:
+        return 1
+
+    def steps_per_chain(self) -> int:
         return 1
 
     def flops_per_step(self) -> float:
@@ -276,6 +312,27 @@ class DecodeJob:
 
     def kernel_key(self) -> str:
         return "decode_step"
+
+    def capture_key(self) -> str:
+        return "decode_step"
+
+    def e2e_setup(self):
+        import torch
+        self.h_in = {k: (None if v is None else v.cpu().pin_memory()) for k, v in self.t.items()}
+        self.h_o = torch.empty(self.t["q"].shape, dtype=self.out_dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in self.h_in.values() if v is not None)
+        d2h = self.h_o.numel() * self.h_o.element_size() + \
+            self.h_in["W0"].numel() * self.h_in["W0"].element_size()
+        return h2d, d2h
+
+    def e2e_step(self):
+        """The public call with host buffers: the state W goes in and comes back
+        updated, with the token's inputs in and o out."""
+        self._call(self.h_in, self.h_in["W0"], self.h_o)
+
+
+def _make_job(name, device, seed_offset=0):
+    return DecodeJob(name, device) if name == "dec" else Job(name, device, seed_offset)
 
 
 def _flush(buf):
@@ -326,7 +383,6 @@ class ClockSampler:
         self.reasons = set()
         self.max_mhz = None
         self._stop = threading.Event()
-        self._nvml = None
 
     def _handle(self):
         import pynvml
@@ -399,14 +455,17 @@ def _fp32_peak(device):
 
 
 def _roofline(job, per_launch_s, peaks, fp32_meas_tflops, n_sm):
+    """Binding roofline of the job's kernel: HBM for the mini-batch, decode and
+    d = 16 kernels, FP32 FMA (plain ALU arithmetic) for the per-token d = 64 ones."""
     launches = job.launches_per_step()
+    head_tokens = job.head_tokens_per_step // launches
+    traffic = _traffic(job.capture_key(), head_tokens)
     if job.bound() == "alu":
         flops = job.flops_per_step() / launches
         achieved = flops / per_launch_s / 1e12
         peak = n_sm * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
         return {"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 2),
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": _traffic(job.kernel_key(), job.w.head_tokens),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                 "algorithmic_flops_per_launch": flops,
                 "peak_basis": f"{n_sm} SM x 128 FP32 lanes x 2 x {peaks['sm_max_mhz']:.0f} MHz",
                 "fp32_probe_tflops": round(fp32_meas_tflops, 2),
@@ -416,98 +475,88 @@ def _roofline(job, per_launch_s, peaks, fp32_meas_tflops, n_sm):
     achieved = byts / per_launch_s / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": _traffic(job.kernel_key(), job.w.head_tokens), "kernel": job.kernel_key(),
+            "traffic": traffic, "kernel": job.kernel_key(),
             "algorithmic_bytes_per_launch": round(byts),
             "peak_basis": f"{peaks['source']} HBM copy bandwidth"}
 
 
-def _oracle_pass(w, inp, passes, heads, threads):
-    """One oracle run over the sampled heads (OpenMP over heads), every pass."""
+# ---------------------------------------------------------------------------
+# The oracle on the host cores (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_heads(job, heads, threads):
+    """One oracle run over the first `heads` heads of the workload (in batch-row
+    order, OpenMP over heads), every pass."""
     import oracle
+    w, inp = job.w, job.inp
     f64 = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
-    sel = lambda a: None if a is None else f64(a[:, :heads] if a.ndim >= 3 else a)
-    rows = heads if heads < w.H else w.H
-    for ps in passes:
+    if job.decode:
+        take = lambda a: None if a is None else a[:, :, :1]
+    else:
+        take = lambda a: a
+    rows = max(1, -(-heads // w.H))
+    hh = min(heads, w.H)
+    sel = lambda a: None if a is None else f64(take(a)[:rows, :hh])
+    m = inp.get("mask")
+    for ps in job.passes:
         mode = (1 if w.minibatch else 0) | (2 if ps["lnjac"] else 0)
-        m = inp.get("mask")
-        if heads >= w.H:
-            oracle.forward(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["eta_logit"]),
-                           f64(inp["gate_logit"]), f64(inp["W0"]), f64(inp["gamma"]),
-                           f64(inp["beta"]), eps=w.eps, mode=mode, b=w.b, mask=m, nthreads=threads)
-        else:
-            oracle.forward(sel(inp["q"][:1]), sel(inp["k"][:1]), sel(inp["v"][:1]),
-                           sel(inp["eta_logit"][:1]), sel(inp["gate_logit"][:1]),
-                           sel(inp["W0"][:1]), f64(inp["gamma"][:rows]), f64(inp["beta"][:rows]),
-                           eps=w.eps, mode=mode, b=w.b, mask=None if m is None else m[:1],
-                           nthreads=threads)
+        oracle.forward(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(inp["eta_logit"]),
+                       sel(inp["gate_logit"]), sel(inp["W0"]), f64(inp["gamma"][:hh]),
+                       f64(inp["beta"][:hh]), eps=w.eps, mode=mode, b=w.b,
+                       mask=None if m is None else m[:rows], nthreads=threads)
+    return rows * hh
 
 
-def _cpu_baseline(job, min_seconds=8.0):
-    """The oracle, as it stands, on the host cores: head-tokens/s over the whole workload."""
+def _oracle_sample(job, budget_s):
+    """Time the oracle, as it stands, on a bounded sample of the workload: whole
+    heads (all T tokens of each), as many as fill about `budget_s` seconds on the
+    host's cores. Returns (head-tokens/s, cores, sample description)."""
     w = job.w
     cores = len(os.sched_getaffinity(0))
-    used = min(cores, w.heads)
+    T = 1 if job.decode else w.T
+    heads = min(w.heads, cores)
     t0 = time.perf_counter()
-    reps = 0
-    while True:
-        _oracle_pass(w, job.inp, job.passes, w.heads, used)
-        reps += 1
+    done = _oracle_heads(job, heads, min(cores, heads))
+    el = time.perf_counter() - t0
+    reps, ht = 1, done * T * len(job.passes)
+    if el < budget_s and heads < w.heads:
+        # scale the sample up to the budget (whole rows of heads), then time it
+        want = int(heads * budget_s / max(el, 1e-3))
+        heads = max(heads, min(w.heads, want))
+        t0 = time.perf_counter()
+        done = _oracle_heads(job, heads, min(cores, heads))
         el = time.perf_counter() - t0
-        if el >= min_seconds or reps >= 8:
-            break
-    return {"value": job.head_tokens_per_step * reps / el, "unit": "head-tokens/s",
-            "cores": used, "kind": "oracle",
-            "sample": f"whole workload {job.name} ({w.heads} heads x T={w.T} x {len(job.passes)} "
-                      f"pass(es)) x {reps} rep(s), fp64, OpenMP over heads, {el:.1f} s"}
+        ht = done * T * len(job.passes)
+    while el < budget_s and done >= w.heads and reps < 1000000:
+        t1 = time.perf_counter()
+        _oracle_heads(job, heads, min(cores, heads))
+        el += time.perf_counter() - t1
+        reps += 1
+    used = min(cores, done)
+    sample = (f"{done} of {w.heads} heads x T={T} x {len(job.passes)} pass(es) x {reps} rep(s) "
+              f"of workload {job.name}, fp64, OpenMP over heads on {used} of {cores} host cores, "
+              f"{el:.1f} s")
+    return ht * reps / el, used, sample
 
 
-def _e2e(job, steps, device):
-    """Same metric through the public API, end to end. Every step copies that
-    step's inputs from pinned host memory to the device (once: the passes share
-    them), runs the passes on their own streams as the device-timed step does,
-    copies every pass's results (o, W_T) back to pinned host memory as soon as
-    that pass ends, and waits for them on the host."""
+def _cpu_baseline(job, budget_s):
+    v, cores, sample = _oracle_sample(job, budget_s)
+    return {"value": v, "unit": "head-tokens/s", "cores": cores, "kind": "oracle",
+            "sample": sample}
+
+
+def _e2e(job, steps):
+    """The same metric through the public call with HOST buffers: every step
+    copies that step's inputs from pinned host memory, runs the kernel and
+    copies the results (o, W_T, or the decode state W) back before the call
+    returns."""
     import torch
-    from test_sequence_layers_02_b200 import ttt_scan
-    t = job.t
-    w = job.w
-    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
-    dev = {k: (None if v is None else torch.empty_like(v)) for k, v in t.items()}
-    n = len(job.passes)
-    o_h = [torch.empty(t["q"].shape, dtype=job.out_dtype).pin_memory() for _ in range(n)]
-    wt_h = [torch.empty(t["W0"].shape, dtype=torch.float32).pin_memory() for _ in range(n)]
-    o_d = [torch.empty_like(t["q"], dtype=job.out_dtype) for _ in range(n)]
-    wt_d = [torch.empty_like(t["W0"]) for _ in range(n)]
-    streams = [torch.cuda.Stream(device) for _ in range(n)]
-    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = sum(o.numel() * o.element_size() + x.numel() * x.element_size()
-              for o, x in zip(o_h, wt_h))
-
-    def step():
-        main = torch.cuda.current_stream(device)
-        for k, v in host.items():
-            if v is not None:
-                dev[k].copy_(v, non_blocking=True)
-        for i, ps in enumerate(job.passes):
-            st = streams[i]
-            st.wait_stream(main)
-            ttt_scan.scan(dev["q"], dev["k"], dev["v"], dev["eta_logit"], dev["gate_logit"],
-                          dev["W0"], dev["gamma"], dev["beta"], eps=w.eps,
-                          minibatch=w.minibatch, b=w.b, mask=dev["mask"],
-                          out_dtype=job.out_dtype, o=o_d[i], W_T=wt_d[i], stream=st, **ps)
-            with torch.cuda.stream(st):
-                o_h[i].copy_(o_d[i], non_blocking=True)
-                wt_h[i].copy_(wt_d[i], non_blocking=True)
-            main.wait_stream(st)
-        rc = ttt_scan.check_device_status(main)   # synchronises: the results are on the host
-        if rc != ttt_scan.TTT_OK:
-            raise ttt_scan.TTTScanError(rc, "device")
-
-    step()
+    h2d, d2h = job.e2e_setup()
+    job.e2e_step()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for _ in range(steps):
-        step()
+        job.e2e_step()
     torch.cuda.synchronize()
     el = time.perf_counter() - t0
     return {"value": job.head_tokens_per_step * steps / el, "unit": "head-tokens/s",
@@ -517,7 +566,7 @@ def _e2e(job, steps, device):
 
 def _workload_desc(job):
     w = job.w
-    if isinstance(job, DecodeJob):
+    if job.decode:
         return (f"TTT-Linear decode step {job.name}: one token per head, W [B,H,d,d] fp32 "
                 f"updated in place, LN-Jacobian gradient, bf16 in, bf16 out, B={w.B} H={w.H} "
                 f"d={w.d}")
@@ -528,6 +577,22 @@ def _workload_desc(job):
     extra = ", SKIP/UPDATE mask ~ Bernoulli(0.5)" if w.mask_p else ""
     return (f"TTT-Linear scan workload {job.name}: {mode}, {grad}, {dt}, B={w.B} H={w.H} "
             f"T={w.T} d={w.d}{extra}")
+
+
+def _measure(job, steps, warmup, flush_buf, peaks, fp32_tflops, n_sm):
+    ts = _time_job(job, steps, warmup, flush_buf)
+    tot = sum(ts)
+    per_launch = tot / (len(ts) * job.launches_per_step())
+    return {
+        "workload": _workload_desc(job),
+        "value": job.head_tokens_per_step * len(ts) / tot, "unit": "head-tokens/s",
+        "ms_per_step": round(tot / len(ts) * 1e3, 4),
+        "roofline": _roofline(job, per_launch, peaks, fp32_tflops, n_sm),
+        # the passes of a step run concurrently: one dependent step of a head's
+        # chain takes the step time over the chain's length
+        "chain_step_ns": round(tot / len(ts) / job.steps_per_chain() * 1e9, 2),
+        "update_fraction": round(job.update_fraction(), 4) if not job.decode else None,
+        "gpu_launches": job.launches_per_step() * len(ts)}, tot
 
 
 def shard_rows(B: int, world: int, rank: int) -> tuple:
@@ -575,7 +640,7 @@ def run_ours(args):
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     fp32_tflops, n_sm = _fp32_peak(device)
 
-    job = Job(args.workload, device, seed_offset=1000 * rank)
+    job = _make_job(args.workload, device, 1000 * rank)
     # --- headline: timed region ---
     if world > 1:
         dist.barrier()
@@ -590,7 +655,7 @@ def run_ours(args):
                                       dist if world > 1 else None)
     per_launch = total / (args.steps * job.launches_per_step())
     roof = _roofline(job, per_launch, peaks, fp32_tflops, n_sm)
-    e2e = _e2e(job, max(2, min(args.steps, 5)), device)
+    e2e = _e2e(job, max(2, min(args.steps, 5)))
     if world > 1:
         ev = torch.tensor([e2e["value"]], dtype=torch.float64, device=device)
         dist.all_reduce(ev, op=dist.ReduceOp.MIN)
@@ -598,20 +663,19 @@ def run_ours(args):
     by_workload = {}
     if world == 1 and not args.headline_only:
         for name in args.extra:
-            ej = DecodeJob(name, device) if name == "dec" else Job(name, device)
-            ts = _time_job(ej, max(3, min(args.steps, 10)), args.warmup, flush_buf)
-            tot = sum(ts)
-            pl = tot / (len(ts) * ej.launches_per_step())
-            by_workload[name] = {
-                "workload": _workload_desc(ej),
-                "value": ej.head_tokens_per_step * len(ts) / tot, "unit": "head-tokens/s",
-                "ms_per_step": round(tot / len(ts) * 1e3, 4),
-                "roofline": _roofline(ej, pl, peaks, fp32_tflops, n_sm),
-                "chain_step_ns": round(pl / max(1, ej.w.n_chunks if ej.w.minibatch else ej.w.T) * 1e9, 2),
-                "gpu_launches": ej.launches_per_step() * len(ts)}
+            if name == args.workload:
+                continue
+            ej = _make_job(name, device)
+            entry, _ = _measure(ej, max(3, min(args.steps, 10)), args.warmup, flush_buf, peaks,
+                                fp32_tflops, n_sm)
+            entry["e2e"] = _e2e(ej, 3)
+            if not args.no_cpu_baseline:
+                entry["cpu_baseline"] = _cpu_baseline(ej, args.cpu_budget_extra)
+            by_workload[name] = entry
             del ej
             torch.cuda.empty_cache()
-    cpu = _cpu_baseline(job) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    cpu = (_cpu_baseline(job, args.cpu_budget)
+           if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None)
     if rank == 0:
         w = job.w
         line = {
@@ -619,7 +683,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t_max / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic (seeded numpy PCG64; no dataset)",
+            "dtype": "bf16" if w.in_bf16 else "f32",
+            "data": "synthetic (seeded numpy PCG64; no dataset)",
             "config": {"workload": _workload_desc(job), "B": w.B, "H": w.H, "T": w.T, "d": w.d,
                        "head_tokens_per_step": job.head_tokens_per_step,
                        "l2": "flushed between timed steps (256 MB device write, untimed)",
@@ -628,9 +693,8 @@ def run_ours(args):
                                   if len(job.passes) == 2 else "one launch"),
                        "parallelism": f"heads sharded across {world} rank(s), no collective"},
             "roofline": roof,
-            # the passes of a step run concurrently, so one chain step takes the
-            # step time over the sequence length
-            "chain_step_ns": round(t_max / args.steps / w.T * 1e9, 2),
+            "chain_step_ns": round(t_max / args.steps / job.steps_per_chain() * 1e9, 2),
+            "update_fraction": None if job.decode else round(job.update_fraction(), 4),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": job.launches_per_step() * args.steps,
@@ -644,42 +708,53 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+class _HostJob:
+    """A workload's host inputs only (the reference arm needs no GPU)."""
+
+    def __init__(self, name):
+        from test_sequence_layers_02_b200.workloads import WORKLOADS, make_workload
+        self.w = WORKLOADS["2s" if name == "2" else name]
+        self.name = name
+        self.decode = False
+        self.passes = ([dict(lnjac=False), dict(lnjac=True)] if name == "2"
+                       else [dict(lnjac=self.w.lnjac)])
+        self.inp = make_workload(self.w)
+
+
 def run_reference(args):
-    """The oracle (CPU, fp64) on the headline workload, as the reference arm (rank 0 only)."""
+    """The oracle (CPU, fp64) on the headline workload, as the reference arm
+    (rank 0 only): every step is a bounded sample of whole heads, sized so that
+    a step takes a few seconds on this host."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    from test_sequence_layers_02_b200.workloads import WORKLOADS, make_workload
-    w = WORKLOADS["2s"]
-    inp = make_workload(w)
+    job = _HostJob(args.workload)
+    w = job.w
     cores = len(os.sched_getaffinity(0))
-    passes = [dict(lnjac=False), dict(lnjac=True)]
-    # one step = both gradient forms over a sample of the heads, sized so that a
-    # step takes about a second on this host (the full run stays within minutes)
     heads = min(w.heads, cores)
     t0 = time.perf_counter()
-    _oracle_pass(w, inp, passes, heads, min(cores, heads))
+    _oracle_heads(job, heads, min(cores, heads))
     first = time.perf_counter() - t0
-    if first > 3.0 and heads > 1:
-        heads = max(1, int(heads * 3.0 / first))
+    if first > args.ref_step_s and heads > 1:
+        heads = max(1, int(heads * args.ref_step_s / first))
     used = min(cores, heads)
     for _ in range(args.warmup):
-        _oracle_pass(w, inp, passes, heads, used)
+        _oracle_heads(job, heads, used)
     t0 = time.perf_counter()
+    done = 0
     for _ in range(args.steps):
-        _oracle_pass(w, inp, passes, heads, used)
+        done = _oracle_heads(job, heads, used)
     el = time.perf_counter() - t0
-    value = 2 * heads * w.T * args.steps / el
-    sample = f"{heads} of {w.heads} heads x T={w.T} x 2 gradient forms per step, fp64"
+    value = done * w.T * len(job.passes) * args.steps / el
+    sample = (f"{done} of {w.heads} heads x T={w.T} x {len(job.passes)} pass(es) per step, fp64, "
+              f"OpenMP over heads on {used} of {cores} host cores")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "head-tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy PCG64; no dataset)",
-            "config": {"workload": "TTT-Linear scan workload 2: per-token, simplified + LN-Jacobian "
-                                   "gradients, fp32 inputs, B=4 H=4 T=2048 d=64",
-                       "sample": sample},
+            "config": {"workload": _workload_desc(job), "sample": sample},
             "cpu_baseline": {"value": value, "unit": "head-tokens/s", "cores": used,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "head-tokens/s", "h2d_bytes_per_step": 0,
@@ -688,9 +763,17 @@ def run_reference(args):
 
 
 PROFILE_CASES = {
-    # kernel -> (make_inputs kwargs, scan kwargs)
+    # name -> (make_inputs kwargs, scan kwargs)
     "tc": (dict(B=4, H=16, T=8192, d=64, seed=7, random_affine=True, in_bf16=True),
            dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
+    # workload 5's kind of launch (mask ~ Bernoulli(0.5), one CTA per SM) at a
+    # quarter of its length: inputs 268 MB > L2
+    "tc_masked": (dict(B=2, H=32, T=8192, d=64, seed=5, random_affine=True, in_bf16=True,
+                       mask_p=0.5, b=16),
+                  dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
+    # workload 4's per-token pass at its full size (384 heads, one CTA per head)
+    "simt_4pt": (dict(B=16, H=24, T=2048, d=64, seed=4, random_affine=True, in_bf16=True),
+                 dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
     "simt": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
              dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False, single_cta=True)),
     "cluster": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
@@ -717,22 +800,16 @@ def run_profile_case(name: str):
         return
     mk, kw = PROFILE_CASES[name]
     inp = make_inputs(**mk)
-    bf = mk.get("in_bf16", False)
 
-    def dev(key):
-        a = inp.get(key)
-        if a is None:
-            return None
-        if bf and key in ("q", "k", "v", "eta_logit", "gate_logit"):
-            return torch.from_numpy(inp[key + "_bf16"].view(np.int16)).view(torch.bfloat16).cuda()
-        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    class _W:
+        in_bf16 = mk.get("in_bf16", False)
 
-    t = {k: dev(k) for k in ("q", "k", "v", "eta_logit", "gate_logit", "W0", "gamma", "beta")}
+    t = _dev_inputs(inp, _W, torch.device("cuda"))
     kw = dict(kw)
     out_dtype = torch.bfloat16 if kw.pop("out_bf16") else torch.float32
     for _ in range(2):
         ttt_scan.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"],
-                      t["beta"], out_dtype=out_dtype, **kw)
+                      t["beta"], mask=t["mask"], out_dtype=out_dtype, **kw)
     rc = ttt_scan.check_device_status()
     print(f"profile case {name}: status {ttt_scan.status_string(rc)}")
     if rc != ttt_scan.TTT_OK:
@@ -745,11 +822,17 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="2", help="headline workload id (default 2)")
-    ap.add_argument("--extra", nargs="*", default=["3", "4", "4pt", "5", "dec"],
+    ap.add_argument("--workload", default=HEADLINE, help="headline workload id (default 5)")
+    ap.add_argument("--extra", nargs="*", default=EXTRA,
                     help="other workloads measured on one GPU (by_workload)")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for the headline's CPU baseline")
+    ap.add_argument("--cpu-budget-extra", type=float, default=3.0,
+                    help="seconds of oracle work for each other workload's CPU baseline")
+    ap.add_argument("--ref-step-s", type=float, default=4.0,
+                    help="reference arm: about this many seconds of oracle work per step")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one kernel on a fixed case for a profiler capture and exit")
     args = ap.parse_args()

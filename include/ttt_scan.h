@@ -30,6 +30,8 @@
 #ifndef TTT_SCAN_H
 #define TTT_SCAN_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -58,10 +60,17 @@ enum {
   TTT_GRAD_ABLATE = 1u << 8,      /* ablation gradient: the LayerNorm Jacobian applied to
                                      -gamma*v, i.e. the prediction's contribution removed
                                      ("Error Correction in Trained TTT Layers", Abstract);
-                                     per-token mode only; invalid with TTT_NO_LN */
-  TTT_GRAD_NORM_MATCH = 1u << 9   /* with TTT_GRAD_ABLATE: rescale each token's gradient to the
+                                     both modes; invalid with TTT_NO_LN */
+  TTT_GRAD_NORM_MATCH = 1u << 9,  /* with TTT_GRAD_ABLATE: rescale each token's gradient to the
                                      L2 norm of its full LN-Jacobian gradient (0 where the
                                      ablated gradient is 0); invalid without TTT_GRAD_ABLATE */
+  TTT_KQ_SILU = 1u << 10          /* the `:mlp` variant ("Edifice.Recurrent.TTT", `build`
+                                     options, `:variant`): k <- SiLU(k), q <- SiLU(q)
+                                     (SiLU(x) = x sigmoid(x)) before the inner model, every
+                                     other step unchanged. The CUDA-core scan kernels take it
+                                     with fp32 inputs only (TTT_ERR_UNSUPPORTED with bf16
+                                     inputs there); the tensor-core kernel applies it to its
+                                     bf16 operands; the decode step takes both dtypes */
 };
 
 /* Kernel identifiers returned by ttt_scan_kernel_choice(). */
@@ -98,10 +107,11 @@ enum {
  * Kernels: per-token mode runs a CUDA-core kernel for any b: at d = 64, when
  *   the B*H heads fit on the device as clusters of 4 CTAs (one per SM), each
  *   head's rows of W are split over such a cluster; otherwise (or with
- *   TTT_KERNEL_SINGLE_CTA, or the ablation gradient) one CTA runs each head. Mini-batch mode runs the
+ *   TTT_KERNEL_SINGLE_CTA) one CTA runs each head. Mini-batch mode runs the
  *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs and a per-token
  *   gate, and otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which
- *   takes b <= 16.
+ *   takes b <= 16. Every gradient form (TTT_GRAD_LNJAC, TTT_NO_LN,
+ *   TTT_GRAD_ABLATE, TTT_GRAD_NORM_MATCH) runs in both modes on every kernel.
  *   Other combinations return TTT_ERR_UNSUPPORTED.
  * The library allocates no device memory per call.
  */
@@ -116,13 +126,15 @@ int ttt_scan_forward(const void* q, const void* k, const void* v,
  * ttt_scan_forward, plus the per-token inner-gradient norms of the ablation
  * study ("Error Correction in Trained TTT Layers", Abstract: the mean ratio of
  * the ablated gradient's norm to the full gradient's norm). Needs
- * TTT_GRAD_ABLATE in per-token mode (else TTT_ERR_INVALID_ARG / _UNSUPPORTED
- * as for the scan); the outputs o, W_T and W_chunks are those of
- * ttt_scan_forward with the same arguments.
+ * TTT_GRAD_ABLATE (else TTT_ERR_INVALID_ARG), in either mode (mini-batch: both
+ * norms at the chunk-start state W_s); the outputs o, W_T and W_chunks are
+ * those of ttt_scan_forward with the same arguments. Per-token calls run on
+ * one CTA per head.
  *   grad_norms  device, [B, H, T, 2] fp32, written: per head-token the L2 norm
  *               of the full LayerNorm-Jacobian gradient J^T(gamma*(pred - v))
  *               and of the ablated gradient J^T(-gamma*v) before any norm
- *               matching, both at that token's state W_{t-1}; zeros on the
+ *               matching, both at the state the token's gradient is taken at
+ *               (W_{t-1} per token, W_s in mini-batch mode); zeros on the
  *               tokens of SKIP chunks, which take no gradient. Must not
  *               overlap any other argument; null only when B*H*T == 0.
  * The call costs one more warp reduction per token on the gradient chain.
@@ -169,7 +181,7 @@ int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b);
  *   o            [B, H, d]      out: fp32, or bf16 with TTT_OUT_BF16
  * No output may overlap an input, and W may overlap nothing else.
  * mode: TTT_GRAD_LNJAC, TTT_NO_LN, TTT_IN_BF16, TTT_OUT_BF16, TTT_GATE_CHANNEL,
- *   TTT_GRAD_ABLATE, TTT_GRAD_NORM_MATCH (as for the scan).
+ *   TTT_GRAD_ABLATE, TTT_GRAD_NORM_MATCH, TTT_KQ_SILU (as for the scan).
  *   TTT_MODE_MINIBATCH returns TTT_ERR_UNSUPPORTED (a one-token step has no
  *   chunk); TTT_KERNEL_SIMT and TTT_KERNEL_SINGLE_CTA are accepted and ignored.
  * Sizes: B, H >= 0, d in {16, 64}, eps >= 0 (finite). Returns TTT_OK or an error
@@ -180,6 +192,52 @@ int ttt_decode_step(const void* q, const void* k, const void* v,
                     const float* gamma, const float* beta, int B, int H, int d,
                     float eps, unsigned mode, const unsigned char* update, void* o,
                     void* cuda_stream);
+
+/*
+ * Backward of the scan: the gradients of L = <dO, o> + <dW_T, W_T> with respect
+ * to every input of a ttt_scan_forward call with the same arguments, by the
+ * chain rule taken through the forward's steps in reverse (no page gives this
+ * pass; it is the reverse of the recurrence in the comment at the top of this
+ * file, for the training both "Edifice.Recurrent.TTT" (Architecture) and
+ * PonderTTT (Technical Architecture) do). Per-token and mini-batch mode, the
+ * SIMPLE, LN-Jacobian, no-LayerNorm and ablation gradients, scalar, per-feature
+ * or no gate, the mask and the SiLU variant. Arithmetic is fp32.
+ *
+ * Enqueue-only on `cuda_stream`. All pointers are DEVICE pointers owned by the
+ * caller, 16-byte aligned, contiguous row-major:
+ *   q, k, v, eta_logit, gate_logit, gamma, beta, mask   as for ttt_scan_forward
+ *   W_chunks     [B, H, ceil(T/b) + 1, d, d] fp32: the W_chunks snapshots written by
+ *                ttt_scan_forward with the same arguments (the state before every chunk
+ *                of b tokens; the backward recomputes each chunk from its snapshot)
+ *   dO           [B, H, T, d] fp32, dL/do
+ *   dW_T         [B, H, d, d] fp32, dL/dW_T; NULL = zero
+ *   dq, dk, dv   [B, H, T, d] fp32 out
+ *   d_eta_logit  [B, H, T] fp32 out (0 on SKIP chunks)
+ *   d_gate_logit fp32 out, the shape of gate_logit; NULL only when gate_logit is NULL
+ *   dW0          [B, H, d, d] fp32 out
+ *   dgamma, dbeta [H, d] fp32 out, summed over the batch rows (in batch-row order, so
+ *                the result is deterministic); unused (may be NULL) with TTT_NO_LN
+ *   workspace    device scratch of at least ttt_scan_backward_workspace_bytes(B, H, d,
+ *                mode) bytes (per-head partial sums of dgamma, dbeta); NULL when that
+ *                is 0. Owned by the caller; calls that share one must not overlap.
+ * No output may overlap an input, another output or the workspace.
+ * Sizes: as for ttt_scan_forward, with b <= 16 (the chunk the backward recomputes
+ *   from one snapshot) and d in {16, 64}. mode: the forward's bits; TTT_OUT_BF16,
+ *   TTT_KERNEL_SIMT and TTT_KERNEL_SINGLE_CTA are ignored, TTT_GRAD_NORM_MATCH returns
+ *   TTT_ERR_UNSUPPORTED. Returns TTT_OK or an error code before launching anything.
+ * Allocates no device memory.
+ */
+size_t ttt_scan_backward_workspace_bytes(int B, int H, int d, unsigned mode);
+
+int ttt_scan_backward(const void* q, const void* k, const void* v,
+                      const void* eta_logit, const void* gate_logit,
+                      const float* gamma, const float* beta,
+                      int B, int H, int T, int d, float eps, unsigned mode, int b,
+                      const unsigned char* mask, const float* W_chunks,
+                      const float* dO, const float* dW_T,
+                      float* dq, float* dk, float* dv, float* d_eta_logit,
+                      float* d_gate_logit, float* dW0, float* dgamma, float* dbeta,
+                      void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
  * Synchronise `cuda_stream`, then report and clear the device status word that

@@ -11,9 +11,16 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libttt_scan.so"
-# Translation units, compiled in parallel and linked into one shared library.
-SOURCES = [CSRC / "ttt_scan.cu", CSRC / "simt_f32.cu", CSRC / "simt_bf16.cu",
-           CSRC / "cluster.cu", CSRC / "probe.cu"]
+# Objects, compiled in parallel and linked into one shared library: (source,
+# object stem, extra defines). simt.cu is built once per input dtype and mode.
+UNITS = [(CSRC / "ttt_scan.cu", "ttt_scan", ()),
+         (CSRC / "cluster.cu", "cluster", ()),
+         (CSRC / "backward.cu", "backward", ()),
+         (CSRC / "probe.cu", "probe", ())]
+UNITS += [(CSRC / "simt.cu", f"simt_{dt}_{md}",
+           (f"-DTTT_SIMT_BF16={int(dt == 'bf16')}", f"-DTTT_SIMT_MINIBATCH={int(md == 'mb')}"))
+          for dt in ("f32", "bf16") for md in ("tok", "mb")]
+SOURCES = sorted({src for src, _, _ in UNITS})
 HEADERS = sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.h")) + sorted((ROOT / "include").glob("*.h"))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -45,14 +52,14 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> Path:
     tag = f"{os.getpid()}"
     objs, procs = [], []
     try:
-        for src in SOURCES:
-            obj = LIB.parent / f".{src.stem}.{tag}.o"
-            cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-c", str(src), "-o", str(obj)]
+        for src, stem, defs in UNITS:
+            obj = LIB.parent / f".{stem}.{tag}.o"
+            cmd = [_nvcc(), *NVCC_FLAGS, *defs, *extra, "-c", str(src), "-o", str(obj)]
             if verbose:
                 print(" ".join(cmd), file=sys.stderr)
             objs.append(obj)
-            procs.append((src, subprocess.Popen(cmd)))
-        failed = [src.name for src, pr in procs if pr.wait() != 0]
+            procs.append((stem, subprocess.Popen(cmd)))
+        failed = [stem for stem, pr in procs if pr.wait() != 0]
         if failed:
             raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
         tmp = LIB.with_suffix(f".so.tmp{tag}")

@@ -58,17 +58,26 @@ struct ClusterLaunch {
   }
 };
 
-template <typename InT, typename OutT>
-int cluster_dispatch(const ttt::ScanParams* p, int gm, cudaStream_t s, int* capacity) {
+template <typename InT, typename OutT, int GM>
+int cluster_one(const ttt::ScanParams* p, cudaStream_t s, int* capacity) {
   if (capacity) {
-    *capacity = gm == 0 ? ClusterLaunch<InT, OutT, 0>::capacity()
-              : gm == 1 ? ClusterLaunch<InT, OutT, 1>::capacity()
-                        : ClusterLaunch<InT, OutT, 2>::capacity();
+    *capacity = ClusterLaunch<InT, OutT, GM>::capacity();
     return TTT_OK;
   }
-  if (gm == 0) return ClusterLaunch<InT, OutT, 0>::launch(*p, s);
-  if (gm == 1) return ClusterLaunch<InT, OutT, 1>::launch(*p, s);
-  return ClusterLaunch<InT, OutT, 2>::launch(*p, s);
+  return ClusterLaunch<InT, OutT, GM>::launch(*p, s);
+}
+
+// gm: 0 simplified, 1 LN Jacobian, 2 no LayerNorm, 3 ablation, 4 ablation with
+// per-token norm matching (the gradient norms are written by the one-CTA kernel).
+template <typename InT, typename OutT>
+int cluster_dispatch(const ttt::ScanParams* p, int gm, cudaStream_t s, int* capacity) {
+  switch (gm) {
+    case 0: return cluster_one<InT, OutT, 0>(p, s, capacity);
+    case 1: return cluster_one<InT, OutT, 1>(p, s, capacity);
+    case 3: return cluster_one<InT, OutT, 3>(p, s, capacity);
+    case 4: return cluster_one<InT, OutT, 4>(p, s, capacity);
+    default: return cluster_one<InT, OutT, 2>(p, s, capacity);
+  }
 }
 
 int call(const ttt::ScanParams* p, unsigned mode, int gm, cudaStream_t s, int* capacity) {

@@ -36,6 +36,7 @@ struct ScanParams {
   int ablate;              // ablation gradient (prediction removed, Jacobian kept)
   int norm_match;          // ... rescaled per token to the full gradient's norm
   float* grad_norms;       // [B, H, T, 2] per-token gradient norms (ablation), may be null
+  int kq_silu;             // the `:mlp` variant: SiLU on every key and query as it is loaded
 };
 
 // Gradient variant of the CUDA-core chain: 0 simplified, 1 LN Jacobian, 2 no
@@ -62,6 +63,10 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 }
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// SiLU(x) = x sigmoid(x), the activation of the `:mlp` variant ("Edifice.Recurrent.TTT",
+// `build` options, `:variant`) on keys and queries.
+__device__ __forceinline__ float siluf_(float x) { return x * sigmoidf_(x); }
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll

@@ -42,6 +42,7 @@ struct DecodeParams {
   float eps;
   int lnjac, no_ln, gate_channel;
   int ablate, norm_match;   // ablation gradient; per-token norm matching
+  int kq_silu;              // the `:mlp` variant: SiLU on k and q as they are loaded
 };
 
 template <int D>
@@ -110,6 +111,13 @@ __global__ void __launch_bounds__(DecodeShape<D>::NT) decode_step_kernel(const D
   float kk[4], qq[4];
   load4<InT>(static_cast<const InT*>(p.k) + bh * D + 4 * cg, kk);
   load4<InT>(static_cast<const InT*>(p.q) + bh * D + 4 * cg, qq);
+  if (p.kq_silu) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      kk[i] = siluf_(kk[i]);
+      qq[i] = siluf_(qq[i]);
+    }
+  }
   // the head row this lane ends up holding after the reductions
   const int rr = 16 * wih + S::RPI * ((lane >> 1) & (S::NI - 1)) + rsub;
   const float vr = to_f32(static_cast<const InT*>(p.v)[bh * D + rr]);

@@ -1,5 +1,5 @@
 // Host-side launchers of the CUDA-core kernels, each compiled in its own
-// translation unit (simt_f32.cu, simt_bf16.cu, cluster.cu) so the library
+// translation unit (four objects of simt.cu, cluster.cu) so the library
 // builds in parallel. Arguments are already checked by the C-ABI entry points;
 // every function returns a ttt_status code.
 #pragma once
@@ -10,13 +10,19 @@
 
 namespace ttt {
 
-// One CTA per head: fp32 inputs / bf16 inputs (output dtype, mode and d from
-// the arguments).
-int launch_simt_f32in(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
-int launch_simt_bf16in(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+// SMs of the current device (0 if the query fails); cached per device.
+int device_sm_count();
+
+// One CTA per head, by input dtype and mode (output dtype, gradient form and d
+// from the arguments).
+int launch_simt_f32_pertoken(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+int launch_simt_f32_minibatch(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+int launch_simt_bf16_pertoken(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
+int launch_simt_bf16_minibatch(const ScanParams& p, unsigned mode, int d, cudaStream_t stream);
 
 // Per-token d = 64, each head over a cluster of CTAs. gm: 0 simplified,
-// 1 LN-Jacobian, 2 no LayerNorm gradient.
+// 1 LN-Jacobian, 2 no LayerNorm gradient, 3 ablation, 4 ablation with
+// per-token norm matching.
 int launch_cluster(const ScanParams& p, unsigned mode, int gm, cudaStream_t stream);
 // Clusters of that kernel that fit on the current device at once (0 if unknown).
 int cluster_capacity(unsigned mode, int gm);

@@ -1,0 +1,627 @@
+// Backward of the TTT-Linear scan on CUDA cores (fp32): the gradients of
+// L = <dO, o> + <dW_T, W_T> with respect to q, k, v, the two logits, W0, gamma
+// and beta, in per-token and mini-batch mode.
+//
+// The forward recurrence ("Edifice.Recurrent.TTT", Equations (TTT-Linear);
+// mini-batch: PonderTTT, Technical Architecture, dual-form updates) is, per
+// token t of a chunk that starts from W_s,
+//     z_t = W_{t-1} k_t,  G_t = G(z_t, v_t),  W_t = W_{t-1} - eta_t G_t k_t^T,
+//     o_t = gate_t (W_t q_t)
+// (mini-batch: every z_t from W_s, o_t = gate_t (W_s q_t - sum_{j<=t} eta_j
+// (k_j.q_t) G_j), one update per chunk). Its reverse, with D = dL/dW at the
+// chunk end (D_e), dy_t = gate_t dO_t and the exact chunk identity
+// W_t = W_s - sum_{j<=t} eta_j G_j k_j^T, is
+//     u_t   = D_e k_t + sum_{j>=t} dy_j (q_j.k_t) + sum_{j>t} dz_j (k_j.k_t)
+//     deta_t = -G_t.u_t,   dG_t = -eta_t u_t,   dz_t = G'(z_t)^T dG_t
+//     dq_t  = W_s^T dy_t - sum_{j<=t} eta_j (G_j.dy_t) k_j
+//     dk_t  = -eta_t (D_e^T G_t + sum_{j>=t} (dy_j.G_t) q_j + sum_{j>t} (dz_j.G_t) k_j)
+//             + W_s^T dz_t - sum_{j<t} eta_j (G_j.dz_t) k_j
+//     D_s   = D_e + sum_t (dy_t q_t^T + dz_t k_t^T)
+// where the terms in dz_j (k_j.k_t) and (G_j.dz_t) are absent in mini-batch
+// mode (its z_t do not depend on the chunk's earlier gradients). Only the dz_t
+// are sequential (the chain, one warp, right to left through the chunk); the
+// d x d work (W_s K^T, W_s Q^T, D_e K^T, W_s^T [dy dz], D_e^T G and the rank-2b
+// update of D) is batched per chunk. The chunk-start states W_s come from the
+// forward's W_chunks snapshots (one per chunk of b tokens); the forward inside a
+// chunk is recomputed from W_s with the same identity.
+//
+// One CTA of 4d threads per (batch row, head). gamma / beta gradients are
+// summed over the head's tokens in the chain warp's registers and written per
+// head to `gb_part`; bwd_reduce_gb_kernel sums them over the batch rows in a
+// fixed order.
+#pragma once
+
+#include "common.cuh"
+#include "scan_simt.cuh"  // kC, butterfly
+
+namespace ttt {
+
+struct BwdParams {
+  const void* q;           // [B, H, T, D] fp32 or bf16 (with eta_logit, gate_logit)
+  const void* k;
+  const void* v;
+  const void* eta_logit;   // [B, H, T]
+  const void* gate_logit;  // [B, H, T], [B, H, T, D] (gate_channel) or null
+  const float* gamma;      // [H, D]; null with no_ln
+  const float* beta;
+  const unsigned char* mask;  // [B, n_chunks] or null
+  const float* W_chunks;   // [B, H, n_chunks + 1, D, D]: W before every chunk of b tokens
+  const float* dO;         // [B, H, T, D]
+  const float* dW_T;       // [B, H, D, D] or null (zero)
+  float* dq;               // [B, H, T, D]
+  float* dk;
+  float* dv;
+  float* deta;             // [B, H, T]
+  float* dgate;            // shape of gate_logit, or null
+  float* dW0;              // [B, H, D, D]
+  float* gb_part;          // [B * H, 2, D]: per head sum of dgamma, dbeta (null with no_ln)
+  int B, H, T;
+  int b;                   // chunk (<= kC)
+  int n_chunks;            // ceil(T / b)
+  float eps;
+  int gate_channel;
+  int kq_silu;
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int NT = 4 * D;   // threads: 256 at d = 64, 64 at d = 16
+  static constexpr int C = kC;       // largest chunk
+  static constexpr int LD = D + 1;   // padded row stride of every [rows][D] array
+  static constexpr int MAT = D * LD; // a d x d matrix
+  static constexpr int TOK = C * LD; // a [C][D] token array
+  static constexpr int GR = C * C;   // a Gram
+  // offsets in floats
+  static constexpr int oW = 0;                 // W_s
+  static constexpr int oDm = oW + MAT;         // D = dL/dW (chunk end, then chunk start)
+  static constexpr int oK = oDm + MAT;         // inner-model keys (after SiLU if asked)
+  static constexpr int oQ = oK + TOK;          // inner-model queries
+  static constexpr int oV = oQ + TOK;
+  static constexpr int oDO = oV + TOK;
+  static constexpr int oZ = oDO + TOK;         // W_s k_t, then z_t
+  static constexpr int oY = oZ + TOK;          // W_s q_t, then y_t = W_t q_t
+  static constexpr int oPB = oY + TOK;         // D_e k_t
+  static constexpr int oG = oPB + TOK;         // G_t
+  static constexpr int oXh = oG + TOK;         // xhat_t (z_t with no LayerNorm)
+  static constexpr int oDy = oXh + TOK;        // dy_t = gate_t dO_t
+  static constexpr int oDz = oDy + TOK;        // dz_t
+  static constexpr int oT1 = oDz + TOK;        // W_s^T dy_t
+  static constexpr int oT2 = oT1 + TOK;        // W_s^T dz_t
+  static constexpr int oT3 = oT2 + TOK;        // D_e^T G_t
+  static constexpr int oKK = oT3 + TOK;        // k_i . k_j
+  static constexpr int oQK = oKK + GR;         // q_i . k_j
+  static constexpr int oGDy = oQK + GR;        // G_j . dy_i
+  static constexpr int oGDz = oGDy + GR;       // G_j . dz_i
+  static constexpr int oEta = oGDz + GR;       // eta_t (0 on SKIP chunks and past the chunk)
+  static constexpr int oSg = oEta + C;         // sigmoid(eta_logit_t)
+  static constexpr int oGate = oSg + C;        // scalar gate_t
+  static constexpr int oS = oGate + C;         // LayerNorm s_t
+  static constexpr int floats = oS + C;
+  static constexpr int bytes = floats * 4;
+};
+
+__device__ __forceinline__ float silu_grad(float x) {
+  const float s = sigmoidf_(x);
+  return s * (1.f + x * (1.f - s));
+}
+
+template <typename InT>
+__device__ __forceinline__ float ld_in(const void* p, size_t i) {
+  return to_f32(static_cast<const InT*>(p)[i]);
+}
+
+// GM: 0 simplified (G = err), 1 LN Jacobian, 2 no LayerNorm (G = z - v),
+// 3 ablation (the Jacobian applied to -gamma v).
+template <int D, typename InT, bool MINIB, int GM>
+__global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int NT = L::NT, C = L::C, LD = L::LD;
+  constexpr int EPL = (D + 31) / 32;
+  constexpr bool kLN = GM != 2;
+  constexpr bool kJac = GM == 1 || GM == 3;
+  extern __shared__ __align__(16) float sm[];
+  float* sW = sm + L::oW;
+  float* sD = sm + L::oDm;
+  float* sK = sm + L::oK;
+  float* sQ = sm + L::oQ;
+  float* sV = sm + L::oV;
+  float* sDO = sm + L::oDO;
+  float* sZ = sm + L::oZ;
+  float* sY = sm + L::oY;
+  float* sPB = sm + L::oPB;
+  float* sG = sm + L::oG;
+  float* sXh = sm + L::oXh;
+  float* sDy = sm + L::oDy;
+  float* sDz = sm + L::oDz;
+  float* sT1 = sm + L::oT1;
+  float* sT2 = sm + L::oT2;
+  float* sT3 = sm + L::oT3;
+  float* sKK = sm + L::oKK;
+  float* sQK = sm + L::oQK;
+  float* sGDy = sm + L::oGDy;
+  float* sGDz = sm + L::oGDz;
+  float* sEta = sm + L::oEta;
+  float* sSg = sm + L::oSg;
+  float* sGate = sm + L::oGate;
+  float* sS = sm + L::oS;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const long long bh = blockIdx.x;
+  const int bi = (int)(bh / p.H);
+  const int h = (int)(bh - (long long)bi * p.H);
+  const int T = p.T, b = p.b, nc = p.n_chunks;
+  const size_t tok0 = (size_t)bh * T;
+  const float inv_d = 1.0f / (float)D;
+  const float* Wc = p.W_chunks + (size_t)bh * (nc + 1) * D * D;
+
+  // chain warp: this lane's features f = lane + 32 e, and gamma / beta sums
+  float gam[EPL], bet[EPL], dgam[EPL], dbet[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int f = lane + 32 * e;
+    const bool ok = f < D && kLN;
+    gam[e] = ok ? p.gamma[(size_t)h * D + f] : 1.f;
+    bet[e] = ok ? p.beta[(size_t)h * D + f] : 0.f;
+    dgam[e] = 0.f;
+    dbet[e] = 0.f;
+  }
+
+  // D = dW_T
+  for (int idx = tid; idx < D * D; idx += NT) {
+    const int r = idx / D, c = idx - r * D;
+    sD[r * LD + c] = p.dW_T ? p.dW_T[(size_t)bh * D * D + idx] : 0.f;
+  }
+
+  for (int ch = nc - 1; ch >= 0; --ch) {
+    const int t0 = ch * b;
+    const int n = min(b, T - t0);
+    const bool upd = p.mask == nullptr || p.mask[(size_t)bi * nc + ch] != 0;
+
+    // ---- chunk inputs (rows past n are zero), W_s, scalars ----
+    for (int idx = tid; idx < D * D; idx += NT) {
+      const int r = idx / D, c = idx - r * D;
+      sW[r * LD + c] = Wc[(size_t)ch * D * D + idx];
+    }
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int t = idx / D, f = idx - t * D;
+      const bool ok = t < n;
+      const size_t g = (tok0 + t0 + t) * D + f;
+      float kv = ok ? ld_in<InT>(p.k, g) : 0.f;
+      float qv = ok ? ld_in<InT>(p.q, g) : 0.f;
+      if (p.kq_silu) {
+        kv = siluf_(kv);
+        qv = siluf_(qv);
+      }
+      sK[t * LD + f] = kv;
+      sQ[t * LD + f] = qv;
+      sV[t * LD + f] = ok ? ld_in<InT>(p.v, g) : 0.f;
+      float gch = 1.f;
+      if (ok && p.gate_logit && p.gate_channel) gch = sigmoidf_(ld_in<InT>(p.gate_logit, g));
+      // dy = gate dO (the scalar gate is applied below, once it is known)
+      sDO[t * LD + f] = ok ? p.dO[g] : 0.f;
+      sDy[t * LD + f] = ok ? gch * p.dO[g] : 0.f;
+    }
+    if (tid < C) {
+      const int t = tid;
+      const bool ok = t < n;
+      const float sg = (ok && upd) ? sigmoidf_(ld_in<InT>(p.eta_logit, tok0 + t0 + t)) : 0.f;
+      sSg[t] = sg;
+      sEta[t] = sg * inv_d;
+      sGate[t] = (ok && p.gate_logit && !p.gate_channel)
+                     ? sigmoidf_(ld_in<InT>(p.gate_logit, tok0 + t0 + t)) : 1.f;
+    }
+    __syncthreads();
+    if (p.gate_logit && !p.gate_channel) {
+      for (int idx = tid; idx < C * D; idx += NT) {
+        const int t = idx / D, f = idx - t * D;
+        sDy[t * LD + f] *= sGate[t];
+      }
+    }
+
+    // ---- batched: W_s k_t, W_s q_t, D_e k_t (thread: row r, tokens tg + 4m) ----
+    {
+      const int r = tid % D, tg = tid / D;
+      constexpr int NTK = C / 4;
+      float az[NTK], ay[NTK], ap[NTK];
+#pragma unroll
+      for (int m = 0; m < NTK; ++m) az[m] = ay[m] = ap[m] = 0.f;
+      for (int c = 0; c < D; ++c) {
+        const float w = sW[r * LD + c], dd = sD[r * LD + c];
+#pragma unroll
+        for (int m = 0; m < NTK; ++m) {
+          const int t = tg + 4 * m;
+          const float kc = sK[t * LD + c];
+          az[m] = fmaf(w, kc, az[m]);
+          ay[m] = fmaf(w, sQ[t * LD + c], ay[m]);
+          ap[m] = fmaf(dd, kc, ap[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NTK; ++m) {
+        const int t = tg + 4 * m;
+        sZ[t * LD + r] = az[m];
+        sY[t * LD + r] = ay[m];
+        sPB[t * LD + r] = ap[m];
+      }
+    }
+    // ---- Grams k_i.k_j and q_i.k_j ----
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int i = idx / C, j = idx - i * C;
+      float kk = 0.f, qk = 0.f;
+      for (int f = 0; f < D; ++f) {
+        const float kj = sK[j * LD + f];
+        kk = fmaf(sK[i * LD + f], kj, kk);
+        qk = fmaf(sQ[i * LD + f], kj, qk);
+      }
+      sKK[idx] = kk;
+      sQK[idx] = qk;
+    }
+    __syncthreads();
+
+    // ---- forward chain (warp 0): z_t, LayerNorm, G_t ----
+    if (warp == 0) {
+      for (int t = 0; t < C; ++t) {
+        if (t >= n || !upd) {
+          // SKIP chunks take no gradient (eta = 0): G plays no part
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const int f = lane + 32 * e;
+            if (f < D) {
+              sG[t * LD + f] = 0.f;
+              sXh[t * LD + f] = 0.f;
+            }
+          }
+          continue;
+        }
+        float z[EPL], v[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const int f = lane + 32 * e;
+          float acc = 0.f;
+          if (f < D) {
+            acc = sZ[t * LD + f];
+            if (!MINIB)
+              for (int j = 0; j < t; ++j) acc = fmaf(-sEta[j] * sKK[t * C + j], sG[j * LD + f], acc);
+          }
+          z[e] = acc;
+          v[e] = f < D ? sV[t * LD + f] : 0.f;
+        }
+        float G[EPL], xh[EPL];
+        if (!kLN) {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            G[e] = z[e] - v[e];
+            xh[e] = z[e];
+          }
+        } else {
+          float m1[1] = {0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) m1[0] += z[e];
+          butterfly<1>(m1);
+          const float mu = m1[0] * inv_d;
+          float m2[1] = {0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const float y = (lane + 32 * e < D) ? z[e] - mu : 0.f;
+            m2[0] = fmaf(y, y, m2[0]);
+          }
+          butterfly<1>(m2);
+          const float s = sqrtf(m2[0] * inv_d + p.eps);
+          float g[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const bool fv = lane + 32 * e < D;
+            xh[e] = fv ? (z[e] - mu) / s : 0.f;
+            const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
+            g[e] = fv ? (GM == 3 ? -gam[e] * v[e] : (GM == 1 ? gam[e] * err : err)) : 0.f;
+          }
+          if (kJac) {
+            float m[2] = {0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              m[0] += g[e];
+              m[1] = fmaf(g[e], xh[e], m[1]);
+            }
+            butterfly<2>(m);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e)
+              G[e] = (g[e] - m[0] * inv_d - xh[e] * (m[1] * inv_d)) / s;
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) G[e] = g[e];
+          }
+          if (lane == 0) sS[t] = s;
+        }
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const int f = lane + 32 * e;
+          if (f < D) {
+            sG[t * LD + f] = G[e];
+            sXh[t * LD + f] = xh[e];
+          }
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+
+    // ---- readout y_t = W_s q_t - sum_{j<=t} eta_j (q_t.k_j) G_j, and the gate gradients ----
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int t = idx / D, f = idx - t * D;
+      float y = sY[t * LD + f];
+      if (upd)
+        for (int j = 0; j <= t; ++j) y = fmaf(-sEta[j] * sQK[t * C + j], sG[j * LD + f], y);
+      sY[t * LD + f] = y;
+      if (p.gate_logit && p.gate_channel && t < n) {
+        const size_t g = (tok0 + t0 + t) * D + f;
+        const float gs = sigmoidf_(ld_in<InT>(p.gate_logit, g));
+        p.dgate[g] = sDO[t * LD + f] * y * gs * (1.f - gs);
+      }
+    }
+    __syncthreads();
+    if (p.gate_logit && !p.gate_channel) {
+      // one warp per token: dL/dgate_logit = (dO . y) gate (1 - gate)
+      for (int t = warp; t < n; t += NT / 32) {
+        float acc[1] = {0.f};
+        for (int f = lane; f < D; f += 32) acc[0] = fmaf(sDO[t * LD + f], sY[t * LD + f], acc[0]);
+        butterfly<1>(acc);
+        if (lane == 0) {
+          const float gs = sGate[t];
+          p.dgate[tok0 + t0 + t] = acc[0] * gs * (1.f - gs);
+        }
+      }
+    }
+
+    // ---- backward chain (warp 0), right to left: u_t, deta_t, dz_t, dv_t ----
+    if (warp == 0) {
+      for (int t = C - 1; t >= 0; --t) {
+        if (t >= n) continue;
+        const size_t gt = tok0 + t0 + t;
+        if (!upd) {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const int f = lane + 32 * e;
+            if (f < D) {
+              sDz[t * LD + f] = 0.f;
+              p.dv[gt * D + f] = 0.f;
+            }
+          }
+          if (lane == 0) p.deta[gt] = 0.f;
+          continue;
+        }
+        float u[EPL], G[EPL], xh[EPL], v[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const int f = lane + 32 * e;
+          float acc = 0.f;
+          if (f < D) {
+            acc = sPB[t * LD + f];
+            for (int j = t; j < n; ++j) acc = fmaf(sQK[j * C + t], sDy[j * LD + f], acc);
+            if (!MINIB)
+              for (int j = t + 1; j < n; ++j) acc = fmaf(sKK[j * C + t], sDz[j * LD + f], acc);
+          }
+          u[e] = acc;
+          G[e] = f < D ? sG[t * LD + f] : 0.f;
+          xh[e] = f < D ? sXh[t * LD + f] : 0.f;
+          v[e] = f < D ? sV[t * LD + f] : 0.f;
+        }
+        float de[1] = {0.f};
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) de[0] = fmaf(-G[e], u[e], de[0]);
+        butterfly<1>(de);
+        const float eta = sEta[t];
+        if (lane == 0) p.deta[gt] = de[0] * sSg[t] * (1.f - sSg[t]) * inv_d;
+        float dG[EPL], dz[EPL], dv[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          dG[e] = (lane + 32 * e < D) ? -eta * u[e] : 0.f;
+          dv[e] = 0.f;
+        }
+        if (!kLN) {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            dz[e] = dG[e];
+            dv[e] = -dG[e];
+          }
+        } else {
+          const float s = sS[t];
+          float derr[EPL], dxh[EPL];
+          float ds = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) dxh[e] = 0.f;
+          if (kJac) {
+            // G = (g - mean g - xhat mean(g xhat)) / s
+            float g[EPL];
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              const bool fv = lane + 32 * e < D;
+              const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
+              g[e] = fv ? (GM == 3 ? -gam[e] * v[e] : gam[e] * err) : 0.f;
+              m[0] += g[e];
+              m[1] = fmaf(g[e], xh[e], m[1]);
+              m[2] += dG[e];
+              m[3] = fmaf(dG[e], xh[e], m[3]);
+            }
+            butterfly<4>(m);
+            const float c_ = m[1] * inv_d, mdG = m[2] * inv_d, mdGx = m[3] * inv_d;
+            float sdGG[1] = {0.f};
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) sdGG[0] = fmaf(dG[e], G[e], sdGG[0]);
+            butterfly<1>(sdGG);
+            ds = -sdGG[0] / s;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              const bool fv = lane + 32 * e < D;
+              const float dg = fv ? (dG[e] - mdG - xh[e] * mdGx) / s : 0.f;
+              dxh[e] = fv ? (-dG[e] * c_ - g[e] * mdGx) / s : 0.f;
+              if (GM == 3) {
+                dgam[e] -= dg * v[e];
+                dv[e] -= dg * gam[e];
+                derr[e] = 0.f;
+              } else {
+                const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
+                dgam[e] = fmaf(dg, err, dgam[e]);
+                derr[e] = dg * gam[e];
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) derr[e] = dG[e];
+          }
+          // err = gamma xhat + beta - v
+          float dxx[1] = {0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            if (lane + 32 * e < D) {
+              dgam[e] = fmaf(derr[e], xh[e], dgam[e]);
+              dbet[e] += derr[e];
+              dv[e] -= derr[e];
+              dxh[e] = fmaf(derr[e], gam[e], dxh[e]);
+            }
+            dxx[0] = fmaf(dxh[e], xh[e], dxx[0]);
+          }
+          butterfly<1>(dxx);
+          // xhat = (z - mu) / s, s = sqrt(var + eps): z - mu = xhat s
+          const float dvar = (ds - dxx[0] / s) / (2.f * s);
+          float dy[EPL];
+          float mdy[1] = {0.f};
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            dy[e] = (lane + 32 * e < D) ? dxh[e] / s + dvar * 2.f * xh[e] * s * inv_d : 0.f;
+            mdy[0] += dy[e];
+          }
+          butterfly<1>(mdy);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) dz[e] = dy[e] - mdy[0] * inv_d;
+        }
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const int f = lane + 32 * e;
+          if (f < D) {
+            sDz[t * LD + f] = dz[e];
+            p.dv[gt * D + f] = dv[e];
+          }
+        }
+        __syncwarp();
+      }
+      // rows past the chunk
+      for (int t = n; t < C; ++t)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          if (lane + 32 * e < D) sDz[t * LD + lane + 32 * e] = 0.f;
+    }
+    __syncthreads();
+
+    // ---- batched: W_s^T dy_t, W_s^T dz_t, D_e^T G_t (thread: column c, tokens tg + 4m);
+    //      Grams G_j.dy_i, G_j.dz_i ----
+    {
+      const int c = tid % D, tg = tid / D;
+      constexpr int NTK = C / 4;
+      float a1[NTK], a2[NTK], a3[NTK];
+#pragma unroll
+      for (int m = 0; m < NTK; ++m) a1[m] = a2[m] = a3[m] = 0.f;
+      for (int r = 0; r < D; ++r) {
+        const float w = sW[r * LD + c], dd = sD[r * LD + c];
+#pragma unroll
+        for (int m = 0; m < NTK; ++m) {
+          const int t = tg + 4 * m;
+          a1[m] = fmaf(w, sDy[t * LD + r], a1[m]);
+          a2[m] = fmaf(w, sDz[t * LD + r], a2[m]);
+          a3[m] = fmaf(dd, sG[t * LD + r], a3[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NTK; ++m) {
+        const int t = tg + 4 * m;
+        sT1[t * LD + c] = a1[m];
+        sT2[t * LD + c] = a2[m];
+        sT3[t * LD + c] = a3[m];
+      }
+    }
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int i = idx / C, j = idx - i * C;
+      float gy = 0.f, gz = 0.f;
+      for (int f = 0; f < D; ++f) {
+        const float gj = sG[j * LD + f];
+        gy = fmaf(gj, sDy[i * LD + f], gy);
+        gz = fmaf(gj, sDz[i * LD + f], gz);
+      }
+      sGDy[idx] = gy;
+      sGDz[idx] = gz;
+    }
+    __syncthreads();
+
+    // ---- dq, dk (chained through SiLU for the `:mlp` variant) ----
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int t = idx / D, c = idx - t * D;
+      if (t >= n) continue;
+      float dq = sT1[t * LD + c];
+      float dk = sT2[t * LD + c];
+      if (upd) {
+        float a = sT3[t * LD + c];
+        for (int j = t; j < n; ++j) a = fmaf(sGDy[j * C + t], sQ[j * LD + c], a);
+        if (!MINIB)
+          for (int j = t + 1; j < n; ++j) a = fmaf(sGDz[j * C + t], sK[j * LD + c], a);
+        dk = fmaf(-sEta[t], a, dk);
+        for (int j = 0; j <= t; ++j) dq = fmaf(-sEta[j] * sGDy[t * C + j], sK[j * LD + c], dq);
+        if (!MINIB)
+          for (int j = 0; j < t; ++j) dk = fmaf(-sEta[j] * sGDz[t * C + j], sK[j * LD + c], dk);
+      }
+      const size_t g = (tok0 + t0 + t) * D + c;
+      if (p.kq_silu) {
+        dq *= silu_grad(ld_in<InT>(p.q, g));
+        dk *= silu_grad(ld_in<InT>(p.k, g));
+      }
+      p.dq[g] = dq;
+      p.dk[g] = dk;
+    }
+    // ---- D_s = D_e + sum_t (dy_t q_t^T + dz_t k_t^T) ----
+    for (int idx = tid; idx < D * D; idx += NT) {
+      const int r = idx / D, c = idx - r * D;
+      float acc = sD[r * LD + c];
+      for (int t = 0; t < n; ++t) {
+        acc = fmaf(sDy[t * LD + r], sQ[t * LD + c], acc);
+        acc = fmaf(sDz[t * LD + r], sK[t * LD + c], acc);
+      }
+      sD[r * LD + c] = acc;
+    }
+    __syncthreads();
+  }
+
+  // ---- dW0 = D, per-head gamma / beta sums ----
+  for (int idx = tid; idx < D * D; idx += NT) {
+    const int r = idx / D, c = idx - r * D;
+    p.dW0[(size_t)bh * D * D + idx] = sD[r * LD + c];
+  }
+  if (kLN && warp == 0 && p.gb_part != nullptr) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int f = lane + 32 * e;
+      if (f < D) {
+        p.gb_part[((size_t)bh * 2) * D + f] = dgam[e];
+        p.gb_part[((size_t)bh * 2 + 1) * D + f] = dbet[e];
+      }
+    }
+  }
+}
+
+// dgamma[h][f] = sum over batch rows of the per-head sums (in batch-row order,
+// so the result does not depend on scheduling); likewise dbeta.
+__global__ void bwd_reduce_gb_kernel(const float* __restrict__ gb_part, int B, int H, int D,
+                                     float* __restrict__ dgamma, float* __restrict__ dbeta) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= H * D) return;
+  const int h = idx / D, f = idx - h * D;
+  float sg = 0.f, sb = 0.f;
+  for (int bi = 0; bi < B; ++bi) {
+    const size_t bh = (size_t)bi * H + h;
+    sg += gb_part[(bh * 2) * D + f];
+    sb += gb_part[(bh * 2 + 1) * D + f];
+  }
+  dgamma[idx] = sg;
+  dbeta[idx] = sb;
+}
+
+}  // namespace ttt

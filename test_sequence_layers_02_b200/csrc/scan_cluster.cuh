@@ -490,6 +490,12 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT, 1)
       finish_scalars(0, issue_scalars(0));
       if (nc > 1) finish_scalars(1, issue_scalars(1));
       cp_async_wait_all();
+      if (p.kq_silu) {
+        tile_silu<D, InT>(tileK(0), chunk_len(0), at, L::NW);
+        tile_silu<D, InT>(tileQ(0), chunk_len(0), at, L::NW);
+        if (nc > 1) tile_silu<D, InT>(tileK(1), chunk_len(1), at, L::NW);
+        if (nc > 2) tile_silu<D, InT>(tileK(2), chunk_len(2), at, L::NW);
+      }
     }
   }
   // every CTA has started and armed its barriers before any remote access
@@ -559,6 +565,10 @@ __global__ void __launch_bounds__(ClusterLayout<InT, CS>::NT, 1)
       if (c >= 1) outputs(c - 1, gpre);
       if (c + 2 < nc) finish_scalars(c + 2, pre);
       cp_async_wait_all();
+      if (p.kq_silu) {
+        if (c + 3 < nc) tile_silu<D, InT>(tileK(c + 3), chunk_len(c + 3), at, L::NW);
+        if (has_next) tile_silu<D, InT>(tileQ(c + 1), chunk_len(c + 1), at, L::NW);
+      }
     }
     __syncthreads();
   }

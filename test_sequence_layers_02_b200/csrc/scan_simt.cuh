@@ -126,6 +126,27 @@ __device__ __forceinline__ void tile_load(unsigned char* tile, const InT* src, i
   }
 }
 
+// SiLU, in place, on the pieces of a tile that tile_load() with the same
+// arguments copied for this thread (the `:mlp` variant's keys and queries).
+// Call after this thread's copies completed (cp.async.wait) and before the
+// barrier that publishes the tile; fp32 tiles only, so every element keeps
+// full precision. Rows past n were zero-filled and SiLU(0) = 0.
+template <int D, typename InT>
+__device__ __forceinline__ void tile_silu(unsigned char* tile, int n, int tid, int nthreads) {
+  if constexpr (sizeof(InT) == 4) {
+    using L = PipeLayout<D, InT, 1>;
+    constexpr int CPR = D * L::ELT / 16;
+    for (int idx = tid; idx < kC * CPR; idx += nthreads) {
+      const int row = idx / CPR;
+      if (row >= n) continue;
+      float4* x = reinterpret_cast<float4*>(tile + row * L::ROWB + (idx - row * CPR) * 16);
+      float4 v = *x;
+      v.x = siluf_(v.x); v.y = siluf_(v.y); v.z = siluf_(v.z); v.w = siluf_(v.w);
+      *x = v;
+    }
+  }
+}
+
 // Four consecutive elements of a shared-memory tile row (16 bytes of fp32 or
 // 8 bytes of bf16), widened to two fp32 pairs.
 template <typename InT>
@@ -881,6 +902,11 @@ __global__ void __launch_bounds__(2 * D * IH + 32, IH == 1 ? 3 : 1)
       finish_scalars(0, issue_scalars(0));
       if (nc > 1) finish_scalars(1, issue_scalars(1));
       cp_async_wait_all();
+      if (p.kq_silu) {
+        tile_silu<D, InT>(tileK(0), chunk_len(0), tid, NBT);
+        tile_silu<D, InT>(tileQ(0), chunk_len(0), tid, NBT);
+        if (nc > 1) tile_silu<D, InT>(tileK(1), chunk_len(1), tid, NBT);
+      }
     }
   } else {
     float sgb = 0.f, sb = 0.f;
@@ -1006,6 +1032,10 @@ __global__ void __launch_bounds__(2 * D * IH + 32, IH == 1 ? 3 : 1)
       }
       if (c + 2 < nc) finish_scalars(c + 2, pre);
       cp_async_wait_all();
+      if (p.kq_silu) {
+        if (c + 2 < nc) tile_silu<D, InT>(tileK(c + 2), chunk_len(c + 2), tid, NBT);
+        if (has_next) tile_silu<D, InT>(tileQ(c + 1), chunk_len(c + 1), tid, NBT);
+      }
     }
     __syncthreads();
 

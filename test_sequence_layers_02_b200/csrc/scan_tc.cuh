@@ -84,8 +84,8 @@ constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
 constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
 constexpr int oGam = oFlag + kSR * 4;              // gamma, beta [2][64] f32, sum gamma^2, sum gamma*beta
 constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
-// tma[NST], g[2], z[2], xm[2], w, wb, gram, pro
-constexpr int kBars = NST + 2 + 2 + 2 + 4;
+// tma[NST], g[2], z[2], xm[2], w, wb, gram, pro, rdy[NST]
+constexpr int kBars = NST + 2 + 2 + 2 + 4 + NST;
 constexpr int oTmem = oBar + kBars * 8;            // two TMEM base addresses
 constexpr int oAbort = oTmem + 8;
 constexpr int kSmemUsed = oAbort + 4;
@@ -159,6 +159,9 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   uint64_t* bar_wb = bar_w + 1;      // W_s bf16 refreshed (bulk, 128 arrivals)
   uint64_t* bar_gram = bar_wb + 1;   // Gram MMA complete (commit)
   uint64_t* bar_pro = bar_gram + 1;  // prologue MMAs complete (commit)
+  // [NST] stage x ready for the MMAs: with the SiLU variant, K_x and Q_{x-1}
+  // transformed in place (bulk, 128 arrivals); otherwise the TMA barrier is used
+  uint64_t* bar_rdy = bar_pro + 1;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + oTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + oAbort);
   auto tKQ = [&](int x) { return smem + oKQ + (x % NST) * 2 * kTile; };  // K_x, then Q_{x-1}
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       if (p.mask) r.m = p.mask[(size_t)bi * p.n_mask_chunks + x];
       const int t = x * CB + i;
       if (t < T) {
-        r.e = gel[t];
+        if (r.m) r.e = gel[t];  // a SKIP chunk takes no gradient: its eta is not read
         if (ggl) r.g = ggl[t];
       }
     }
@@ -233,11 +236,16 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   // ---- issuer helpers ----
   int tma_issued = 0;  // TMA loads [0, tma_issued) issued (chunk x = {K_x, Q_{x-1}, V_x})
   int w_issued = 0;    // commits to bar_w
+  // A SKIP chunk's keys and values are never used (its z, gradient and update
+  // are not formed), so only its queries are loaded; the K_x / V_x slots keep
+  // stale data that only reaches TMEM columns nobody reads (P_x; the Gram rows
+  // of Xg_x and M_x are zeroed by gram_extract).
   auto issue_tma = [&](int x) {
     uint64_t* bar = &bar_tma[x % NST];
-    const uint32_t bytes = (x < nc ? 2 * kTile : 0) + (x >= 1 ? kTile : 0);
+    const bool kv = x < nc && sFlag[x & (kSR - 1)] != 0;
+    const uint32_t bytes = (kv ? 2 * kTile : 0) + (x >= 1 ? kTile : 0);
     mbar_arrive_expect_tx(bar, bytes);
-    if (x < nc) {
+    if (kv) {
       tma_load_3d(tKQ(x), &maps.k, bar, 0, x * CB, (int)bh);
       tma_load_3d(tV(x), &maps.v, bar, 0, x * CB, (int)bh);
     }
@@ -245,6 +253,28 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     tma_issued = x + 1;
   };
   auto tma_parity = [&](int x) { return (uint32_t)((x / NST) & 1); };
+  // stage x ready for the MMAs (see bar_rdy)
+  auto wait_stage = [&](int x) {
+    return mbar_wait_bounded(p.kq_silu ? &bar_rdy[x % NST] : &bar_tma[x % NST], tma_parity(x),
+                             lim);
+  };
+  // The `:mlp` variant: SiLU in place on stage x (K_x and Q_{x-1}; bulk
+  // threads, 32 bytes each). The operands stay bf16, as the MMAs read them.
+  auto silu_stage = [&](int x) {
+    unsigned char* st = tKQ(x);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      uint4* ptr = reinterpret_cast<uint4*>(st + (gt + 128 * u) * 16);
+      uint4 w = *ptr;
+      uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        wv[e] = pack_bf16(siluf_(__uint_as_float(wv[e] << 16)),
+                          siluf_(__uint_as_float(wv[e] & 0xffff0000u)));
+      *ptr = w;
+    }
+    fence_proxy_async_smem();
+  };
   const uint32_t idescN16 = idesc_bf16_f32(128, 16, false, false);
   const uint32_t idescN32 = idesc_bf16_f32(128, 32, false, false);
   const uint32_t idescW = idesc_bf16_f32(128, 64, false, true);
@@ -276,10 +306,13 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     float r[16];
     tmem_ld16(tmem2 + 16u * (uint32_t)(x & 1), r);
     tmem_wait_ld();
-    const int n0 = chunk_len(x);
+    // Xg_{x+1} and M_x are used only when chunk x updates (Xg also needs
+    // chunk x+1 to update); the rows of a SKIP chunk are zero, which also
+    // discards the stale keys its stage holds
+    const int n0 = sFlag[x & (kSR - 1)] ? chunk_len(x) : 0;
     float v[16];
     if (lane < CB) {
-      const int n1 = (x + 1 < nc) ? chunk_len(x + 1) : 0;
+      const int n1 = (x + 1 < nc && sFlag[(x + 1) & (kSR - 1)]) ? chunk_len(x + 1) : 0;
 #pragma unroll
       for (int j = 0; j < CB; ++j) v[j] = (lane < n1 && j < n0) ? r[j] : 0.f;
     } else {
@@ -317,6 +350,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     mbar_init(bar_wb, 128);
     mbar_init(bar_gram, 1);
     mbar_init(bar_pro, 1);
+    for (int s = 0; s < NST; ++s) mbar_init(&bar_rdy[s], 128);
     mbar_init_fence();
     *sAbort = 0;
   }
@@ -384,6 +418,15 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   if (!mbar_wait_bounded(&bar_tma[0], 0, lim)) bad = true;
   if (!mbar_wait_bounded(&bar_tma[1], 0, lim)) bad = true;
   if (nc > 1 && !mbar_wait_bounded(&bar_tma[2], 0, lim)) bad = true;
+  if (p.kq_silu && is_bulk) {
+    // stages 0 .. min(3, nc) (the prologue MMAs and the first Gram read them)
+    for (int x = 0; x <= nc && x < 4; ++x) {
+      if (x == 3 && !mbar_wait_bounded(&bar_tma[3], 0, lim)) bad = true;
+      if (bad) break;
+      silu_stage(x);
+      mbar_arrive(&bar_rdy[x]);
+    }
+  }
   tc_fence_before();
   const bool pro_bad = __syncthreads_or(bad);
   tc_fence_after();
@@ -424,7 +467,8 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       // per-feature coefficients that do not depend on Z_k, formed before
       // waiting for it: LNJAC a = gamma^2, c = gamma (beta - v);
       // simplified a = gamma, c = beta - v; no LayerNorm c = -v
-      float a8[8], c8[8];
+      // ablation (GM 3, and GM 4 next to the full Jacobian form): a = 0, c = -gamma v
+      float a8[8], c8[8], cb8[8];
       {
         const unsigned char* Vt = tV(k) + tm_m * D * 2;
 #pragma unroll
@@ -432,9 +476,13 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           const int f = tm_p + 8 * u;
           const float v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Vt + f * 2));
           const float g = sGam[f];
-          if (GM == 1) {
+          cb8[u] = -g * v;
+          if (GM == 1 || GM == 4) {
             a8[u] = g * g;
             c8[u] = g * (sBet[f] - v);
+          } else if (GM == 3) {
+            a8[u] = 0.f;
+            c8[u] = cb8[u];
           } else if (GM == 0) {
             a8[u] = g;
             c8[u] = sBet[f] - v;
@@ -475,43 +523,81 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           for (int u = 0; u < 8; ++u) G[u] = z[u] + c8[u];
         } else {
           // shift by one element of the token, then all moments in one round
+          // (Jacobian forms: sums of a y, a y^2, c y, c; GM 4 also c_b y, c_b)
+          constexpr bool kJac = GM == 1 || GM == 3 || GM == 4;
+          constexpr int NM = GM == 4 ? 8 : (kJac ? 6 : 2);
           const float c0 = __shfl_sync(0xffffffffu, z[0], lane & ~7);
-          float m[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float m[NM];
+#pragma unroll
+          for (int i = 0; i < NM; ++i) m[i] = 0.f;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float y = z[u] - c0;
             z[u] = y;
             m[0] += y;
             m[1] = fmaf(y, y, m[1]);
-            if (GM == 1) {
+            if (kJac) {
               const float ay = a8[u] * y;
               m[2] += ay;
               m[3] = fmaf(ay, y, m[3]);
               m[4] = fmaf(c8[u], y, m[4]);
               m[5] += c8[u];
             }
+            if (GM == 4) {
+              m[6] = fmaf(cb8[u], y, m[6]);
+              m[7] += cb8[u];
+            }
           }
 #pragma unroll
           for (int off = 1; off < 8; off <<= 1) {
 #pragma unroll
-            for (int i = 0; i < (GM == 1 ? 6 : 2); ++i)
-              m[i] += __shfl_xor_sync(0xffffffffu, m[i], off);
+            for (int i = 0; i < NM; ++i) m[i] += __shfl_xor_sync(0xffffffffu, m[i], off);
           }
           const float inv_d = 1.0f / D;
           const float mu1 = m[0] * inv_d;                    // mean of the shifted values
           const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
           const float rs = rsqrtf(var + p.eps);
-          if (GM == 1) {
-            // moments of the centred values y - mu1
-            const float sg2y = m[2] - mu1 * sg2;
-            const float sg2yy = m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sg2;
-            const float swy = m[4] - mu1 * m[5];
-            const float mg = (rs * sg2y + m[5]) * inv_d;     // mean of g = gamma^2 xhat + w
-            const float mgx = rs * (rs * sg2yy + swy) * inv_d;
+          if (kJac) {
+            // J^T g with g = a xhat / rs + c (a = gamma^2, c = gamma (beta - v): the
+            // full form; a = 0, c = -gamma v: the ablation), from the moments of
+            // the centred values y - mu1
+            const float sa = (GM == 3) ? 0.f : sg2;          // sum of a
+            const float say = m[2] - mu1 * sa;
+            const float sayy = m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa;
+            const float scy = m[4] - mu1 * m[5];
+            const float mg = (rs * say + m[5]) * inv_d;      // mean of g
+            const float mgx = rs * (rs * sayy + scy) * inv_d;
             const float rs2 = rs * rs;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               G[u] = rs2 * (a8[u] - mgx) * (z[u] - mu1) + rs * (c8[u] - mg);
+            if (GM == 4) {
+              // the ablation (a = 0) next to the full form: both norms, then
+              // the ablation, rescaled to the full norm with norm matching
+              const float mgb = m[7] * inv_d;
+              const float mgxb = rs * (m[6] - mu1 * m[7]) * inv_d;
+              float nf = 0.f, nb = 0.f;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float gb = -rs2 * mgxb * (z[u] - mu1) + rs * (cb8[u] - mgb);
+                nf = fmaf(G[u], G[u], nf);
+                nb = fmaf(gb, gb, nb);
+                G[u] = gb;
+              }
+#pragma unroll
+              for (int off = 1; off < 8; off <<= 1) {
+                nf += __shfl_xor_sync(0xffffffffu, nf, off);
+                nb += __shfl_xor_sync(0xffffffffu, nb, off);
+              }
+              if (p.grad_norms != nullptr && tm_p == 0 && tm_m < n) {
+                float* gn = p.grad_norms + (tok0 + (size_t)k * CB + tm_m) * 2;
+                gn[0] = sqrtf(nf);
+                gn[1] = sqrtf(nb);
+              }
+              const float scale = !p.norm_match ? 1.f : (nb > 0.f ? sqrtf(nf / nb) : 0.f);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) G[u] *= scale;
+            }
           } else {
 #pragma unroll
             for (int u = 0; u < 8; ++u) G[u] = fmaf(a8[u] * rs, z[u] - mu1, c8[u]);
@@ -526,6 +612,11 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           *reinterpret_cast<__nv_bfloat16*>(An + core_off(f + 64, tm_m)) = a;
         }
         fence_proxy_async_smem();
+      } else if (GM == 4 && p.grad_norms != nullptr && tm_p == 0 && tm_m < n) {
+        // a SKIP chunk takes no gradient: zero norms for its tokens
+        float* gn = p.grad_norms + (tok0 + (size_t)k * CB + tm_m) * 2;
+        gn[0] = 0.f;
+        gn[1] = 0.f;
       }
       mbar_arrive(&bar_g[k & 1]);
     }
@@ -591,6 +682,15 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         fence_proxy_async_smem();
         issue_tma(c + NST);
       }
+      // SiLU variant: stage c+4, read first by the issuer's next iteration
+      if (p.kq_silu && c + 4 <= nc) {
+        if (mbar_wait_bounded(&bar_tma[(c + 4) % NST], tma_parity(c + 4), lim)) {
+          silu_stage(c + 4);
+          mbar_arrive(&bar_rdy[(c + 4) % NST]);
+        } else if (lane == 0) {
+          fail();
+        }
+      }
       // ---- Gram of chunk c+2 -> [Xg_{c+3}; M_{c+2}]. Its buffer held the
       // operand of chunk c's MMAc, complete since bar_w ----
       // (warp 4 alone: the other bulk warps go on to the outputs; a failed
@@ -646,8 +746,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
 
       if (c + 2 < nc) {
         // Gram of chunk c+2 (stages c+2, c+3) into TMEM slot c & 1
-        ok = mbar_wait_bounded(&bar_tma[(c + 2) % NST], tma_parity(c + 2), lim) &&
-             mbar_wait_bounded(&bar_tma[(c + 3) % NST], tma_parity(c + 3), lim);
+        ok = wait_stage(c + 2) && wait_stage(c + 3);
         if (!ok || *sAbort) {
           fail();
           break;
@@ -658,8 +757,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       }
       if (next) {
         // W_{s,c+1} in bf16, then [P_{c+2} | Q0_{c+1}] = W_{s,c+1} [K_{c+2}; Q_{c+1}]^T
-        ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) &&
-             mbar_wait_bounded(&bar_tma[(c + 2) % NST], tma_parity(c + 2), lim);
+        ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) && wait_stage(c + 2);
         if (!ok || *sAbort) {
           fail();
           break;

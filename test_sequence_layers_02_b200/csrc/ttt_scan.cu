@@ -11,6 +11,7 @@
 #include "scan_tc.cuh"
 #include "decode.cuh"
 #include "launch.h"
+#include "abi_util.h"
 
 #include <cudaTypedefs.h>
 
@@ -21,7 +22,7 @@ long long g_wait_limit = 1LL << 20;
 constexpr unsigned kKnownModes = TTT_MODE_MINIBATCH | TTT_GRAD_LNJAC | TTT_NO_LN |
                                  TTT_IN_BF16 | TTT_OUT_BF16 | TTT_KERNEL_SIMT |
                                  TTT_GATE_CHANNEL | TTT_KERNEL_SINGLE_CTA | TTT_GRAD_ABLATE |
-                                 TTT_GRAD_NORM_MATCH;
+                                 TTT_GRAD_NORM_MATCH | TTT_KQ_SILU;
 
 // Gradient-mode combinations that make no sense, whatever the kernel.
 bool bad_grad_mode(unsigned mode) {
@@ -30,13 +31,8 @@ bool bad_grad_mode(unsigned mode) {
   return false;
 }
 
-bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
-
-bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
-  if (!a || !b || na == 0 || nb == 0) return false;
-  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
-  return a0 < b0 + nb && b0 < a0 + na;
-}
+using ttt::abi::misaligned;
+using ttt::abi::overlaps;
 
 // Largest divisor of b that is <= cap.
 int largest_divisor_upto(int b, int cap) {
@@ -45,18 +41,36 @@ int largest_divisor_upto(int b, int cap) {
   return 1;
 }
 
+// Gradient variant of a call (as ttt::grad_variant): 0 simplified, 1 LN
+// Jacobian, 2 no LayerNorm, 3 ablation, 4 ablation with norm matching or with
+// the gradient norms written.
+int grad_variant_of(unsigned mode, bool norms) {
+  if (mode & TTT_NO_LN) return 2;
+  if (mode & TTT_GRAD_ABLATE) return ((mode & TTT_GRAD_NORM_MATCH) || norms) ? 4 : 3;
+  return (mode & TTT_GRAD_LNJAC) ? 1 : 0;
+}
+
 // Which kernel a valid call runs (see ttt_scan_kernel_choice in the header).
-int choose_kernel(long long heads, int T, int d, unsigned mode, int b) {
+// `norms`: the gradient norms are asked for (ttt_scan_forward_grad_norms).
+int choose_kernel(long long heads, int T, int d, unsigned mode, int b, bool norms) {
   if (heads == 0) return TTT_KERNEL_NONE;
   const bool minibatch = mode & TTT_MODE_MINIBATCH;
   if (minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
       !(mode & (TTT_KERNEL_SIMT | TTT_GATE_CHANNEL)) && T > 0)
     return TTT_KERNEL_ID_TENSOR_CORE;
-  if (!minibatch && d == 64 && !(mode & (TTT_KERNEL_SINGLE_CTA | TTT_GRAD_ABLATE)) && T > 0) {
-    const int gm = (mode & TTT_NO_LN) ? 2 : ((mode & TTT_GRAD_LNJAC) ? 1 : 0);
-    if (heads <= ttt::cluster_capacity(mode, gm)) return TTT_KERNEL_ID_CUDA_CORE_CLUSTER;
+  if (!minibatch && d == 64 && !(mode & TTT_KERNEL_SINGLE_CTA) && !norms && T > 0) {
+    if (heads <= ttt::cluster_capacity(mode, grad_variant_of(mode, norms)))
+      return TTT_KERNEL_ID_CUDA_CORE_CLUSTER;
   }
   return TTT_KERNEL_ID_CUDA_CORE;
+}
+
+// The CUDA-core kernels apply the SiLU variant to fp32 tiles only (a bf16
+// tile would round SiLU(k) back to bf16); the tensor-core kernel reads bf16
+// operands anyway.
+bool silu_unsupported(int kernel, unsigned mode) {
+  return (mode & TTT_KQ_SILU) && (mode & TTT_IN_BF16) && kernel != TTT_KERNEL_ID_TENSOR_CORE &&
+         kernel != TTT_KERNEL_NONE;
 }
 
 // ---- tensor-core kernel: tensor maps and launch ----
@@ -89,18 +103,6 @@ bool encode_qkv_map(CUtensorMap* map, const void* base, int T, long long heads, 
   return r == CUDA_SUCCESS;
 }
 
-// SMs of the current device (0 if the query fails).
-int device_sm_count() {
-  static int cache[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
-  return n;
-}
-
 template <typename OutT, int GM>
 int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   ttt::TcMaps maps;
@@ -111,7 +113,7 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
     return TTT_ERR_CUDA;
   // up to one head per SM: the one-CTA-per-SM build (more registers per
   // thread); beyond that, three CTAs share an SM
-  auto kernel = heads <= device_sm_count() ? ttt::scan_tc_kernel<OutT, GM, 1>
+  auto kernel = heads <= ttt::device_sm_count() ? ttt::scan_tc_kernel<OutT, GM, 1>
                                            : ttt::scan_tc_kernel<OutT, GM, 3>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ttt::tc::kSmemBytes) != cudaSuccess)
@@ -120,16 +122,19 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
-int dispatch_tc(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
-  const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
-  if (mode & TTT_OUT_BF16) {
-    if (gm == 0) return launch_tc<__nv_bfloat16, 0>(p, s);
-    if (gm == 1) return launch_tc<__nv_bfloat16, 1>(p, s);
-    return launch_tc<__nv_bfloat16, 2>(p, s);
+template <typename OutT>
+int dispatch_tc_gm(const ttt::ScanParams& p, cudaStream_t s) {
+  switch (ttt::grad_variant(p)) {
+    case 0: return launch_tc<OutT, 0>(p, s);
+    case 1: return launch_tc<OutT, 1>(p, s);
+    case 3: return launch_tc<OutT, 3>(p, s);
+    case 4: return launch_tc<OutT, 4>(p, s);
+    default: return launch_tc<OutT, 2>(p, s);
   }
-  if (gm == 0) return launch_tc<float, 0>(p, s);
-  if (gm == 1) return launch_tc<float, 1>(p, s);
-  return launch_tc<float, 2>(p, s);
+}
+
+int dispatch_tc(const ttt::ScanParams& p, unsigned mode, cudaStream_t s) {
+  return (mode & TTT_OUT_BF16) ? dispatch_tc_gm<__nv_bfloat16>(p, s) : dispatch_tc_gm<float>(p, s);
 }
 
 template <int D, typename InT, typename OutT>
@@ -150,6 +155,21 @@ int dispatch_decode(const ttt::DecodeParams& p, unsigned mode, cudaStream_t s) {
 }
 
 }  // namespace
+
+namespace ttt {
+
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace ttt
 
 extern "C" {
 
@@ -206,7 +226,10 @@ static int scan_forward(const void* q, const void* k, const void* v, const void*
     if (misaligned(p)) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
-  if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
+  const int which = choose_kernel((long long)B * H, T, d, mode, b, grad_norms != nullptr);
+  if (silu_unsupported(which, mode)) return TTT_ERR_UNSUPPORTED;
+  if (which == TTT_KERNEL_ID_CUDA_CORE && (mode & TTT_MODE_MINIBATCH) && b > ttt::kC)
+    return TTT_ERR_UNSUPPORTED;
 
   const size_t heads = (size_t)B * H;
   const int n_mask_chunks = (T + b - 1) / b;
@@ -260,23 +283,23 @@ static int scan_forward(const void* q, const void* k, const void* v, const void*
   p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
   p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
   p.grad_norms = grad_norms;
+  p.kq_silu = (mode & TTT_KQ_SILU) ? 1 : 0;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  const int which = choose_kernel((long long)heads, T, d, mode, b);
   if (which == TTT_KERNEL_ID_TENSOR_CORE) return dispatch_tc(p, mode, stream);
   if (p.minibatch) {
-    if (b > ttt::kC) return TTT_ERR_UNSUPPORTED;
     p.C = b;
   } else {
     // chunks must not straddle a mask / snapshot boundary when either is asked for
     p.C = (mask || W_chunks) ? largest_divisor_upto(b, ttt::kC) : ttt::kC;
   }
-  if (which == TTT_KERNEL_ID_CUDA_CORE_CLUSTER) {
-    const int gm = p.no_ln ? 2 : (p.lnjac ? 1 : 0);
-    return ttt::launch_cluster(p, mode, gm, stream);
-  }
-  return (mode & TTT_IN_BF16) ? ttt::launch_simt_bf16in(p, mode, d, stream)
-                              : ttt::launch_simt_f32in(p, mode, d, stream);
+  if (which == TTT_KERNEL_ID_CUDA_CORE_CLUSTER)
+    return ttt::launch_cluster(p, mode, ttt::grad_variant(p), stream);
+  if (mode & TTT_IN_BF16)
+    return p.minibatch ? ttt::launch_simt_bf16_minibatch(p, mode, d, stream)
+                       : ttt::launch_simt_bf16_pertoken(p, mode, d, stream);
+  return p.minibatch ? ttt::launch_simt_f32_minibatch(p, mode, d, stream)
+                     : ttt::launch_simt_f32_pertoken(p, mode, d, stream);
 }
 
 int ttt_scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,
@@ -304,8 +327,8 @@ int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b) {
   if (B < 0 || H < 0 || T < 0 || b < 1 || d <= 0) return TTT_ERR_INVALID_ARG;
   if (d != 16 && d != 64) return TTT_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
-  if ((mode & TTT_GRAD_ABLATE) && (mode & TTT_MODE_MINIBATCH)) return TTT_ERR_UNSUPPORTED;
-  const int which = choose_kernel((long long)B * H, T, d, mode, b);
+  const int which = choose_kernel((long long)B * H, T, d, mode, b, false);
+  if (silu_unsupported(which, mode)) return TTT_ERR_UNSUPPORTED;
   if (which == TTT_KERNEL_ID_CUDA_CORE && (mode & TTT_MODE_MINIBATCH) && b > ttt::kC)
     return TTT_ERR_UNSUPPORTED;
   return which;
@@ -361,6 +384,7 @@ int ttt_decode_step(const void* q, const void* k, const void* v, const void* eta
   p.gate_channel = (mode & TTT_GATE_CHANNEL) ? 1 : 0;
   p.ablate = (mode & TTT_GRAD_ABLATE) ? 1 : 0;
   p.norm_match = (mode & TTT_GRAD_NORM_MATCH) ? 1 : 0;
+  p.kq_silu = (mode & TTT_KQ_SILU) ? 1 : 0;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   return d == 64 ? dispatch_decode<64>(p, mode, stream) : dispatch_decode<16>(p, mode, stream);
 }

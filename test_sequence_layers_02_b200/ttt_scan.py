@@ -2,8 +2,8 @@
 
 Every step of the scan runs in the library's CUDA kernels; this module checks
 shapes and dtypes, allocates outputs with torch, and passes raw device pointers
-and the current CUDA stream to ``ttt_scan_forward`` and ``ttt_decode_step``
-(include/ttt_scan.h). There
+and the current CUDA stream to ``ttt_scan_forward``, ``ttt_scan_backward`` and
+``ttt_decode_step`` (include/ttt_scan.h). There
 is no CPU fallback: if the library cannot be loaded, the first call raises.
 """
 
@@ -28,6 +28,7 @@ GATE_CHANNEL = 1 << 6
 KERNEL_SINGLE_CTA = 1 << 7
 GRAD_ABLATE = 1 << 8
 GRAD_NORM_MATCH = 1 << 9
+KQ_SILU = 1 << 10
 
 # Kernel identifiers of ttt_scan_kernel_choice.
 KERNEL_NONE, KERNEL_CUDA_CORE, KERNEL_CUDA_CORE_CLUSTER, KERNEL_TENSOR_CORE = 0, 1, 2, 3
@@ -75,6 +76,12 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.ttt_set_wait_limit.restype = i
+        L.ttt_scan_backward_workspace_bytes.argtypes = [i, i, i, u]
+        L.ttt_scan_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_scan_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, ctypes.c_float,
+                                        u, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        vp, ctypes.c_size_t, vp]
+        L.ttt_scan_backward.restype = i
         L.ttt_probe_ffma.argtypes = [i, i, i, vp, ctypes.POINTER(ctypes.c_double), vp]
         L.ttt_probe_ffma.restype = i
         _lib = L
@@ -105,9 +112,9 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
          minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
          b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
          force_simt: bool = False, single_cta: bool = False, ablate: bool = False,
-         norm_match: bool = False, want_chunks: bool = False, want_grad_norms: bool = False,
-         o: Optional[torch.Tensor] = None, W_T: Optional[torch.Tensor] = None,
-         stream: Optional[torch.cuda.Stream] = None):
+         norm_match: bool = False, kq_silu: bool = False, want_chunks: bool = False,
+         want_grad_norms: bool = False, o: Optional[torch.Tensor] = None,
+         W_T: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
     """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
 
     q, k, v: [B, H, T, d] fp32 or bf16; eta_logit: [B, H, T] with the same
@@ -119,24 +126,29 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     per-token mode on one CTA per head (see ``kernel_choice``). ``ablate``
     selects the ablation gradient (the LayerNorm Jacobian applied to
     -gamma * v), ``norm_match`` rescales it per token to the full gradient's norm.
-    ``want_grad_norms`` (with ``ablate``, per-token) also returns [B, H, T, 2]
+    ``kq_silu`` runs the `:mlp` variant (SiLU on every key and query).
+    ``want_grad_norms`` (with ``ablate``) also returns [B, H, T, 2]
     fp32: per token the norms of the full and of the ablated gradient (zeros
     on SKIP chunks), after W_T (and the chunk snapshots, if asked for).
 
     CUDA tensors run on ``stream`` (default: the current stream) and return
     without synchronising. CPU tensors take the end-to-end path: inputs are
     copied to the current CUDA device, the scan runs there, and o / W_T are
-    copied back to host memory before returning.
+    copied back to host memory before returning; the copies and the scan are
+    all issued on ``stream``, so they are ordered.
     """
     host = not q.is_cuda
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
-        mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
-        q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask = map(
-            mv, (q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask))
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(s):
+            mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+            q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask = map(
+                mv, (q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask))
         o_dev, wt_dev = None, None
     else:
         o_dev, wt_dev = o, W_T
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
     if q.dim() != 4:
         raise ValueError("q must be [B, H, T, d]")
     B, H, T, d = q.shape
@@ -167,16 +179,17 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
             (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
             (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0) |
             (KERNEL_SINGLE_CTA if single_cta else 0) | (GRAD_ABLATE if ablate else 0) |
-            (GRAD_NORM_MATCH if norm_match else 0) | (GATE_CHANNEL if channel else 0))
-    if o_dev is None:
-        o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
-    if wt_dev is None:
-        wt_dev = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
-    wc = (torch.empty((B, H, n_chunks + 1, d, d), dtype=torch.float32, device=q.device)
-          if want_chunks else None)
-    gn = (torch.empty((B, H, T, 2), dtype=torch.float32, device=q.device)
-          if want_grad_norms else None)
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+            (GRAD_NORM_MATCH if norm_match else 0) | (GATE_CHANNEL if channel else 0) |
+            (KQ_SILU if kq_silu else 0))
+    with torch.cuda.stream(s):
+        if o_dev is None:
+            o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
+        if wt_dev is None:
+            wt_dev = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+        wc = (torch.empty((B, H, n_chunks + 1, d, d), dtype=torch.float32, device=q.device)
+              if want_chunks else None)
+        gn = (torch.empty((B, H, T, 2), dtype=torch.float32, device=q.device)
+              if want_grad_norms else None)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W0), _ptr(gamma),
             _ptr(beta), B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(o_dev),
             _ptr(wt_dev), _ptr(wc))
@@ -190,26 +203,95 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
         o_h = o if o is not None else torch.empty(o_dev.shape, dtype=o_dev.dtype, pin_memory=True)
         wt_h = W_T if W_T is not None else torch.empty(wt_dev.shape, dtype=torch.float32,
                                                        pin_memory=True)
-        o_h.copy_(o_dev, non_blocking=True)
-        wt_h.copy_(wt_dev, non_blocking=True)
+        with torch.cuda.stream(s):
+            o_h.copy_(o_dev, non_blocking=True)
+            wt_h.copy_(wt_dev, non_blocking=True)
+            extra = tuple(x.to("cpu") for x in (wc, gn) if x is not None)
         rc = check_device_status(s)
         if rc != TTT_OK:
             raise TTTScanError(rc, "device")
-        extra = ((wc.cpu(),) if want_chunks else ()) + ((gn.cpu(),) if want_grad_norms else ())
         return (o_h, wt_h) + extra
     extra = ((wc,) if want_chunks else ()) + ((gn,) if want_grad_norms else ())
     return (o_dev, wt_dev) + extra
 
 
+def scan_backward(q, k, v, eta_logit, gate_logit, gamma, beta, W_chunks, dO, dW_T=None, *,
+                  eps: float = 1e-6, minibatch: bool = False, lnjac: bool = False,
+                  no_ln: bool = False, ablate: bool = False, kq_silu: bool = False, b: int = 16,
+                  mask=None, workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of ``<dO, o> + <dW_T, W_T>`` for a ``scan`` with the same arguments.
+
+    Inputs as for ``scan`` (CUDA tensors), plus ``W_chunks`` [B, H, ceil(T/b) + 1,
+    d, d] (the snapshots ``scan(..., want_chunks=True)`` returns), ``dO`` [B, H, T,
+    d] fp32 and ``dW_T`` [B, H, d, d] fp32 or None (zero). ``workspace`` (optional)
+    is a device tensor of at least ``backward_workspace_bytes`` bytes; by default
+    one is allocated here. Returns a dict of fp32 tensors dq, dk, dv, deta_logit,
+    dgate_logit (None without a gate), dW0, dgamma, dbeta (None with ``no_ln``).
+    Runs on ``stream`` (default: the current stream) without synchronising.
+    """
+    if q.dim() != 4 or not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor [B, H, T, d]")
+    B, H, T, d = q.shape
+    in_dtype = q.dtype
+    channel = gate_logit is not None and gate_logit.dim() == 4
+    n_chunks = -(-T // b) if b > 0 else 0
+    for name, t, shp, dt in (("k", k, (B, H, T, d), in_dtype), ("v", v, (B, H, T, d), in_dtype),
+                             ("eta_logit", eta_logit, (B, H, T), in_dtype),
+                             ("gate_logit", gate_logit, (B, H, T, d) if channel else (B, H, T),
+                              in_dtype),
+                             ("W_chunks", W_chunks, (B, H, n_chunks + 1, d, d), torch.float32),
+                             ("dO", dO, (B, H, T, d), torch.float32),
+                             ("dW_T", dW_T, (B, H, d, d), torch.float32),
+                             ("mask", mask, (B, n_chunks), torch.uint8)):
+        if t is None and name in ("gate_logit", "dW_T", "mask"):
+            continue
+        if tuple(t.shape) != shp or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous {shp} {dt}")
+    mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
+            (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
+            (GRAD_ABLATE if ablate else 0) | (GATE_CHANNEL if channel else 0) |
+            (KQ_SILU if kq_silu else 0))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    need = int(lib().ttt_scan_backward_workspace_bytes(B, H, d, mode))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    with torch.cuda.stream(s):
+        out = dict(dq=torch.empty((B, H, T, d), **f32), dk=torch.empty((B, H, T, d), **f32),
+                   dv=torch.empty((B, H, T, d), **f32), deta_logit=torch.empty((B, H, T), **f32),
+                   dgate_logit=None if gate_logit is None else torch.empty(gate_logit.shape, **f32),
+                   dW0=torch.empty((B, H, d, d), **f32),
+                   dgamma=None if no_ln else torch.empty((H, d), **f32),
+                   dbeta=None if no_ln else torch.empty((H, d), **f32))
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().ttt_scan_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(gamma), _ptr(beta),
+        B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(W_chunks), _ptr(dO), _ptr(dW_T),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["deta_logit"]),
+        _ptr(out["dgate_logit"]), _ptr(out["dW0"]), _ptr(out["dgamma"]), _ptr(out["dbeta"]),
+        _ptr(workspace), ws_bytes, ctypes.c_void_p(s.cuda_stream))
+    if rc != TTT_OK:
+        raise TTTScanError(rc, "ttt_scan_backward")
+    return out
+
+
+def backward_workspace_bytes(B: int, H: int, d: int, *, no_ln: bool = False) -> int:
+    """Bytes of device workspace ``ttt_scan_backward`` needs for these sizes."""
+    return int(lib().ttt_scan_backward_workspace_bytes(B, H, d, NO_LN if no_ln else 0))
+
+
 def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
                   lnjac: bool = False, no_ln: bool = False, in_bf16: bool = False,
                   out_bf16: bool = False, b: int = 16, force_simt: bool = False,
-                  single_cta: bool = False, ablate: bool = False, norm_match: bool = False) -> int:
+                  single_cta: bool = False, ablate: bool = False, norm_match: bool = False,
+                  kq_silu: bool = False) -> int:
     """The KERNEL_* identifier ``scan`` would run for these sizes (launches nothing)."""
     mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_bf16 else 0) | (OUT_BF16 if out_bf16 else 0) |
             (KERNEL_SIMT if force_simt else 0) | (KERNEL_SINGLE_CTA if single_cta else 0) |
-            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0))
+            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0) |
+            (KQ_SILU if kq_silu else 0))
     rc = lib().ttt_scan_kernel_choice(B, H, T, d, mode, b)
     if rc < 0:
         raise TTTScanError(rc, "ttt_scan_kernel_choice")
@@ -218,7 +300,7 @@ def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
 
 def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 1e-6,
                 lnjac: bool = False, no_ln: bool = False, ablate: bool = False,
-                norm_match: bool = False, update=None,
+                norm_match: bool = False, kq_silu: bool = False, update=None,
                 out_dtype: Optional[torch.dtype] = None, o: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None):
     """One streaming step ``o = decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta)``.
@@ -231,19 +313,24 @@ def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 
 
     CUDA tensors run on ``stream`` without synchronising. CPU tensors take the
     end-to-end path: inputs and W go to the current CUDA device, the step runs
-    there, and o and the new W come back (W is overwritten in host memory).
+    there, and o and the new W come back (W is overwritten in host memory); the
+    copies and the step are all issued on ``stream``, so they are ordered.
+    ``kq_silu`` runs the `:mlp` variant (SiLU on k and q).
     """
     host = not q.is_cuda
     W_host = None
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
-        mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
         W_host = W
-        q, k, v, eta_logit, gate_logit, W, gamma, beta, update = map(
-            mv, (q, k, v, eta_logit, gate_logit, W, gamma, beta, update))
+        with torch.cuda.stream(s):
+            mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+            q, k, v, eta_logit, gate_logit, W, gamma, beta, update = map(
+                mv, (q, k, v, eta_logit, gate_logit, W, gamma, beta, update))
         o_dev = None
     else:
         o_dev = o
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
     if q.dim() != 3:
         raise ValueError("q must be [B, H, d]")
     B, H, d = q.shape
@@ -269,10 +356,11 @@ def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 
     mode = ((GRAD_LNJAC if lnjac else 0) | (NO_LN if no_ln else 0) |
             (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
             (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (GATE_CHANNEL if channel else 0) |
-            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0))
+            (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0) |
+            (KQ_SILU if kq_silu else 0))
     if o_dev is None:
-        o_dev = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        with torch.cuda.stream(s):
+            o_dev = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
     rc = lib().ttt_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W), _ptr(gamma),
         _ptr(beta), B, H, d, float(eps), mode, _ptr(update), _ptr(o_dev),
@@ -281,8 +369,9 @@ def decode_step(q, k, v, eta_logit, gate_logit, W, gamma, beta, *, eps: float = 
         raise TTTScanError(rc, "ttt_decode_step")
     if host:
         o_h = o if o is not None else torch.empty(o_dev.shape, dtype=o_dev.dtype, pin_memory=True)
-        o_h.copy_(o_dev, non_blocking=True)
-        W_host.copy_(W, non_blocking=True)
+        with torch.cuda.stream(s):
+            o_h.copy_(o_dev, non_blocking=True)
+            W_host.copy_(W, non_blocking=True)
         rc = check_device_status(s)
         if rc != TTT_OK:
             raise TTTScanError(rc, "device")

@@ -80,7 +80,7 @@ INVALID, UNSUPPORTED = -1, -2
     dict(q=addr(0, 4)), dict(o=addr(8, 8)), dict(mask=addr(10, 1)), dict(W_chunks=addr(11, 2)),
     dict(B=-1), dict(H=-1), dict(T=-1), dict(b=0), dict(b=-3), dict(d=0), dict(d=-64),
     dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")),
-    dict(mode=1 << 10), dict(mode=1 << 31),
+    dict(mode=1 << 11), dict(mode=1 << 31),
     dict(mode=(1 << 8) | 4),              # ablation without a LayerNorm
     dict(mode=1 << 9),                    # norm matching without the ablation
     dict(o=addr(0)),                      # output over an input
@@ -95,7 +95,8 @@ def test_invalid_arguments_rejected(lib, over):
 
 @pytest.mark.parametrize("over", [dict(d=32), dict(d=128), dict(d=17),
                                   dict(mode=1, b=17), dict(mode=1 | 32, b=32),
-                                  dict(mode=1 | (1 << 8))])
+                                  dict(mode=(1 << 10) | 8),            # SiLU, bf16, per-token
+                                  dict(mode=(1 << 10) | 8 | 1 | 32)])  # SiLU, bf16, CUDA-core mini-batch
 def test_unsupported_shapes(lib, over):
     assert call(lib, **over) == UNSUPPORTED
 
@@ -122,7 +123,7 @@ def call_gn(lib, **over):
     (dict(gn=addr(8)), INVALID),                   # over o
     (dict(gn=addr(9)), INVALID),                   # over W_T
     (dict(gn=addr(2, 1 << 10)), INVALID),          # inside v
-    (dict(mode=(1 << 8) | 1), UNSUPPORTED),        # mini-batch has no ablation form
+    (dict(mode=(1 << 8) | 8 | (1 << 10)), UNSUPPORTED),   # SiLU on bf16 CUDA-core tiles
     (dict(d=32), UNSUPPORTED),
     (dict(B=0), 0), (dict(B=0, gn=None), 0), (dict(T=0, B=0), 0),   # empty: nothing launched
 ], ids=lambda x: ",".join(x) if isinstance(x, dict) else str(x))
@@ -156,7 +157,7 @@ def dcall(lib, **over):
     dict(gamma=None), dict(beta=None),
     dict(q=addr(0, 4)), dict(W=addr(5, 8)), dict(update=addr(10, 1)), dict(o=addr(8, 2)),
     dict(B=-1), dict(H=-1), dict(d=0), dict(eps=-1.0), dict(eps=float("nan")),
-    dict(mode=1 << 10), dict(mode=(1 << 8) | 4), dict(mode=1 << 9),
+    dict(mode=1 << 11), dict(mode=(1 << 8) | 4), dict(mode=1 << 9),
     dict(o=addr(1)),                      # output over an input
     dict(W=addr(8)),                      # state over the output
     dict(W=addr(2, 64)),                  # state inside v
@@ -185,11 +186,17 @@ def test_kernel_choice_without_launching(lib):
     assert f(2, 3, 40, 16, 0, 16) == 1                               # d = 16: one CTA per head
     assert f(2, 3, 40, 64, 1 << 7, 16) == 1                          # single CTA asked for
     assert f(0, 3, 40, 64, 0, 16) == 0                               # nothing to launch
-    assert f(2, 3, 40, 64, 1 << 10, 16) == INVALID
+    assert f(2, 3, 40, 64, 1 << 11, 16) == INVALID
     assert f(2, 3, 40, 64, 1 << 9, 16) == INVALID                     # norm match alone
     assert f(2, 3, 40, 64, (1 << 8) | 4, 16) == INVALID               # ablation without LN
-    assert f(2, 3, 40, 64, 1 | (1 << 8), 16) == UNSUPPORTED           # mini-batch ablation
-    assert f(2, 3, 40, 64, 1 << 8, 16) == 1                           # ablation: one CTA per head
+    assert f(2, 3, 40, 64, 1 | (1 << 8), 16) == 1                     # mini-batch ablation, fp32
+    assert f(2, 3, 40, 64, MINIB | BF16 | (1 << 8), 16) == 3          # ... bf16: tensor cores
+    assert f(2, 3, 40, 64, MINIB | BF16 | (1 << 8) | (1 << 9), 16) == 3
+    assert f(2, 3, 40, 64, 1 << 8, 16) in (1, 2)                      # per-token ablation
+    assert f(2, 3, 40, 64, (1 << 10) | BF16, 16) == UNSUPPORTED       # SiLU on bf16 CUDA-core tiles
+    assert f(2, 3, 40, 64, (1 << 10) | BF16 | MINIB, 16) == 3         # ... on the tensor cores
+    assert f(2, 3, 40, 64, 1 << 10, 16) in (1, 2)                     # SiLU, fp32, per-token
+    assert f(2, 3, 40, 16, (1 << 10) | MINIB, 16) == 1
     assert f(2, 3, 40, 64, 0, 0) == INVALID
     assert f(2, 3, 40, 32, 0, 16) == UNSUPPORTED
     assert f(2, 3, 40, 64, MINIB, 17) == UNSUPPORTED
@@ -216,3 +223,47 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(ts, "_LIB_PATH", tmp_path / "missing.so")
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         ts.lib()
+
+
+def bcall(lib, **over):
+    """ttt_scan_backward with fake, non-overlapping device addresses."""
+    a = dict(q=addr(0), k=addr(1), v=addr(2), eta=addr(3), gate=addr(4), gamma=addr(6),
+             beta=addr(7), B=2, H=3, T=40, d=64, eps=1e-6, mode=2, b=16, mask=None,
+             Wc=addr(13), dO=addr(14), dWT=None, dq=addr(15), dk=addr(16), dv=addr(17),
+             deta=addr(18), dgate=addr(19), dW0=addr(20), dgamma=addr(21), dbeta=addr(22),
+             ws=addr(23), ws_bytes=1 << 20)
+    a.update(over)
+    return lib.ttt_scan_backward(a["q"], a["k"], a["v"], a["eta"], a["gate"], a["gamma"],
+                                 a["beta"], a["B"], a["H"], a["T"], a["d"], a["eps"], a["mode"],
+                                 a["b"], a["mask"], a["Wc"], a["dO"], a["dWT"], a["dq"], a["dk"],
+                                 a["dv"], a["deta"], a["dgate"], a["dW0"], a["dgamma"],
+                                 a["dbeta"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(dO=None), dict(Wc=None), dict(dq=None), dict(dW0=None),
+    dict(dgate=None),                     # a gate needs its gradient
+    dict(dgamma=None), dict(ws=None),     # LayerNorm: gamma / beta gradients and workspace
+    dict(ws_bytes=2 * 3 * 2 * 64 * 4 - 4),
+    dict(dq=addr(15, 4)), dict(B=-1), dict(b=0), dict(eps=-1.0), dict(mode=1 << 11),
+    dict(mode=(1 << 8) | 4), dict(mode=1 << 9),
+    dict(dq=addr(0)),                     # output over an input
+    dict(dk=addr(15)),                    # two outputs on one buffer
+    dict(ws=addr(21)),                    # workspace over dgamma
+], ids=lambda o: ",".join(f"{k}" for k in o))
+def test_backward_invalid_arguments_rejected(lib, over):
+    assert bcall(lib, **over) == INVALID
+
+
+@pytest.mark.parametrize("over", [dict(d=32), dict(b=17), dict(mode=(1 << 8) | (1 << 9) | 2)])
+def test_backward_unsupported(lib, over):
+    assert bcall(lib, **over) == UNSUPPORTED
+
+
+def test_backward_workspace_bytes_and_no_ln(lib):
+    f = lib.ttt_scan_backward_workspace_bytes
+    assert f(2, 3, 64, 2) == 2 * 3 * 2 * 64 * 4
+    assert f(2, 3, 64, 4) == 0                       # no LayerNorm: no gamma / beta
+    assert f(0, 3, 64, 2) == 0
+    # no LayerNorm: gamma, beta, their gradients and the workspace may be absent
+    assert bcall(lib, B=0, mode=4, gamma=None, beta=None, dgamma=None, dbeta=None, ws=None) == 0

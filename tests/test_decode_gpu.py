@@ -39,7 +39,7 @@ def step_inputs(B, H, d, *, seed, in_bf16, gate="scalar", update_p=None):
     return out
 
 
-def gpu_step(inp, *, in_bf16, out_bf16, lnjac, no_ln, eps, W=None):
+def gpu_step(inp, *, in_bf16, out_bf16, lnjac, no_ln, eps, W=None, kq_silu=False):
     import torch
     from test_sequence_layers_02_b200 import ttt_scan
     t = to_torch(inp, "cuda", in_bf16)
@@ -47,7 +47,7 @@ def gpu_step(inp, *, in_bf16, out_bf16, lnjac, no_ln, eps, W=None):
     upd = None if inp.get("update") is None else torch.from_numpy(inp["update"]).cuda()
     o = ttt_scan.decode_step(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], W_dev,
                              t["gamma"], t["beta"], eps=eps, lnjac=lnjac, no_ln=no_ln,
-                             update=upd,
+                             update=upd, kq_silu=kq_silu,
                              out_dtype=torch.bfloat16 if out_bf16 else torch.float32)
     torch.cuda.synchronize()
     assert ttt_scan.check_device_status() == ttt_scan.TTT_OK
@@ -67,7 +67,8 @@ def np64(t):
 
 
 def assert_out_close(got, ref, out_bf16, what):
-    """fp32 bound; a bf16 output adds its own rounding (half an ulp, 2^-9 relative)."""
+    """fp32 bound; a bf16 output adds its own rounding to nearest, half an ulp,
+    which is at most 2^-8 of the value (bf16 keeps 8 significant bits)."""
     if not out_bf16:
         assert_fp32_close(got, ref, what)
         return
@@ -210,3 +211,16 @@ def test_decode_empty_and_bad_arguments():
     with pytest.raises(ValueError):
         ttt_scan.decode_step(z(1, 2, 64), z(1, 2, 64), z(1, 2, 64), z(1, 2), None,
                              z(1, 2, 64, 16), z(2, 64), z(2, 64))
+
+
+@pytest.mark.parametrize("d", [16, 64])
+@pytest.mark.parametrize("dtypes", [(False, False), (True, True)], ids=["f32", "bf16io"])
+def test_decode_kq_silu_variant(d, dtypes):
+    """The `:mlp` variant's decode step (SiLU on k and q) against the oracle."""
+    in_bf16, out_bf16 = dtypes
+    inp = step_inputs(3, 5, d, seed=560 + d, in_bf16=in_bf16, update_p=0.7)
+    o, W = gpu_step(inp, in_bf16=in_bf16, out_bf16=out_bf16, lnjac=True, no_ln=False, eps=1e-6,
+                    kq_silu=True)
+    ro, rW = oracle_step(inp, mode=LNJAC | (1 << 10), eps=1e-6)
+    assert_out_close(np64(o), ro, out_bf16, "o")
+    assert_fp32_close(np64(W), rW, "W")
