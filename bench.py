@@ -38,7 +38,7 @@ sys.path.insert(0, str(ROOT))
 
 METRIC = "TTT-Linear scan head-tokens/sec at d=64 on 1 B200; % of binding roofline"
 HEADLINE = "5"
-EXTRA = ["1", "2", "3", "4", "4pt", "dec"]
+EXTRA = ["1", "2", "3", "4", "4pt", "dec", "bwd2", "bwd3"]
 L2_FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PROFILE_TRAFFIC = ROOT / "profiles" / "dram_traffic.json"
 
@@ -64,6 +64,7 @@ _KERNEL_SOURCES = {
     "scan_tc": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
     "decode_step": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h",
                     "common.cuh"],
+    "scan_bwd": ["backward.cu", "scan_bwd.cuh", "scan_simt.cuh", "abi_util.h", "common.cuh"],
 }
 # Captures: a kernel may have several (e.g. the tensor-core kernel with and
 # without a SKIP/UPDATE mask); each names the kernel whose sources it covers.
@@ -331,8 +332,116 @@ class DecodeJob:
         self._call(self.h_in, self.h_in["W0"], self.h_o)
 
 
+class BwdJob:
+    """The backward pass of a scan workload (gradients of <dO, o> + <dW_T, W_T>
+    for every input), from the forward's chunk snapshots; the forward runs once
+    before timing, outside the timed region."""
+
+    decode = False
+    BWD_OF = {"bwd2": "2j", "bwd3": "3"}
+
+    def __init__(self, name: str, device):
+        import torch
+        from test_sequence_layers_02_b200 import ttt_scan
+        from test_sequence_layers_02_b200.workloads import WORKLOADS, make_workload
+        self.name = name
+        self.w = w = WORKLOADS[self.BWD_OF[name]]
+        self.passes = [dict(lnjac=w.lnjac)]
+        self.inp = make_workload(w)
+        self.mask_np = self.inp.get("mask")
+        self.t = _dev_inputs(self.inp, w, device)
+        t = self.t
+        rng = np.random.default_rng(w.seed + 77)
+        self.t["dO"] = torch.from_numpy(
+            rng.standard_normal((w.B, w.H, w.T, w.d), dtype=np.float32)).to(device)
+        self.t["dW_T"] = torch.from_numpy(
+            (0.1 * rng.standard_normal((w.B, w.H, w.d, w.d))).astype(np.float32)).to(device)
+        self.kw = dict(eps=w.eps, minibatch=w.minibatch, lnjac=w.lnjac, b=w.b)
+        _, _, self.t["W_chunks"] = ttt_scan.scan(
+            t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"],
+            t["beta"], mask=t["mask"], want_chunks=True, force_simt=True,
+            out_dtype=torch.float32, **self.kw)
+        self.ws = torch.empty(ttt_scan.backward_workspace_bytes(w.B, w.H, w.d), dtype=torch.uint8,
+                              device=device)
+        self.bwd = ttt_scan.scan_backward
+        torch.cuda.synchronize()
+
+    @property
+    def head_tokens_per_step(self) -> int:
+        return self.w.head_tokens
+
+    def _call(self, t):
+        return self.bwd(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["gamma"],
+                        t["beta"], t["W_chunks"], t["dO"], t["dW_T"], mask=t["mask"],
+                        workspace=self.ws, **self.kw)
+
+    def step(self):
+        self.out = self._call(self.t)
+
+    def launches_per_step(self) -> int:
+        return 2  # the per-head kernel and the gamma / beta reduction
+
+    def steps_per_chain(self) -> int:
+        return self.w.T
+
+    def update_fraction(self) -> float:
+        return 1.0 if self.mask_np is None else float(self.mask_np.mean())
+
+    def flops_per_step(self) -> float:
+        # per head-token: the forward recomputed from W_s (W_s k, W_s q: 4 d^2),
+        # D_e k (2 d^2), W_s^T dy, W_s^T dz, D_e^T G (6 d^2), the rank-2 update of
+        # D (4 d^2); the O(b d) Gram terms are left out
+        return 16.0 * self.w.d * self.w.d * self.w.head_tokens
+
+    def bytes_per_step(self) -> float:
+        w = self.w
+        d = w.d
+        ie = 2 if w.in_bf16 else 4
+        per_tok = 3 * d * ie + 2 * ie + d * 4 + 3 * d * 4 + 2 * 4   # inputs, dO; dq, dk, dv, dlogits
+        snaps = (w.n_chunks + 1) * d * d * 4 * w.heads               # W_chunks
+        return float(per_tok * w.head_tokens + snaps + 2 * d * d * 4 * w.heads)
+
+    def bound(self):
+        return "alu"
+
+    def kernel_key(self) -> str:
+        return "scan_bwd"
+
+    def capture_key(self) -> str:
+        return "scan_bwd"
+
+    def e2e_setup(self):
+        """Pinned host copies of the inputs (with the forward's snapshots and dO)
+        and of the gradients."""
+        import torch
+        self.h_in = {k: (None if v is None else v.cpu().pin_memory()) for k, v in self.t.items()}
+        self.d_in = {k: (None if v is None else torch.empty_like(v)) for k, v in self.t.items()}
+        out = self._call(self.t)
+        self.h_out = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory())
+                      for k, v in out.items()}
+        h2d = sum(v.numel() * v.element_size() for v in self.h_in.values() if v is not None)
+        d2h = sum(v.numel() * v.element_size() for v in self.h_out.values() if v is not None)
+        return h2d, d2h
+
+    def e2e_step(self):
+        """Inputs in, the public backward call, every gradient back to the host."""
+        import torch
+        for k, v in self.h_in.items():
+            if v is not None:
+                self.d_in[k].copy_(v, non_blocking=True)
+        out = self._call(self.d_in)
+        for k, v in out.items():
+            if v is not None:
+                self.h_out[k].copy_(v, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+
 def _make_job(name, device, seed_offset=0):
-    return DecodeJob(name, device) if name == "dec" else Job(name, device, seed_offset)
+    if name == "dec":
+        return DecodeJob(name, device)
+    if name in BwdJob.BWD_OF:
+        return BwdJob(name, device)
+    return Job(name, device, seed_offset)
 
 
 def _flush(buf):
@@ -486,17 +595,28 @@ def _roofline(job, per_launch_s, peaks, fp32_meas_tflops, n_sm):
 
 def _oracle_heads(job, heads, threads):
     """One oracle run over the first `heads` heads of the workload (in batch-row
-    order, OpenMP over heads), every pass."""
+    order, OpenMP over heads), every pass (the backward job: the oracle's
+    backward, one head after another)."""
     import oracle
     w, inp = job.w, job.inp
+    if isinstance(job, BwdJob):
+        rows = max(1, -(-heads // w.H))
+        hh = min(heads, w.H)
+        f64 = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
+        sel = lambda a: None if a is None else f64(a[:rows, :hh])
+        m = inp.get("mask")
+        oracle.backward(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(inp["eta_logit"]),
+                        sel(inp["gate_logit"]), sel(inp["W0"]), f64(inp["gamma"][:hh]),
+                        f64(inp["beta"][:hh]), sel(job.t["dO"].cpu().numpy()),
+                        sel(job.t["dW_T"].cpu().numpy()), eps=w.eps,
+                        mode=(1 if w.minibatch else 0) | (2 if w.lnjac else 0), b=w.b,
+                        mask=None if m is None else m[:rows])
+        return rows * hh
     f64 = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
-    if job.decode:
-        take = lambda a: None if a is None else a[:, :, :1]
-    else:
-        take = lambda a: a
     rows = max(1, -(-heads // w.H))
     hh = min(heads, w.H)
-    sel = lambda a: None if a is None else f64(take(a)[:rows, :hh])
+    # the decode workload's inputs hold one token per head already ([B, H, 1, ...])
+    sel = lambda a: None if a is None else f64(a[:rows, :hh])
     m = inp.get("mask")
     for ps in job.passes:
         mode = (1 if w.minibatch else 0) | (2 if ps["lnjac"] else 0)
@@ -515,24 +635,21 @@ def _oracle_sample(job, budget_s):
     cores = len(os.sched_getaffinity(0))
     T = 1 if job.decode else w.T
     heads = min(w.heads, cores)
-    t0 = time.perf_counter()
-    done = _oracle_heads(job, heads, min(cores, heads))
-    el = time.perf_counter() - t0
-    reps, ht = 1, done * T * len(job.passes)
-    if el < budget_s and heads < w.heads:
-        # scale the sample up to the budget (whole rows of heads), then time it
-        want = int(heads * budget_s / max(el, 1e-3))
-        heads = max(heads, min(w.heads, want))
+    while True:
+        # grow the sample (whole rows of heads) until it fills the budget
         t0 = time.perf_counter()
         done = _oracle_heads(job, heads, min(cores, heads))
         el = time.perf_counter() - t0
-        ht = done * T * len(job.passes)
+        if el >= 0.5 * budget_s or done >= w.heads:
+            break
+        heads = min(w.heads, max(2 * heads, int(heads * budget_s / max(el, 1e-3))))
+    reps, ht = 1, done * T * len(job.passes)
     while el < budget_s and done >= w.heads and reps < 1000000:
         t1 = time.perf_counter()
         _oracle_heads(job, heads, min(cores, heads))
         el += time.perf_counter() - t1
         reps += 1
-    used = min(cores, done)
+    used = 1 if isinstance(job, BwdJob) else min(cores, done)   # the backward oracle is serial
     sample = (f"{done} of {w.heads} heads x T={T} x {len(job.passes)} pass(es) x {reps} rep(s) "
               f"of workload {job.name}, fp64, OpenMP over heads on {used} of {cores} host cores, "
               f"{el:.1f} s")
@@ -566,6 +683,13 @@ def _e2e(job, steps):
 
 def _workload_desc(job):
     w = job.w
+    if isinstance(job, BwdJob):
+        mode = "mini-batch b=%d" % w.b if w.minibatch else "per-token"
+        dt = "bf16 in" if w.in_bf16 else "fp32 in"
+        extra = ", SKIP/UPDATE mask" if w.mask_p else ""
+        return (f"TTT-Linear scan backward ({job.name}: the gradients of workload "
+                f"{job.BWD_OF[job.name]}): {mode}, LN-Jacobian gradient, {dt}, fp32 gradients, "
+                f"B={w.B} H={w.H} T={w.T} d={w.d}{extra}")
     if job.decode:
         return (f"TTT-Linear decode step {job.name}: one token per head, W [B,H,d,d] fp32 "
                 f"updated in place, LN-Jacobian gradient, bf16 in, bf16 out, B={w.B} H={w.H} "

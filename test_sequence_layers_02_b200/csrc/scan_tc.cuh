@@ -60,6 +60,7 @@ namespace tc {
 constexpr int D = 64;
 constexpr int CB = 16;              // chunk (b)
 constexpr int NT = 288;             // 4 chain + 4 bulk + 1 issuer warps
+constexpr int kMinbMany = 3;        // CTAs per SM of the build for more heads than SMs
 constexpr int NST = 5;              // TMA stages
 constexpr int kSR = 32;             // scalar ring (chunks)
 constexpr uint32_t kTmemCols = 128;
@@ -91,6 +92,8 @@ constexpr int oAbort = oTmem + 8;
 constexpr int kSmemUsed = oAbort + 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
 static_assert(kSmemBytes <= 75 * 1024, "three CTAs per SM must fit in shared memory");
+template <int MINB>
+constexpr int smem_bytes() { return kSmemBytes; }
 static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
 static_assert(3 * (kTmemCols + kTmemGramCols) <= 512, "three CTAs per SM must fit in TMEM");
 // The 128-row A operand of the Gram MMA starts at a stage's K tile and runs
@@ -216,7 +219,8 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       if (p.mask) r.m = p.mask[(size_t)bi * p.n_mask_chunks + x];
       const int t = x * CB + i;
       if (t < T) {
-        if (r.m) r.e = gel[t];  // a SKIP chunk takes no gradient: its eta is not read
+        r.e = gel[t];  // (read whatever the mask says: a load that waited for the
+                       // mask byte would stall these warps once per 8 chunks)
         if (ggl) r.g = ggl[t];
       }
     }

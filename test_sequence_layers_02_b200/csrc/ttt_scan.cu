@@ -112,13 +112,15 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
       !encode_qkv_map(&maps.v, p.v, p.T, heads, false))
     return TTT_ERR_CUDA;
   // up to one head per SM: the one-CTA-per-SM build (more registers per
-  // thread); beyond that, three CTAs share an SM
-  auto kernel = heads <= ttt::device_sm_count() ? ttt::scan_tc_kernel<OutT, GM, 1>
-                                           : ttt::scan_tc_kernel<OutT, GM, 3>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           ttt::tc::kSmemBytes) != cudaSuccess)
+  // thread); beyond that, several CTAs share an SM
+  const bool one = heads <= ttt::device_sm_count();
+  auto kernel = one ? ttt::scan_tc_kernel<OutT, GM, 1>
+                    : ttt::scan_tc_kernel<OutT, GM, ttt::tc::kMinbMany>;
+  const int smem = one ? ttt::tc::smem_bytes<1>() : ttt::tc::smem_bytes<ttt::tc::kMinbMany>();
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
     return TTT_ERR_CUDA;
-  kernel<<<(unsigned)heads, ttt::tc::NT, ttt::tc::kSmemBytes, stream>>>(p, maps);
+  kernel<<<(unsigned)heads, ttt::tc::NT, smem, stream>>>(p, maps);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
