@@ -240,6 +240,39 @@ int ttt_scan_backward(const void* q, const void* k, const void* v,
                       void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * ttt_scan_backward for callers that cannot allocate device memory. (The
+ * pages have no counterpart; this is an interface of this library.) Some
+ * callers cannot call cudaMalloc: code that runs inside a framework whose
+ * allocator owns all of the device's memory, or a loop that cannot afford the
+ * implicit device synchronisation of cudaMalloc. This entry point takes the
+ * arguments of ttt_scan_backward without the workspace: the per-head
+ * dgamma / dbeta partial sums live in a fixed array of 2^20 floats (4 MiB) of
+ * device memory that the library defines, which every GPU that loads the
+ * library holds until the process exits. It allocates nothing and calls no
+ * allocating routine.
+ *   - Limit: B * H * 2 * d <= 2^20 (8192 heads at d = 64, 32768 at d = 16);
+ *     larger problems return TTT_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its partial sums
+ *     there; nothing in it needs to start at zero (each call writes every
+ *     partial sum it reads). Calls whose kernels overlap on the GPU (on
+ *     different streams, with no ordering between them) race on the array;
+ *     order them on one stream.
+ * Everything else, including the results, is as for ttt_scan_backward.
+ */
+int ttt_scan_backward_noalloc(const void* q, const void* k, const void* v,
+                              const void* eta_logit, const void* gate_logit,
+                              const float* gamma, const float* beta,
+                              int B, int H, int T, int d, float eps, unsigned mode, int b,
+                              const unsigned char* mask, const float* W_chunks,
+                              const float* dO, const float* dW_T,
+                              float* dq, float* dk, float* dv, float* d_eta_logit,
+                              float* d_gate_logit, float* dW0, float* dgamma, float* dbeta,
+                              void* cuda_stream);
+
+/*
  * Synchronise `cuda_stream`, then report and clear the device status word that
  * the kernels set when a bounded wait gives up. Returns TTT_OK,
  * TTT_ERR_DEVICE_TIMEOUT, or TTT_ERR_CUDA (a sticky or asynchronous CUDA error).

@@ -150,3 +150,49 @@ int ttt_scan_backward(const void* q, const void* k, const void* v, const void* e
 }
 
 }  // extern "C"
+
+// ---- The no-allocation variant: the same backward with its scratch in a fixed
+// device array, for callers that cannot call cudaMalloc. ----
+namespace {
+
+// The per-head dgamma / dbeta partial sums of ttt_scan_backward_noalloc: room
+// for 2^20 floats (4 MiB), i.e. B * H * 2 * d <= 2^20 (8192 heads at d = 64,
+// 32768 at d = 16). A file-scope device array: every GPU that loads the
+// library holds it until the process exits.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_bwd_scratch[kNoAllocScratchFloats];
+
+// Device address of g_bwd_scratch on the current device. In host code the
+// array's name stands for a host-side shadow, not for device memory, so the
+// address is looked up (once per device, with that device current) and cached.
+float* noalloc_scratch_current_device() {
+  static float* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cache[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<float*>(ptr);
+  }
+  return cache[dev];
+}
+
+}  // namespace
+
+extern "C" int ttt_scan_backward_noalloc(
+    const void* q, const void* k, const void* v, const void* eta_logit, const void* gate_logit,
+    const float* gamma, const float* beta, int B, int H, int T, int d, float eps, unsigned mode,
+    int b, const unsigned char* mask, const float* W_chunks, const float* dO, const float* dW_T,
+    float* dq, float* dk, float* dv, float* d_eta_logit, float* d_gate_logit, float* dW0,
+    float* dgamma, float* dbeta, void* cuda_stream) {
+  const size_t need = workspace_bytes_for(B, H, d, mode);
+  if (need > sizeof(g_bwd_scratch)) return TTT_ERR_UNSUPPORTED;
+  float* scratch = nullptr;
+  if (need > 0) {
+    scratch = noalloc_scratch_current_device();
+    if (scratch == nullptr) return TTT_ERR_CUDA;
+  }
+  return ttt_scan_backward(q, k, v, eta_logit, gate_logit, gamma, beta, B, H, T, d, eps, mode, b,
+                           mask, W_chunks, dO, dW_T, dq, dk, dv, d_eta_logit, d_gate_logit, dW0,
+                           dgamma, dbeta, scratch, need, cuda_stream);
+}
