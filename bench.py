@@ -903,6 +903,13 @@ PROFILE_CASES = {
     "cluster": (dict(B=4, H=4, T=2048, d=64, seed=2, qk_l2norm=True),
                 dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),
     "decode": (None, None),
+    # the backward pass at workload 2's shape, a quarter of its length (per-token,
+    # LN Jacobian, fp32) and at workload 3's shape, a quarter of its length
+    # (mini-batch, bf16 inputs); the forward's snapshots are taken first
+    "bwd2": (dict(B=4, H=4, T=512, d=64, seed=2, qk_l2norm=True),
+             dict(eps=1e-6, minibatch=False, lnjac=True, b=16)),
+    "bwd3": (dict(B=8, H=12, T=1024, d=64, seed=3, random_affine=True, in_bf16=True),
+             dict(eps=1e-6, minibatch=True, lnjac=True, b=16)),
 }
 
 
@@ -929,6 +936,19 @@ def run_profile_case(name: str):
         in_bf16 = mk.get("in_bf16", False)
 
     t = _dev_inputs(inp, _W, torch.device("cuda"))
+    if name.startswith("bwd"):
+        _, _, Wc = ttt_scan.scan(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"],
+                                 t["gamma"], t["beta"], mask=t["mask"], want_chunks=True,
+                                 force_simt=True, out_dtype=torch.float32, **kw)
+        dO = torch.randn(t["q"].shape, dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            ttt_scan.scan_backward(t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"],
+                                   t["gamma"], t["beta"], Wc, dO, None, mask=t["mask"], **kw)
+        rc = ttt_scan.check_device_status()
+        print(f"profile case {name}: status {ttt_scan.status_string(rc)}")
+        if rc != ttt_scan.TTT_OK:
+            raise SystemExit(1)
+        return
     kw = dict(kw)
     out_dtype = torch.bfloat16 if kw.pop("out_bf16") else torch.float32
     for _ in range(2):

@@ -25,10 +25,15 @@
 // forward's W_chunks snapshots (one per chunk of b tokens); the forward inside a
 // chunk is recomputed from W_s with the same identity.
 //
+// Every LayerNorm gradient step of the reverse chain takes one warp reduction:
+// the sums it needs are closed forms in a few sums over u (formed together)
+// and in per-token sums the forward recompute leaves behind. In mini-batch
+// mode no token's chain step depends on another's, so all warps take tokens.
+//
 // One CTA of 4d threads per (batch row, head). gamma / beta gradients are
-// summed over the head's tokens in the chain warp's registers and written per
-// head to `gb_part`; bwd_reduce_gb_kernel sums them over the batch rows in a
-// fixed order.
+// summed over the head's tokens in the chain warps' registers, then over the
+// warps in a fixed order, and written per head to `gb_part`;
+// bwd_reduce_gb_kernel sums them over the batch rows in a fixed order.
 #pragma once
 
 #include "common.cuh"
@@ -95,8 +100,13 @@ struct BwdLayout {
   static constexpr int oEta = oGDz + GR;       // eta_t (0 on SKIP chunks and past the chunk)
   static constexpr int oSg = oEta + C;         // sigmoid(eta_logit_t)
   static constexpr int oGate = oSg + C;        // scalar gate_t
-  static constexpr int oS = oGate + C;         // LayerNorm s_t
-  static constexpr int floats = oS + C;
+  static constexpr int oS = oGate + C;         // per token of the forward: LayerNorm s_t,
+  static constexpr int oA = oS + C;            //   mean(g), mean(g xhat) (Jacobian forms),
+  static constexpr int oCg = oA + C;           //   sum gamma^2 xhat, sum gamma^2 xhat^2
+  static constexpr int oP1 = oCg + C;          //   (LN Jacobian) and sum xhat
+  static constexpr int oP2 = oP1 + C;
+  static constexpr int oPx = oP2 + C;
+  static constexpr int floats = oPx + C;
   static constexpr int bytes = floats * 4;
 };
 
@@ -116,6 +126,7 @@ template <int D, typename InT, bool MINIB, int GM>
 __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int NT = L::NT, C = L::C, LD = L::LD;
+  constexpr int NW = NT / 32;
   constexpr int EPL = (D + 31) / 32;
   constexpr bool kLN = GM != 2;
   constexpr bool kJac = GM == 1 || GM == 3;
@@ -144,6 +155,11 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
   float* sSg = sm + L::oSg;
   float* sGate = sm + L::oGate;
   float* sS = sm + L::oS;
+  float* sA = sm + L::oA;
+  float* sCg = sm + L::oCg;
+  float* sP1 = sm + L::oP1;
+  float* sP2 = sm + L::oP2;
+  float* sPx = sm + L::oPx;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -155,8 +171,9 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
   const float inv_d = 1.0f / (float)D;
   const float* Wc = p.W_chunks + (size_t)bh * (nc + 1) * D * D;
 
-  // chain warp: this lane's features f = lane + 32 e, and gamma / beta sums
+  // chain warps: this lane's features f = lane + 32 e, and gamma / beta sums
   float gam[EPL], bet[EPL], dgam[EPL], dbet[EPL];
+  float sg2 = 0.f;  // sum of gamma^2 over the head's features
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
     const int f = lane + 32 * e;
@@ -165,7 +182,16 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
     bet[e] = ok ? p.beta[(size_t)h * D + f] : 0.f;
     dgam[e] = 0.f;
     dbet[e] = 0.f;
+    if (f < D) sg2 = fmaf(gam[e], gam[e], sg2);
   }
+  {
+    float t1[1] = {sg2};
+    butterfly<1>(t1);
+    sg2 = t1[0];
+  }
+  // per-token mode: warp 0 walks the tokens in order; mini-batch: every warp
+  const bool chain_warp = MINIB || warp == 0;
+  const int t_first = MINIB ? warp : 0, t_step = MINIB ? NW : 1;
 
   // D = dW_T
   for (int idx = tid; idx < D * D; idx += NT) {
@@ -259,9 +285,10 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
     }
     __syncthreads();
 
-    // ---- forward chain (warp 0): z_t, LayerNorm, G_t ----
-    if (warp == 0) {
-      for (int t = 0; t < C; ++t) {
+    // ---- forward chain: z_t, LayerNorm (one reduction of shifted moments),
+    //      G_t, and the per-token sums the reverse chain needs ----
+    if (chain_warp) {
+      for (int t = t_first; t < C; t += t_step) {
         if (t >= n || !upd) {
           // SKIP chunks take no gradient (eta = 0): G plays no part
 #pragma unroll
@@ -295,43 +322,64 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
             xh[e] = z[e];
           }
         } else {
-          float m1[1] = {0.f};
+          // shift by one element of the token; moments of y = z - shift:
+          // sum y, sum y^2 and (Jacobian forms) sum a y, sum a y^2, sum c y, sum c
+          // with g = a xhat + c (LN Jacobian: a = gamma^2, c = gamma (beta - v);
+          // ablation: a = 0, c = -gamma v)
+          const float c0 = __shfl_sync(0xffffffffu, z[0], 0);
+          constexpr int NM = kJac ? 6 : 2;
+          float m[NM], y[EPL], aa[EPL], cc[EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) m1[0] += z[e];
-          butterfly<1>(m1);
-          const float mu = m1[0] * inv_d;
-          float m2[1] = {0.f};
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            const float y = (lane + 32 * e < D) ? z[e] - mu : 0.f;
-            m2[0] = fmaf(y, y, m2[0]);
-          }
-          butterfly<1>(m2);
-          const float s = sqrtf(m2[0] * inv_d + p.eps);
-          float g[EPL];
+          for (int i = 0; i < NM; ++i) m[i] = 0.f;
 #pragma unroll
           for (int e = 0; e < EPL; ++e) {
             const bool fv = lane + 32 * e < D;
-            xh[e] = fv ? (z[e] - mu) / s : 0.f;
-            const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
-            g[e] = fv ? (GM == 3 ? -gam[e] * v[e] : (GM == 1 ? gam[e] * err : err)) : 0.f;
+            y[e] = fv ? z[e] - c0 : 0.f;
+            aa[e] = (fv && GM == 1) ? gam[e] * gam[e] : 0.f;
+            cc[e] = !fv ? 0.f : (GM == 3 ? -gam[e] * v[e] : gam[e] * (bet[e] - v[e]));
+            m[0] += y[e];
+            m[1] = fmaf(y[e], y[e], m[1]);
+            if (kJac) {
+              const float ay = aa[e] * y[e];
+              m[2] += ay;
+              m[3] = fmaf(ay, y[e], m[3]);
+              m[4] = fmaf(cc[e], y[e], m[4]);
+              m[5] += cc[e];
+            }
           }
+          butterfly<NM>(m);
+          const float mu1 = m[0] * inv_d;
+          const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
+          const float s = sqrtf(var + p.eps);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e)
+            xh[e] = (lane + 32 * e < D) ? (y[e] - mu1) / s : 0.f;
           if (kJac) {
-            float m[2] = {0.f, 0.f};
+            const float sa = (GM == 1) ? sg2 : 0.f;                       // sum of a
+            const float p1 = (m[2] - mu1 * sa) / s;                       // sum a xhat
+            const float p2 = (m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa) / (s * s);  // sum a xhat^2
+            const float a_ = (p1 + m[5]) * inv_d;                         // mean g
+            const float cg = (p2 + (m[4] - mu1 * m[5]) / s) * inv_d;      // mean g xhat
 #pragma unroll
             for (int e = 0; e < EPL; ++e) {
-              m[0] += g[e];
-              m[1] = fmaf(g[e], xh[e], m[1]);
+              const float g = fmaf(aa[e], xh[e], cc[e]);
+              G[e] = (lane + 32 * e < D) ? (g - a_ - xh[e] * cg) / s : 0.f;
             }
-            butterfly<2>(m);
-#pragma unroll
-            for (int e = 0; e < EPL; ++e)
-              G[e] = (g[e] - m[0] * inv_d - xh[e] * (m[1] * inv_d)) / s;
+            if (lane == 0) {
+              sA[t] = a_;
+              sCg[t] = cg;
+              sP1[t] = p1;
+              sP2[t] = p2;
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) G[e] = g[e];
+            for (int e = 0; e < EPL; ++e)
+              G[e] = (lane + 32 * e < D) ? fmaf(gam[e], xh[e], bet[e]) - v[e] : 0.f;
           }
-          if (lane == 0) sS[t] = s;
+          if (lane == 0) {
+            sS[t] = s;
+            sPx[t] = (m[0] - (float)D * mu1) / s;  // sum xhat
+          }
         }
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -373,9 +421,11 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
       }
     }
 
-    // ---- backward chain (warp 0), right to left: u_t, deta_t, dz_t, dv_t ----
-    if (warp == 0) {
-      for (int t = C - 1; t >= 0; --t) {
+    // ---- reverse chain: u_t, deta_t, dz_t, dv_t (per-token mode: warp 0,
+    //      right to left; mini-batch: every warp, any order) ----
+    if (chain_warp) {
+      for (int i = t_first; i < C; i += t_step) {
+        const int t = MINIB ? i : C - 1 - i;
         if (t >= n) continue;
         const size_t gt = tok0 + t0 + t;
         if (!upd) {
@@ -406,95 +456,83 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
           xh[e] = f < D ? sXh[t * LD + f] : 0.f;
           v[e] = f < D ? sV[t * LD + f] : 0.f;
         }
-        float de[1] = {0.f};
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) de[0] = fmaf(-G[e], u[e], de[0]);
-        butterfly<1>(de);
-        const float eta = sEta[t];
-        if (lane == 0) p.deta[gt] = de[0] * sSg[t] * (1.f - sSg[t]) * inv_d;
-        float dG[EPL], dz[EPL], dv[EPL];
+        // one reduction: sum G u, sum u, sum u xhat, sum u w, sum u w xhat with
+        // w = gamma^2 (LN Jacobian) or gamma (simplified gradient)
+        float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
-          dG[e] = (lane + 32 * e < D) ? -eta * u[e] : 0.f;
-          dv[e] = 0.f;
+          const float w = GM == 1 ? gam[e] * gam[e] : gam[e];
+          m[0] = fmaf(G[e], u[e], m[0]);
+          m[1] += u[e];
+          m[2] = fmaf(u[e], xh[e], m[2]);
+          m[3] = fmaf(u[e], w, m[3]);
+          m[4] = fmaf(u[e] * w, xh[e], m[4]);
         }
+        butterfly<5>(m);
+        const float eta = sEta[t];
+        if (lane == 0) p.deta[gt] = -m[0] * sSg[t] * (1.f - sSg[t]) * inv_d;
+        float dz[EPL], dv[EPL];
         if (!kLN) {
 #pragma unroll
           for (int e = 0; e < EPL; ++e) {
-            dz[e] = dG[e];
-            dv[e] = -dG[e];
+            dz[e] = -eta * u[e];
+            dv[e] = eta * u[e];
           }
         } else {
+          // dG = -eta u; the sums of the LayerNorm backward in closed form
           const float s = sS[t];
-          float derr[EPL], dxh[EPL];
-          float ds = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) dxh[e] = 0.f;
+          const float mdG = -eta * m[1] * inv_d, mdGx = -eta * m[2] * inv_d;
+          float ds = 0.f, s_jx = 0.f, s_j = 0.f, s_ex = 0.f, s_e = 0.f;
           if (kJac) {
-            // G = (g - mean g - xhat mean(g xhat)) / s
-            float g[EPL];
-            float m[4] = {0.f, 0.f, 0.f, 0.f};
+            const float a_ = sA[t], cg = sCg[t];
+            ds = eta * m[0] / s;                         // -(sum dG G) / s
+            s_jx = -2.f * (float)D * cg * mdGx / s;      // sum over f of the Jacobian part of dxhat * xhat
+            s_j = -(float)D * (cg * mdG + a_ * mdGx) / s;  // ... and of that part alone
+          }
+          if (GM == 1) {         // derr = dg gamma: sums of derr gamma xhat, derr gamma
+            s_ex = (-eta * m[4] - mdG * sP1[t] - mdGx * sP2[t]) / s;
+            s_e = (-eta * m[3] - mdG * sg2 - mdGx * sP1[t]) / s;
+          } else if (GM == 0) {  // derr = dG
+            s_ex = -eta * m[4];
+            s_e = -eta * m[3];
+          }
+          const float dxx = s_jx + s_ex;
+          const float dvar = (ds - dxx / s) / (2.f * s);
+          const float mdy = ((s_j + s_e) / s + dvar * 2.f * s * sPx[t] * inv_d) * inv_d;
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-              const bool fv = lane + 32 * e < D;
-              const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
-              g[e] = fv ? (GM == 3 ? -gam[e] * v[e] : gam[e] * err) : 0.f;
-              m[0] += g[e];
-              m[1] = fmaf(g[e], xh[e], m[1]);
-              m[2] += dG[e];
-              m[3] = fmaf(dG[e], xh[e], m[3]);
-            }
-            butterfly<4>(m);
-            const float c_ = m[1] * inv_d, mdG = m[2] * inv_d, mdGx = m[3] * inv_d;
-            float sdGG[1] = {0.f};
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) sdGG[0] = fmaf(dG[e], G[e], sdGG[0]);
-            butterfly<1>(sdGG);
-            ds = -sdGG[0] / s;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-              const bool fv = lane + 32 * e < D;
-              const float dg = fv ? (dG[e] - mdG - xh[e] * mdGx) / s : 0.f;
-              dxh[e] = fv ? (-dG[e] * c_ - g[e] * mdGx) / s : 0.f;
+          for (int e = 0; e < EPL; ++e) {
+            const bool fv = lane + 32 * e < D;
+            const float dG = -eta * u[e];
+            float derr, dxh = 0.f;
+            dv[e] = 0.f;
+            if (kJac) {
+              const float g = GM == 3 ? -gam[e] * v[e]
+                                      : gam[e] * (fmaf(gam[e], xh[e], bet[e]) - v[e]);
+              const float dg = (dG - mdG - xh[e] * mdGx) / s;
+              dxh = (-dG * sCg[t] - g * mdGx) / s;
               if (GM == 3) {
-                dgam[e] -= dg * v[e];
-                dv[e] -= dg * gam[e];
-                derr[e] = 0.f;
+                if (fv) {
+                  dgam[e] -= dg * v[e];
+                  dv[e] -= dg * gam[e];
+                }
+                derr = 0.f;
               } else {
-                const float err = fmaf(gam[e], xh[e], bet[e]) - v[e];
-                dgam[e] = fmaf(dg, err, dgam[e]);
-                derr[e] = dg * gam[e];
+                if (fv) dgam[e] = fmaf(dg, fmaf(gam[e], xh[e], bet[e]) - v[e], dgam[e]);
+                derr = dg * gam[e];
               }
+            } else {
+              derr = dG;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) derr[e] = dG[e];
-          }
-          // err = gamma xhat + beta - v
-          float dxx[1] = {0.f};
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            if (lane + 32 * e < D) {
-              dgam[e] = fmaf(derr[e], xh[e], dgam[e]);
-              dbet[e] += derr[e];
-              dv[e] -= derr[e];
-              dxh[e] = fmaf(derr[e], gam[e], dxh[e]);
+            // err = gamma xhat + beta - v
+            if (fv) {
+              dgam[e] = fmaf(derr, xh[e], dgam[e]);
+              dbet[e] += derr;
             }
-            dxx[0] = fmaf(dxh[e], xh[e], dxx[0]);
+            dv[e] -= derr;
+            dxh = fmaf(derr, gam[e], dxh);
+            // xhat = (z - mu) / s, s = sqrt(var + eps), z - mu = xhat s
+            dz[e] = fv ? dxh / s + dvar * 2.f * xh[e] * s * inv_d - mdy : 0.f;
           }
-          butterfly<1>(dxx);
-          // xhat = (z - mu) / s, s = sqrt(var + eps): z - mu = xhat s
-          const float dvar = (ds - dxx[0] / s) / (2.f * s);
-          float dy[EPL];
-          float mdy[1] = {0.f};
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            dy[e] = (lane + 32 * e < D) ? dxh[e] / s + dvar * 2.f * xh[e] * s * inv_d : 0.f;
-            mdy[0] += dy[e];
-          }
-          butterfly<1>(mdy);
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) dz[e] = dy[e] - mdy[0] * inv_d;
         }
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -507,10 +545,11 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
         __syncwarp();
       }
       // rows past the chunk
-      for (int t = n; t < C; ++t)
+      if (warp == 0)
+        for (int t = n; t < C; ++t)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          if (lane + 32 * e < D) sDz[t * LD + lane + 32 * e] = 0.f;
+          for (int e = 0; e < EPL; ++e)
+            if (lane + 32 * e < D) sDz[t * LD + lane + 32 * e] = 0.f;
     }
     __syncthreads();
 
@@ -595,14 +634,25 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
     const int r = idx / D, c = idx - r * D;
     p.dW0[(size_t)bh * D * D + idx] = sD[r * LD + c];
   }
-  if (kLN && warp == 0 && p.gb_part != nullptr) {
+  if (kLN && p.gb_part != nullptr) {
+    // the chain warps' sums, added over the warps in warp order
+    float* red = sT1;  // [NW][2][D] (free after the last chunk)
+    if (chain_warp) {
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const int f = lane + 32 * e;
-      if (f < D) {
-        p.gb_part[((size_t)bh * 2) * D + f] = dgam[e];
-        p.gb_part[((size_t)bh * 2 + 1) * D + f] = dbet[e];
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        if (f < D) {
+          red[(warp * 2) * D + f] = dgam[e];
+          red[(warp * 2 + 1) * D + f] = dbet[e];
+        }
       }
+    }
+    __syncthreads();
+    if (tid < 2 * D) {
+      const int which = tid / D, f = tid - which * D;
+      float acc = 0.f;
+      for (int w = 0; w < (MINIB ? NW : 1); ++w) acc += red[(w * 2 + which) * D + f];
+      p.gb_part[((size_t)bh * 2 + which) * D + f] = acc;
     }
   }
 }
