@@ -123,7 +123,7 @@ __device__ __forceinline__ float ld_in(const void* p, size_t i) {
 // GM: 0 simplified (G = err), 1 LN Jacobian, 2 no LayerNorm (G = z - v),
 // 3 ablation (the Jacobian applied to -gamma v).
 template <int D, typename InT, bool MINIB, int GM>
-__global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int NT = L::NT, C = L::C, LD = L::LD;
   constexpr int NW = NT / 32;
@@ -191,7 +191,6 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
   }
   // per-token mode: warp 0 walks the tokens in order; mini-batch: every warp
   const bool chain_warp = MINIB || warp == 0;
-  const int t_first = MINIB ? warp : 0, t_step = MINIB ? NW : 1;
 
   // D = dW_T
   for (int idx = tid; idx < D * D; idx += NT) {
@@ -287,114 +286,139 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
 
     // ---- forward chain: z_t, LayerNorm (one reduction of shifted moments),
     //      G_t, and the per-token sums the reverse chain needs ----
-    if (chain_warp) {
-      for (int t = t_first; t < C; t += t_step) {
-        if (t >= n || !upd) {
-          // SKIP chunks take no gradient (eta = 0): G plays no part
+    // One token's LayerNorm and gradient from its z (this lane's features):
+    // writes G, xhat and the per-token sums, returns G.
+    auto fwd_token = [&](int t, const float (&z)[EPL], float (&G)[EPL]) {
+      float v[EPL], xh[EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            const int f = lane + 32 * e;
-            if (f < D) {
-              sG[t * LD + f] = 0.f;
-              sXh[t * LD + f] = 0.f;
-            }
-          }
-          continue;
-        }
-        float z[EPL], v[EPL];
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        v[e] = f < D ? sV[t * LD + f] : 0.f;
+      }
+      if (!kLN) {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
-          const int f = lane + 32 * e;
-          float acc = 0.f;
-          if (f < D) {
-            acc = sZ[t * LD + f];
-            if (!MINIB)
-              for (int j = 0; j < t; ++j) acc = fmaf(-sEta[j] * sKK[t * C + j], sG[j * LD + f], acc);
-          }
-          z[e] = acc;
-          v[e] = f < D ? sV[t * LD + f] : 0.f;
+          G[e] = (lane + 32 * e < D) ? z[e] - v[e] : 0.f;
+          xh[e] = z[e];
         }
-        float G[EPL], xh[EPL];
-        if (!kLN) {
+      } else {
+        // shift by one element of the token; moments of y = z - shift:
+        // sum y, sum y^2 and (Jacobian forms) sum a y, sum a y^2, sum c y, sum c
+        // with g = a xhat + c (LN Jacobian: a = gamma^2, c = gamma (beta - v);
+        // ablation: a = 0, c = -gamma v)
+        const float c0 = __shfl_sync(0xffffffffu, z[0], 0);
+        constexpr int NM = kJac ? 6 : 2;
+        float m[NM], y[EPL], aa[EPL], cc[EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            G[e] = z[e] - v[e];
-            xh[e] = z[e];
-          }
-        } else {
-          // shift by one element of the token; moments of y = z - shift:
-          // sum y, sum y^2 and (Jacobian forms) sum a y, sum a y^2, sum c y, sum c
-          // with g = a xhat + c (LN Jacobian: a = gamma^2, c = gamma (beta - v);
-          // ablation: a = 0, c = -gamma v)
-          const float c0 = __shfl_sync(0xffffffffu, z[0], 0);
-          constexpr int NM = kJac ? 6 : 2;
-          float m[NM], y[EPL], aa[EPL], cc[EPL];
+        for (int i = 0; i < NM; ++i) m[i] = 0.f;
 #pragma unroll
-          for (int i = 0; i < NM; ++i) m[i] = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            const bool fv = lane + 32 * e < D;
-            y[e] = fv ? z[e] - c0 : 0.f;
-            aa[e] = (fv && GM == 1) ? gam[e] * gam[e] : 0.f;
-            cc[e] = !fv ? 0.f : (GM == 3 ? -gam[e] * v[e] : gam[e] * (bet[e] - v[e]));
-            m[0] += y[e];
-            m[1] = fmaf(y[e], y[e], m[1]);
-            if (kJac) {
-              const float ay = aa[e] * y[e];
-              m[2] += ay;
-              m[3] = fmaf(ay, y[e], m[3]);
-              m[4] = fmaf(cc[e], y[e], m[4]);
-              m[5] += cc[e];
-            }
-          }
-          butterfly<NM>(m);
-          const float mu1 = m[0] * inv_d;
-          const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
-          const float s = sqrtf(var + p.eps);
-#pragma unroll
-          for (int e = 0; e < EPL; ++e)
-            xh[e] = (lane + 32 * e < D) ? (y[e] - mu1) / s : 0.f;
+        for (int e = 0; e < EPL; ++e) {
+          const bool fv = lane + 32 * e < D;
+          y[e] = fv ? z[e] - c0 : 0.f;
+          aa[e] = (fv && GM == 1) ? gam[e] * gam[e] : 0.f;
+          cc[e] = !fv ? 0.f : (GM == 3 ? -gam[e] * v[e] : gam[e] * (bet[e] - v[e]));
+          m[0] += y[e];
+          m[1] = fmaf(y[e], y[e], m[1]);
           if (kJac) {
-            const float sa = (GM == 1) ? sg2 : 0.f;                       // sum of a
-            const float p1 = (m[2] - mu1 * sa) / s;                       // sum a xhat
-            const float p2 = (m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa) / (s * s);  // sum a xhat^2
-            const float a_ = (p1 + m[5]) * inv_d;                         // mean g
-            const float cg = (p2 + (m[4] - mu1 * m[5]) / s) * inv_d;      // mean g xhat
+            const float ay = aa[e] * y[e];
+            m[2] += ay;
+            m[3] = fmaf(ay, y[e], m[3]);
+            m[4] = fmaf(cc[e], y[e], m[4]);
+            m[5] += cc[e];
+          }
+        }
+        butterfly<NM>(m);
+        const float mu1 = m[0] * inv_d;
+        const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
+        const float s = sqrtf(var + p.eps);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-              const float g = fmaf(aa[e], xh[e], cc[e]);
-              G[e] = (lane + 32 * e < D) ? (g - a_ - xh[e] * cg) / s : 0.f;
-            }
-            if (lane == 0) {
-              sA[t] = a_;
-              sCg[t] = cg;
-              sP1[t] = p1;
-              sP2[t] = p2;
-            }
-          } else {
+        for (int e = 0; e < EPL; ++e) xh[e] = (lane + 32 * e < D) ? (y[e] - mu1) / s : 0.f;
+        if (kJac) {
+          const float sa = (GM == 1) ? sg2 : 0.f;                                 // sum of a
+          const float p1 = (m[2] - mu1 * sa) / s;                                 // sum a xhat
+          const float p2 = (m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa) / (s * s);  // sum a xhat^2
+          const float a_ = (p1 + m[5]) * inv_d;                                   // mean g
+          const float cg = (p2 + (m[4] - mu1 * m[5]) / s) * inv_d;                // mean g xhat
 #pragma unroll
-            for (int e = 0; e < EPL; ++e)
-              G[e] = (lane + 32 * e < D) ? fmaf(gam[e], xh[e], bet[e]) - v[e] : 0.f;
+          for (int e = 0; e < EPL; ++e) {
+            const float g = fmaf(aa[e], xh[e], cc[e]);
+            G[e] = (lane + 32 * e < D) ? (g - a_ - xh[e] * cg) / s : 0.f;
           }
           if (lane == 0) {
-            sS[t] = s;
-            sPx[t] = (m[0] - (float)D * mu1) / s;  // sum xhat
+            sA[t] = a_;
+            sCg[t] = cg;
+            sP1[t] = p1;
+            sP2[t] = p2;
           }
-        }
+        } else {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const int f = lane + 32 * e;
-          if (f < D) {
-            sG[t * LD + f] = G[e];
-            sXh[t * LD + f] = xh[e];
-          }
+          for (int e = 0; e < EPL; ++e)
+            G[e] = (lane + 32 * e < D) ? fmaf(gam[e], xh[e], bet[e]) - v[e] : 0.f;
         }
-        __syncwarp();
+        if (lane == 0) {
+          sS[t] = s;
+          sPx[t] = (m[0] - (float)D * mu1) / s;  // sum xhat
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        if (f < D) {
+          sG[t * LD + f] = G[e];
+          sXh[t * LD + f] = xh[e];
+        }
+      }
+    };
+    auto zero_rows = [&](float* a, int t) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e)
+        if (lane + 32 * e < D) a[t * LD + lane + 32 * e] = 0.f;
+    };
+    if (MINIB) {
+      // every token's z is W_s k_t: every warp takes tokens
+      for (int t = warp; t < C; t += NW) {
+        if (t >= n || !upd) {  // SKIP chunks take no gradient (eta = 0)
+          zero_rows(sG, t);
+          zero_rows(sXh, t);
+          continue;
+        }
+        float z[EPL], G[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) z[e] = (lane + 32 * e < D) ? sZ[t * LD + lane + 32 * e] : 0.f;
+        fwd_token(t, z, G);
+      }
+    } else if (warp == 0) {
+      // z of every token in registers; each G_t goes at once into the later
+      // tokens' z (z_m -= eta_t (k_m . k_t) G_t)
+      float zr[C][EPL];
+#pragma unroll
+      for (int t = 0; t < C; ++t)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          zr[t][e] = (t < n && lane + 32 * e < D) ? sZ[t * LD + lane + 32 * e] : 0.f;
+#pragma unroll
+      for (int t = 0; t < C; ++t) {
+        if (t < n && upd) {
+          float G[EPL];
+          fwd_token(t, zr[t], G);
+          const float et = sEta[t];
+#pragma unroll
+          for (int m2 = t + 1; m2 < C; ++m2) {
+            const float a = -et * sKK[m2 * C + t];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) zr[m2][e] = fmaf(a, G[e], zr[m2][e]);
+          }
+        } else {
+          zero_rows(sG, t);
+          zero_rows(sXh, t);
+        }
       }
     }
     __syncthreads();
 
-    // ---- readout y_t = W_s q_t - sum_{j<=t} eta_j (q_t.k_j) G_j, and the gate gradients ----
+    // ---- readout y_t = W_s q_t - sum_{j<=t} eta_j (q_t.k_j) G_j and the gate
+    //      gradients; the part of u_t that does not wait for the chain,
+    //      D_e k_t + sum_{j>=t} dy_j (q_j.k_t), into sPB ----
     for (int idx = tid; idx < C * D; idx += NT) {
       const int t = idx / D, f = idx - t * D;
       float y = sY[t * LD + f];
@@ -406,6 +430,9 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
         const float gs = sigmoidf_(ld_in<InT>(p.gate_logit, g));
         p.dgate[g] = sDO[t * LD + f] * y * gs * (1.f - gs);
       }
+      float u = sPB[t * LD + f];
+      for (int j = t; j < n; ++j) u = fmaf(sQK[j * C + t], sDy[j * LD + f], u);
+      sPB[t * LD + f] = u;
     }
     __syncthreads();
     if (p.gate_logit && !p.gate_channel) {
@@ -421,135 +448,161 @@ __global__ void __launch_bounds__(4 * D) scan_bwd_kernel(const BwdParams p) {
       }
     }
 
-    // ---- reverse chain: u_t, deta_t, dz_t, dv_t (per-token mode: warp 0,
-    //      right to left; mini-batch: every warp, any order) ----
-    if (chain_warp) {
-      for (int i = t_first; i < C; i += t_step) {
-        const int t = MINIB ? i : C - 1 - i;
-        if (t >= n) continue;
-        const size_t gt = tok0 + t0 + t;
-        if (!upd) {
+    // ---- reverse chain: deta_t, dz_t, dv_t from u_t (per-token mode: warp 0,
+    //      right to left, u in registers; mini-batch: every warp) ----
+    // One token's step: the LayerNorm backward of dG = -eta u in closed form
+    // (one warp reduction); writes deta, dz, dv and adds to the gamma / beta sums.
+    auto bwd_token = [&](int t, const float (&u)[EPL], float (&dz)[EPL]) {
+      const size_t gt = tok0 + t0 + t;
+      float G[EPL], xh[EPL], v[EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            const int f = lane + 32 * e;
-            if (f < D) {
-              sDz[t * LD + f] = 0.f;
-              p.dv[gt * D + f] = 0.f;
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        G[e] = f < D ? sG[t * LD + f] : 0.f;
+        xh[e] = f < D ? sXh[t * LD + f] : 0.f;
+        v[e] = f < D ? sV[t * LD + f] : 0.f;
+      }
+      // sum G u, sum u, sum u xhat, sum u w, sum u w xhat with w = gamma^2 (LN
+      // Jacobian) or gamma (simplified gradient)
+      float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const float w = GM == 1 ? gam[e] * gam[e] : gam[e];
+        m[0] = fmaf(G[e], u[e], m[0]);
+        m[1] += u[e];
+        m[2] = fmaf(u[e], xh[e], m[2]);
+        m[3] = fmaf(u[e], w, m[3]);
+        m[4] = fmaf(u[e] * w, xh[e], m[4]);
+      }
+      butterfly<5>(m);
+      const float eta = sEta[t];
+      if (lane == 0) p.deta[gt] = -m[0] * sSg[t] * (1.f - sSg[t]) * inv_d;
+      float dv[EPL];
+      if (!kLN) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          dz[e] = -eta * u[e];
+          dv[e] = eta * u[e];
+        }
+      } else {
+        // dG = -eta u; the sums of the LayerNorm backward in closed form
+        const float s = sS[t];
+        const float mdG = -eta * m[1] * inv_d, mdGx = -eta * m[2] * inv_d;
+        float ds = 0.f, s_jx = 0.f, s_j = 0.f, s_ex = 0.f, s_e = 0.f;
+        if (kJac) {
+          const float a_ = sA[t], cg = sCg[t];
+          ds = eta * m[0] / s;                           // -(sum dG G) / s
+          s_jx = -2.f * (float)D * cg * mdGx / s;        // sum of the Jacobian part of dxhat * xhat
+          s_j = -(float)D * (cg * mdG + a_ * mdGx) / s;  // ... and of that part alone
+        }
+        if (GM == 1) {         // derr = dg gamma: sums of derr gamma xhat, derr gamma
+          s_ex = (-eta * m[4] - mdG * sP1[t] - mdGx * sP2[t]) / s;
+          s_e = (-eta * m[3] - mdG * sg2 - mdGx * sP1[t]) / s;
+        } else if (GM == 0) {  // derr = dG
+          s_ex = -eta * m[4];
+          s_e = -eta * m[3];
+        }
+        const float dxx = s_jx + s_ex;
+        const float dvar = (ds - dxx / s) / (2.f * s);
+        const float mdy = ((s_j + s_e) / s + dvar * 2.f * s * sPx[t] * inv_d) * inv_d;
+        const float cgt = kJac ? sCg[t] : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const bool fv = lane + 32 * e < D;
+          const float dG = -eta * u[e];
+          float derr, dxh = 0.f;
+          dv[e] = 0.f;
+          if (kJac) {
+            const float g = GM == 3 ? -gam[e] * v[e] : gam[e] * (fmaf(gam[e], xh[e], bet[e]) - v[e]);
+            const float dg = (dG - mdG - xh[e] * mdGx) / s;
+            dxh = (-dG * cgt - g * mdGx) / s;
+            if (GM == 3) {
+              if (fv) {
+                dgam[e] -= dg * v[e];
+                dv[e] -= dg * gam[e];
+              }
+              derr = 0.f;
+            } else {
+              if (fv) dgam[e] = fmaf(dg, fmaf(gam[e], xh[e], bet[e]) - v[e], dgam[e]);
+              derr = dg * gam[e];
             }
+          } else {
+            derr = dG;
           }
-          if (lane == 0) p.deta[gt] = 0.f;
+          // err = gamma xhat + beta - v
+          if (fv) {
+            dgam[e] = fmaf(derr, xh[e], dgam[e]);
+            dbet[e] += derr;
+          }
+          dv[e] -= derr;
+          dxh = fmaf(derr, gam[e], dxh);
+          // xhat = (z - mu) / s, s = sqrt(var + eps), z - mu = xhat s
+          dz[e] = fv ? dxh / s + dvar * 2.f * xh[e] * s * inv_d - mdy : 0.f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        if (f < D) {
+          sDz[t * LD + f] = dz[e];
+          p.dv[gt * D + f] = dv[e];
+        }
+      }
+    };
+    auto skip_token = [&](int t) {  // a SKIP chunk takes no gradient
+      const size_t gt = tok0 + t0 + t;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int f = lane + 32 * e;
+        if (f < D) {
+          sDz[t * LD + f] = 0.f;
+          p.dv[gt * D + f] = 0.f;
+        }
+      }
+      if (lane == 0) p.deta[gt] = 0.f;
+    };
+    if (MINIB) {
+      for (int t = warp; t < C; t += NW) {
+        if (t >= n) {
+          zero_rows(sDz, t);
           continue;
         }
-        float u[EPL], G[EPL], xh[EPL], v[EPL];
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const int f = lane + 32 * e;
-          float acc = 0.f;
-          if (f < D) {
-            acc = sPB[t * LD + f];
-            for (int j = t; j < n; ++j) acc = fmaf(sQK[j * C + t], sDy[j * LD + f], acc);
-            if (!MINIB)
-              for (int j = t + 1; j < n; ++j) acc = fmaf(sKK[j * C + t], sDz[j * LD + f], acc);
-          }
-          u[e] = acc;
-          G[e] = f < D ? sG[t * LD + f] : 0.f;
-          xh[e] = f < D ? sXh[t * LD + f] : 0.f;
-          v[e] = f < D ? sV[t * LD + f] : 0.f;
+        if (!upd) {
+          skip_token(t);
+          continue;
         }
-        // one reduction: sum G u, sum u, sum u xhat, sum u w, sum u w xhat with
-        // w = gamma^2 (LN Jacobian) or gamma (simplified gradient)
-        float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+        float u[EPL], dz[EPL];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const float w = GM == 1 ? gam[e] * gam[e] : gam[e];
-          m[0] = fmaf(G[e], u[e], m[0]);
-          m[1] += u[e];
-          m[2] = fmaf(u[e], xh[e], m[2]);
-          m[3] = fmaf(u[e], w, m[3]);
-          m[4] = fmaf(u[e] * w, xh[e], m[4]);
-        }
-        butterfly<5>(m);
-        const float eta = sEta[t];
-        if (lane == 0) p.deta[gt] = -m[0] * sSg[t] * (1.f - sSg[t]) * inv_d;
-        float dz[EPL], dv[EPL];
-        if (!kLN) {
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            dz[e] = -eta * u[e];
-            dv[e] = eta * u[e];
-          }
-        } else {
-          // dG = -eta u; the sums of the LayerNorm backward in closed form
-          const float s = sS[t];
-          const float mdG = -eta * m[1] * inv_d, mdGx = -eta * m[2] * inv_d;
-          float ds = 0.f, s_jx = 0.f, s_j = 0.f, s_ex = 0.f, s_e = 0.f;
-          if (kJac) {
-            const float a_ = sA[t], cg = sCg[t];
-            ds = eta * m[0] / s;                         // -(sum dG G) / s
-            s_jx = -2.f * (float)D * cg * mdGx / s;      // sum over f of the Jacobian part of dxhat * xhat
-            s_j = -(float)D * (cg * mdG + a_ * mdGx) / s;  // ... and of that part alone
-          }
-          if (GM == 1) {         // derr = dg gamma: sums of derr gamma xhat, derr gamma
-            s_ex = (-eta * m[4] - mdG * sP1[t] - mdGx * sP2[t]) / s;
-            s_e = (-eta * m[3] - mdG * sg2 - mdGx * sP1[t]) / s;
-          } else if (GM == 0) {  // derr = dG
-            s_ex = -eta * m[4];
-            s_e = -eta * m[3];
-          }
-          const float dxx = s_jx + s_ex;
-          const float dvar = (ds - dxx / s) / (2.f * s);
-          const float mdy = ((s_j + s_e) / s + dvar * 2.f * s * sPx[t] * inv_d) * inv_d;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            const bool fv = lane + 32 * e < D;
-            const float dG = -eta * u[e];
-            float derr, dxh = 0.f;
-            dv[e] = 0.f;
-            if (kJac) {
-              const float g = GM == 3 ? -gam[e] * v[e]
-                                      : gam[e] * (fmaf(gam[e], xh[e], bet[e]) - v[e]);
-              const float dg = (dG - mdG - xh[e] * mdGx) / s;
-              dxh = (-dG * sCg[t] - g * mdGx) / s;
-              if (GM == 3) {
-                if (fv) {
-                  dgam[e] -= dg * v[e];
-                  dv[e] -= dg * gam[e];
-                }
-                derr = 0.f;
-              } else {
-                if (fv) dgam[e] = fmaf(dg, fmaf(gam[e], xh[e], bet[e]) - v[e], dgam[e]);
-                derr = dg * gam[e];
-              }
-            } else {
-              derr = dG;
-            }
-            // err = gamma xhat + beta - v
-            if (fv) {
-              dgam[e] = fmaf(derr, xh[e], dgam[e]);
-              dbet[e] += derr;
-            }
-            dv[e] -= derr;
-            dxh = fmaf(derr, gam[e], dxh);
-            // xhat = (z - mu) / s, s = sqrt(var + eps), z - mu = xhat s
-            dz[e] = fv ? dxh / s + dvar * 2.f * xh[e] * s * inv_d - mdy : 0.f;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const int f = lane + 32 * e;
-          if (f < D) {
-            sDz[t * LD + f] = dz[e];
-            p.dv[gt * D + f] = dv[e];
-          }
-        }
-        __syncwarp();
+        for (int e = 0; e < EPL; ++e) u[e] = (lane + 32 * e < D) ? sPB[t * LD + lane + 32 * e] : 0.f;
+        bwd_token(t, u, dz);
       }
-      // rows past the chunk
-      if (warp == 0)
-        for (int t = n; t < C; ++t)
+    } else if (warp == 0) {
+      // u of every token in registers; each dz_t goes at once into the earlier
+      // tokens' u (u_m += (k_t . k_m) dz_t)
+      float ur[C][EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e)
-            if (lane + 32 * e < D) sDz[t * LD + lane + 32 * e] = 0.f;
+      for (int t = 0; t < C; ++t)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          ur[t][e] = (t < n && lane + 32 * e < D) ? sPB[t * LD + lane + 32 * e] : 0.f;
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        const int t = C - 1 - i;
+        if (t >= n) {
+          zero_rows(sDz, t);
+        } else if (!upd) {
+          skip_token(t);
+        } else {
+          float dz[EPL];
+          bwd_token(t, ur[t], dz);
+#pragma unroll
+          for (int m2 = 0; m2 < t; ++m2) {
+            const float a = sKK[t * C + m2];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) ur[m2][e] = fmaf(a, dz[e], ur[m2][e]);
+          }
+        }
+      }
     }
     __syncthreads();
 
