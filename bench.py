@@ -62,6 +62,7 @@ _KERNEL_SOURCES = {
     "scan_simt": ["simt.cu", "scan_simt.cuh", "launch.h", "common.cuh"],
     # one translation unit holds the tensor-core and decode kernels
     "scan_tc": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h", "common.cuh"],
+    "scan_tc_many": ["tc_many.cu", "scan_tc_many.cuh", "sm100.cuh", "launch.h", "common.cuh"],
     "decode_step": ["scan_tc.cuh", "sm100.cuh", "decode.cuh", "scan_simt.cuh", "launch.h",
                     "common.cuh"],
     "scan_bwd": ["backward.cu", "scan_bwd.cuh", "scan_simt.cuh", "abi_util.h", "common.cuh"],
@@ -69,6 +70,17 @@ _KERNEL_SOURCES = {
 # Captures: a kernel may have several (e.g. the tensor-core kernel with and
 # without a SKIP/UPDATE mask); each names the kernel whose sources it covers.
 _CAPTURE_KERNEL = {"scan_tc_masked": "scan_tc", "scan_simt_4pt": "scan_simt"}
+
+
+def _tc_takes_many(heads: int) -> bool:
+    """Whether the tensor-core launcher picks its three-CTAs-per-SM kernel for
+    this many heads: where that saves a wave, (waves at three per SM) * 1.5 <
+    (waves at two per SM), the rule of the launcher in ttt_scan.cu."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    waves2 = -(-heads // (2 * sms))
+    waves3 = -(-heads // (3 * sms))
+    return 3 * waves3 < 2 * waves2
 
 
 def _kernel_hash(kernel_key: str) -> str:
@@ -232,6 +244,8 @@ class Job:
 
     def capture_key(self) -> str:
         k = self.kernel_key()
+        if k == "scan_tc" and _tc_takes_many(self.w.B * self.w.H):
+            return "scan_tc_many"
         if k == "scan_tc" and self.mask_np is not None:
             return "scan_tc_masked"
         if k == "scan_simt" and self.name == "4pt":
@@ -895,6 +909,10 @@ PROFILE_CASES = {
     "tc_masked": (dict(B=2, H=32, T=8192, d=64, seed=5, random_affine=True, in_bf16=True,
                        mask_p=0.5, b=16),
                   dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
+    # workload 4's mini-batch launch at its full size (384 heads: the kernel
+    # built for three CTAs per SM); inputs 302 MB > L2
+    "tc_many": (dict(B=16, H=24, T=2048, d=64, seed=4, random_affine=True, in_bf16=True),
+                dict(eps=1e-6, minibatch=True, lnjac=True, b=16, out_bf16=True)),
     # workload 4's per-token pass at its full size (384 heads, one CTA per head)
     "simt_4pt": (dict(B=16, H=24, T=2048, d=64, seed=4, random_affine=True, in_bf16=True),
                  dict(eps=1e-6, minibatch=False, lnjac=True, b=16, out_bf16=False)),

@@ -1,9 +1,10 @@
 // Host-side launchers of the CUDA-core kernels, each compiled in its own
-// translation unit (four objects of simt.cu, cluster.cu) so the library
+// translation unit (four objects of simt.cu, cluster.cu, tc_many.cu) so the library
 // builds in parallel. Arguments are already checked by the C-ABI entry points;
 // every function returns a ttt_status code.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -29,5 +30,13 @@ int cluster_capacity(unsigned mode, int gm);
 // Read and clear that kernel's device status word: 0 clean, > 0 a bounded wait
 // gave up, < 0 the copy failed.
 int cluster_status_take();
+
+// Mini-batch d = 64 on the tensor cores, the build for three CTAs per SM
+// (scan_tc_many.cuh); q, k, v are the tensor maps of the three inputs. gm as
+// for launch_cluster.
+int launch_tc_many(const ScanParams& p, const CUtensorMap* q, const CUtensorMap* k,
+                   const CUtensorMap* v, bool out_bf16, int gm, cudaStream_t stream);
+// Read and clear that kernel's device status word (as cluster_status_take).
+int tc_many_status_take();
 
 }  // namespace ttt

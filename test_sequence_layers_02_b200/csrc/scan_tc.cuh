@@ -7,38 +7,48 @@
 //     TTT Layers", Abstract),  o_i = W_s q_i - sum_{j<=i} eta_j (k_j.q_i) G_j,
 //     W_e = W_s - sum_j eta_j G_j k_j^T.
 //
-// Look-ahead. With Aneg_c[f][j] = -eta_j G_j[f] and W_{s,c+1} = W_{s,c} + Aneg_c K_c,
-//     Z_{c+1}^T = W_{s,c+1} K_{c+1}^T = P_{c+1}^T + Aneg_c Xg_{c+1}^T,
-//     P_{c+1}^T = W_{s,c} K_{c+1}^T,   Xg_{c+1}[m][j] = k_{c+1,m} . k_{c,j},
-// so P_{c+1} comes from the tensor core a chunk early and the correction is
-// one more small MMA accumulated into the same TMEM columns. Between two
-// LayerNorms only: the chain's Aneg -> three MMAs -> TMEM read of the next Z.
+// Two-chunk look-ahead. With Aneg_c[f][j] = -eta_j G_j[f] (bf16, written by the
+// chain) and W_{s,c+1} = W_{s,c} + Aneg_c K_c,
+//     Z_x^T  = W_{s,x-2} K_x^T + Aneg_{x-2} (K_x K_{x-2}^T)^T + Aneg_{x-1} (K_x K_{x-1}^T)^T
+//     O_x^T  = W_{s,x-1} Q_x^T + Aneg_{x-1} (Q_x K_{x-1}^T)^T + Aneg_x tril(Q_x K_x^T)^T
+// The W_s products (MMA1) run two chunks early on an older W, and only the
+// small corrections (MMAc, K = 16) follow the chain. Per chunk c the chain's
+// Aneg_c feeds three MMAs:
+//     MMAc_a  B(c+1) (+)= Aneg_c [Xg_{c+1}; M_c]^T    (Xg_{c+1} = K_{c+1} K_c^T, M_c = tril(Q_c K_c^T))
+//     MMAc_b  B(c+2)  = Aneg_c [Y_{c+2}; N_{c+1}]^T   (Y_{c+2} = K_{c+2} K_c^T, N_{c+1} = Q_{c+1} K_c^T)
+//     MMA3    W += Aneg_c K_c                          (fp32 state in TMEM)
+// and MMA1 A(c+2) = W_{s,c} [K_{c+2}; Q_{c+1}]^T. The chain reads Z_x = A(x) +
+// B(x) (P halves) and the bulk reads O_x = A(x+1) + B(x+1) (Q halves).
+// The Grams [Xg; M; Y; N] (64 rows x 16, all against K_c) are formed one or two
+// chunks ahead by a warp of their own with mma.sync, so no Gram MMA or TMEM
+// round trip sits on any loop. The loops per chunk:
+//     chain:  Z_c -> LayerNorm -> Aneg_c -> MMAc_a -> Z_{c+1}
+//     state:  MMA3_c -> W_{s,c+1} fp32 -> bf16 (bulk) -> MMA3_{c+1}
+// (W_s in bf16 is double-buffered, so MMA1 reading one copy overlaps the refresh
+// of the other).
 //
-// Warps (288 threads):
-//   chain 0-3   read Z_k^T (TMEM, feature-major), transpose through shared
+// Warps (320 threads):
+//   chain 0-3   read Z_k (TMEM, feature-major), transpose through shared
 //               memory, token-major LayerNorm + gradient (8 lanes per token,
 //               one shuffle round of shifted moments), write Aneg_k (bf16).
-//   bulk 4-7    W (fp32 TMEM) -> bf16 operand W_s; Gram products two chunks
-//               ahead -> bf16 operand [Xg_{c+3}; M_{c+2}]; outputs o_c = gate * O_c^T;
+//   bulk 4-7    W (fp32 TMEM) -> bf16 W_s; outputs o_c = gate * O_c^T;
 //               per-chunk scalars; one thread issues every TMA load of chunk
-//               x = {K_x, Q_{x-1}, V_x}, NST chunks ahead.
-//   issuer 8    (one thread) every tcgen05.mma, per chunk c in this order:
-//               MMAc [P_{c+1} | O_c]^T += Aneg_c [Xg_{c+1}; M_c]^T (one N = 32 MMA,
-//               committed alone: the chain's next Z waits for nothing else);
-//               MMA3 W += Aneg_c K_c (K as an MN-major operand); the Gram
-//               [K_{c+3}; Q_{c+2}] K_{c+2}^T; once W_s is refreshed, MMA1
-//               [P_{c+2} | Q0_{c+1}]^T = W_s [K_{c+2}; Q_{c+1}]^T.
-// One chunk period is then the longer of two loops from MMAc: the chain's
-// (Z -> LayerNorm -> Aneg) and the W refresh's (MMA3 -> bf16 W_s -> MMA1,
-// which must precede the next MMAc); the Grams and the outputs stay off both.
+//               x = {K_x, Q_{x-1}, V_x} (only Q_{x-1} for a SKIP chunk x),
+//               NST chunks ahead; SiLU variant: the in-place SiLU of a stage.
+//   issuer 8    (one thread) every tcgen05.mma and commit.
+//   gram 9      the Gram operand of chunk c (mma.sync, 64 x 16 x 64), as soon
+//               as its buffer is free (two chunks ahead of its use).
 // M = 128 everywhere: A operands stack two copies of their 64 rows, so TMEM
 // lanes 0-63 and 64-127 hold identical d-row results and every warp quarter
 // reads its own lanes.
 //
-// Handoffs are mbarriers in rings of two (a producer can never run two phases
-// ahead of its consumer). Every wait is bounded: on expiry the CTA records the
-// timeout status, all warps leave their loops, the issuer drains its MMAs and
-// the TMA thread its copies (each with a bound of its own) and TMEM is freed.
+// SKIP chunks (PonderTTT, "Core Idea"): no K/V load, no LayerNorm, no MMAc, no
+// MMA3, no W refresh (the bf16 copy of W_s stays valid); only the outputs
+// W_s q, which MMA1 computes anyway.
+//
+// Every wait is bounded: on expiry the CTA records the timeout status, all
+// warps leave their loops, the issuer drains its MMAs and the TMA thread its
+// copies (each with a bound of its own) and TMEM is freed.
 #pragma once
 
 #include "common.cuh"
@@ -59,46 +69,53 @@ namespace tc {
 
 constexpr int D = 64;
 constexpr int CB = 16;              // chunk (b)
-constexpr int NT = 288;             // 4 chain + 4 bulk + 1 issuer warps
-constexpr int kMinbMany = 3;        // CTAs per SM of the build for more heads than SMs
-constexpr int NST = 5;              // TMA stages
+constexpr int NT = 320;             // 4 chain + 4 bulk + 1 issuer + 1 Gram warps
+constexpr int kMinbMany = 2;        // CTAs per SM of the build for more heads than SMs
 constexpr int kSR = 32;             // scalar ring (chunks)
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kTmemGramCols = 32;
+constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColW = 0;       // W accumulator (64 columns)
-// slot s = 0, 1: [P^T | Q0^T / O^T] at 64 + 32 s (16 + 16 columns); the Gram
-// of chunk x in columns 16 (x & 1) of the second allocation
-__device__ __forceinline__ uint32_t col_p(int s) { return 64u + 32u * (uint32_t)s; }
-__device__ __forceinline__ uint32_t col_o(int s) { return 80u + 32u * (uint32_t)s; }
+// A(x): MMA1 results [P | Q0] (16 + 16 columns), three slots; B(x): the
+// corrections, two slots
+__device__ __forceinline__ uint32_t col_a(int x) { return 64u + 32u * (uint32_t)(x % 3); }
+__device__ __forceinline__ uint32_t col_b(int x) { return 160u + 32u * (uint32_t)(x & 1); }
 constexpr int kTile = CB * D * 2;   // 2048 bytes
 constexpr int kZS = 72;             // row stride (floats) of the token-major Z tile
 
+// TMA stages: the Gram operand of chunk c needs the keys of chunk c+2 about
+// two chunk periods before MMA3 of chunk c, and a load issued once stage c
+// frees takes a few microseconds here, so the stages run deep. The per-chunk
+// scalars are stored up to 11 chunks ahead of every TMA issue (16 ahead, in
+// blocks of 8), which bounds NST at 11.
+__host__ __device__ constexpr int nst_for(int minb) { return minb == 1 ? 10 : 6; }
+
 // shared memory (bytes from a 1024-aligned base)
-constexpr int oKQ = 0;                             // [NST][K_x | Q_{x-1}] 128B-swizzled
-constexpr int oV = oKQ + NST * 2 * kTile;          // [NST] V_x, row-major
-constexpr int oWb = oV + NST * kTile;              // W_s bf16, 128 rows x 128 B, 128B-swizzled
-constexpr int oAneg = oWb + 128 * 128;             // [2] 128 rows x 16 bf16 (core matrices)
-constexpr int oXM = oAneg + 2 * 128 * 32;          // [2] [Xg_{x+1}; M_x] 32 x 16 bf16 (core matrices)
-constexpr int oZ = oXM + 2 * 1024;                 // [2][16][kZS] f32
-constexpr int oEta = oZ + 2 * CB * kZS * 4;        // [kSR][16] f32 (mask folded in)
-constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
-constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
-constexpr int oGam = oFlag + kSR * 4;              // gamma, beta [2][64] f32, sum gamma^2, sum gamma*beta
-constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
-// tma[NST], g[2], z[2], xm[2], w, wb, gram, pro, rdy[NST]
-constexpr int kBars = NST + 2 + 2 + 2 + 4 + NST;
-constexpr int oTmem = oBar + kBars * 8;            // two TMEM base addresses
-constexpr int oAbort = oTmem + 8;
-constexpr int kSmemUsed = oAbort + 4;
-constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
-static_assert(kSmemBytes <= 75 * 1024, "three CTAs per SM must fit in shared memory");
+template <int NST>
+struct TcLayout {
+  static_assert(NST <= 11, "the scalar ring must run ahead of every TMA issue");
+  static constexpr int oKQ = 0;                             // [NST][K_x | Q_{x-1}] 128B-swizzled
+  static constexpr int oV = oKQ + NST * 2 * kTile;          // [NST] V_x, row-major
+  static constexpr int oWb = oV + NST * kTile;              // [2] W_s bf16, 128 rows x 128 B, 128B-swizzled
+  static constexpr int oAneg = oWb + 2 * 128 * 128;         // [2] 128 rows x 16 bf16 (core matrices)
+  static constexpr int oXM = oAneg + 2 * 128 * 32;          // [3] {[Xg; M], [Y; N]}: 2 x 32 x 16 bf16
+  static constexpr int oZ = oXM + 3 * 2048;                 // [2][16][kZS] f32
+  static constexpr int oEta = oZ + 2 * CB * kZS * 4;        // [kSR][16] f32 (mask folded in)
+  static constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
+  static constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
+  static constexpr int oGam = oFlag + kSR * 4;              // gamma, beta [2][64] f32, sum gamma^2, sum gamma*beta
+  static constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
+  // tma[NST], rdy[NST], g[2], z[2], xm[3], w, wb, pro
+  static constexpr int kBars = 2 * NST + 2 + 2 + 3 + 3;
+  static constexpr int oTmem = oBar + kBars * 8;            // TMEM base address
+  static constexpr int oAbort = oTmem + 8;
+  static constexpr int kSmemUsed = oAbort + 4;
+  static constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
+  static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
+};
 template <int MINB>
-constexpr int smem_bytes() { return kSmemBytes; }
-static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
-static_assert(3 * (kTmemCols + kTmemGramCols) <= 512, "three CTAs per SM must fit in TMEM");
-// The 128-row A operand of the Gram MMA starts at a stage's K tile and runs
-// 16 KB forward: it must stay inside this CTA's shared memory.
-static_assert(oKQ + (NST - 1) * 2 * kTile + 128 * 128 <= kSmemUsed, "Gram operand in bounds");
+constexpr int smem_bytes() { return TcLayout<nst_for(MINB)>::kSmemBytes; }
+static_assert(smem_bytes<1>() <= 227 * 1024, "one CTA per SM must fit in shared memory");
+static_assert(2 * smem_bytes<kMinbMany>() <= 227 * 1024, "two CTAs per SM must fit in shared memory");
+static_assert(2 * kTmemCols <= 512, "two CTAs per SM must fit in TMEM");
 
 __device__ __forceinline__ int core_off(int row, int k) {
   return (row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
@@ -124,29 +141,54 @@ __device__ __forceinline__ bool bar_any(int bar_id, int count, bool v) {
       : "memory");
   return r != 0;
 }
-__device__ __forceinline__ void bar_sync(int bar_id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(count) : "memory");
-}
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(bar))
                : "memory");
+}
+// One arrival for the whole warp: the lanes converge, which orders their
+// earlier shared-memory writes before lane 0's arrival (a release). A barrier
+// fed this way counts warps, not threads; one arrival per thread would put 32
+// atomic updates of the same word in line.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+// Four 8x8 b16 matrices from shared memory (one row address per lane).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 constexpr int kBarChain = 2;  // named barriers (0 is __syncthreads)
 constexpr int kBarBulk = 3;
 
 }  // namespace tc
 
-// MINB = 3: three CTAs share an SM (heads above the SM count; 72 registers);
+// MINB = 2: two CTAs share an SM (heads above the SM count);
 // MINB = 1: one CTA per SM, for up to one head per SM (more registers).
 template <typename OutT, int GM, int MINB>
 __global__ void __launch_bounds__(tc::NT, MINB)
     scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps) {
   using namespace tc;
   using namespace sm100;
+  constexpr int NST = nst_for(MINB);
+  using Lt = TcLayout<NST>;
+  constexpr int oKQ = Lt::oKQ, oV = Lt::oV, oWb = Lt::oWb, oAneg = Lt::oAneg, oXM = Lt::oXM,
+                oZ = Lt::oZ, oEta = Lt::oEta, oGate = Lt::oGate, oFlag = Lt::oFlag,
+                oGam = Lt::oGam, oBar = Lt::oBar, oTmem = Lt::oTmem, oAbort = Lt::oAbort;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sWb = smem + oWb;
   float* sZ = reinterpret_cast<float*>(smem + oZ);
   float* sEta = reinterpret_cast<float*>(smem + oEta);
   float* sGate = reinterpret_cast<float*>(smem + oGate);
@@ -155,22 +197,23 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   float* sBet = sGam + D;
   float* sGamSums = sGam + 2 * D;  // [0] sum gamma^2, [1] sum gamma*beta
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + oBar);  // [NST] chunk x -> x % NST
-  uint64_t* bar_g = bar_tma + NST;   // [2] Aneg_k written (chain, 128 arrivals)
+  // [NST] stage x ready for its readers: with the SiLU variant K_x and Q_{x-1}
+  // transformed in place (bulk, one arrival per warp); otherwise the TMA
+  // barrier is used
+  uint64_t* bar_rdy = bar_tma + NST;
+  uint64_t* bar_g = bar_rdy + NST;   // [2] Aneg_k written (chain, one arrival per warp)
   uint64_t* bar_z = bar_g + 2;       // [2] Z_k complete in TMEM (commit)
-  uint64_t* bar_xm = bar_z + 2;      // [2] [Xg_{x+1}; M_x] written (bulk warp 4, 32 arrivals)
-  uint64_t* bar_w = bar_xm + 2;      // a chunk's MMAc and MMA3 complete (commit)
-  uint64_t* bar_wb = bar_w + 1;      // W_s bf16 refreshed (bulk, 128 arrivals)
-  uint64_t* bar_gram = bar_wb + 1;   // Gram MMA complete (commit)
-  uint64_t* bar_pro = bar_gram + 1;  // prologue MMAs complete (commit)
-  // [NST] stage x ready for the MMAs: with the SiLU variant, K_x and Q_{x-1}
-  // transformed in place (bulk, 128 arrivals); otherwise the TMA barrier is used
-  uint64_t* bar_rdy = bar_pro + 1;
+  uint64_t* bar_xm = bar_z + 2;      // [3] Gram operand of chunk x written (Gram warp, 1 arrival)
+  uint64_t* bar_w = bar_xm + 3;      // a chunk's MMAs complete (commit)
+  uint64_t* bar_wb = bar_w + 1;      // W read from TMEM and W_s bf16 refreshed (bulk, 4 warps)
+  uint64_t* bar_pro = bar_wb + 1;    // prologue MMAs complete (commit)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + oTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + oAbort);
   auto tKQ = [&](int x) { return smem + oKQ + (x % NST) * 2 * kTile; };  // K_x, then Q_{x-1}
   auto tV = [&](int x) { return smem + oV + (x % NST) * kTile; };
+  auto sWb = [&](int i) { return smem + oWb + i * 128 * 128; };
   auto aneg = [&](int c) { return smem + oAneg + (c & 1) * 4096; };
-  auto xm = [&](int x) { return smem + oXM + (x & 1) * 1024; };  // [Xg_{x+1}; M_x]
+  auto xm = [&](int x) { return smem + oXM + (x % 3) * 2048; };  // [Xg_{x+1}; M_x], then [Y_{x+2}; N_{x+1}]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -178,6 +221,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   const bool is_chain = warp < 4;
   const bool is_bulk = warp >= 4 && warp < 8;
   const bool issuer = (tid == 256);
+  const bool is_gram = warp == 9;
   const bool tma_thread = (tid == 224);        // bulk warp 7, lane 0
   const int wq = warp & 3;                     // TMEM lane quarter of this warp
   const uint32_t tlane = (uint32_t)(wq * 32) << 16;
@@ -197,7 +241,11 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const long long lim = p.wait_limit;
   const long long drain_lim = 1LL << 24;
-  auto chunk_len = [&](int c) { return min(CB, T - c * CB); };
+  // tokens of chunk x (0 outside the sequence)
+  auto chunk_len = [&](int x) { return (x >= 0 && x < nc) ? min(CB, T - x * CB) : 0; };
+  auto upd_of = [&](int x) { return x >= 0 && x < nc && sFlag[x & (kSR - 1)] != 0; };
+  // B(x) holds corrections iff chunk x-2 or x-1 updated
+  auto b_valid = [&](int x) { return upd_of(x - 2) || upd_of(x - 1); };
   auto fail = [&]() {
     *sAbort = 1;
     atomicExch(&g_ttt_status, (int)kStatusTimeout);
@@ -237,16 +285,15 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     }
   };
 
-  // ---- issuer helpers ----
+  // ---- TMA ----
   int tma_issued = 0;  // TMA loads [0, tma_issued) issued (chunk x = {K_x, Q_{x-1}, V_x})
   int w_issued = 0;    // commits to bar_w
-  // A SKIP chunk's keys and values are never used (its z, gradient and update
-  // are not formed), so only its queries are loaded; the K_x / V_x slots keep
-  // stale data that only reaches TMEM columns nobody reads (P_x; the Gram rows
-  // of Xg_x and M_x are zeroed by gram_extract).
+  // A SKIP chunk's keys and values are never read by anything whose result is
+  // used (its z, gradient and update are not formed; the Gram rows against its
+  // keys are zeroed), so only its queries are loaded.
   auto issue_tma = [&](int x) {
     uint64_t* bar = &bar_tma[x % NST];
-    const bool kv = x < nc && sFlag[x & (kSR - 1)] != 0;
+    const bool kv = upd_of(x);
     const uint32_t bytes = (kv ? 2 * kTile : 0) + (x >= 1 ? kTile : 0);
     mbar_arrive_expect_tx(bar, bytes);
     if (kv) {
@@ -257,7 +304,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     tma_issued = x + 1;
   };
   auto tma_parity = [&](int x) { return (uint32_t)((x / NST) & 1); };
-  // stage x ready for the MMAs (see bar_rdy)
+  // stage x ready for the MMAs and the Grams (see bar_rdy)
   auto wait_stage = [&](int x) {
     return mbar_wait_bounded(p.kq_silu ? &bar_rdy[x % NST] : &bar_tma[x % NST], tma_parity(x),
                              lim);
@@ -279,60 +326,79 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     }
     fence_proxy_async_smem();
   };
-  const uint32_t idescN16 = idesc_bf16_f32(128, 16, false, false);
+
+  // ---- issuer helpers ----
   const uint32_t idescN32 = idesc_bf16_f32(128, 32, false, false);
   const uint32_t idescW = idesc_bf16_f32(128, 64, false, true);
-  const uint32_t aWb = smem_u32(sWb);
-  // D (+)= W_s . R^T, R = `n` rows (16 or 32) of a 128B-swizzled K-major tile
-  auto mma_ws = [&](uint32_t d, const unsigned char* rows, int n) {
-    const uint32_t ar = smem_u32(rows);
+  // D = W_s (bf16 copy `wb`) . [32 rows of stage x]^T (N = 32)
+  auto mma_ws = [&](uint32_t d, int wb, int x) {
+    const uint32_t aw = smem_u32(sWb(wb)), ar = smem_u32(tKQ(x));
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ss(d, smem_desc(aWb + kk * 32, 16, 1024, kLayoutSw128),
-                  smem_desc(ar + kk * 32, 16, 1024, kLayoutSw128), n == 32 ? idescN32 : idescN16,
-                  kk > 0 ? 1u : 0u);
+      mma_bf16_ss(d, smem_desc(aw + kk * 32, 16, 1024, kLayoutSw128),
+                  smem_desc(ar + kk * 32, 16, 1024, kLayoutSw128), idescN32, kk > 0 ? 1u : 0u);
   };
-  // Gram for chunk x into TMEM columns 16 (x & 1) of the second allocation:
-  // A = [K_{x+1}; Q_x] (stage x+1; the 128-row operand reads on into the
-  // following shared memory, whose rows land in TMEM lanes that are never
-  // read), B = K_x:  lanes 0-15 k_{x+1,m}.k_{x,j}, lanes 16-31 q_{x,i}.k_{x,j}
-  auto mma_gram = [&](uint32_t tmem2, int x) {
-    const uint32_t a = smem_u32(tKQ(x + 1)), b = smem_u32(tKQ(x));
+
+  // ---- Gram warp: the operand of chunk c (c < nc, c updates), rows
+  // [Xg_{c+1}; M_c] and [Y_{c+2}; N_{c+1}] against the keys of chunk c: row
+  // block w = 0..3 holds stage c+1 rows 0-15 / 16-31, stage c+2 rows 0-15 /
+  // 16-31 (16 rows x 16 keys each, by mma.sync); zero wherever a factor is
+  // outside a chunk or belongs to a SKIP chunk (whose stage holds stale keys) ----
+  auto gram_operand = [&](int c) {
+    const uint32_t right = smem_u32(tKQ(c));  // K_c, rows 0-15
+    const int ra = lane & 15, ha = lane >> 4;                            // A: row, 8-column half
+    const int rb = (lane & 7) + 8 * (lane >> 4), hb = (lane >> 3) & 1;  // B: key row, half
+    // all four row blocks and both key halves at once: eight independent
+    // accumulator chains of four k-steps each, so the latency of one mma.sync
+    // overlaps the others
+    float acc[4][2][4];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ss(tmem2 + 16u * (uint32_t)(x & 1), smem_desc(a + kk * 32, 16, 1024, kLayoutSw128),
-                  smem_desc(b + kk * 32, 16, 1024, kLayoutSw128), idescN16, kk > 0 ? 1u : 0u);
-  };
-  // bulk warp with TMEM lane quarter 0: Gram rows -> the 32-row operand
-  // [Xg_{x+1}; M_x] (bf16): rows 0-15 Xg_{x+1}[m][j] (zero past the chunk
-  // lengths), rows 16-31 M_x[i][j] (causal), row = lane
-  auto gram_extract = [&](uint32_t tmem2, int x) {
-    float r[16];
-    tmem_ld16(tmem2 + 16u * (uint32_t)(x & 1), r);
-    tmem_wait_ld();
-    // Xg_{x+1} and M_x are used only when chunk x updates (Xg also needs
-    // chunk x+1 to update); the rows of a SKIP chunk are zero, which also
-    // discards the stale keys its stage holds
-    const int n0 = sFlag[x & (kSR - 1)] ? chunk_len(x) : 0;
-    float v[16];
-    if (lane < CB) {
-      const int n1 = (x + 1 < nc && sFlag[(x + 1) & (kSR - 1)]) ? chunk_len(x + 1) : 0;
+    for (int w = 0; w < 4; ++w)
 #pragma unroll
-      for (int j = 0; j < CB; ++j) v[j] = (lane < n1 && j < n0) ? r[j] : 0.f;
-    } else {
-      const int i = lane - CB;
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int j = 0; j < CB; ++j) v[j] = (j <= i && i < n0) ? r[j] : 0.f;
+        for (int i = 0; i < 4; ++i) acc[w][nt][i] = 0.f;
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      uint32_t bq[4], a[4][4];
+      ldsm_x4(right + (uint32_t)rb * 128u + (uint32_t)(((2 * kb + hb) ^ (rb & 7)) << 4), bq);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t left = smem_u32(tKQ(c + 1 + (w >> 1))) + (uint32_t)((w & 1) * 16) * 128u;
+        const int rla = (w & 1) * 16 + ra;  // row within the stage
+        ldsm_x4(left + (uint32_t)ra * 128u + (uint32_t)(((2 * kb + ha) ^ (rla & 7)) << 4), a[w]);
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        mma_16816(acc[w][0], a[w], bq[0], bq[1]);
+        mma_16816(acc[w][1], a[w], bq[2], bq[3]);
+      }
     }
-    unsigned char* dst = xm(x);
+    const int n0 = chunk_len(c);
+    const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int j0 = 0; j0 < CB; j0 += 8) {
-      uint4 u;
-      u.x = pack_bf16(v[j0 + 0], v[j0 + 1]);
-      u.y = pack_bf16(v[j0 + 2], v[j0 + 3]);
-      u.z = pack_bf16(v[j0 + 4], v[j0 + 5]);
-      u.w = pack_bf16(v[j0 + 6], v[j0 + 7]);
-      *reinterpret_cast<uint4*>(dst + core_off(lane, j0)) = u;
+    for (int w = 0; w < 4; ++w) {
+      int nrow;  // rows of this block in a chunk whose keys / queries are used
+      if (w == 0) nrow = upd_of(c + 1) ? chunk_len(c + 1) : 0;       // Xg_{c+1}
+      else if (w == 1) nrow = n0;                                    // M_c
+      else if (w == 2) nrow = upd_of(c + 2) ? chunk_len(c + 2) : 0;  // Y_{c+2}
+      else nrow = chunk_len(c + 1);                                  // N_{c+1}
+      unsigned char* dst = xm(c) + (w >> 1) * 1024;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int r = g + 8 * hr, j = 8 * nt + 2 * t4;
+          const bool okr = r < nrow;
+          float v0 = (okr && j < n0) ? acc[w][nt][2 * hr] : 0.f;
+          float v1 = (okr && j + 1 < n0) ? acc[w][nt][2 * hr + 1] : 0.f;
+          if (w == 1) {  // causal: key j <= query r
+            v0 = (j <= r) ? v0 : 0.f;
+            v1 = (j + 1 <= r) ? v1 : 0.f;
+          }
+          *reinterpret_cast<uint32_t*>(dst + core_off((w & 1) * 16 + r, j)) = pack_bf16(v0, v1);
+        }
+      }
     }
     fence_proxy_async_smem();
   };
@@ -340,21 +406,21 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   // =========================== prologue ===========================
   if (warp == 0) {
     tmem_alloc(sTmem, kTmemCols);
-    tmem_alloc(sTmem + 1, kTmemGramCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) mbar_init(&bar_tma[s], 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar_g[s], 128);
-      mbar_init(&bar_z[s], 1);
-      mbar_init(&bar_xm[s], 32);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bar_tma[s], 1);
+      mbar_init(&bar_rdy[s], 4);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_g[s], 4);
+      mbar_init(&bar_z[s], 1);
+    }
+    for (int s = 0; s < 3; ++s) mbar_init(&bar_xm[s], 1);
     mbar_init(bar_w, 1);
-    mbar_init(bar_wb, 128);
-    mbar_init(bar_gram, 1);
+    mbar_init(bar_wb, 4);
     mbar_init(bar_pro, 1);
-    for (int s = 0; s < NST; ++s) mbar_init(&bar_rdy[s], 128);
     mbar_init_fence();
     *sAbort = 0;
   }
@@ -369,7 +435,6 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sTmem[0];
-  const uint32_t tmem2 = sTmem[1];
   if (tma_thread) {
     prefetch_tensormap(&maps.q);
     prefetch_tensormap(&maps.k);
@@ -386,7 +451,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     sGamSums[1] = sgb;
   }
   if (is_bulk) {
-    // W0 -> TMEM (both row copies) and the bf16 operand W_s
+    // W0 -> TMEM (both row copies) and the bf16 operand W_{s,0} (copy 0)
     const int row = wq * 32 + lane;
     const float* src = p.W0 + ((size_t)bh * D + (row & 63)) * D;  // may alias W_T
 #pragma unroll
@@ -405,7 +470,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         u.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
         u.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
         u.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
-        *reinterpret_cast<uint4*>(sWb + sw128_off(row, 4 * hf + ch)) = u;
+        *reinterpret_cast<uint4*>(sWb(0) + sw128_off(row, 4 * hf + ch)) = u;
       }
       if (Wc && row < 64) {
         float* dst = Wc + (size_t)row * D + 32 * hf;
@@ -417,18 +482,18 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     tmem_wait_st();
     fence_proxy_async_smem();
   }
-  // tiles of chunks 0, 1 (chunk 1 carries Q_0) and, for the Gram of chunk 1, 2
+  // stages 0, 1, 2 (read by the prologue MMAs and the first Gram operand)
   bool bad = false;
-  if (!mbar_wait_bounded(&bar_tma[0], 0, lim)) bad = true;
-  if (!mbar_wait_bounded(&bar_tma[1], 0, lim)) bad = true;
-  if (nc > 1 && !mbar_wait_bounded(&bar_tma[2], 0, lim)) bad = true;
+  for (int x = 0; x < 3 && x <= nc; ++x)
+    if (!mbar_wait_bounded(&bar_tma[x], 0, lim)) bad = true;
   if (p.kq_silu && is_bulk) {
-    // stages 0 .. min(3, nc) (the prologue MMAs and the first Gram read them)
+    // stages 0 .. min(3, nc), each marked ready
     for (int x = 0; x <= nc && x < 4; ++x) {
       if (x == 3 && !mbar_wait_bounded(&bar_tma[3], 0, lim)) bad = true;
+      bad = __any_sync(0xffffffffu, bad);
       if (bad) break;
       silu_stage(x);
-      mbar_arrive(&bar_rdy[x]);
+      mbar_arrive_warp(&bar_rdy[x]);
     }
   }
   tc_fence_before();
@@ -436,24 +501,13 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   tc_fence_after();
   if (pro_bad && tid == 0) fail();
   if (issuer && !pro_bad) {
-    mma_gram(tmem2, 0);                        // Xg_1, M_0
-    if (nc > 1) mma_gram(tmem2, 1);            // Xg_2, M_1
-    mma_ws(tmem + col_p(0), tKQ(0), 16);       // P_0
-    mma_ws(tmem + col_p(1), tKQ(1), 32);       // [P_1 | Q0_0]
+    mma_ws(tmem + col_a(0), 0, 0);  // A(0) = W0 [K_0; -]^T
+    mma_ws(tmem + col_a(1), 0, 1);  // A(1) = W0 [K_1; Q_0]^T (stage 1 holds only Q_0 if nc = 1)
     mma_commit(bar_pro);
   }
-  if (warp == 4 && !pro_bad) {
-    if (mbar_wait_bounded(bar_pro, 0, lim)) {
-      tc_fence_after();
-      gram_extract(tmem2, 0);
-      if (nc > 1) gram_extract(tmem2, 1);
-    } else if (lane == 0) {
-      fail();
-    }
-  }
-  if (warp == 4 && !pro_bad) {
-    mbar_arrive(&bar_xm[0]);
-    mbar_arrive(&bar_xm[1]);
+  if (is_gram && !pro_bad) {
+    if (upd_of(0)) gram_operand(0);
+    mbar_arrive_warp(&bar_xm[0]);
   }
   tc_fence_before();
   __syncthreads();
@@ -465,15 +519,18 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     // =========================== chain ===========================
     const float sg2 = sGamSums[0], sgb = sGamSums[1];
     const int tm_m = gt >> 3, tm_p = gt & 7;  // token-major role: token, feature part
+    (void)sgb;
     for (int k = 0; k < nc; ++k) {
       const int n = chunk_len(k);
-      const bool upd = sFlag[k & (kSR - 1)] != 0;
+      const bool upd = upd_of(k);
       // per-feature coefficients that do not depend on Z_k, formed before
-      // waiting for it: LNJAC a = gamma^2, c = gamma (beta - v);
-      // simplified a = gamma, c = beta - v; no LayerNorm c = -v
-      // ablation (GM 3, and GM 4 next to the full Jacobian form): a = 0, c = -gamma v
+      // waiting for it: LNJAC a = gamma^2, c = gamma (beta - v); simplified
+      // a = gamma, c = beta - v; no LayerNorm c = -v; ablation (GM 3, and GM 4
+      // next to the full Jacobian form) a = 0, c = -gamma v
       float a8[8], c8[8], cb8[8];
-      {
+      bool vok = true;
+      if (upd) vok = mbar_wait_bounded(&bar_tma[k % NST], tma_parity(k), lim);  // V_k landed
+      if (upd && vok) {
         const unsigned char* Vt = tV(k) + tm_m * D * 2;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -500,15 +557,18 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       bool ok;
       if (k == 0) ok = mbar_wait_bounded(bar_pro, 0, lim);
       else ok = mbar_wait_bounded(&bar_z[k & 1], (uint32_t)(((k - 1) >> 1) & 1), lim);
+      ok = ok && vok;
       if (upd && ok) {
-        // Z_k^T (feature-major) -> token-major tile
+        // Z_k^T = A(k) + B(k) (feature-major) -> token-major tile
         tc_fence_after();
-        float z[8];
-        tmem_ld8(tmem + tlane + col_p(k & 1) + 8 * half, z);
+        float z[8], zb[8];
+        tmem_ld8(tmem + tlane + col_a(k) + 8 * half, z);
+        const bool bv = b_valid(k);
+        if (bv) tmem_ld8(tmem + tlane + col_b(k) + 8 * half, zb);
         tmem_wait_ld();
         float* Zk = sZ + (k & 1) * CB * kZS + 8 * half * kZS + fm;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) Zk[u * kZS] = z[u];
+        for (int u = 0; u < 8; ++u) Zk[u * kZS] = bv ? z[u] + zb[u] : z[u];
       }
       tc_fence_before();
       if (bar_any(kBarChain, 128, !ok || *sAbort)) {
@@ -519,7 +579,6 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         // token-major LayerNorm + gradient: token tm_m, features tm_p + 8u
         const float* Zk = sZ + (k & 1) * CB * kZS + tm_m * kZS;
         float z[8], G[8];
-        (void)sgb;
 #pragma unroll
         for (int u = 0; u < 8; ++u) z[u] = Zk[tm_p + 8 * u];
         if (GM == 2) {
@@ -622,26 +681,67 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         gn[0] = 0.f;
         gn[1] = 0.f;
       }
-      mbar_arrive(&bar_g[k & 1]);
+      mbar_arrive_warp(&bar_g[k & 1]);
+    }
+  } else if (is_gram && run) {
+    // =========================== Gram ===========================
+    // the operand of chunk c goes to buffer c % 3, last read by the MMAs of
+    // chunk c-3, all complete once Z_{c-1} is (its commit follows them). It
+    // reads stages c .. c+2; a stage this warp has seen land (seen > x) needs
+    // no second wait (each wait costs a few hundred cycles even when the phase
+    // is long complete)
+    int seen = 3;  // stages 0 .. 2: waited by every thread in the prologue
+    for (int c = 1; c < nc; ++c) {
+      bool ok = (c == 1) ? mbar_wait_bounded(bar_pro, 0, lim)
+                         : mbar_wait_bounded(&bar_z[(c - 1) & 1], (uint32_t)(((c - 2) >> 1) & 1),
+                                             lim);
+      if (ok && upd_of(c)) {
+        const int top = min(c + 2, nc);
+        for (int x = max(seen, c); x <= top; ++x) ok = ok && wait_stage(x);
+        seen = max(seen, top + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) gram_operand(c);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) fail();
+        break;
+      }
+      if (__any_sync(0xffffffffu, *sAbort != 0)) break;
+      mbar_arrive_warp(&bar_xm[c % 3]);
     }
   } else if (is_bulk && run) {
     // =========================== bulk ===========================
     Raw pre{};
+    int wbuf = 0;  // the bf16 copy holding W_{s,c}
     for (int c = 0; c < nc; ++c) {
-      const bool upd = sFlag[c & (kSR - 1)] != 0;
+      const bool upd = upd_of(c);
       if ((c & 7) == 0) pre = fetch_block(c + 16);
-      // ---- MMAc and MMA3 of chunk c complete ----
+      // ---- the MMAs of chunk c complete ----
       bool ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
       if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
         if (gt == 0) fail();
         break;
       }
       tc_fence_after();
-      // ---- W_{s,c+1} (fp32 TMEM) -> bf16 operand; snapshot ----
+      // ---- outputs O_c = A(c+1) + B(c+1) (query halves) ----
+      float ov[8];
+      {
+        float ob[8];
+        tmem_ld8(tmem + tlane + col_a(c + 1) + 16 + 8 * half, ov);
+        const bool bv = b_valid(c + 1);
+        if (bv) tmem_ld8(tmem + tlane + col_b(c + 1) + 16 + 8 * half, ob);
+        tmem_wait_ld();
+        if (bv) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ov[u] += ob[u];
+        }
+      }
+      // ---- W_{s,c+1} (fp32 TMEM) -> the other bf16 copy; snapshot ----
       const int row = wq * 32 + lane;
       if (upd) {
-        // two 32-column TMEM loads; the second is in flight while the first
-        // half is packed to bf16 and stored
+        wbuf ^= 1;
+        unsigned char* dstw = sWb(wbuf);
         float w[32];
         uint4 packed[4];
 #pragma unroll
@@ -650,7 +750,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           if (hf == 1) {
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch)
-              *reinterpret_cast<uint4*>(sWb + sw128_off(row, ch)) = packed[ch];
+              *reinterpret_cast<uint4*>(dstw + sw128_off(row, ch)) = packed[ch];
           }
           tmem_wait_ld();
 #pragma unroll
@@ -669,7 +769,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         }
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch)
-          *reinterpret_cast<uint4*>(sWb + sw128_off(row, 4 + ch)) = packed[ch];
+          *reinterpret_cast<uint4*>(dstw + sw128_off(row, 4 + ch)) = packed[ch];
         fence_proxy_async_smem();
       } else if (Wc && row < 64) {
         const float* srcw = Wc + ((size_t)c * D + row) * D;  // W unchanged: repeat the snapshot
@@ -678,41 +778,26 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           *reinterpret_cast<float4*>(dst + k) = *reinterpret_cast<const float4*>(srcw + k);
       }
       tc_fence_before();
-      mbar_arrive(bar_wb);
+      mbar_arrive_warp(bar_wb);
       // refill stage c % NST with load c + NST: every reader of its tiles (MMA1
-      // and the Grams of chunks c-1 and c, MMA3 of chunk c, the chain's V_c)
-      // completed before bar_w of this chunk
+      // of chunk c-2, the Gram operands of chunks c-1 and c, MMA3 of chunk c,
+      // the chain's V_c) completed before bar_w of this chunk
       if (tma_thread && c + NST <= nc) {
         fence_proxy_async_smem();
         issue_tma(c + NST);
       }
-      // SiLU variant: stage c+4, read first by the issuer's next iteration
+      // SiLU variant: stage c+4, read first by the chain after chunk c+1
       if (p.kq_silu && c + 4 <= nc) {
-        if (mbar_wait_bounded(&bar_tma[(c + 4) % NST], tma_parity(c + 4), lim)) {
+        if (__all_sync(0xffffffffu,
+                       mbar_wait_bounded(&bar_tma[(c + 4) % NST], tma_parity(c + 4), lim))) {
           silu_stage(c + 4);
-          mbar_arrive(&bar_rdy[(c + 4) % NST]);
-        } else if (lane == 0) {
-          fail();
-        }
-      }
-      // ---- Gram of chunk c+2 -> [Xg_{c+3}; M_{c+2}]. Its buffer held the
-      // operand of chunk c's MMAc, complete since bar_w ----
-      // (warp 4 alone: the other bulk warps go on to the outputs; a failed
-      // wait is seen by all at the next bar_any)
-      if (c + 2 < nc && wq == 0) {
-        if (mbar_wait_bounded(bar_gram, (uint32_t)(c & 1), lim)) {
-          tc_fence_after();
-          gram_extract(tmem2, c + 2);
-          mbar_arrive(&bar_xm[c & 1]);
+          mbar_arrive_warp(&bar_rdy[(c + 4) % NST]);
         } else if (lane == 0) {
           fail();
         }
       }
       // ---- outputs o_c = gate * O_c^T ----
       {
-        float ov[8];
-        tmem_ld8(tmem + tlane + col_o((c + 1) & 1) + 8 * half, ov);
-        tmem_wait_ld();
         const float* gte = sGate + (c & (kSR - 1)) * CB + 8 * half;
         const int n = chunk_len(c);
         OutT* dst = go + (size_t)c * CB * D;
@@ -726,11 +811,11 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     }
   } else if (issuer && run) {
     // =========================== issuer ===========================
+    int wbuf = 0;  // the bf16 copy holding W_{s,c}
     for (int c = 0; c < nc; ++c) {
-      const bool upd = sFlag[c & (kSR - 1)] != 0;
-      const bool next = c + 1 < nc;
-      // the operand [Xg_{c+1}; M_c] (its Gram has left TMEM slot c & 1), Aneg_c
-      bool ok = mbar_wait_bounded(&bar_xm[c & 1], (uint32_t)((c >> 1) & 1), lim) &&
+      const bool upd = upd_of(c);
+      // the Gram operand of chunk c and Aneg_c
+      bool ok = mbar_wait_bounded(&bar_xm[c % 3], (uint32_t)((c / 3) & 1), lim) &&
                 mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim);
       if (!ok || *sAbort) {
         fail();
@@ -738,37 +823,41 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       }
       tc_fence_after();
       const uint64_t da = smem_desc(smem_u32(aneg(c)), 128, 256, kLayoutNone);
-      if (upd)
-        mma_bf16_ss(tmem + col_p((c + 1) & 1), da,
-                    smem_desc(smem_u32(xm(c)), 128, 256, kLayoutNone), idescN32, 1u);
-      if (next) mma_commit(&bar_z[(c + 1) & 1]);
-      if (upd)
+      if (upd)  // B(c+1) (+)= Aneg_c [Xg_{c+1}; M_c]^T
+        mma_bf16_ss(tmem + col_b(c + 1), da, smem_desc(smem_u32(xm(c)), 128, 256, kLayoutNone),
+                    idescN32, upd_of(c - 1) ? 1u : 0u);
+      if (c + 1 < nc) mma_commit(&bar_z[(c + 1) & 1]);
+      // the bulk has read O_{c-1} (from A(c), B(c)) and W_{s,c} from TMEM, and
+      // written the bf16 copy of W_{s,c}
+      if (c > 0) {
+        ok = mbar_wait_bounded(bar_wb, (uint32_t)((c - 1) & 1), lim);
+        if (!ok || *sAbort) {
+          fail();
+          break;
+        }
+        tc_fence_after();
+      }
+      if (upd && c + 1 < nc)  // B(c+2) = Aneg_c [Y_{c+2}; N_{c+1}]^T (slot of B(c), read)
+        mma_bf16_ss(tmem + col_b(c + 2), da,
+                    smem_desc(smem_u32(xm(c) + 1024), 128, 256, kLayoutNone), idescN32, 0u);
+      if (upd)  // W += Aneg_c K_c (K as an MN-major operand)
         mma_bf16_ss(tmem + kColW, da, smem_desc(smem_u32(tKQ(c)), 2048, 1024, kLayoutSw128),
                     idescW, 1u);
       mma_commit(bar_w);
       ++w_issued;
-
-      if (c + 2 < nc) {
-        // Gram of chunk c+2 (stages c+2, c+3) into TMEM slot c & 1
-        ok = wait_stage(c + 2) && wait_stage(c + 3);
+      if (c + 1 < nc) {
+        // A(c+2) = W_{s,c} [K_{c+2}; Q_{c+1}]^T from the bf16 copy of W_{s,c}.
+        // Stage c+2 has landed: the Gram warp saw it before it wrote the operand
+        // of an updating chunk c (waited for above); otherwise wait here
+        ok = upd || c + 2 <= 2 || wait_stage(c + 2);
         if (!ok || *sAbort) {
           fail();
           break;
         }
         tc_fence_after();
-        mma_gram(tmem2, c + 2);
-        mma_commit(bar_gram);
+        mma_ws(tmem + col_a(c + 2), wbuf, c + 2);
       }
-      if (next) {
-        // W_{s,c+1} in bf16, then [P_{c+2} | Q0_{c+1}] = W_{s,c+1} [K_{c+2}; Q_{c+1}]^T
-        ok = mbar_wait_bounded(bar_wb, (uint32_t)(c & 1), lim) && wait_stage(c + 2);
-        if (!ok || *sAbort) {
-          fail();
-          break;
-        }
-        tc_fence_after();
-        mma_ws(tmem + col_p((c + 2) & 1), tKQ(c + 2), 32);
-      }
+      if (upd) wbuf ^= 1;
     }
   }
 
@@ -803,10 +892,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) {
-    tmem_dealloc(tmem, kTmemCols);
-    tmem_dealloc(tmem2, kTmemGramCols);
-  }
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace ttt

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <type_traits>
 
 #include "ttt_scan.h"
 #include "common.cuh"
@@ -111,9 +112,20 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
       !encode_qkv_map(&maps.k, p.k, p.T, heads, true) ||
       !encode_qkv_map(&maps.v, p.v, p.T, heads, false))
     return TTT_ERR_CUDA;
-  // up to one head per SM: the one-CTA-per-SM build (more registers per
-  // thread); beyond that, several CTAs share an SM
-  const bool one = heads <= ttt::device_sm_count();
+  // Up to one head per SM: the one-CTA-per-SM build (more registers per
+  // thread, deeper staging); beyond that two CTAs share an SM. The kernel of
+  // scan_tc_many.cuh fits three per SM, with a chunk loop about 1.5 times as
+  // long: it goes where it saves a wave, (waves at three per SM) * 1.5 <
+  // (waves at two per SM), i.e. for 2 to 3 heads per SM.
+  const long long sms = ttt::device_sm_count();
+  const bool one = heads <= sms;
+  if (sms > 0) {
+    const long long waves2 = (heads + 2 * sms - 1) / (2 * sms);
+    const long long waves3 = (heads + 3 * sms - 1) / (3 * sms);
+    if (3 * waves3 < 2 * waves2)
+      return ttt::launch_tc_many(p, &maps.q, &maps.k, &maps.v,
+                                 std::is_same<OutT, __nv_bfloat16>::value, GM, stream);
+  }
   auto kernel = one ? ttt::scan_tc_kernel<OutT, GM, 1>
                     : ttt::scan_tc_kernel<OutT, GM, ttt::tc::kMinbMany>;
   const int smem = one ? ttt::tc::smem_bytes<1>() : ttt::tc::smem_bytes<ttt::tc::kMinbMany>();
@@ -202,8 +214,9 @@ int ttt_check_device_status(void* cuda_stream) {
     if (cudaMemcpyToSymbol(ttt::g_ttt_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
   }
   const int hc = ttt::cluster_status_take();
-  if (hc < 0) return TTT_ERR_CUDA;
-  return (h != 0 || hc != 0) ? TTT_ERR_DEVICE_TIMEOUT : TTT_OK;
+  const int hm = ttt::tc_many_status_take();
+  if (hc < 0 || hm < 0) return TTT_ERR_CUDA;
+  return (h != 0 || hc != 0 || hm != 0) ? TTT_ERR_DEVICE_TIMEOUT : TTT_OK;
 }
 
 static int scan_forward(const void* q, const void* k, const void* v, const void* eta_logit,

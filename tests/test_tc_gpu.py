@@ -36,11 +36,13 @@ def test_tc_matches_oracle(grad, out_bf16, T):
 
 
 @pytest.mark.parametrize("grad", [LNJAC, 0, NO_LN], ids=["lnjac", "simple", "no_ln"])
-@pytest.mark.parametrize("BH", [(4, 37), (10, 15)], ids=["148heads", "150heads"])
-def test_tc_both_occupancy_builds(grad, BH):
-    """Up to one head per SM runs the one-CTA-per-SM build, more heads the
-    three-CTAs-per-SM build (B200: 148 SMs); both against the oracle, with a
-    ragged tail and a SKIP/UPDATE mask."""
+@pytest.mark.parametrize("BH", [(4, 37), (10, 15), (10, 30), (10, 45)],
+                         ids=["148heads", "150heads", "300heads", "450heads"])
+def test_tc_all_occupancy_builds(grad, BH):
+    """On B200's 148 SMs: up to 148 heads run the one-CTA-per-SM build, 150
+    the two-per-SM build, 300 the three-per-SM kernel (one wave instead of
+    two), 450 the two-per-SM build again (two waves either way); each against
+    the oracle, with a ragged tail and a SKIP/UPDATE mask."""
     B, H = BH
     inp = make_inputs(B, H, 40, 64, seed=250 + grad + B, random_affine=True, in_bf16=True,
                       mask_p=0.7, b=16)
@@ -90,14 +92,16 @@ def test_tc_eta_zero_and_no_gate():
     assert_rrms(o, ref, "o", tol=5e-3)
 
 
-def test_tc_wait_timeout_reports_and_recovers():
+@pytest.mark.parametrize("BH", [(1, 2), (10, 30)], ids=["2heads", "300heads"])
+def test_tc_wait_timeout_reports_and_recovers(BH):
     """With a wait limit of 0 every bounded wait gives up at once: the kernel
-    must report TTT_ERR_DEVICE_TIMEOUT (no hang, no trap), and the context must
+    (either tensor-core kernel: 300 heads take the three-per-SM one) must
+    report TTT_ERR_DEVICE_TIMEOUT (no hang, no trap), and the context must
     stay usable for a normal call afterwards."""
     import torch
     from test_sequence_layers_02_b200 import ttt_scan
     from tests.helpers import to_torch
-    inp = make_inputs(1, 2, 48, 64, seed=402, random_affine=True, in_bf16=True)
+    inp = make_inputs(*BH, 48, 64, seed=402, random_affine=True, in_bf16=True)
     t = to_torch(inp, "cuda", True)
     args = (t["q"], t["k"], t["v"], t["eta_logit"], t["gate_logit"], t["W0"], t["gamma"], t["beta"])
     ttt_scan.set_wait_limit(0)
