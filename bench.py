@@ -69,7 +69,8 @@ _KERNEL_SOURCES = {
 }
 # Captures: a kernel may have several (e.g. the tensor-core kernel with and
 # without a SKIP/UPDATE mask); each names the kernel whose sources it covers.
-_CAPTURE_KERNEL = {"scan_tc_masked": "scan_tc", "scan_simt_4pt": "scan_simt"}
+_CAPTURE_KERNEL = {"scan_tc_masked": "scan_tc", "scan_simt_4pt": "scan_simt",
+                   "scan_bwd_pertoken": "scan_bwd", "scan_bwd_minibatch": "scan_bwd"}
 
 
 def _tc_takes_many(heads: int) -> bool:
@@ -422,7 +423,7 @@ class BwdJob:
         return "scan_bwd"
 
     def capture_key(self) -> str:
-        return "scan_bwd"
+        return "scan_bwd_minibatch" if self.w.minibatch else "scan_bwd_pertoken"
 
     def e2e_setup(self):
         """Pinned host copies of the inputs (with the forward's snapshots and dO)
