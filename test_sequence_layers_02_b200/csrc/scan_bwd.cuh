@@ -106,7 +106,8 @@ struct BwdLayout {
   static constexpr int oP1 = oCg + C;          //   (LN Jacobian) and sum xhat
   static constexpr int oP2 = oP1 + C;
   static constexpr int oPx = oP2 + C;
-  static constexpr int floats = oPx + C;
+  static constexpr int oRs = oPx + C;          //   and 1 / s_t
+  static constexpr int floats = oRs + C;
   static constexpr int bytes = floats * 4;
 };
 
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
   float* sP1 = sm + L::oP1;
   float* sP2 = sm + L::oP2;
   float* sPx = sm + L::oPx;
+  float* sRs = sm + L::oRs;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -329,20 +331,21 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         }
         butterfly<NM>(m);
         const float mu1 = m[0] * inv_d;
-        const float var = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f);
-        const float s = sqrtf(var + p.eps);
+        const float ve = fmaxf(fmaf(m[1], inv_d, -mu1 * mu1), 0.f) + p.eps;
+        const float rs = rsqrtf(ve);  // 1 / s, s = sqrt(var + eps)
+        const float s = ve * rs;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) xh[e] = (lane + 32 * e < D) ? (y[e] - mu1) / s : 0.f;
+        for (int e = 0; e < EPL; ++e) xh[e] = (lane + 32 * e < D) ? (y[e] - mu1) * rs : 0.f;
         if (kJac) {
           const float sa = (GM == 1) ? sg2 : 0.f;                                 // sum of a
-          const float p1 = (m[2] - mu1 * sa) / s;                                 // sum a xhat
-          const float p2 = (m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa) / (s * s);  // sum a xhat^2
+          const float p1 = (m[2] - mu1 * sa) * rs;                                // sum a xhat
+          const float p2 = (m[3] - 2.f * mu1 * m[2] + mu1 * mu1 * sa) * (rs * rs);  // sum a xhat^2
           const float a_ = (p1 + m[5]) * inv_d;                                   // mean g
-          const float cg = (p2 + (m[4] - mu1 * m[5]) / s) * inv_d;                // mean g xhat
+          const float cg = fmaf(m[4] - mu1 * m[5], rs, p2) * inv_d;               // mean g xhat
 #pragma unroll
           for (int e = 0; e < EPL; ++e) {
             const float g = fmaf(aa[e], xh[e], cc[e]);
-            G[e] = (lane + 32 * e < D) ? (g - a_ - xh[e] * cg) / s : 0.f;
+            G[e] = (lane + 32 * e < D) ? (g - a_ - xh[e] * cg) * rs : 0.f;
           }
           if (lane == 0) {
             sA[t] = a_;
@@ -357,7 +360,8 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         }
         if (lane == 0) {
           sS[t] = s;
-          sPx[t] = (m[0] - (float)D * mu1) / s;  // sum xhat
+          sRs[t] = rs;
+          sPx[t] = (m[0] - (float)D * mu1) * rs;  // sum xhat
         }
       }
 #pragma unroll
@@ -486,25 +490,25 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         }
       } else {
         // dG = -eta u; the sums of the LayerNorm backward in closed form
-        const float s = sS[t];
+        const float s = sS[t], rs = sRs[t];
         const float mdG = -eta * m[1] * inv_d, mdGx = -eta * m[2] * inv_d;
         float ds = 0.f, s_jx = 0.f, s_j = 0.f, s_ex = 0.f, s_e = 0.f;
         if (kJac) {
           const float a_ = sA[t], cg = sCg[t];
-          ds = eta * m[0] / s;                           // -(sum dG G) / s
-          s_jx = -2.f * (float)D * cg * mdGx / s;        // sum of the Jacobian part of dxhat * xhat
-          s_j = -(float)D * (cg * mdG + a_ * mdGx) / s;  // ... and of that part alone
+          ds = eta * m[0] * rs;                           // -(sum dG G) / s
+          s_jx = -2.f * (float)D * cg * mdGx * rs;        // sum of the Jacobian part of dxhat * xhat
+          s_j = -(float)D * (cg * mdG + a_ * mdGx) * rs;  // ... and of that part alone
         }
         if (GM == 1) {         // derr = dg gamma: sums of derr gamma xhat, derr gamma
-          s_ex = (-eta * m[4] - mdG * sP1[t] - mdGx * sP2[t]) / s;
-          s_e = (-eta * m[3] - mdG * sg2 - mdGx * sP1[t]) / s;
+          s_ex = (-eta * m[4] - mdG * sP1[t] - mdGx * sP2[t]) * rs;
+          s_e = (-eta * m[3] - mdG * sg2 - mdGx * sP1[t]) * rs;
         } else if (GM == 0) {  // derr = dG
           s_ex = -eta * m[4];
           s_e = -eta * m[3];
         }
         const float dxx = s_jx + s_ex;
-        const float dvar = (ds - dxx / s) / (2.f * s);
-        const float mdy = ((s_j + s_e) / s + dvar * 2.f * s * sPx[t] * inv_d) * inv_d;
+        const float dvar = (ds - dxx * rs) * (0.5f * rs);
+        const float mdy = ((s_j + s_e) * rs + dvar * 2.f * s * sPx[t] * inv_d) * inv_d;
         const float cgt = kJac ? sCg[t] : 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -514,8 +518,8 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
           dv[e] = 0.f;
           if (kJac) {
             const float g = GM == 3 ? -gam[e] * v[e] : gam[e] * (fmaf(gam[e], xh[e], bet[e]) - v[e]);
-            const float dg = (dG - mdG - xh[e] * mdGx) / s;
-            dxh = (-dG * cgt - g * mdGx) / s;
+            const float dg = (dG - mdG - xh[e] * mdGx) * rs;
+            dxh = (-dG * cgt - g * mdGx) * rs;
             if (GM == 3) {
               if (fv) {
                 dgam[e] -= dg * v[e];
@@ -537,7 +541,7 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
           dv[e] -= derr;
           dxh = fmaf(derr, gam[e], dxh);
           // xhat = (z - mu) / s, s = sqrt(var + eps), z - mu = xhat s
-          dz[e] = fv ? dxh / s + dvar * 2.f * xh[e] * s * inv_d - mdy : 0.f;
+          dz[e] = fv ? fmaf(dxh, rs, dvar * 2.f * xh[e] * s * inv_d) - mdy : 0.f;
         }
       }
 #pragma unroll
