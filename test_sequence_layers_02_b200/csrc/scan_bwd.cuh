@@ -200,44 +200,74 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
     sD[r * LD + c] = p.dW_T ? p.dW_T[(size_t)bh * D * D + idx] : 0.f;
   }
 
+  // ---- a chunk's global inputs, loaded into registers one chunk ahead (the
+  // loads of chunk ch-1 are in flight while chunk ch computes): this thread's
+  // elements idx = tid + NT i of W_s and of the [C][D] token arrays, and (tid
+  // < C) token tid's logits. Rows past the chunk and SKIP chunks' eta are
+  // zeroed when the registers are stored. ----
+  constexpr int kWpt = D * D / NT, kTpt = C * D / NT;
+  float rw[kWpt], rk[kTpt], rq[kTpt], rv[kTpt], ro[kTpt], rgc[kTpt];
+  float rel = 0.f, rgl = 0.f;
+  auto fetch = [&](int ch) {
+    const int t0 = ch * b;
+    const int n = min(b, T - t0);
+#pragma unroll
+    for (int i = 0; i < kWpt; ++i) rw[i] = Wc[(size_t)ch * D * D + tid + NT * i];
+#pragma unroll
+    for (int i = 0; i < kTpt; ++i) {
+      const int idx = tid + NT * i, t = idx / D;
+      const bool ok = t < n;
+      const size_t g = (tok0 + t0 + t) * D + (idx - t * D);
+      rk[i] = ok ? ld_in<InT>(p.k, g) : 0.f;
+      rq[i] = ok ? ld_in<InT>(p.q, g) : 0.f;
+      rv[i] = ok ? ld_in<InT>(p.v, g) : 0.f;
+      ro[i] = ok ? p.dO[g] : 0.f;
+      rgc[i] = (ok && p.gate_logit && p.gate_channel) ? ld_in<InT>(p.gate_logit, g) : 0.f;
+    }
+    if (tid < C && tid < n) {
+      rel = ld_in<InT>(p.eta_logit, tok0 + t0 + tid);
+      rgl = (p.gate_logit && !p.gate_channel) ? ld_in<InT>(p.gate_logit, tok0 + t0 + tid) : 0.f;
+    }
+  };
+  if (nc > 0) fetch(nc - 1);
+
   for (int ch = nc - 1; ch >= 0; --ch) {
     const int t0 = ch * b;
     const int n = min(b, T - t0);
     const bool upd = p.mask == nullptr || p.mask[(size_t)bi * nc + ch] != 0;
 
     // ---- chunk inputs (rows past n are zero), W_s, scalars ----
-    for (int idx = tid; idx < D * D; idx += NT) {
-      const int r = idx / D, c = idx - r * D;
-      sW[r * LD + c] = Wc[(size_t)ch * D * D + idx];
+#pragma unroll
+    for (int i = 0; i < kWpt; ++i) {
+      const int idx = tid + NT * i, r = idx / D;
+      sW[r * LD + idx - r * D] = rw[i];
     }
-    for (int idx = tid; idx < C * D; idx += NT) {
-      const int t = idx / D, f = idx - t * D;
+#pragma unroll
+    for (int i = 0; i < kTpt; ++i) {
+      const int idx = tid + NT * i, t = idx / D, f = idx - t * D;
       const bool ok = t < n;
-      const size_t g = (tok0 + t0 + t) * D + f;
-      float kv = ok ? ld_in<InT>(p.k, g) : 0.f;
-      float qv = ok ? ld_in<InT>(p.q, g) : 0.f;
-      if (p.kq_silu) {
+      float kv = rk[i], qv = rq[i];
+      if (p.kq_silu && ok) {
         kv = siluf_(kv);
         qv = siluf_(qv);
       }
       sK[t * LD + f] = kv;
       sQ[t * LD + f] = qv;
-      sV[t * LD + f] = ok ? ld_in<InT>(p.v, g) : 0.f;
-      float gch = 1.f;
-      if (ok && p.gate_logit && p.gate_channel) gch = sigmoidf_(ld_in<InT>(p.gate_logit, g));
+      sV[t * LD + f] = rv[i];
+      const float gch = (ok && p.gate_logit && p.gate_channel) ? sigmoidf_(rgc[i]) : 1.f;
       // dy = gate dO (the scalar gate is applied below, once it is known)
-      sDO[t * LD + f] = ok ? p.dO[g] : 0.f;
-      sDy[t * LD + f] = ok ? gch * p.dO[g] : 0.f;
+      sDO[t * LD + f] = ro[i];
+      sDy[t * LD + f] = gch * ro[i];
     }
     if (tid < C) {
       const int t = tid;
       const bool ok = t < n;
-      const float sg = (ok && upd) ? sigmoidf_(ld_in<InT>(p.eta_logit, tok0 + t0 + t)) : 0.f;
+      const float sg = (ok && upd) ? sigmoidf_(rel) : 0.f;
       sSg[t] = sg;
       sEta[t] = sg * inv_d;
-      sGate[t] = (ok && p.gate_logit && !p.gate_channel)
-                     ? sigmoidf_(ld_in<InT>(p.gate_logit, tok0 + t0 + t)) : 1.f;
+      sGate[t] = (ok && p.gate_logit && !p.gate_channel) ? sigmoidf_(rgl) : 1.f;
     }
+    if (ch > 0) fetch(ch - 1);
     __syncthreads();
     if (p.gate_logit && !p.gate_channel) {
       for (int idx = tid; idx < C * D; idx += NT) {
@@ -673,15 +703,35 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
       p.dq[g] = dq;
       p.dk[g] = dk;
     }
-    // ---- D_s = D_e + sum_t (dy_t q_t^T + dz_t k_t^T) ----
-    for (int idx = tid; idx < D * D; idx += NT) {
-      const int r = idx / D, c = idx - r * D;
-      float acc = sD[r * LD + c];
+    // ---- D_s = D_e + sum_t (dy_t q_t^T + dz_t k_t^T): a TS x TS tile of D
+    //      per thread, so each value read from shared memory feeds TS FMAs ----
+    {
+      constexpr int TS = (D == 64) ? 4 : 2;  // TS * TS = D * D / NT
+      static_assert(TS * TS * NT == D * D, "one tile per thread");
+      const int r0 = TS * (tid / (D / TS)), c0 = TS * (tid % (D / TS));
+      float acc[TS][TS];
+#pragma unroll
+      for (int i = 0; i < TS; ++i)
+#pragma unroll
+        for (int j = 0; j < TS; ++j) acc[i][j] = sD[(r0 + i) * LD + c0 + j];
       for (int t = 0; t < n; ++t) {
-        acc = fmaf(sDy[t * LD + r], sQ[t * LD + c], acc);
-        acc = fmaf(sDz[t * LD + r], sK[t * LD + c], acc);
+        float dy[TS], dz[TS], q[TS], k[TS];
+#pragma unroll
+        for (int i = 0; i < TS; ++i) {
+          dy[i] = sDy[t * LD + r0 + i];
+          dz[i] = sDz[t * LD + r0 + i];
+          q[i] = sQ[t * LD + c0 + i];
+          k[i] = sK[t * LD + c0 + i];
+        }
+#pragma unroll
+        for (int i = 0; i < TS; ++i)
+#pragma unroll
+          for (int j = 0; j < TS; ++j) acc[i][j] = fmaf(dz[i], k[j], fmaf(dy[i], q[j], acc[i][j]));
       }
-      sD[r * LD + c] = acc;
+#pragma unroll
+      for (int i = 0; i < TS; ++i)
+#pragma unroll
+        for (int j = 0; j < TS; ++j) sD[(r0 + i) * LD + c0 + j] = acc[i][j];
     }
     __syncthreads();
   }
