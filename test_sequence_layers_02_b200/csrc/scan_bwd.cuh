@@ -72,7 +72,10 @@ template <int D>
 struct BwdLayout {
   static constexpr int NT = 4 * D;   // threads: 256 at d = 64, 64 at d = 16
   static constexpr int C = kC;       // largest chunk
-  static constexpr int LD = D + 1;   // padded row stride of every [rows][D] array
+  // padded row stride of every [rows][D] array: rows stay 16-byte aligned
+  // (float4 reads along a row), and rows r and r+8 of a column fall in
+  // different banks
+  static constexpr int LD = D + 4;
   static constexpr int MAT = D * LD; // a d x d matrix
   static constexpr int TOK = C * LD; // a [C][D] token array
   static constexpr int GR = C * C;   // a Gram
@@ -109,7 +112,15 @@ struct BwdLayout {
   static constexpr int oRs = oPx + C;          //   and 1 / s_t
   static constexpr int floats = oRs + C;
   static constexpr int bytes = floats * 4;
+  static_assert(LD % 4 == 0 && oDm % 4 == 0 && oK % 4 == 0 && oQ % 4 == 0 && oG % 4 == 0 &&
+                    oDy % 4 == 0 && oDz % 4 == 0,
+                "arrays read as float4 start on 16 bytes");
 };
+
+__device__ __forceinline__ float4 ld4(const float* a) { return *reinterpret_cast<const float4*>(a); }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
 
 __device__ __forceinline__ float silu_grad(float x) {
   const float s = sigmoidf_(x);
@@ -201,13 +212,19 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
   }
 
   // ---- a chunk's global inputs, loaded into registers one chunk ahead (the
-  // loads of chunk ch-1 are in flight while chunk ch computes): this thread's
+  // loads of chunk ch-1 are in flight while chunk ch finishes): this thread's
   // elements idx = tid + NT i of W_s and of the [C][D] token arrays, and (tid
   // < C) token tid's logits. Rows past the chunk and SKIP chunks' eta are
   // zeroed when the registers are stored. ----
+  // (Raw values of the input type: converting at the load would wait for it.)
   constexpr int kWpt = D * D / NT, kTpt = C * D / NT;
-  float rw[kWpt], rk[kTpt], rq[kTpt], rv[kTpt], ro[kTpt], rgc[kTpt];
-  float rel = 0.f, rgl = 0.f;
+  const InT* pk = static_cast<const InT*>(p.k);
+  const InT* pq = static_cast<const InT*>(p.q);
+  const InT* pv = static_cast<const InT*>(p.v);
+  const InT* pel = static_cast<const InT*>(p.eta_logit);
+  const InT* pgl = static_cast<const InT*>(p.gate_logit);
+  float rw[kWpt], ro[kTpt];
+  InT rk[kTpt], rq[kTpt], rv[kTpt], rgc[kTpt], rel, rgl;
   auto fetch = [&](int ch) {
     const int t0 = ch * b;
     const int n = min(b, T - t0);
@@ -216,17 +233,21 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
     for (int i = 0; i < kTpt; ++i) {
       const int idx = tid + NT * i, t = idx / D;
-      const bool ok = t < n;
       const size_t g = (tok0 + t0 + t) * D + (idx - t * D);
-      rk[i] = ok ? ld_in<InT>(p.k, g) : 0.f;
-      rq[i] = ok ? ld_in<InT>(p.q, g) : 0.f;
-      rv[i] = ok ? ld_in<InT>(p.v, g) : 0.f;
-      ro[i] = ok ? p.dO[g] : 0.f;
-      rgc[i] = (ok && p.gate_logit && p.gate_channel) ? ld_in<InT>(p.gate_logit, g) : 0.f;
+      rk[i] = rq[i] = rv[i] = rgc[i] = from_f32<InT>(0.f);
+      ro[i] = 0.f;
+      if (t < n) {
+        rk[i] = pk[g];
+        rq[i] = pq[g];
+        rv[i] = pv[g];
+        ro[i] = p.dO[g];
+        if (pgl && p.gate_channel) rgc[i] = pgl[g];
+      }
     }
+    rel = rgl = from_f32<InT>(0.f);
     if (tid < C && tid < n) {
-      rel = ld_in<InT>(p.eta_logit, tok0 + t0 + tid);
-      rgl = (p.gate_logit && !p.gate_channel) ? ld_in<InT>(p.gate_logit, tok0 + t0 + tid) : 0.f;
+      rel = pel[tok0 + t0 + tid];
+      if (pgl && !p.gate_channel) rgl = pgl[tok0 + t0 + tid];
     }
   };
   if (nc > 0) fetch(nc - 1);
@@ -246,15 +267,15 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
     for (int i = 0; i < kTpt; ++i) {
       const int idx = tid + NT * i, t = idx / D, f = idx - t * D;
       const bool ok = t < n;
-      float kv = rk[i], qv = rq[i];
+      float kv = to_f32(rk[i]), qv = to_f32(rq[i]);
       if (p.kq_silu && ok) {
         kv = siluf_(kv);
         qv = siluf_(qv);
       }
       sK[t * LD + f] = kv;
       sQ[t * LD + f] = qv;
-      sV[t * LD + f] = rv[i];
-      const float gch = (ok && p.gate_logit && p.gate_channel) ? sigmoidf_(rgc[i]) : 1.f;
+      sV[t * LD + f] = to_f32(rv[i]);
+      const float gch = (ok && p.gate_logit && p.gate_channel) ? sigmoidf_(to_f32(rgc[i])) : 1.f;
       // dy = gate dO (the scalar gate is applied below, once it is known)
       sDO[t * LD + f] = ro[i];
       sDy[t * LD + f] = gch * ro[i];
@@ -262,12 +283,11 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
     if (tid < C) {
       const int t = tid;
       const bool ok = t < n;
-      const float sg = (ok && upd) ? sigmoidf_(rel) : 0.f;
+      const float sg = (ok && upd) ? sigmoidf_(to_f32(rel)) : 0.f;
       sSg[t] = sg;
       sEta[t] = sg * inv_d;
-      sGate[t] = (ok && p.gate_logit && !p.gate_channel) ? sigmoidf_(rgl) : 1.f;
+      sGate[t] = (ok && p.gate_logit && !p.gate_channel) ? sigmoidf_(to_f32(rgl)) : 1.f;
     }
-    if (ch > 0) fetch(ch - 1);
     __syncthreads();
     if (p.gate_logit && !p.gate_channel) {
       for (int idx = tid; idx < C * D; idx += NT) {
@@ -283,15 +303,15 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
       float az[NTK], ay[NTK], ap[NTK];
 #pragma unroll
       for (int m = 0; m < NTK; ++m) az[m] = ay[m] = ap[m] = 0.f;
-      for (int c = 0; c < D; ++c) {
-        const float w = sW[r * LD + c], dd = sD[r * LD + c];
+      for (int c = 0; c < D; c += 4) {
+        const float4 w = ld4(sW + r * LD + c), dd = ld4(sD + r * LD + c);
 #pragma unroll
         for (int m = 0; m < NTK; ++m) {
           const int t = tg + 4 * m;
-          const float kc = sK[t * LD + c];
-          az[m] = fmaf(w, kc, az[m]);
-          ay[m] = fmaf(w, sQ[t * LD + c], ay[m]);
-          ap[m] = fmaf(dd, kc, ap[m]);
+          const float4 kc = ld4(sK + t * LD + c);
+          az[m] = dot4(w, kc, az[m]);
+          ay[m] = dot4(w, ld4(sQ + t * LD + c), ay[m]);
+          ap[m] = dot4(dd, kc, ap[m]);
         }
       }
 #pragma unroll
@@ -306,10 +326,10 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
     for (int idx = tid; idx < C * C; idx += NT) {
       const int i = idx / C, j = idx - i * C;
       float kk = 0.f, qk = 0.f;
-      for (int f = 0; f < D; ++f) {
-        const float kj = sK[j * LD + f];
-        kk = fmaf(sK[i * LD + f], kj, kk);
-        qk = fmaf(sQ[i * LD + f], kj, qk);
+      for (int f = 0; f < D; f += 4) {
+        const float4 kj = ld4(sK + j * LD + f);
+        kk = dot4(ld4(sK + i * LD + f), kj, kk);
+        qk = dot4(ld4(sQ + i * LD + f), kj, qk);
       }
       sKK[idx] = kk;
       sQK[idx] = qk;
@@ -422,26 +442,22 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         fwd_token(t, z, G);
       }
     } else if (warp == 0) {
-      // z of every token in registers; each G_t goes at once into the later
-      // tokens' z (z_m -= eta_t (k_m . k_t) G_t)
-      float zr[C][EPL];
-#pragma unroll
-      for (int t = 0; t < C; ++t)
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          zr[t][e] = (t < n && lane + 32 * e < D) ? sZ[t * LD + lane + 32 * e] : 0.f;
-#pragma unroll
+      // token by token: z_t = W_s k_t - sum_{j<t} eta_j (k_t . k_j) G_j, the
+      // earlier G_j read back from shared memory (this lane wrote them); a
+      // rolled loop keeps the chain's code small
+#pragma unroll 1
       for (int t = 0; t < C; ++t) {
         if (t < n && upd) {
-          float G[EPL];
-          fwd_token(t, zr[t], G);
-          const float et = sEta[t];
+          float z[EPL], G[EPL];
 #pragma unroll
-          for (int m2 = t + 1; m2 < C; ++m2) {
-            const float a = -et * sKK[m2 * C + t];
+          for (int e = 0; e < EPL; ++e) z[e] = (lane + 32 * e < D) ? sZ[t * LD + lane + 32 * e] : 0.f;
+          for (int j = 0; j < t; ++j) {
+            const float a = -sEta[j] * sKK[t * C + j];
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) zr[m2][e] = fmaf(a, G[e], zr[m2][e]);
+            for (int e = 0; e < EPL; ++e)
+              if (lane + 32 * e < D) z[e] = fmaf(a, sG[j * LD + lane + 32 * e], z[e]);
           }
+          fwd_token(t, z, G);
         } else {
           zero_rows(sG, t);
           zero_rows(sXh, t);
@@ -611,15 +627,9 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         bwd_token(t, u, dz);
       }
     } else if (warp == 0) {
-      // u of every token in registers; each dz_t goes at once into the earlier
-      // tokens' u (u_m += (k_t . k_m) dz_t)
-      float ur[C][EPL];
-#pragma unroll
-      for (int t = 0; t < C; ++t)
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          ur[t][e] = (t < n && lane + 32 * e < D) ? sPB[t * LD + lane + 32 * e] : 0.f;
-#pragma unroll
+      // right to left: u_t = (the part in sPB) + sum_{j>t} (k_j . k_t) dz_j,
+      // the later dz_j read back from shared memory (this lane wrote them)
+#pragma unroll 1
       for (int i = 0; i < C; ++i) {
         const int t = C - 1 - i;
         if (t >= n) {
@@ -627,17 +637,22 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
         } else if (!upd) {
           skip_token(t);
         } else {
-          float dz[EPL];
-          bwd_token(t, ur[t], dz);
+          float u[EPL], dz[EPL];
 #pragma unroll
-          for (int m2 = 0; m2 < t; ++m2) {
-            const float a = sKK[t * C + m2];
+          for (int e = 0; e < EPL; ++e) u[e] = (lane + 32 * e < D) ? sPB[t * LD + lane + 32 * e] : 0.f;
+          for (int j = n - 1; j > t; --j) {
+            const float a = sKK[j * C + t];
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) ur[m2][e] = fmaf(a, dz[e], ur[m2][e]);
+            for (int e = 0; e < EPL; ++e)
+              if (lane + 32 * e < D) u[e] = fmaf(a, sDz[j * LD + lane + 32 * e], u[e]);
           }
+          bwd_token(t, u, dz);
         }
       }
     }
+    // the next chunk's loads, issued once the chains (whose registers they
+    // would crowd) are done
+    if (ch > 0) fetch(ch - 1);
     __syncthreads();
 
     // ---- batched: W_s^T dy_t, W_s^T dz_t, D_e^T G_t (thread: column c, tokens tg + 4m);
@@ -648,14 +663,17 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
       float a1[NTK], a2[NTK], a3[NTK];
 #pragma unroll
       for (int m = 0; m < NTK; ++m) a1[m] = a2[m] = a3[m] = 0.f;
-      for (int r = 0; r < D; ++r) {
-        const float w = sW[r * LD + c], dd = sD[r * LD + c];
+      for (int r = 0; r < D; r += 4) {
+        const float4 w = make_float4(sW[r * LD + c], sW[(r + 1) * LD + c], sW[(r + 2) * LD + c],
+                                     sW[(r + 3) * LD + c]);
+        const float4 dd = make_float4(sD[r * LD + c], sD[(r + 1) * LD + c], sD[(r + 2) * LD + c],
+                                      sD[(r + 3) * LD + c]);
 #pragma unroll
         for (int m = 0; m < NTK; ++m) {
           const int t = tg + 4 * m;
-          a1[m] = fmaf(w, sDy[t * LD + r], a1[m]);
-          a2[m] = fmaf(w, sDz[t * LD + r], a2[m]);
-          a3[m] = fmaf(dd, sG[t * LD + r], a3[m]);
+          a1[m] = dot4(w, ld4(sDy + t * LD + r), a1[m]);
+          a2[m] = dot4(w, ld4(sDz + t * LD + r), a2[m]);
+          a3[m] = dot4(dd, ld4(sG + t * LD + r), a3[m]);
         }
       }
 #pragma unroll
@@ -669,10 +687,10 @@ __global__ void __launch_bounds__(4 * D, 1) scan_bwd_kernel(const BwdParams p) {
     for (int idx = tid; idx < C * C; idx += NT) {
       const int i = idx / C, j = idx - i * C;
       float gy = 0.f, gz = 0.f;
-      for (int f = 0; f < D; ++f) {
-        const float gj = sG[j * LD + f];
-        gy = fmaf(gj, sDy[i * LD + f], gy);
-        gz = fmaf(gj, sDz[i * LD + f], gz);
+      for (int f = 0; f < D; f += 4) {
+        const float4 gj = ld4(sG + j * LD + f);
+        gy = dot4(gj, ld4(sDy + i * LD + f), gy);
+        gz = dot4(gj, ld4(sDz + i * LD + f), gz);
       }
       sGDy[idx] = gy;
       sGDz[idx] = gz;
