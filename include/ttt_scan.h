@@ -155,6 +155,48 @@ int ttt_scan_forward_grad_norms(const void* q, const void* k, const void* v,
 int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b);
 
 /*
+ * ttt_scan_forward with its inputs and outputs in HOST memory: the end-to-end
+ * call of a caller whose tensors live on the host. No page has this call; it
+ * is plumbing around the same scan. The sequence is cut into segments of
+ * `seg_tokens` tokens (0: the library's choice, about an eighth of T, at
+ * least 256, a multiple of b); segment i+1's inputs are copied in while
+ * segment i is scanned and segment i-1's outputs are copied out, and the
+ * state W passes from one segment to the next on the device, exactly. o and
+ * W_T are those of ttt_scan_forward on the whole sequence up to rounding (the
+ * kernels' look-ahead products restart at a segment boundary, where the first
+ * chunk's z comes straight from the state), and bit for bit when one segment
+ * covers the sequence.
+ *
+ * Arguments as for ttt_scan_forward, except:
+ *   q .. mask, o, W_T   HOST pointers (page-locked memory lets the copies run
+ *                       asynchronously; pageable memory works, more slowly).
+ *                       W_T may equal W0. They must stay valid, and o / W_T
+ *                       unread, until `cuda_stream` has completed the call.
+ *   seg_tokens          0, or a positive multiple of b.
+ *   workspace           DEVICE memory of at least
+ *                       ttt_scan_forward_host_workspace_bytes(B, H, T, d, mode, b,
+ *                       seg_tokens) bytes, 16-byte aligned, owned by the caller and
+ *                       not touched by anything else until the call completes on
+ *                       `cuda_stream`.
+ * There is no W_chunks output. Enqueue-only: the copies run on two streams of
+ * the library's own (created on first use on each device, kept until exit) and
+ * the scans on `cuda_stream`, which waits for the last copy, so synchronising
+ * `cuda_stream` completes the call. Calls from several host threads are
+ * enqueued one at a time. Errors: TTT_ERR_INVALID_ARG for arguments the scan
+ * rejects, for seg_tokens that is negative or not a multiple of b, or for a
+ * workspace that is too small or misaligned (nothing is enqueued);
+ * TTT_ERR_CUDA if a copy or a stream operation fails to enqueue.
+ */
+size_t ttt_scan_forward_host_workspace_bytes(int B, int H, int T, int d, unsigned mode, int b,
+                                             int seg_tokens);
+int ttt_scan_forward_host(const void* q, const void* k, const void* v,
+                          const void* eta_logit, const void* gate_logit,
+                          const float* W0, const float* gamma, const float* beta,
+                          int B, int H, int T, int d, float eps, unsigned mode, int b,
+                          const unsigned char* mask, void* o, float* W_T, int seg_tokens,
+                          void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * One streaming decode step: the per-token recurrence above for a single token
  * of every (batch row, head), with the fast weights carried between calls and
  * updated IN PLACE (the state-in, state-out step of cortex_rust

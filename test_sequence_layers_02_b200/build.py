@@ -17,7 +17,8 @@ UNITS = [(CSRC / "ttt_scan.cu", "ttt_scan", ()),
          (CSRC / "cluster.cu", "cluster", ()),
          (CSRC / "backward.cu", "backward", ()),
          (CSRC / "probe.cu", "probe", ()),
-         (CSRC / "tc_many.cu", "tc_many", ())]
+         (CSRC / "tc_many.cu", "tc_many", ()),
+         (CSRC / "host_scan.cu", "host_scan", ())]
 UNITS += [(CSRC / "simt.cu", f"simt_{dt}_{md}",
            (f"-DTTT_SIMT_BF16={int(dt == 'bf16')}", f"-DTTT_SIMT_MINIBATCH={int(md == 'mb')}"))
           for dt in ("f32", "bf16") for md in ("tok", "mb")]

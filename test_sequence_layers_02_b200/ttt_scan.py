@@ -76,6 +76,12 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.ttt_set_wait_limit.restype = i
+        L.ttt_scan_forward_host_workspace_bytes.argtypes = [i, i, i, i, u, i, i]
+        L.ttt_scan_forward_host_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_scan_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                            ctypes.c_float, u, i, vp, vp, vp, i, vp,
+                                            ctypes.c_size_t, vp]
+        L.ttt_scan_forward_host.restype = i
         L.ttt_scan_backward_workspace_bytes.argtypes = [i, i, i, u]
         L.ttt_scan_backward_workspace_bytes.restype = ctypes.c_size_t
         L.ttt_scan_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, ctypes.c_float,
@@ -108,47 +114,8 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
-         minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
-         b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
-         force_simt: bool = False, single_cta: bool = False, ablate: bool = False,
-         norm_match: bool = False, kq_silu: bool = False, want_chunks: bool = False,
-         want_grad_norms: bool = False, o: Optional[torch.Tensor] = None,
-         W_T: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
-    """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
-
-    q, k, v: [B, H, T, d] fp32 or bf16; eta_logit: [B, H, T] with the same
-    dtype; gate_logit: [B, H, T], or [B, H, T, d] for a per-feature gate, or
-    None; W0: [B, H, d, d] fp32 (z = W k);
-    gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
-    uint8 or None. ``out_dtype`` defaults to the input dtype. ``force_simt``
-    keeps mini-batch mode on the CUDA-core kernel; ``single_cta`` keeps
-    per-token mode on one CTA per head (see ``kernel_choice``). ``ablate``
-    selects the ablation gradient (the LayerNorm Jacobian applied to
-    -gamma * v), ``norm_match`` rescales it per token to the full gradient's norm.
-    ``kq_silu`` runs the `:mlp` variant (SiLU on every key and query).
-    ``want_grad_norms`` (with ``ablate``) also returns [B, H, T, 2]
-    fp32: per token the norms of the full and of the ablated gradient (zeros
-    on SKIP chunks), after W_T (and the chunk snapshots, if asked for).
-
-    CUDA tensors run on ``stream`` (default: the current stream) and return
-    without synchronising. CPU tensors take the end-to-end path: inputs are
-    copied to the current CUDA device, the scan runs there, and o / W_T are
-    copied back to host memory before returning; the copies and the scan are
-    all issued on ``stream``, so they are ordered.
-    """
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        s = stream if stream is not None else torch.cuda.current_stream(dev)
-        with torch.cuda.stream(s):
-            mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
-            q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask = map(
-                mv, (q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask))
-        o_dev, wt_dev = None, None
-    else:
-        o_dev, wt_dev = o, W_T
-        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+def _check_inputs(q, k, v, eta_logit, gate_logit, W0, gamma, beta, b, mask):
+    """Shapes, dtypes and contiguity of a scan's inputs; returns the sizes."""
     if q.dim() != 4:
         raise ValueError("q must be [B, H, T, d]")
     B, H, T, d = q.shape
@@ -174,13 +141,119 @@ def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
     if mask is not None:
         if tuple(mask.shape) != (B, n_chunks) or mask.dtype != torch.uint8 or not mask.is_contiguous():
             raise ValueError(f"mask: expected contiguous [B, {n_chunks}] uint8")
-    out_dtype = out_dtype or in_dtype
-    mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
+    return B, H, T, d, in_dtype, channel, n_chunks
+
+
+def _mode_bits(minibatch, lnjac, no_ln, in_dtype, out_dtype, force_simt, single_cta, ablate,
+               norm_match, channel, kq_silu) -> int:
+    return ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_dtype == torch.bfloat16 else 0) |
             (OUT_BF16 if out_dtype == torch.bfloat16 else 0) | (KERNEL_SIMT if force_simt else 0) |
             (KERNEL_SINGLE_CTA if single_cta else 0) | (GRAD_ABLATE if ablate else 0) |
             (GRAD_NORM_MATCH if norm_match else 0) | (GATE_CHANNEL if channel else 0) |
             (KQ_SILU if kq_silu else 0))
+
+
+def host_workspace_bytes(B: int, H: int, T: int, d: int, mode: int, b: int,
+                         seg_tokens: int = 0) -> int:
+    """Device workspace of ``ttt_scan_forward_host`` (0 for invalid sizes)."""
+    return int(lib().ttt_scan_forward_host_workspace_bytes(B, H, T, d, mode, b, seg_tokens))
+
+
+def _scan_host(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps, minibatch, lnjac, no_ln,
+               b, mask, out_dtype, force_simt, single_cta, ablate, norm_match, kq_silu, o, W_T,
+               stream, seg_tokens: int = 0):
+    """The end-to-end scan of host tensors through ``ttt_scan_forward_host``."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("eta_logit", eta_logit),
+                    ("gate_logit", gate_logit), ("W0", W0), ("gamma", gamma), ("beta", beta),
+                    ("mask", mask), ("o", o), ("W_T", W_T)):
+        if t is not None and t.is_cuda:
+            raise ValueError(f"{name}: with host inputs every tensor must be in host memory")
+    B, H, T, d, in_dtype, channel, n_chunks = _check_inputs(q, k, v, eta_logit, gate_logit, W0,
+                                                            gamma, beta, b, mask)
+    out_dtype = out_dtype or in_dtype
+    mode = _mode_bits(minibatch, lnjac, no_ln, in_dtype, out_dtype, force_simt, single_cta,
+                      ablate, norm_match, channel, kq_silu)
+    if o is None:
+        o = torch.empty((B, H, T, d), dtype=out_dtype, pin_memory=True)
+    if W_T is None:
+        W_T = torch.empty((B, H, d, d), dtype=torch.float32, pin_memory=True)
+    if (tuple(o.shape) != (B, H, T, d) or o.dtype != out_dtype or not o.is_contiguous() or
+            tuple(W_T.shape) != (B, H, d, d) or W_T.dtype != torch.float32 or
+            not W_T.is_contiguous()):
+        raise ValueError("o / W_T: expected contiguous [B, H, T, d] out_dtype / [B, H, d, d] float32")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    nbytes = host_workspace_bytes(B, H, T, d, mode, b, seg_tokens)
+    with torch.cuda.stream(s):
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    rc = lib().ttt_scan_forward_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(eta_logit), _ptr(gate_logit), _ptr(W0), _ptr(gamma),
+        _ptr(beta), B, H, T, d, float(eps), mode, int(b), _ptr(mask), _ptr(o), _ptr(W_T),
+        int(seg_tokens), _ptr(ws), ctypes.c_size_t(ws.numel()), ctypes.c_void_p(s.cuda_stream))
+    if rc != TTT_OK:
+        raise TTTScanError(rc)
+    rc = check_device_status(s)  # synchronises the stream: o and W_T are in host memory
+    if rc != TTT_OK:
+        raise TTTScanError(rc, "device")
+    return o, W_T
+
+
+def scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta, *, eps: float = 1e-6,
+         minibatch: bool = False, lnjac: bool = False, no_ln: bool = False,
+         b: int = 16, mask=None, out_dtype: Optional[torch.dtype] = None,
+         force_simt: bool = False, single_cta: bool = False, ablate: bool = False,
+         norm_match: bool = False, kq_silu: bool = False, want_chunks: bool = False,
+         want_grad_norms: bool = False, o: Optional[torch.Tensor] = None,
+         W_T: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """TTT-Linear scan ``(o, W_T) = scan(q, k, v, eta_logit, gate_logit, W0, gamma, beta)``.
+
+    q, k, v: [B, H, T, d] fp32 or bf16; eta_logit: [B, H, T] with the same
+    dtype; gate_logit: [B, H, T], or [B, H, T, d] for a per-feature gate, or
+    None; W0: [B, H, d, d] fp32 (z = W k);
+    gamma, beta: [H, d] fp32 (may be None with ``no_ln``); mask: [B, ceil(T/b)]
+    uint8 or None. ``out_dtype`` defaults to the input dtype. ``force_simt``
+    keeps mini-batch mode on the CUDA-core kernel; ``single_cta`` keeps
+    per-token mode on one CTA per head (see ``kernel_choice``). ``ablate``
+    selects the ablation gradient (the LayerNorm Jacobian applied to
+    -gamma * v), ``norm_match`` rescales it per token to the full gradient's norm.
+    ``kq_silu`` runs the `:mlp` variant (SiLU on every key and query).
+    ``want_grad_norms`` (with ``ablate``) also returns [B, H, T, 2]
+    fp32: per token the norms of the full and of the ablated gradient (zeros
+    on SKIP chunks), after W_T (and the chunk snapshots, if asked for).
+
+    CUDA tensors run on ``stream`` (default: the current stream) and return
+    without synchronising. CPU tensors take the end-to-end path, the library's
+    ``ttt_scan_forward_host``: the sequence is copied to the current CUDA device
+    in segments that overlap the scan of the previous segment and the copy-back
+    of the one before, and the call returns once o / W_T are in host memory
+    (page-locked host tensors make the copies asynchronous). With
+    ``want_chunks`` or ``want_grad_norms``, CPU tensors are copied in whole,
+    scanned and copied back on ``stream``.
+    """
+    host = not q.is_cuda
+    if host and not want_chunks and not want_grad_norms:
+        return _scan_host(q, k, v, eta_logit, gate_logit, W0, gamma, beta, eps=eps,
+                          minibatch=minibatch, lnjac=lnjac, no_ln=no_ln, b=b, mask=mask,
+                          out_dtype=out_dtype, force_simt=force_simt, single_cta=single_cta,
+                          ablate=ablate, norm_match=norm_match, kq_silu=kq_silu, o=o, W_T=W_T,
+                          stream=stream)
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(s):
+            mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+            q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask = map(
+                mv, (q, k, v, eta_logit, gate_logit, W0, gamma, beta, mask))
+        o_dev, wt_dev = None, None
+    else:
+        o_dev, wt_dev = o, W_T
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    B, H, T, d, in_dtype, channel, n_chunks = _check_inputs(q, k, v, eta_logit, gate_logit, W0,
+                                                            gamma, beta, b, mask)
+    out_dtype = out_dtype or in_dtype
+    mode = _mode_bits(minibatch, lnjac, no_ln, in_dtype, out_dtype, force_simt, single_cta,
+                      ablate, norm_match, channel, kq_silu)
     with torch.cuda.stream(s):
         if o_dev is None:
             o_dev = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)

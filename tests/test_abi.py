@@ -267,3 +267,55 @@ def test_backward_workspace_bytes_and_no_ln(lib):
     assert f(0, 3, 64, 2) == 0
     # no LayerNorm: gamma, beta, their gradients and the workspace may be absent
     assert bcall(lib, B=0, mode=4, gamma=None, beta=None, dgamma=None, dbeta=None, ws=None) == 0
+
+
+# ---- ttt_scan_forward_host: the end-to-end entry point (host buffers) ----
+def call_host(lib, **over):
+    """ttt_scan_forward_host with fake host addresses; every call below is
+    rejected (or is empty) before any copy is enqueued."""
+    a = dict(q=addr(0), k=addr(1), v=addr(2), eta=addr(3), gate=addr(4), W0=addr(5),
+             gamma=addr(6), beta=addr(7), B=2, H=3, T=40, d=64, eps=1e-6, mode=1 | 2 | 8 | 16,
+             b=16, mask=None, o=addr(8), W_T=addr(9), seg=0, ws=addr(12), ws_bytes=None)
+    a.update(over)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = lib.ttt_scan_forward_host_workspace_bytes(
+            a["B"], a["H"], a["T"], a["d"], a["mode"], a["b"], max(a["seg"], 0))
+    return lib.ttt_scan_forward_host(a["q"], a["k"], a["v"], a["eta"], a["gate"], a["W0"],
+                                     a["gamma"], a["beta"], a["B"], a["H"], a["T"], a["d"],
+                                     a["eps"], a["mode"], a["b"], a["mask"], a["o"], a["W_T"],
+                                     a["seg"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(seg=5), INVALID),                    # not a multiple of b
+    (dict(seg=-16), INVALID),
+    (dict(B=-1), INVALID), (dict(T=-1), INVALID), (dict(b=0), INVALID),
+    (dict(eps=float("nan")), INVALID), (dict(mode=1 << 11), INVALID),
+    (dict(q=None), INVALID), (dict(W0=None), INVALID), (dict(o=None), INVALID),
+    (dict(gamma=None), INVALID),
+    (dict(ws=None), INVALID), (dict(ws=addr(12, 8)), INVALID),   # missing / misaligned workspace
+    (dict(ws_bytes=1024), INVALID),            # workspace too small
+    (dict(o=addr(0)), INVALID),                # output over an input
+    (dict(W_T=addr(8)), INVALID),              # W_T over o
+    (dict(W_T=addr(5, 256)), INVALID),         # W_T partially over W0
+    (dict(d=32), UNSUPPORTED),
+    (dict(B=0), 0),                            # no heads: nothing to do
+], ids=lambda x: ",".join(x) if isinstance(x, dict) else str(x))
+def test_host_entry_checks(lib, over, want):
+    assert call_host(lib, **over) == want
+
+
+def test_host_workspace_bytes(lib):
+    f = lib.ttt_scan_forward_host_workspace_bytes
+    MB = 1 | 2 | 8 | 16
+    assert f(2, 32, 32768, 64, MB, 16, 5) == 0           # not a multiple of b
+    assert f(2, 32, 32768, 64, MB, 16, -16) == 0
+    assert f(-1, 32, 32768, 64, MB, 16, 0) == 0
+    default = f(2, 32, 32768, 64, MB, 16, 0)
+    assert default == f(2, 32, 32768, 64, MB, 16, 4096)  # the default: an eighth of T
+    # two segments' worth of inputs and outputs, plus the state
+    per_seg = 2 * 32 * 4096 * (3 * 64 * 2 + 2 * 2 + 64 * 2)
+    assert 2 * per_seg < default < 2 * per_seg + 2 * 32 * 64 * 64 * 4 + (1 << 20)
+    assert f(2, 32, 32768, 64, MB, 16, 1024) < default < f(2, 32, 32768, 64, MB, 16, 32768)
+    # a segment never exceeds the sequence
+    assert f(1, 1, 40, 64, MB, 16, 0) == f(1, 1, 40, 64, MB, 16, 1024)
