@@ -84,15 +84,26 @@ def _tc_takes_many(heads: int) -> bool:
     return 3 * waves3 < 2 * waves2
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments (a comment edit leaves the binary alone)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.sub(r"//[^\n]*", "", text)
+
+
 def _kernel_hash(kernel_key: str) -> str:
+    """Hash of what a kernel's binary is built from: its sources and includes,
+    the launcher, the public header (comments stripped) and the compiler flags."""
+    from test_sequence_layers_02_b200 import build
     kernel_key = _CAPTURE_KERNEL.get(kernel_key, kernel_key)
     pkg = ROOT / "test_sequence_layers_02_b200"
     files = sorted(set(_KERNEL_SOURCES[kernel_key] + ["ttt_scan.cu"]))
-    paths = [pkg / "csrc" / f for f in files] + [pkg / "build.py", ROOT / "include" / "ttt_scan.h"]
+    paths = [pkg / "csrc" / f for f in files] + [ROOT / "include" / "ttt_scan.h"]
     h = hashlib.sha256()
     for p in paths:
         h.update(p.name.encode())
-        h.update(p.read_bytes())
+        h.update(_code_only(p.read_text()).encode())
+    h.update(" ".join(build.NVCC_FLAGS).replace(str(ROOT), "").encode())
     return h.hexdigest()[:16]
 
 

@@ -158,7 +158,7 @@ int ttt_scan_kernel_choice(int B, int H, int T, int d, unsigned mode, int b);
  * ttt_scan_forward with its inputs and outputs in HOST memory: the end-to-end
  * call of a caller whose tensors live on the host. No page has this call; it
  * is plumbing around the same scan. The sequence is cut into segments of
- * `seg_tokens` tokens (0: the library's choice, about a sixteenth of T,
+ * `seg_tokens` tokens (0: the library's choice, about an eighth of T,
  * at least 256, a multiple of b and of 16); segment i+1's inputs are copied in while
  * segment i is scanned and segment i-1's outputs are copied out, and the
  * state W passes from one segment to the next on the device, exactly. o and

@@ -65,8 +65,8 @@ struct Layout {
   size_t total = 0;
 };
 
-// The default segment: about a sixteenth of the sequence (the last segment's
-// scan and copy-out are the part of the call no copy-in hides), at least 256 tokens,
+// The default segment: about an eighth of the sequence (measured at workload 5
+// against a sixteenth, a quarter and whole: the fastest), at least 256 tokens,
 // a multiple of b and of 16 (the per-token kernels' own chunk of up to 16
 // tokens then never straddles a segment boundary either).
 int segment_tokens(int T, int b, int seg_tokens) {
@@ -78,7 +78,7 @@ int segment_tokens(int T, int b, int seg_tokens) {
     r = t;
   }
   const long long unit = (long long)b / g * 16;
-  const long long part = ((long long)T + 15) / 16;
+  const long long part = ((long long)T + 7) / 8;
   const long long want = part > 256 ? part : 256;
   const long long s = (want + unit - 1) / unit * unit;
   return s > 0x40000000LL ? 0x40000000 : (int)s;

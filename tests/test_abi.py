@@ -312,9 +312,9 @@ def test_host_workspace_bytes(lib):
     assert f(2, 32, 32768, 64, MB, 16, -16) == 0
     assert f(-1, 32, 32768, 64, MB, 16, 0) == 0
     default = f(2, 32, 32768, 64, MB, 16, 0)
-    assert default == f(2, 32, 32768, 64, MB, 16, 2048)  # the default: a sixteenth of T
+    assert default == f(2, 32, 32768, 64, MB, 16, 4096)  # the default: an eighth of T
     # two segments' worth of inputs and outputs, plus the state
-    per_seg = 2 * 32 * 2048 * (3 * 64 * 2 + 2 * 2 + 64 * 2)
+    per_seg = 2 * 32 * 4096 * (3 * 64 * 2 + 2 * 2 + 64 * 2)
     assert 2 * per_seg < default < 2 * per_seg + 2 * 32 * 64 * 64 * 4 + (1 << 20)
     assert f(2, 32, 32768, 64, MB, 16, 1024) < default < f(2, 32, 32768, 64, MB, 16, 32768)
     # a segment never exceeds the sequence
