@@ -63,6 +63,7 @@ __device__ int g_ttt_status;
 
 struct TcMaps {
   CUtensorMap q, k, v;  // [B*H][T][64] bf16 as {64, T, B*H}, box {64, 16, 1}
+  CUtensorMap o;        // [B*H][T][64] of the output type, the same view and box
 };
 
 namespace tc {
@@ -97,7 +98,8 @@ struct TcLayout {
   static constexpr int oWb = oV + NST * kTile;              // [2] W_s bf16, 128 rows x 128 B, 128B-swizzled
   static constexpr int oAneg = oWb + 2 * 128 * 128;         // [2] 128 rows x 16 bf16 (core matrices)
   static constexpr int oXM = oAneg + 2 * 128 * 32;          // [3] {[Xg; M], [Y; N]}: 2 x 32 x 16 bf16
-  static constexpr int oZ = oXM + 3 * 2048;                 // [2][16][kZS] f32
+  static constexpr int oOut = oXM + 3 * 2048;               // [2][16][64] outputs (<= f32), TMA-stored
+  static constexpr int oZ = oOut + 2 * CB * D * 4;          // [2][16][kZS] f32
   static constexpr int oEta = oZ + 2 * CB * kZS * 4;        // [kSR][16] f32 (mask folded in)
   static constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
   static constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
@@ -140,6 +142,10 @@ __device__ __forceinline__ bool bar_any(int bar_id, int count, bool v) {
       : "r"((int)v), "r"(bar_id), "r"(count)
       : "memory");
   return r != 0;
+}
+// Named barrier over `count` threads.
+__device__ __forceinline__ void bar_sync(int bar_id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(bar))
@@ -184,6 +190,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   constexpr int NST = nst_for(MINB);
   using Lt = TcLayout<NST>;
   constexpr int oKQ = Lt::oKQ, oV = Lt::oV, oWb = Lt::oWb, oAneg = Lt::oAneg, oXM = Lt::oXM,
+                oOut = Lt::oOut,
                 oZ = Lt::oZ, oEta = Lt::oEta, oGate = Lt::oGate, oFlag = Lt::oFlag,
                 oGam = Lt::oGam, oBar = Lt::oBar, oTmem = Lt::oTmem, oAbort = Lt::oAbort;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -237,7 +244,6 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   const __nv_bfloat16* gel = static_cast<const __nv_bfloat16*>(p.eta_logit) + tok0;
   const __nv_bfloat16* ggl =
       p.gate_logit ? static_cast<const __nv_bfloat16*>(p.gate_logit) + tok0 : nullptr;
-  OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const long long lim = p.wait_limit;
   const long long drain_lim = 1LL << 24;
@@ -718,6 +724,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       const bool upd = upd_of(c);
       if ((c & 7) == 0) pre = fetch_block(c + 16);
       // ---- the MMAs of chunk c complete ----
+      if (tma_thread) bulk_wait_group_read<1>();  // the store of chunk c-2 has read its tile
       bool ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
       if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
         if (gt == 0) fail();
@@ -796,19 +803,25 @@ __global__ void __launch_bounds__(tc::NT, MINB)
           fail();
         }
       }
-      // ---- outputs o_c = gate * O_c^T ----
+      // ---- outputs o_c = gate * O_c^T: into a token-major tile, then one TMA
+      // store of the tile (rows past the sequence are outside the tensor map
+      // and are not written). The tile of chunk c-2 was last read by its store,
+      // which the storing thread waited for before this chunk's first barrier.
       {
         const float* gte = sGate + (c & (kSR - 1)) * CB + 8 * half;
-        const int n = chunk_len(c);
-        OutT* dst = go + (size_t)c * CB * D;
+        OutT* tile = reinterpret_cast<OutT*>(smem + oOut) + (c & 1) * CB * D;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = 8 * half + u;
-          if (t < n) dst[(size_t)t * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+        for (int u = 0; u < 8; ++u) tile[(8 * half + u) * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+        fence_proxy_async_smem();
+        bar_sync(kBarBulk, 128);
+        if (tma_thread) {
+          tma_store_3d(&maps.o, tile, 0, c * CB, (int)bh);
+          bulk_commit_group();
         }
       }
       if ((c & 7) == 4) store_block(c + 12, pre);
     }
+    if (tma_thread) bulk_wait_group<0>();  // every output store complete before the CTA ends
   } else if (issuer && run) {
     // =========================== issuer ===========================
     int wbuf = 0;  // the bf16 copy holding W_{s,c}

@@ -104,13 +104,31 @@ bool encode_qkv_map(CUtensorMap* map, const void* base, int T, long long heads, 
   return r == CUDA_SUCCESS;
 }
 
+// The output [B*H][T][64] (bf16 or fp32) in the same view and box, no swizzle:
+// the kernel stores a token-major tile of 16 rows per chunk.
+bool encode_out_map(CUtensorMap* map, void* base, int T, long long heads, bool bf16) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t elt = bf16 ? 2 : 4;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {64 * elt, (cuuint64_t)T * 64 * elt};
+  const cuuint32_t box[3] = {64, 16, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename OutT, int GM>
 int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   ttt::TcMaps maps;
   const long long heads = (long long)p.B * p.H;
   if (!encode_qkv_map(&maps.q, p.q, p.T, heads, true) ||
       !encode_qkv_map(&maps.k, p.k, p.T, heads, true) ||
-      !encode_qkv_map(&maps.v, p.v, p.T, heads, false))
+      !encode_qkv_map(&maps.v, p.v, p.T, heads, false) ||
+      !encode_out_map(&maps.o, p.o, p.T, heads, std::is_same<OutT, __nv_bfloat16>::value))
     return TTT_ERR_CUDA;
   // Up to one head per SM: the one-CTA-per-SM build (more registers per
   // thread, deeper staging); beyond that two CTAs share an SM. The kernel of
