@@ -31,10 +31,12 @@
 //   chain 0-3   read Z_k (TMEM, feature-major), transpose through shared
 //               memory, token-major LayerNorm + gradient (8 lanes per token,
 //               one shuffle round of shifted moments), write Aneg_k (bf16).
-//   bulk 4-7    W (fp32 TMEM) -> bf16 W_s; outputs o_c = gate * O_c^T;
-//               per-chunk scalars; one thread issues every TMA load of chunk
-//               x = {K_x, Q_{x-1}, V_x} (only Q_{x-1} for a SKIP chunk x),
-//               NST chunks ahead; SiLU variant: the in-place SiLU of a stage.
+//   bulk 4-7    W (fp32 TMEM) -> bf16 W_s; outputs o_c = gate * O_c^T into a
+//               token-major shared-memory tile (two, alternating), written to
+//               global memory by one TMA store per chunk; per-chunk scalars;
+//               one thread issues every TMA load of chunk x = {K_x, Q_{x-1},
+//               V_x} (only Q_{x-1} for a SKIP chunk x), NST chunks ahead, and
+//               every output store; SiLU variant: the in-place SiLU of a stage.
 //   issuer 8    (one thread) every tcgen05.mma and commit.
 //   gram 9      the Gram operand of chunk c (mma.sync, 64 x 16 x 64), as soon
 //               as its buffer is free (two chunks ahead of its use).
