@@ -108,8 +108,8 @@ enum {
  *   the B*H heads fit on the device as clusters of 4 CTAs (one per SM), each
  *   head's rows of W are split over such a cluster; otherwise (or with
  *   TTT_KERNEL_SINGLE_CTA) one CTA runs each head. Mini-batch mode runs the
- *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs and a per-token
- *   gate, and otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which
+ *   tcgen05 tensor-core kernel for d = 64, b = 16 with bf16 inputs (either gate
+ *   form), and otherwise (or with TTT_KERNEL_SIMT) the CUDA-core kernel, which
  *   takes b <= 16. Every gradient form (TTT_GRAD_LNJAC, TTT_NO_LN,
  *   TTT_GRAD_ABLATE, TTT_GRAD_NORM_MATCH) runs in both modes on every kernel.
  *   Other combinations return TTT_ERR_UNSUPPORTED.

@@ -92,7 +92,8 @@ constexpr int kZS = 72;             // row stride (floats) of the token-major Z 
 __host__ __device__ constexpr int nst_for(int minb) { return minb == 1 ? 10 : 6; }
 
 // shared memory (bytes from a 1024-aligned base)
-template <int NST>
+// GCH: the build for a per-feature gate (room for its logit tiles).
+template <int NST, bool GCH>
 struct TcLayout {
   static_assert(NST <= 11, "the scalar ring must run ahead of every TMA issue");
   static constexpr int oKQ = 0;                             // [NST][K_x | Q_{x-1}] 128B-swizzled
@@ -101,7 +102,8 @@ struct TcLayout {
   static constexpr int oAneg = oWb + 2 * 128 * 128;         // [2] 128 rows x 16 bf16 (core matrices)
   static constexpr int oXM = oAneg + 2 * 128 * 32;          // [3] {[Xg; M], [Y; N]}: 2 x 32 x 16 bf16
   static constexpr int oOut = oXM + 3 * 2048;               // [2][16][64] outputs (<= f32), TMA-stored
-  static constexpr int oZ = oOut + 2 * CB * D * 4;          // [2][16][kZS] f32
+  static constexpr int oGch = oOut + 2 * CB * D * 4;        // [3][16][64] bf16 per-feature gate logits
+  static constexpr int oZ = oGch + (GCH ? 3 * CB * D * 2 : 0);  // [2][16][kZS] f32
   static constexpr int oEta = oZ + 2 * CB * kZS * 4;        // [kSR][16] f32 (mask folded in)
   static constexpr int oGate = oEta + kSR * CB * 4;         // [kSR][16] f32
   static constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
@@ -115,10 +117,11 @@ struct TcLayout {
   static constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
   static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
 };
-template <int MINB>
-constexpr int smem_bytes() { return TcLayout<nst_for(MINB)>::kSmemBytes; }
-static_assert(smem_bytes<1>() <= 227 * 1024, "one CTA per SM must fit in shared memory");
-static_assert(2 * smem_bytes<kMinbMany>() <= 227 * 1024, "two CTAs per SM must fit in shared memory");
+template <int MINB, bool GCH>
+constexpr int smem_bytes() { return TcLayout<nst_for(MINB), GCH>::kSmemBytes; }
+static_assert(smem_bytes<1, true>() <= 227 * 1024, "one CTA per SM must fit in shared memory");
+static_assert(2 * smem_bytes<kMinbMany, true>() <= 227 * 1024,
+              "two CTAs per SM must fit in shared memory");
 static_assert(2 * kTmemCols <= 512, "two CTAs per SM must fit in TMEM");
 
 __device__ __forceinline__ int core_off(int row, int k) {
@@ -184,15 +187,17 @@ constexpr int kBarBulk = 3;
 
 // MINB = 2: two CTAs share an SM (heads above the SM count);
 // MINB = 1: one CTA per SM, for up to one head per SM (more registers).
-template <typename OutT, int GM, int MINB>
+// GCH: a per-feature gate (p.gate_channel); the build without it has none of
+// its shared memory or code.
+template <typename OutT, int GM, int MINB, bool GCH>
 __global__ void __launch_bounds__(tc::NT, MINB)
     scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps) {
   using namespace tc;
   using namespace sm100;
   constexpr int NST = nst_for(MINB);
-  using Lt = TcLayout<NST>;
+  using Lt = TcLayout<NST, GCH>;
   constexpr int oKQ = Lt::oKQ, oV = Lt::oV, oWb = Lt::oWb, oAneg = Lt::oAneg, oXM = Lt::oXM,
-                oOut = Lt::oOut,
+                oOut = Lt::oOut, oGch = Lt::oGch,
                 oZ = Lt::oZ, oEta = Lt::oEta, oGate = Lt::oGate, oFlag = Lt::oFlag,
                 oGam = Lt::oGam, oBar = Lt::oBar, oTmem = Lt::oTmem, oAbort = Lt::oAbort;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -244,8 +249,14 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   const int nc = (T + CB - 1) / CB;
   const size_t tok0 = (size_t)bh * T;
   const __nv_bfloat16* gel = static_cast<const __nv_bfloat16*>(p.eta_logit) + tok0;
-  const __nv_bfloat16* ggl =
-      p.gate_logit ? static_cast<const __nv_bfloat16*>(p.gate_logit) + tok0 : nullptr;
+  // the gate: one logit per token (through the scalar ring) or, with a
+  // per-feature gate, one per token and feature (a [16][64] tile per chunk)
+  const __nv_bfloat16* ggl = (p.gate_logit && !GCH)
+                                 ? static_cast<const __nv_bfloat16*>(p.gate_logit) + tok0
+                                 : nullptr;
+  const __nv_bfloat16* gch = (GCH && p.gate_logit)
+                                 ? static_cast<const __nv_bfloat16*>(p.gate_logit) + tok0 * D
+                                 : nullptr;
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const long long lim = p.wait_limit;
   const long long drain_lim = 1LL << 24;
@@ -720,11 +731,32 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     }
   } else if (is_bulk && run) {
     // =========================== bulk ===========================
+    // Per-feature gate: chunk x's [16][64] bf16 logits, one 16-byte piece per
+    // bulk thread, copied into tile x % 3 two chunks ahead (rows past the
+    // sequence zero-filled). One cp.async group per chunk, committed whether or
+    // not it copies anything, so the group count matches the chunk count. A
+    // call without that gate runs none of it: a cp.async wait would also wait
+    // for this warp's other loads in flight (the scalar ring's, which are
+    // meant to take four chunks).
+    auto load_gch = [&](int x) {
+      if (!gch) return;
+      if (x < nc) {
+        const int row = gt >> 3, piece = gt & 7;
+        const bool ok = x * CB + row < T;
+        const __nv_bfloat16* src = gch + (ok ? (size_t)(x * CB + row) * D + piece * 8 : 0);
+        cp_async16_zfill(smem + oGch + (x % 3) * CB * D * 2 + row * D * 2 + piece * 16, src,
+                         ok ? 16 : 0);
+      }
+      cp_async_commit_group();
+    };
+    load_gch(0);
+    load_gch(1);
     Raw pre{};
     int wbuf = 0;  // the bf16 copy holding W_{s,c}
     for (int c = 0; c < nc; ++c) {
       const bool upd = upd_of(c);
       if ((c & 7) == 0) pre = fetch_block(c + 16);
+      if (gch) cp_async_wait_group<1>();  // this thread's piece of chunk c's gate tile (the barrier below shares it)
       // ---- the MMAs of chunk c complete ----
       if (tma_thread) bulk_wait_group_read<1>();  // the store of chunk c-2 has read its tile
       bool ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
@@ -811,9 +843,20 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       // which the storing thread waited for before this chunk's first barrier.
       {
         const float* gte = sGate + (c & (kSR - 1)) * CB + 8 * half;
+        const __nv_bfloat16* gtile =
+            reinterpret_cast<const __nv_bfloat16*>(smem + oGch) + (c % 3) * CB * D;
         OutT* tile = reinterpret_cast<OutT*>(smem + oOut) + (c & 1) * CB * D;
+        if (gch) {  // (one branch per chunk: a per-element select would evaluate both sides)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) tile[(8 * half + u) * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+          for (int u = 0; u < 8; ++u) {
+            const int t = 8 * half + u;
+            const float g = sigmoidf_(__bfloat162float(gtile[t * D + fm]));
+            tile[t * D + fm] = from_f32<OutT>(g * ov[u]);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) tile[(8 * half + u) * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+        }
         fence_proxy_async_smem();
         bar_sync(kBarBulk, 128);
         if (tma_thread) {
@@ -822,7 +865,11 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         }
       }
       if ((c & 7) == 4) store_block(c + 12, pre);
+      // tile (c+2) % 3 was last read by the outputs of chunk c-1, before this
+      // chunk's first barrier
+      load_gch(c + 2);
     }
+    if (gch) cp_async_wait_group<0>();     // no gate copy in flight when the CTA ends
     if (tma_thread) bulk_wait_group<0>();  // every output store complete before the CTA ends
   } else if (issuer && run) {
     // =========================== issuer ===========================

@@ -1,5 +1,6 @@
 // Thin wrappers over the sm_100a instructions used by the tensor-core scan:
-// mbarriers (with bounded waits), TMA tile loads, tcgen05 TMEM allocation,
+// mbarriers (with bounded waits), TMA tile loads and stores, cp.async copies,
+// tcgen05 TMEM allocation,
 // MMA issue/commit and TMEM loads/stores, and the UMMA shared-memory and
 // instruction descriptors. No multicast form is used anywhere.
 #pragma once
@@ -77,6 +78,21 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// 16-byte asynchronous copy global -> shared; bytes past `src_bytes` (0 or
+// 16) are zero-filled and not read.
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's cp.async groups are incomplete.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

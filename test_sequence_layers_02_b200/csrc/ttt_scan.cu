@@ -57,7 +57,7 @@ int choose_kernel(long long heads, int T, int d, unsigned mode, int b, bool norm
   if (heads == 0) return TTT_KERNEL_NONE;
   const bool minibatch = mode & TTT_MODE_MINIBATCH;
   if (minibatch && (mode & TTT_IN_BF16) && d == 64 && b == ttt::tc::CB &&
-      !(mode & (TTT_KERNEL_SIMT | TTT_GATE_CHANNEL)) && T > 0)
+      !(mode & TTT_KERNEL_SIMT) && T > 0)
     return TTT_KERNEL_ID_TENSOR_CORE;
   if (!minibatch && d == 64 && !(mode & TTT_KERNEL_SINGLE_CTA) && !norms && T > 0) {
     if (heads <= ttt::cluster_capacity(mode, grad_variant_of(mode, norms)))
@@ -137,16 +137,22 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   // (waves at two per SM), i.e. for 2 to 3 heads per SM.
   const long long sms = ttt::device_sm_count();
   const bool one = heads <= sms;
-  if (sms > 0) {
+  if (sms > 0 && !p.gate_channel) {  // (the three-per-SM kernel has no per-feature gate)
     const long long waves2 = (heads + 2 * sms - 1) / (2 * sms);
     const long long waves3 = (heads + 3 * sms - 1) / (3 * sms);
     if (3 * waves3 < 2 * waves2)
       return ttt::launch_tc_many(p, &maps.q, &maps.k, &maps.v,
                                  std::is_same<OutT, __nv_bfloat16>::value, GM, stream);
   }
-  auto kernel = one ? ttt::scan_tc_kernel<OutT, GM, 1>
-                    : ttt::scan_tc_kernel<OutT, GM, ttt::tc::kMinbMany>;
-  const int smem = one ? ttt::tc::smem_bytes<1>() : ttt::tc::smem_bytes<ttt::tc::kMinbMany>();
+  constexpr int kMany = ttt::tc::kMinbMany;
+  const bool g = p.gate_channel != 0;
+  auto kernel = one ? (g ? ttt::scan_tc_kernel<OutT, GM, 1, true>
+                         : ttt::scan_tc_kernel<OutT, GM, 1, false>)
+                    : (g ? ttt::scan_tc_kernel<OutT, GM, kMany, true>
+                         : ttt::scan_tc_kernel<OutT, GM, kMany, false>);
+  const int smem = one ? (g ? ttt::tc::smem_bytes<1, true>() : ttt::tc::smem_bytes<1, false>())
+                       : (g ? ttt::tc::smem_bytes<kMany, true>()
+                            : ttt::tc::smem_bytes<kMany, false>());
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return TTT_ERR_CUDA;

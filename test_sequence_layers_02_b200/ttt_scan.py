@@ -358,13 +358,13 @@ def kernel_choice(B: int, H: int, T: int, d: int, *, minibatch: bool = False,
                   lnjac: bool = False, no_ln: bool = False, in_bf16: bool = False,
                   out_bf16: bool = False, b: int = 16, force_simt: bool = False,
                   single_cta: bool = False, ablate: bool = False, norm_match: bool = False,
-                  kq_silu: bool = False) -> int:
+                  kq_silu: bool = False, gate_channel: bool = False) -> int:
     """The KERNEL_* identifier ``scan`` would run for these sizes (launches nothing)."""
     mode = ((MODE_MINIBATCH if minibatch else 0) | (GRAD_LNJAC if lnjac else 0) |
             (NO_LN if no_ln else 0) | (IN_BF16 if in_bf16 else 0) | (OUT_BF16 if out_bf16 else 0) |
             (KERNEL_SIMT if force_simt else 0) | (KERNEL_SINGLE_CTA if single_cta else 0) |
             (GRAD_ABLATE if ablate else 0) | (GRAD_NORM_MATCH if norm_match else 0) |
-            (KQ_SILU if kq_silu else 0))
+            (KQ_SILU if kq_silu else 0) | (GATE_CHANNEL if gate_channel else 0))
     rc = lib().ttt_scan_kernel_choice(B, H, T, d, mode, b)
     if rc < 0:
         raise TTTScanError(rc, "ttt_scan_kernel_choice")

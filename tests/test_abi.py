@@ -200,7 +200,7 @@ def test_kernel_choice_without_launching(lib):
     assert f(2, 3, 40, 64, 0, 0) == INVALID
     assert f(2, 3, 40, 32, 0, 16) == UNSUPPORTED
     assert f(2, 3, 40, 64, MINIB, 17) == UNSUPPORTED
-    assert f(2, 3, 40, 64, MINIB | LNJAC | BF16 | (1 << 6), 16) == 1 # per-feature gate: CUDA cores
+    assert f(2, 3, 40, 64, MINIB | LNJAC | BF16 | (1 << 6), 16) == 3 # per-feature gate: tensor cores
     # per-token d = 64 picks the cluster kernel only where clusters fit on a device
     assert f(2, 3, 40, 64, LNJAC, 16) in (1, 2)
 

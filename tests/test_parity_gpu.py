@@ -441,23 +441,28 @@ GATE_CHANNEL = 1 << 6
     (2, 3, 77, 64, LNJAC, 16, False, True),      # per-token, one CTA per head
     (2, 3, 53, 16, 0, 16, False, False),          # d = 16
     (2, 3, 53, 64, MINIB | LNJAC, 16, False, False),
-    (2, 3, 77, 64, MINIB | LNJAC, 16, True, False),   # bf16 mini-batch: CUDA-core kernel
+    (2, 3, 77, 64, MINIB | LNJAC, 16, True, False),   # bf16 mini-batch: tensor-core kernel
 ], ids=["cluster", "single_cta", "d16", "minibatch_f32", "minibatch_bf16"])
 @pytest.mark.parametrize("with_mask", [False, True])
 def test_per_feature_gate(case, with_mask):
     from test_sequence_layers_02_b200 import ttt_scan
     B, H, T, d, mode, b, in_bf16, single_cta = case
-    want = (ttt_scan.KERNEL_CUDA_CORE if (single_cta or d != 64 or mode & MINIB)
+    tc = bool(mode & MINIB) and in_bf16
+    want = (ttt_scan.KERNEL_TENSOR_CORE if tc else
+            ttt_scan.KERNEL_CUDA_CORE if (single_cta or d != 64 or mode & MINIB)
             else ttt_scan.KERNEL_CUDA_CORE_CLUSTER)
-    assert ttt_scan.kernel_choice(B, H, T, d, minibatch=bool(mode & MINIB), lnjac=bool(mode & LNJAC),
-                                  in_bf16=in_bf16, b=b, single_cta=single_cta) in (want, ttt_scan.KERNEL_TENSOR_CORE)
+    got = ttt_scan.kernel_choice(B, H, T, d, minibatch=bool(mode & MINIB), lnjac=bool(mode & LNJAC),
+                                 in_bf16=in_bf16, b=b, single_cta=single_cta, gate_channel=True)
+    assert got == want or (want == ttt_scan.KERNEL_CUDA_CORE_CLUSTER and
+                           got == ttt_scan.KERNEL_CUDA_CORE)
     inp = make_inputs(B, H, T, d, seed=700 + T + d + mode, random_affine=True, in_bf16=in_bf16,
                       gate_channel=True, mask_p=0.5 if with_mask else None, b=b)
     o, W_T = gpu_scan(inp, in_bf16=in_bf16, eps=1e-6, b=b, lnjac=bool(mode & LNJAC),
                       minibatch=bool(mode & MINIB), single_cta=single_cta)
     ro, rW = oracle_scan(inp, eps=1e-6, mode=mode | GATE_CHANNEL, b=b)
-    assert_fp32_close(o, ro, "o")
-    assert_fp32_close(W_T, rW, "W_T")
+    check = assert_rrms if tc else assert_fp32_close   # bf16 operands on the tensor cores
+    check(o, ro, "o")
+    check(W_T, rW, "W_T")
 
 
 # ---------------------------------------------------------------------------

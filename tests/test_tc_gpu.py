@@ -116,3 +116,25 @@ def test_tc_wait_timeout_reports_and_recovers(BH):
     assert ttt_scan.check_device_status() == ttt_scan.TTT_OK
     ro, rW = oracle_scan(inp, eps=1e-6, mode=MINIB | LNJAC, b=16)
     assert_rrms(o.float().cpu().numpy(), ro, "o")
+
+
+@pytest.mark.parametrize("BH,T,out_bf16", [((2, 3), 77, True), ((2, 3), 160, False),
+                                            ((10, 30), 40, True)],
+                         ids=["6heads_ragged", "6heads_o32", "300heads"])
+def test_tc_per_feature_gate(BH, T, out_bf16):
+    """A per-feature gate [B, H, T, d] on the tensor-core kernel (its bulk warps
+    stage each chunk's gate logits in shared memory), with a mask and a ragged
+    tail; 300 heads keep to the two-per-SM build (the three-per-SM kernel has
+    no per-feature gate)."""
+    from test_sequence_layers_02_b200 import ttt_scan
+    B, H = BH
+    inp = make_inputs(B, H, T, 64, seed=600 + T + B, random_affine=True, in_bf16=True,
+                      gate_channel=True, mask_p=0.6, b=16)
+    assert ttt_scan.kernel_choice(B, H, T, 64, minibatch=True, lnjac=True, in_bf16=True,
+                                  out_bf16=out_bf16, b=16, gate_channel=True) == \
+        ttt_scan.KERNEL_TENSOR_CORE
+    o, W_T = gpu_scan(inp, in_bf16=True, out_bf16=out_bf16, eps=1e-6, b=16, minibatch=True,
+                      lnjac=True)
+    ro, rW = oracle_scan(inp, eps=1e-6, mode=MINIB | LNJAC | (1 << 6), b=16)
+    assert_rrms(o, ro, "o")
+    assert_rrms(W_T, rW, "W_T")
