@@ -32,10 +32,11 @@ int cluster_capacity(unsigned mode, int gm);
 int cluster_status_take();
 
 // Mini-batch d = 64 on the tensor cores, the build for three CTAs per SM
-// (scan_tc_many.cuh); q, k, v are the tensor maps of the three inputs. gm as
-// for launch_cluster.
+// (scan_tc_many.cuh); q, k, v, o are the tensor maps of the three inputs and
+// of the output. gm as for launch_cluster.
 int launch_tc_many(const ScanParams& p, const CUtensorMap* q, const CUtensorMap* k,
-                   const CUtensorMap* v, bool out_bf16, int gm, cudaStream_t stream);
+                   const CUtensorMap* v, const CUtensorMap* o, bool out_bf16, int gm,
+                   cudaStream_t stream);
 // Read and clear that kernel's device status word (as cluster_status_take).
 int tc_many_status_take();
 

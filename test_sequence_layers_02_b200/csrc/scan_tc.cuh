@@ -116,6 +116,7 @@ struct TcLayout {
   static constexpr int kSmemUsed = oAbort + 4;
   static constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
   static_assert(oWb % 1024 == 0, "128B-swizzled operands are 1024-aligned");
+  static_assert(oOut % 128 == 0 && oGch % 16 == 0, "TMA store source on 128 bytes; cp.async on 16");
 };
 template <int MINB, bool GCH>
 constexpr int smem_bytes() { return TcLayout<nst_for(MINB), GCH>::kSmemBytes; }

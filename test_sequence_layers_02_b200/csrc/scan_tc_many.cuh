@@ -60,6 +60,7 @@ __device__ int g_tcm_status;
 
 struct TcMaps {
   CUtensorMap q, k, v;  // [B*H][T][64] bf16 as {64, T, B*H}, box {64, 16, 1}
+  CUtensorMap o;        // [B*H][T][64] of the output type, the same view and box
 };
 
 namespace tc {
@@ -96,7 +97,11 @@ constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
 constexpr int kBars = NST + 2 + 2 + 2 + 4 + NST;
 constexpr int oTmem = oBar + kBars * 8;            // two TMEM base addresses
 constexpr int oAbort = oTmem + 8;
-constexpr int kSmemUsed = oAbort + 4;
+// [2][16][64] bf16 outputs (bf16 output only), TMA-stored a chunk later; a
+// tensor copy's shared-memory operand starts on 128 bytes
+constexpr int oOut = (oAbort + 4 + 127) & ~127;
+constexpr int kSmemUsed = oOut + 2 * CB * D * 2;
+static_assert(oOut % 128 == 0 && (CB * D * 2) % 128 == 0, "TMA store source on 128 bytes");
 constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
 static_assert(kSmemBytes <= 75 * 1024, "three CTAs per SM must fit in shared memory");
 template <int MINB>
@@ -201,6 +206,13 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   const __nv_bfloat16* ggl =
       p.gate_logit ? static_cast<const __nv_bfloat16*>(p.gate_logit) + tok0 : nullptr;
   OutT* go = static_cast<OutT*>(p.o) + tok0 * D;
+  // bf16 outputs go through a shared-memory tile and a TMA store (one thread,
+  // one store per chunk, issued after the next chunk's first bulk barrier);
+  // fp32 outputs (whose tile would not fit three CTAs per SM) are stored directly
+  constexpr bool kTileOut = sizeof(OutT) == 2;
+  auto out_tile = [&](int x) {
+    return reinterpret_cast<OutT*>(smem + oOut) + (x & 1) * CB * D;
+  };
   float* Wc = p.W_chunks ? p.W_chunks + (size_t)bh * (p.n_mask_chunks + 1) * D * D : nullptr;
   const long long lim = p.wait_limit;
   const long long drain_lim = 1LL << 24;
@@ -634,16 +646,25 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   } else if (is_bulk && run) {
     // =========================== bulk ===========================
     Raw pre{};
+    bool finished = true;
     for (int c = 0; c < nc; ++c) {
       const bool upd = sFlag[c & (kSR - 1)] != 0;
       if ((c & 7) == 0) pre = fetch_block(c + 16);
+      // the store of chunk c-2 has read its tile (chunk c writes it again)
+      if (kTileOut && tma_thread) bulk_wait_group_read<0>();
       // ---- MMAc and MMA3 of chunk c complete ----
       bool ok = mbar_wait_bounded(bar_w, (uint32_t)(c & 1), lim);
       if (bar_any(kBarBulk, 128, !ok || *sAbort)) {
         if (gt == 0) fail();
+        finished = false;
         break;
       }
       tc_fence_after();
+      // chunk c-1's outputs, written to its tile before the barrier above
+      if (kTileOut && tma_thread && c >= 1) {
+        tma_store_3d(&maps.o, out_tile(c - 1), 0, (c - 1) * CB, (int)bh);
+        bulk_commit_group();
+      }
       // ---- W_{s,c+1} (fp32 TMEM) -> bf16 operand; snapshot ----
       const int row = wq * 32 + lane;
       if (upd) {
@@ -721,15 +742,33 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         tmem_ld8(tmem + tlane + col_o((c + 1) & 1) + 8 * half, ov);
         tmem_wait_ld();
         const float* gte = sGate + (c & (kSR - 1)) * CB + 8 * half;
-        const int n = chunk_len(c);
-        OutT* dst = go + (size_t)c * CB * D;
+        if (kTileOut) {  // rows past the sequence are outside the tensor map
+          OutT* tile = out_tile(c);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = 8 * half + u;
-          if (t < n) dst[(size_t)t * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+          for (int u = 0; u < 8; ++u)
+            tile[(8 * half + u) * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+          fence_proxy_async_smem();
+        } else {
+          const int n = chunk_len(c);
+          OutT* dst = go + (size_t)c * CB * D;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int t = 8 * half + u;
+            if (t < n) dst[(size_t)t * D + fm] = from_f32<OutT>(gte[u] * ov[u]);
+          }
         }
       }
       if ((c & 7) == 4) store_block(c + 12, pre);
+    }
+    if (kTileOut) {
+      bar_sync(kBarBulk, 128);  // every bulk thread's last tile written
+      if (tma_thread) {
+        if (finished && nc > 0) {
+          tma_store_3d(&maps.o, out_tile(nc - 1), 0, (nc - 1) * CB, (int)bh);
+          bulk_commit_group();
+        }
+        bulk_wait_group<0>();  // every output store complete before the CTA ends
+      }
     }
   } else if (issuer && run) {
     // =========================== issuer ===========================

@@ -35,11 +35,13 @@ int by_gm(const ttt::ScanParams& p, const ttt::tcm::TcMaps& maps, int gm, cudaSt
 namespace ttt {
 
 int launch_tc_many(const ScanParams& p, const CUtensorMap* q, const CUtensorMap* k,
-                   const CUtensorMap* v, bool out_bf16, int gm, cudaStream_t stream) {
+                   const CUtensorMap* v, const CUtensorMap* o, bool out_bf16, int gm,
+                   cudaStream_t stream) {
   tcm::TcMaps maps;
   maps.q = *q;
   maps.k = *k;
   maps.v = *v;
+  maps.o = *o;
   return out_bf16 ? by_gm<__nv_bfloat16>(p, maps, gm, stream) : by_gm<float>(p, maps, gm, stream);
 }
 

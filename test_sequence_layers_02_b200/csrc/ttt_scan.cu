@@ -141,7 +141,7 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
     const long long waves2 = (heads + 2 * sms - 1) / (2 * sms);
     const long long waves3 = (heads + 3 * sms - 1) / (3 * sms);
     if (3 * waves3 < 2 * waves2)
-      return ttt::launch_tc_many(p, &maps.q, &maps.k, &maps.v,
+      return ttt::launch_tc_many(p, &maps.q, &maps.k, &maps.v, &maps.o,
                                  std::is_same<OutT, __nv_bfloat16>::value, GM, stream);
   }
   constexpr int kMany = ttt::tc::kMinbMany;
