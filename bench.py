@@ -92,12 +92,16 @@ def _code_only(text: str) -> str:
 
 
 def _kernel_hash(kernel_key: str) -> str:
-    """Hash of what a kernel's binary is built from: its sources and includes,
-    the launcher, the public header (comments stripped) and the compiler flags."""
+    """Hash of what a kernel's binary is built from: its sources and includes
+    (with ttt_scan.cu where that unit builds or configures it), the public
+    header (comments stripped) and the compiler flags."""
     from test_sequence_layers_02_b200 import build
     kernel_key = _CAPTURE_KERNEL.get(kernel_key, kernel_key)
     pkg = ROOT / "test_sequence_layers_02_b200"
-    files = sorted(set(_KERNEL_SOURCES[kernel_key] + ["ttt_scan.cu"]))
+    # ttt_scan.cu builds the tensor-core and decode kernels and encodes the
+    # tensor maps; the other kernels are objects of their own
+    own = ["ttt_scan.cu"] if kernel_key in ("scan_tc", "scan_tc_many", "decode_step") else []
+    files = sorted(set(_KERNEL_SOURCES[kernel_key] + own))
     paths = [pkg / "csrc" / f for f in files] + [ROOT / "include" / "ttt_scan.h"]
     h = hashlib.sha256()
     for p in paths:
