@@ -72,7 +72,10 @@ namespace tc {
 
 constexpr int D = 64;
 constexpr int CB = 16;              // chunk (b)
-constexpr int NT = 320;             // 4 chain + 4 bulk + 1 issuer + 1 Gram warps
+// threads: 4 chain + 4 bulk + 1 issuer + 1 Gram warps, and with one CTA per SM
+// a producer warp for the TMA loads (two CTAs per SM issue them from a bulk
+// thread: a further warp would cap the registers below what that build needs)
+__host__ __device__ constexpr int nt_for(int minb) { return minb == 1 ? 352 : 320; }
 constexpr int kMinbMany = 2;        // CTAs per SM of the build for more heads than SMs
 constexpr int kSR = 32;             // scalar ring (chunks)
 constexpr uint32_t kTmemCols = 256;
@@ -109,8 +112,8 @@ struct TcLayout {
   static constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
   static constexpr int oGam = oFlag + kSR * 4;              // gamma, beta [2][64] f32, sum gamma^2, sum gamma*beta
   static constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
-  // tma[NST], rdy[NST], g[2], z[2], xm[3], w, wb, pro
-  static constexpr int kBars = 2 * NST + 2 + 2 + 3 + 3;
+  // tma[NST], rdy[NST], free[NST], g[2], z[2], xm[3], w, wb, pro
+  static constexpr int kBars = 3 * NST + 2 + 2 + 3 + 3;
   static constexpr int oTmem = oBar + kBars * 8;            // TMEM base address
   static constexpr int oAbort = oTmem + 8;
   static constexpr int kSmemUsed = oAbort + 4;
@@ -191,11 +194,12 @@ constexpr int kBarBulk = 3;
 // GCH: a per-feature gate (p.gate_channel); the build without it has none of
 // its shared memory or code.
 template <typename OutT, int GM, int MINB, bool GCH>
-__global__ void __launch_bounds__(tc::NT, MINB)
+__global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
     scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps) {
   using namespace tc;
   using namespace sm100;
   constexpr int NST = nst_for(MINB);
+  constexpr bool kProducer = MINB == 1;  // a warp of its own issues the TMA loads
   using Lt = TcLayout<NST, GCH>;
   constexpr int oKQ = Lt::oKQ, oV = Lt::oV, oWb = Lt::oWb, oAneg = Lt::oAneg, oXM = Lt::oXM,
                 oOut = Lt::oOut, oGch = Lt::oGch,
@@ -216,7 +220,10 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   // transformed in place (bulk, one arrival per warp); otherwise the TMA
   // barrier is used
   uint64_t* bar_rdy = bar_tma + NST;
-  uint64_t* bar_g = bar_rdy + NST;   // [2] Aneg_k written (chain, one arrival per warp)
+  // [NST] stage x % NST no longer read: every reader of chunk x's stage
+  // completed before bar_w of chunk x (bulk, one arrival once it saw bar_w)
+  uint64_t* bar_free = bar_rdy + NST;
+  uint64_t* bar_g = bar_free + NST;  // [2] Aneg_k written (chain, one arrival per warp)
   uint64_t* bar_z = bar_g + 2;       // [2] Z_k complete in TMEM (commit)
   uint64_t* bar_xm = bar_z + 2;      // [3] Gram operand of chunk x written (Gram warp, 1 arrival)
   uint64_t* bar_w = bar_xm + 3;      // a chunk's MMAs complete (commit)
@@ -237,7 +244,9 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   const bool is_bulk = warp >= 4 && warp < 8;
   const bool issuer = (tid == 256);
   const bool is_gram = warp == 9;
-  const bool tma_thread = (tid == 224);        // bulk warp 7, lane 0
+  const bool tma_thread = (tid == 224);        // bulk warp 7, lane 0: the output stores
+  // every TMA load: warp 10, lane 0 (one CTA per SM) or the store thread
+  const bool producer = kProducer ? (tid == 320) : tma_thread;
   const int wq = warp & 3;                     // TMEM lane quarter of this warp
   const uint32_t tlane = (uint32_t)(wq * 32) << 16;
   const int fm = (wq & 1) * 32 + lane;         // feature-major role: feature
@@ -432,6 +441,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar_tma[s], 1);
       mbar_init(&bar_rdy[s], 4);
+      mbar_init(&bar_free[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_g[s], 4);
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sTmem[0];
-  if (tma_thread) {
+  if (producer) {
     prefetch_tensormap(&maps.q);
     prefetch_tensormap(&maps.k);
     prefetch_tensormap(&maps.v);
@@ -766,6 +776,10 @@ __global__ void __launch_bounds__(tc::NT, MINB)
         break;
       }
       tc_fence_after();
+      // stage c may be refilled: every reader of its tiles (MMA1 of chunk c-2,
+      // the Gram operands of chunks c-2 .. c, MMA3 of chunk c, the chain's V_c)
+      // completed before bar_w of this chunk
+      if (kProducer && gt == 0) mbar_arrive(&bar_free[c % NST]);
       // ---- outputs O_c = A(c+1) + B(c+1) (query halves) ----
       float ov[8];
       {
@@ -821,10 +835,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       }
       tc_fence_before();
       mbar_arrive_warp(bar_wb);
-      // refill stage c % NST with load c + NST: every reader of its tiles (MMA1
-      // of chunk c-2, the Gram operands of chunks c-1 and c, MMA3 of chunk c,
-      // the chain's V_c) completed before bar_w of this chunk
-      if (tma_thread && c + NST <= nc) {
+      if (!kProducer && tma_thread && c + NST <= nc) {  // refill stage c (see above)
         fence_proxy_async_smem();
         issue_tma(c + NST);
       }
@@ -872,6 +883,20 @@ __global__ void __launch_bounds__(tc::NT, MINB)
     }
     if (gch) cp_async_wait_group<0>();     // no gate copy in flight when the CTA ends
     if (tma_thread) bulk_wait_group<0>();  // every output store complete before the CTA ends
+  } else if (kProducer && producer && run) {
+    // =========================== producer ===========================
+    // load x goes into stage x % NST once the bulk has seen bar_w of chunk
+    // x - NST. Phase x - NST of that stage's barrier cannot be overtaken: its
+    // next phase needs chunk x's MMAs, which need load x.
+    for (int x = NST; x <= nc; ++x) {
+      const int y = x - NST;
+      if (!mbar_wait_bounded(&bar_free[y % NST], (uint32_t)((y / NST) & 1), lim) || *sAbort) {
+        fail();
+        break;
+      }
+      fence_proxy_async_smem();
+      issue_tma(x);
+    }
   } else if (issuer && run) {
     // =========================== issuer ===========================
     int wbuf = 0;  // the bf16 copy holding W_{s,c}
@@ -934,7 +959,7 @@ __global__ void __launch_bounds__(tc::NT, MINB)
       mma_commit(bar_w);
       if (w_issued > 0) mbar_wait_bounded(bar_w, (uint32_t)((w_issued - 1) & 1), drain_lim);
       mbar_wait_bounded(bar_w, (uint32_t)(w_issued & 1), drain_lim);
-    } else if (tma_thread) {
+    } else if (producer) {
       // every TMA stage that may still be loading
       for (int x = (tma_issued > NST ? tma_issued - NST : 0); x < tma_issued; ++x)
         mbar_wait_bounded(&bar_tma[x % NST], tma_parity(x), drain_lim);

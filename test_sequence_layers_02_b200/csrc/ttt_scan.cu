@@ -156,7 +156,7 @@ int launch_tc(const ttt::ScanParams& p, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return TTT_ERR_CUDA;
-  kernel<<<(unsigned)heads, ttt::tc::NT, smem, stream>>>(p, maps);
+  kernel<<<(unsigned)heads, ttt::tc::nt_for(one ? 1 : kMany), smem, stream>>>(p, maps);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
