@@ -27,19 +27,22 @@
 // (W_s in bf16 is double-buffered, so MMA1 reading one copy overlaps the refresh
 // of the other).
 //
-// Warps (320 threads):
+// Warps (352 threads with one CTA per SM, 320 with two):
 //   chain 0-3   read Z_k (TMEM, feature-major), transpose through shared
 //               memory, token-major LayerNorm + gradient (8 lanes per token,
 //               one shuffle round of shifted moments), write Aneg_k (bf16).
 //   bulk 4-7    W (fp32 TMEM) -> bf16 W_s; outputs o_c = gate * O_c^T into a
 //               token-major shared-memory tile (two, alternating), written to
-//               global memory by one TMA store per chunk; per-chunk scalars;
-//               one thread issues every TMA load of chunk x = {K_x, Q_{x-1},
-//               V_x} (only Q_{x-1} for a SKIP chunk x), NST chunks ahead, and
-//               every output store; SiLU variant: the in-place SiLU of a stage.
+//               global memory by one TMA store per chunk (one thread issues
+//               every output store); per-chunk scalars; SiLU variant: the
+//               in-place SiLU of a stage.
 //   issuer 8    (one thread) every tcgen05.mma and commit.
 //   gram 9      the Gram operand of chunk c (mma.sync, 64 x 16 x 64), as soon
 //               as its buffer is free (two chunks ahead of its use).
+//   producer 10 (one thread; one CTA per SM) every TMA load of chunk x =
+//               {K_x, Q_{x-1}, V_x} (only Q_{x-1} for a SKIP chunk x), NST
+//               chunks ahead, once the bulk has freed the stage; with two CTAs
+//               per SM the bulk's store thread issues them instead.
 // M = 128 everywhere: A operands stack two copies of their 64 rows, so TMEM
 // lanes 0-63 and 64-127 hold identical d-row results and every warp quarter
 // reads its own lanes.
