@@ -115,8 +115,8 @@ struct TcLayout {
   static constexpr int oFlag = oGate + kSR * CB * 4;        // [kSR] int
   static constexpr int oGam = oFlag + kSR * 4;              // gamma, beta [2][64] f32, sum gamma^2, sum gamma*beta
   static constexpr int oBar = oGam + 2 * D * 4 + 16;        // mbarriers
-  // tma[NST], rdy[NST], free[NST], g[2], z[2], xm[3], w, wb, pro
-  static constexpr int kBars = 3 * NST + 2 + 2 + 3 + 3;
+  // tma[NST], rdy[NST], free[NST], g[2], z[2], w, wb, pro
+  static constexpr int kBars = 3 * NST + 2 + 2 + 3;
   static constexpr int oTmem = oBar + kBars * 8;            // TMEM base address
   static constexpr int oAbort = oTmem + 8;
   static constexpr int kSmemUsed = oAbort + 4;
@@ -226,10 +226,12 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
   // [NST] stage x % NST no longer read: every reader of chunk x's stage
   // completed before bar_w of chunk x (bulk, one arrival once it saw bar_w)
   uint64_t* bar_free = bar_rdy + NST;
-  uint64_t* bar_g = bar_free + NST;  // [2] Aneg_k written (chain, one arrival per warp)
+  // [2] chunk k ready for the issuer: Aneg_k written (chain, one arrival per
+  // warp) and the Gram operand of chunk k written, stage k+2 landed (Gram
+  // warp, one arrival): five arrivals
+  uint64_t* bar_g = bar_free + NST;
   uint64_t* bar_z = bar_g + 2;       // [2] Z_k complete in TMEM (commit)
-  uint64_t* bar_xm = bar_z + 2;      // [3] Gram operand of chunk x written (Gram warp, 1 arrival)
-  uint64_t* bar_w = bar_xm + 3;      // a chunk's MMAs complete (commit)
+  uint64_t* bar_w = bar_z + 2;       // a chunk's MMAs complete (commit)
   uint64_t* bar_wb = bar_w + 1;      // W read from TMEM and W_s bf16 refreshed (bulk, 4 warps)
   uint64_t* bar_pro = bar_wb + 1;    // prologue MMAs complete (commit)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + oTmem);
@@ -447,10 +449,9 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
       mbar_init(&bar_free[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar_g[s], 4);
+      mbar_init(&bar_g[s], 5);
       mbar_init(&bar_z[s], 1);
     }
-    for (int s = 0; s < 3; ++s) mbar_init(&bar_xm[s], 1);
     mbar_init(bar_w, 1);
     mbar_init(bar_wb, 4);
     mbar_init(bar_pro, 1);
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
   }
   if (is_gram && !pro_bad) {
     if (upd_of(0)) gram_operand(0);
-    mbar_arrive_warp(&bar_xm[0]);
+    mbar_arrive_warp(&bar_g[0]);  // (stages 0 .. 2 were waited above)
   }
   tc_fence_before();
   __syncthreads();
@@ -722,16 +723,21 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
     // chunk c-3, all complete once Z_{c-1} is (its commit follows them). It
     // reads stages c .. c+2; a stage this warp has seen land (seen > x) needs
     // no second wait (each wait costs a few hundred cycles even when the phase
-    // is long complete)
+    // is long complete). Every chunk, SKIP or not, waits through stage c+2
+    // before its arrival, so the issuer's wait for chunk c also covers the
+    // stage its MMA1 reads (a stage is reloaded only after bar_w of its chunk,
+    // which needs this warp's arrival for that chunk, so no phase is missed)
     int seen = 3;  // stages 0 .. 2: waited by every thread in the prologue
     for (int c = 1; c < nc; ++c) {
       bool ok = (c == 1) ? mbar_wait_bounded(bar_pro, 0, lim)
                          : mbar_wait_bounded(&bar_z[(c - 1) & 1], (uint32_t)(((c - 2) >> 1) & 1),
                                              lim);
-      if (ok && upd_of(c)) {
+      if (ok) {
         const int top = min(c + 2, nc);
         for (int x = max(seen, c); x <= top; ++x) ok = ok && wait_stage(x);
         seen = max(seen, top + 1);
+      }
+      if (ok && upd_of(c)) {
         ok = __all_sync(0xffffffffu, ok);
         if (ok) gram_operand(c);
       }
@@ -741,7 +747,7 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
         break;
       }
       if (__any_sync(0xffffffffu, *sAbort != 0)) break;
-      mbar_arrive_warp(&bar_xm[c % 3]);
+      mbar_arrive_warp(&bar_g[c & 1]);
     }
   } else if (is_bulk && run) {
     // =========================== bulk ===========================
@@ -906,8 +912,8 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
     for (int c = 0; c < nc; ++c) {
       const bool upd = upd_of(c);
       // the Gram operand of chunk c and Aneg_c
-      bool ok = mbar_wait_bounded(&bar_xm[c % 3], (uint32_t)((c / 3) & 1), lim) &&
-                mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim);
+      // (one barrier: the Gram operand, Aneg_c and stage c+2)
+      bool ok = mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim);
       if (!ok || *sAbort) {
         fail();
         break;
@@ -938,14 +944,8 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
       ++w_issued;
       if (c + 1 < nc) {
         // A(c+2) = W_{s,c} [K_{c+2}; Q_{c+1}]^T from the bf16 copy of W_{s,c}.
-        // Stage c+2 has landed: the Gram warp saw it before it wrote the operand
-        // of an updating chunk c (waited for above); otherwise wait here
-        ok = upd || c + 2 <= 2 || wait_stage(c + 2);
-        if (!ok || *sAbort) {
-          fail();
-          break;
-        }
-        tc_fence_after();
+        // Stage c+2 has landed: the Gram warp saw it before its arrival for
+        // chunk c, waited for above
         mma_ws(tmem + col_a(c + 2), wbuf, c + 2);
       }
       if (upd) wbuf ^= 1;
