@@ -53,6 +53,28 @@ def test_tc_all_occupancy_builds(grad, BH):
     assert_rrms(W_T, rW, "W_T")
 
 
+@pytest.mark.parametrize("BH,T", [((2, 3), 161), ((2, 3), 176), ((2, 3), 177), ((2, 3), 330),
+                                  ((10, 15), 97), ((10, 15), 112), ((10, 15), 113),
+                                  ((10, 15), 330)],
+                         ids=["1perSM-11chunks", "1perSM-11full", "1perSM-12chunks",
+                              "1perSM-21chunks", "2perSM-7chunks", "2perSM-7full",
+                              "2perSM-8chunks", "2perSM-21chunks"])
+def test_tc_stage_ring_boundaries(BH, T):
+    """The TMA stage ring refills stage x % NST with chunk x once chunk x - NST
+    has finished: ten stages with one CTA per SM (6 heads), six with two (150
+    heads on 148 SMs). Lengths just past the ring (the first refills, a full
+    last chunk or a one-token one) and several times around it, with a
+    SKIP/UPDATE mask, against the oracle."""
+    B, H = BH
+    inp = make_inputs(B, H, T, 64, seed=270 + T + B, random_affine=True, in_bf16=True,
+                      mask_p=0.6, b=16)
+    o, W_T = gpu_scan(inp, in_bf16=True, out_bf16=True, eps=1e-6, b=16, minibatch=True,
+                      lnjac=True)
+    ro, rW = oracle_scan(inp, eps=1e-6, mode=MINIB | LNJAC, b=16)
+    assert_rrms(o, ro, "o")
+    assert_rrms(W_T, rW, "W_T")
+
+
 @pytest.mark.parametrize("T", [64, 77])
 def test_tc_mask_is_bit_exact_on_skipped_chunks(T):
     B, H, b = 2, 3, 16
