@@ -55,16 +55,19 @@ def test_tc_all_occupancy_builds(grad, BH):
 
 @pytest.mark.parametrize("BH,T", [((2, 3), 161), ((2, 3), 176), ((2, 3), 177), ((2, 3), 330),
                                   ((10, 15), 97), ((10, 15), 112), ((10, 15), 113),
-                                  ((10, 15), 330)],
+                                  ((10, 15), 330), ((10, 30), 80), ((10, 30), 81),
+                                  ((10, 30), 97), ((10, 30), 330)],
                          ids=["1perSM-11chunks", "1perSM-11full", "1perSM-12chunks",
                               "1perSM-21chunks", "2perSM-7chunks", "2perSM-7full",
-                              "2perSM-8chunks", "2perSM-21chunks"])
+                              "2perSM-8chunks", "2perSM-21chunks", "3perSM-5chunks",
+                              "3perSM-6chunks", "3perSM-7chunks", "3perSM-21chunks"])
 def test_tc_stage_ring_boundaries(BH, T):
     """The TMA stage ring refills stage x % NST with chunk x once chunk x - NST
     has finished: ten stages with one CTA per SM (6 heads), six with two (150
-    heads on 148 SMs). Lengths just past the ring (the first refills, a full
-    last chunk or a one-token one) and several times around it, with a
-    SKIP/UPDATE mask, against the oracle."""
+    heads on 148 SMs), five in the three-per-SM kernel (300 heads). Lengths at
+    and just past the ring (the first refills, a full last chunk or a
+    one-token one) and several times around it, with a SKIP/UPDATE mask,
+    against the oracle."""
     B, H = BH
     inp = make_inputs(B, H, T, 64, seed=270 + T + B, random_affine=True, in_bf16=True,
                       mask_p=0.6, b=16)
