@@ -911,7 +911,8 @@ __global__ void __launch_bounds__(tc::nt_for(MINB), MINB)
     int wbuf = 0;  // the bf16 copy holding W_{s,c}
     for (int c = 0; c < nc; ++c) {
       const bool upd = upd_of(c);
-      // the Gram operand of chunk c, Aneg_c and stage c+2 (one barrier)
+      // the Gram operand of chunk c, Aneg_c and stage c+2
+      // (one barrier for the three)
       bool ok = mbar_wait_bounded(&bar_g[c & 1], (uint32_t)((c >> 1) & 1), lim);
       if (!ok || *sAbort) {
         fail();
